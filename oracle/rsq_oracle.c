@@ -1,0 +1,441 @@
+/*
+ * rsq_oracle.c -- CPU oracle for the quantized recurrent-state decode step.
+ *
+ * TEST INFRASTRUCTURE.  Only the test suite, the package smoke check and the
+ * benchmark's CPU-baseline / reference arm may load this library.  The product
+ * path (the CUDA library) never calls it and shares no code with it.
+ *
+ * Plain, single-threaded, obviously-correct C.  Every function cites the passage
+ * of the method description it follows.  Sources:
+ *   [LoReS]  "Quantizing Recurrent Language Models Is Easier Than You Think"
+ *            (blog post of the LoReS paper): sections "(1/4) Scale grouping",
+ *            "(2/4) Mixed precision", "(3/4) Rounding", "(4/4) Rotations".
+ *   [LRB]    "Preserving Updates in Low-Bit Recurrent State Quantization",
+ *            abstract (state requantized after every update).
+ *   [FEED]   "When Dynamic Scaling Fails: A Scale-State Feedback Governs
+ *            Recurrent-State Quantization ...", key points (dynamic scale).
+ *   [PHILOX] Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as
+ *            1, 2, 3", SC'11 -- Philox4x32-10 block function.
+ *   Recurrences: gated delta rule and Mamba-2 scalar-decay SSM as named in
+ *   [LRB] abstract and [LoReS] Table 1.
+ *
+ * Orientation.  The state of one head is stored with the key / SSM-state axis i
+ * as rows (dk rows) and the value / head-dim axis j as columns (dv columns):
+ *     GDN     S_t = alpha*(I - beta k k^T) S_{t-1} + beta k v^T,   o_j = sum_i S_ij q_i
+ *     Mamba-2 S_t = exp(dt*A) S_{t-1} + dt B x^T,                  y_j = sum_i S_ij C_i + D x_j
+ * A value channel is a column; its scale is s_j = max_i |S_ij| / r with
+ * r = 2^(b-1) - 1 ([LoReS] (1/4), Proposition "per-channel readout error").
+ *
+ * Two evaluation modes, both in binary32 (the workloads fix FP32 math):
+ *   ORC_PLAIN      the literal definition: dequantize (c*s), sequential sums
+ *                  over i, update, read out from the full-precision S_t,
+ *                  quantize x = S/s with round-to-nearest or floor(x + U), clamp.
+ *   ORC_CANONICAL  the same mathematics in the fixed FP32 evaluation order of
+ *                  the GPU library (partial sums over i = rho (mod R) merged by
+ *                  an XOR butterfly; c-form update; reciprocal multiplier
+ *                  rounded toward zero), so results can be compared bit for bit.
+ * In exact arithmetic both modes compute the same thing.
+ *
+ * Build: gcc -O1 -fPIC -shared -ffp-contract=off -fno-fast-math (see build.py).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_PLAIN 0
+#define ORC_CANONICAL 1
+#define ORC_RTN 0
+#define ORC_SR 1
+
+/* ------------------------------------------------------------------------- */
+/* Philox4x32-10 [PHILOX]: 10 rounds of two 32x32->64 multiplies; the key is
+ * bumped by the Weyl constants between rounds.                              */
+/* ------------------------------------------------------------------------- */
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+    const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+    const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+    uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+    uint32_t k0 = key[0], k1 = key[1];
+    for (int round = 0; round < 10; ++round) {
+        if (round > 0) {
+            k0 += W0;
+            k1 += W1;
+        }
+        uint64_t p0 = (uint64_t)M0 * (uint64_t)x0;
+        uint64_t p1 = (uint64_t)M1 * (uint64_t)x2;
+        uint32_t y0 = (uint32_t)(p1 >> 32) ^ x1 ^ k0;
+        uint32_t y1 = (uint32_t)p1;
+        uint32_t y2 = (uint32_t)(p0 >> 32) ^ x3 ^ k1;
+        uint32_t y3 = (uint32_t)p0;
+        x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+    }
+    out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+/* The 16-bit uniform that stochastic rounding of element (i, j) of head (b, h)
+ * at decode step `step` consumes.  One Philox block serves 8 elements: rows
+ * i' and i' + dk/2 (i' = i mod dk/2) of the four columns 4g..4g+3 (g = j/4).
+ *   counter = { i' | g << 16, h, b, step },  key = { seed_lo, seed_hi }
+ *   chunk   = 4*[i >= dk/2] + (j mod 4);  word chunk/2, low half first.    */
+uint32_t orc_sr_uniform16(uint64_t seed, uint32_t b, uint32_t h, uint32_t step,
+                          int dk, int i, int j)
+{
+    int half = dk / 2;
+    uint32_t ip = (uint32_t)(i % half);
+    uint32_t g = (uint32_t)(j / 4);
+    uint32_t ctr[4] = {ip | (g << 16), h, b, step};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    orc_philox4x32_10(ctr, key, out);
+    int chunk = 4 * (i >= half ? 1 : 0) + (j % 4);
+    uint32_t word = out[chunk / 2];
+    return (chunk % 2 == 0) ? (word & 0xFFFFu) : (word >> 16);
+}
+
+/* bfloat16 -> binary32 widening (exact): the bf16 bits are the upper half. */
+void orc_bf16_to_f32(const uint16_t* src, float* dst, int64_t n)
+{
+    for (int64_t t = 0; t < n; ++t) {
+        uint32_t u = (uint32_t)src[t] << 16;
+        memcpy(&dst[t], &u, 4);
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Sums over the key axis.                                                    */
+/* ------------------------------------------------------------------------- */
+
+/* sum_i a[i*stride] * b[i] accumulated with one fused multiply-add per term.
+ * R == 1: sequential in increasing i.  R > 1 (canonical order): partial p sums
+ * rows i = p, p+R, p+2R, ... sequentially; then for d = 1, 2, ..., R/2 every
+ * partial p becomes P[p] + P[p ^ d]; the result is P[0].                     */
+static float orc_dot_rows(const float* a, int stride, const float* b, int n, int R)
+{
+    float part[64];
+    for (int p = 0; p < R; ++p) {
+        float acc = 0.0f;
+        for (int i = p; i < n; i += R)
+            acc = fmaf(a[(int64_t)i * stride], b[i], acc);
+        part[p] = acc;
+    }
+    for (int d = 1; d < R; d *= 2) {
+        float next[64];
+        for (int p = 0; p < R; ++p)
+            next[p] = part[p] + part[p ^ d];
+        memcpy(part, next, sizeof(float) * (size_t)R);
+    }
+    return part[0];
+}
+
+/* ------------------------------------------------------------------------- */
+/* Per-column scale and quantizer ([LoReS] (1/4), (3/4); [FEED]).             */
+/* ------------------------------------------------------------------------- */
+
+/* Largest representable code r = 2^(b-1) - 1 ([LoReS] (1/4), below the
+ * proposition).  Codes are symmetric in [-r, r].                            */
+static int orc_rmax(int bits) { return (1 << (bits - 1)) - 1; }
+
+/* Reciprocal multiplier r/m rounded toward zero (canonical mode).  With it
+ * |S| * inv <= r for every |S| <= m, so no code exceeds r.                  */
+static float orc_inv_rz(float r, float m)
+{
+    float q = r / m; /* round to nearest */
+    if ((double)q * (double)m > (double)r)
+        q = nextafterf(q, 0.0f);
+    return q;
+}
+
+/* Quantize one element S of a column whose absolute maximum is m (> 0 and
+ * finite) to a symmetric b-bit code.  `u` is the element's 16-bit uniform
+ * (used by stochastic rounding only).
+ *   plain:      x = S / s with s = m / r;  RTN: nearest (ties to even);
+ *               SR: floor(x + u/2^16), i.e. up with probability frac(x)
+ *               ([LoReS] (3/4): SR is conditionally unbiased); clamp to [-r, r].
+ *   canonical:  inv = r/m rounded toward zero;  RTN: nearest integer (ties to
+ *               even) of the exact product S*inv;  SR: t = S*inv + (o + u/2^16)
+ *               rounded once to binary32, c = floor(t) - o, with the offset
+ *               o = 128 (8-bit) or 136 (4-bit) so that t stays in [1, 256).  */
+int orc_quantize_scalar(float S, float m, int bits, int rounding, int mode, uint32_t u)
+{
+    const int r = orc_rmax(bits);
+    const float rf = (float)r;
+    int c;
+    if (mode == ORC_PLAIN) {
+        const float s = m / rf;
+        const float x = S / s;
+        if (rounding == ORC_RTN)
+            c = (int)rintf(x);
+        else
+            c = (int)floor((double)x + (double)u / 65536.0);
+        if (c > r) c = r;
+        if (c < -r) c = -r;
+    } else {
+        const float inv = orc_inv_rz(rf, m);
+        if (rounding == ORC_RTN) {
+            c = (int)rint((double)S * (double)inv);
+        } else {
+            const float off = (bits == 8) ? 128.0f : 136.0f;
+            const float V = off + (float)u / 65536.0f; /* exact */
+            const float t = fmaf(S, inv, V);
+            c = (int)floorf(t) - (int)off;
+        }
+    }
+    return c;
+}
+
+/* Quantize column j of the full-precision state S (dk x dv, row-major) with
+ * the dynamic scale computed from S itself: the "noisy" scale of [LoReS]
+ * (4/4), through which earlier errors feed back [FEED].                     */
+static void orc_quantize_column(const float* S, int dk, int dv, int j, int bits, int rounding,
+                                int mode, uint64_t seed, uint32_t b, uint32_t h,
+                                uint32_t step, int8_t* codes, float* scale_out)
+{
+    const float rf = (float)orc_rmax(bits);
+    /* m_j = max_i |S_ij|; a NaN anywhere in the column makes m NaN. */
+    float m = 0.0f;
+    for (int i = 0; i < dk; ++i) {
+        float a = fabsf(S[(int64_t)i * dv + j]);
+        if (isnan(a) || isnan(m))
+            m = NAN;
+        else if (a > m)
+            m = a;
+    }
+    *scale_out = m / rf; /* s_j = max_i |S_ij| / r */
+    /* An all-zero column has scale 0 and codes 0; a non-finite column keeps
+     * its non-finite scale and gets codes 0.                                */
+    const int usable = (m > 0.0f) && isfinite(m);
+    for (int i = 0; i < dk; ++i) {
+        int c = 0;
+        if (usable) {
+            uint32_t u = (rounding == ORC_SR) ? orc_sr_uniform16(seed, b, h, step, dk, i, j) : 0u;
+            c = orc_quantize_scalar(S[(int64_t)i * dv + j], m, bits, rounding, mode, u);
+        }
+        codes[(int64_t)i * dv + j] = (int8_t)c;
+    }
+}
+
+/* ------------------------------------------------------------------------- */
+/* One decode step of one head.                                              */
+/* ------------------------------------------------------------------------- */
+typedef struct {
+    int dk, dv;       /* rows (key / SSM-state axis) and columns (value / head-dim axis) */
+    int bits;         /* 4, 8 (quantized) or 32 (full-precision state) */
+    int rounding;     /* ORC_RTN or ORC_SR */
+    int mode;         /* ORC_PLAIN or ORC_CANONICAL */
+    int R;            /* canonical partial-sum count (power of two, <= 64); 1 = sequential */
+    uint64_t seed;    /* stochastic-rounding key */
+    uint32_t b, h, step;
+} orc_head;
+
+/* Gated delta rule decode step ([LRB] abstract: Gated DeltaNet; the LoReS
+ * scheme keeps the update in full precision and quantizes the stored state,
+ * [LoReS] "LoReS: State Quantization").
+ *   inputs  c_in (dk*dv codes) + s_in (dv scales) for bits 4/8, or f_in (dk*dv floats) for 32;
+ *           q, k (dk), v (dv) widened to binary32; alpha, beta gates.
+ *   outputs c_out + s_out (or f_out), o (dv): readout from the FP32 S_t.    */
+int orc_gdn_head_step(const orc_head* hd, const int8_t* c_in, const float* s_in,
+                      const float* f_in, const float* q, const float* k, const float* v,
+                      float alpha, float beta, int8_t* c_out, float* s_out, float* f_out,
+                      float* o)
+{
+    const int dk = hd->dk, dv = hd->dv;
+    const int R = (hd->mode == ORC_PLAIN) ? 1 : hd->R;
+    float* S = (float*)malloc(sizeof(float) * (size_t)dk * (size_t)dv);
+    float* Sh = (float*)malloc(sizeof(float) * (size_t)dk * (size_t)dv);
+    float* cf = (float*)malloc(sizeof(float) * (size_t)dk * (size_t)dv);
+    if (!S || !Sh || !cf) { free(S); free(Sh); free(cf); return 1; }
+
+    if (hd->bits == 32) {
+        /* Full-precision state: S_t = alpha*S + k w^T with w = beta*(v - alpha*S^T k). */
+        for (int64_t t = 0; t < (int64_t)dk * dv; ++t) Sh[t] = f_in[t];
+        for (int j = 0; j < dv; ++j) {
+            float u = orc_dot_rows(Sh + j, dv, k, dk, R);
+            float w = beta * fmaf(-alpha, u, v[j]);
+            for (int i = 0; i < dk; ++i)
+                S[(int64_t)i * dv + j] = fmaf(alpha, Sh[(int64_t)i * dv + j], k[i] * w);
+        }
+    } else if (hd->mode == ORC_PLAIN) {
+        /* Dequantize: S^_ij = c_ij * s_j. */
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j)
+                Sh[(int64_t)i * dv + j] = (float)c_in[(int64_t)i * dv + j] * s_in[j];
+        for (int j = 0; j < dv; ++j) {
+            float u = orc_dot_rows(Sh + j, dv, k, dk, 1);        /* u = S^T k */
+            float w = beta * fmaf(-alpha, u, v[j]);            /* w = beta (v - alpha u) */
+            for (int i = 0; i < dk; ++i)                        /* S = alpha S^ + k w^T */
+                S[(int64_t)i * dv + j] = fmaf(alpha, Sh[(int64_t)i * dv + j], k[i] * w);
+        }
+    } else {
+        /* Canonical c-form: u_j = s_j * sum_i c_ij k_i, S_ij = c_ij*(alpha s_j) + k_i w_j. */
+        for (int64_t t = 0; t < (int64_t)dk * dv; ++t) cf[t] = (float)c_in[t];
+        for (int j = 0; j < dv; ++j) {
+            float ck = orc_dot_rows(cf + j, dv, k, dk, R);
+            float u = s_in[j] * ck;
+            float w = beta * fmaf(-alpha, u, v[j]);
+            float a = alpha * s_in[j];
+            for (int i = 0; i < dk; ++i)
+                S[(int64_t)i * dv + j] = fmaf(cf[(int64_t)i * dv + j], a, k[i] * w);
+        }
+    }
+    /* Readout from the full-precision S_t: o_j = sum_i S_ij q_i. */
+    for (int j = 0; j < dv; ++j)
+        o[j] = orc_dot_rows(S + j, dv, q, dk, R);
+
+    if (hd->bits == 32) {
+        for (int64_t t = 0; t < (int64_t)dk * dv; ++t) f_out[t] = S[t];
+    } else {
+        for (int j = 0; j < dv; ++j)
+            orc_quantize_column(S, dk, dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
+                                hd->b, hd->h, hd->step, c_out, &s_out[j]);
+    }
+    free(S); free(Sh); free(cf);
+    return 0;
+}
+
+/* Mamba-2 scalar-decay decode step ([LRB] abstract: Mamba2; [LoReS] Table 1).
+ *   decay a = exp(dt*A) (computed here with libm expf unless `decay` >= 0 is
+ *   given), x (dv = P), Bv, Cv (dk = N), D.                                 */
+int orc_mamba2_head_step(const orc_head* hd, const int8_t* c_in, const float* s_in,
+                         const float* f_in, const float* x, const float* Bv, const float* Cv,
+                         float dt, float A, float D, float decay, int8_t* c_out,
+                         float* s_out, float* f_out, float* y)
+{
+    const int dk = hd->dk, dv = hd->dv;
+    const int R = (hd->mode == ORC_PLAIN) ? 1 : hd->R;
+    float* S = (float*)malloc(sizeof(float) * (size_t)dk * (size_t)dv);
+    float* cf = (float*)malloc(sizeof(float) * (size_t)dk * (size_t)dv);
+    if (!S || !cf) { free(S); free(cf); return 1; }
+    const float a = (decay >= 0.0f) ? decay : expf(dt * A);
+
+    if (hd->bits == 32) {
+        for (int j = 0; j < dv; ++j) {
+            float xd = dt * x[j];
+            for (int i = 0; i < dk; ++i)
+                S[(int64_t)i * dv + j] = fmaf(a, f_in[(int64_t)i * dv + j], Bv[i] * xd);
+        }
+    } else if (hd->mode == ORC_PLAIN) {
+        for (int j = 0; j < dv; ++j) {
+            float xd = dt * x[j];
+            for (int i = 0; i < dk; ++i) {
+                float sh = (float)c_in[(int64_t)i * dv + j] * s_in[j];      /* dequantize */
+                S[(int64_t)i * dv + j] = fmaf(a, sh, Bv[i] * xd);           /* a S^ + dt x B^T */
+            }
+        }
+    } else {
+        for (int64_t t = 0; t < (int64_t)dk * dv; ++t) cf[t] = (float)c_in[t];
+        for (int j = 0; j < dv; ++j) {
+            float xd = dt * x[j];
+            float g = a * s_in[j];
+            for (int i = 0; i < dk; ++i)
+                S[(int64_t)i * dv + j] = fmaf(cf[(int64_t)i * dv + j], g, Bv[i] * xd);
+        }
+    }
+    /* y_j = sum_i S_ij C_i + D x_j, from the full-precision S_t. */
+    for (int j = 0; j < dv; ++j)
+        y[j] = fmaf(D, x[j], orc_dot_rows(S + j, dv, Cv, dk, R));
+
+    if (hd->bits == 32) {
+        for (int64_t t = 0; t < (int64_t)dk * dv; ++t) f_out[t] = S[t];
+    } else {
+        for (int j = 0; j < dv; ++j)
+            orc_quantize_column(S, dk, dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
+                                hd->b, hd->h, hd->step, c_out, &s_out[j]);
+    }
+    free(S); free(cf);
+    return 0;
+}
+
+/* Quantize a full-precision head state (initialisation / checkpoint), with the
+ * same per-column scale and rounding as the decode step.                    */
+int orc_quantize_head(const orc_head* hd, const float* S, int8_t* c_out, float* s_out)
+{
+    if (hd->bits != 4 && hd->bits != 8) return 1;
+    for (int j = 0; j < hd->dv; ++j)
+        orc_quantize_column(S, hd->dk, hd->dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
+                            hd->b, hd->h, hd->step, c_out, &s_out[j]);
+    return 0;
+}
+
+/* Dequantize: S^_ij = c_ij * s_j. */
+void orc_dequantize_head(int dk, int dv, const int8_t* c, const float* s, float* S)
+{
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j)
+            S[(int64_t)i * dv + j] = (float)c[(int64_t)i * dv + j] * s[j];
+}
+
+/* ------------------------------------------------------------------------- */
+/* Storage format of the library, written out independently.                 */
+/*   A head's dv columns are cut into blocks of CB = min(64, dv) columns.     */
+/*   Block cb holds rows i = 0..dk-1 of columns cb*CB .. cb*CB+CB-1, row by   */
+/*   row.  8-bit code c is stored as the byte c + 128; 4-bit codes as the     */
+/*   nibble c + 8, column 2t in the low nibble of byte t of the row segment   */
+/*   and column 2t+1 in the high nibble.  32-bit heads store binary32 values  */
+/*   in the same block order.                                                 */
+/* ------------------------------------------------------------------------- */
+static int orc_cb(int dv) { return dv < 64 ? dv : 64; }
+
+int64_t orc_head_bytes(int dk, int dv, int bits) { return (int64_t)dk * dv * bits / 8; }
+
+void orc_pack_head(int dk, int dv, int bits, const int8_t* c, const float* f, uint8_t* out)
+{
+    const int CB = orc_cb(dv);
+    int64_t pos = 0;
+    for (int cb = 0; cb < dv / CB; ++cb) {
+        for (int i = 0; i < dk; ++i) {
+            for (int jj = 0; jj < CB; ++jj) {
+                int j = cb * CB + jj;
+                int64_t e = (int64_t)i * dv + j;
+                if (bits == 8) {
+                    out[pos++] = (uint8_t)(c[e] + 128);
+                } else if (bits == 4) {
+                    uint8_t nib = (uint8_t)(c[e] + 8);
+                    if (jj % 2 == 0) out[pos] = nib;
+                    else out[pos++] |= (uint8_t)(nib << 4);
+                } else {
+                    memcpy(out + pos, &f[e], 4);
+                    pos += 4;
+                }
+            }
+        }
+    }
+}
+
+void orc_unpack_head(int dk, int dv, int bits, const uint8_t* in, int8_t* c, float* f)
+{
+    const int CB = orc_cb(dv);
+    int64_t pos = 0;
+    for (int cb = 0; cb < dv / CB; ++cb) {
+        for (int i = 0; i < dk; ++i) {
+            for (int jj = 0; jj < CB; ++jj) {
+                int j = cb * CB + jj;
+                int64_t e = (int64_t)i * dv + j;
+                if (bits == 8) {
+                    c[e] = (int8_t)((int)in[pos++] - 128);
+                } else if (bits == 4) {
+                    int nib = (jj % 2 == 0) ? (in[pos] & 0xF) : (in[pos++] >> 4);
+                    c[e] = (int8_t)(nib - 8);
+                } else {
+                    memcpy(&f[e], in + pos, 4);
+                    pos += 4;
+                }
+            }
+        }
+    }
+}
+
+/* Decay-based mixed precision ([LoReS] (2/4): more bits for the slowest-
+ * decaying heads).  Brute force: head h gets `hi` bits when fewer than
+ * n_hi heads have a larger decay score (ties: the lower head index ranks
+ * first), otherwise `lo` bits.                                               */
+void orc_allocate_bits(const double* score, int H, int n_hi, int hi, int lo, int8_t* bits)
+{
+    for (int h = 0; h < H; ++h) {
+        int ahead = 0;
+        for (int g = 0; g < H; ++g)
+            if (score[g] > score[h] || (score[g] == score[h] && g < h)) ++ahead;
+        bits[h] = (int8_t)(ahead < n_hi ? hi : lo);
+    }
+}
