@@ -1,0 +1,487 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized recurrent-state decode step (one JSON line on rank 0).
+
+A step is one decode step of one layer of the Gated DeltaNet workload
+B=64, H=16, d_k=d_v=128, INT8 state with per-value-column scales, Philox
+stochastic rounding, bf16 q/k/v (the workload the head-updates/s metric is
+quoted on).  Consecutive steps cycle through enough independent layer states
+(and input sets) that their footprint is >= 3x the L2 cache, as the layers of a
+model do, so every step reads its state from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched by torchrun (one process per GPU); every rank runs its own
+requests (weak scaling, no collective on the data path); the time is the max
+over ranks.  --impl reference times the CPU oracle on the host cores instead.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+DEFAULT_WORKLOAD = "gdn_b64_h16_d128_int8_sr"
+
+
+def algorithmic_bytes_per_head(w: W.Workload, bits: int) -> int:
+    """Bytes the method must move per head update: codes and scales read and
+    written, the input vectors and gates, and the float output."""
+    esz = 2 if w.in_dtype == "bf16" else 4
+    codes = w.dk * w.dv * bits // 8
+    scales = 4 * w.dv
+    out = 4 * w.dv
+    if w.family == "gdn":
+        vecs = esz * (2 * w.dk + w.dv) + 8          # q, k, v, alpha, beta
+    else:
+        vecs = esz * w.dv + 4                       # x, dt (B, C, A, D added per request / head)
+    return 2 * codes + 2 * scales + vecs + out
+
+
+def step_bytes(w: W.Workload, head_bits) -> int:
+    per = sum(algorithmic_bytes_per_head(w, int(b)) for b in head_bits) * w.B
+    if w.family == "mamba2":
+        esz = 2 if w.in_dtype == "bf16" else 4
+        per += w.B * w.ngroups * 2 * w.dk * esz + 8 * w.H   # B, C per request; A, D per head
+    return per
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "ssm_decode_02_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+class ClockSampler:
+    """nvidia-smi SM clocks and throttle reasons, sampled every 100 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: str):
+        self.index = index
+        self.proc = None
+        self.lines: list[str] = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.Q,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (FileNotFoundError, OSError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, f[5:9]):
+                if val.lower() in ("active", "1", "yes"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def measured_peak_gbs():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def profiled_traffic(kernel_tag: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
+    current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d.get(kernel_tag)
+        if e and e.get("source_hash") == source_hash():
+            return float(e["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
+        pass
+    return None
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_rate(w: W.Workload, head_bits, budget_s: float, heads_per_call: int = 8):
+    """Head updates per second of the single-threaded CPU oracle on a bounded sample
+    of the workload (the first requests of a few steps, from the zero state)."""
+    import oracle
+    R = 8 if w.dk <= 128 else 16
+    rounding = oracle.SR if w.rounding == "sr" else oracle.RTN
+    n_done, t_used, t = 0, 0.0, 0
+    nb = max(1, min(w.B, heads_per_call // w.H + 1))
+    st = oracle.zero_state(nb, w.H, w.dk, w.dv, fp32=w.state == "fp32")
+    while t_used < budget_s:
+        inp = W.inputs(w, t, B=nb)
+        heads = [(b, h) for b in range(nb) for h in range(w.H)][:heads_per_call]
+        t0 = time.perf_counter()
+        if w.family == "gdn":
+            st, _ = oracle.gdn_step(st, inp, head_bits, rounding=rounding, seed=w.sr_seed, step=t,
+                                    R=R, heads=heads)
+        else:
+            st, _ = oracle.mamba2_step(st, inp, head_bits, rounding=rounding, seed=w.sr_seed,
+                                       step=t, R=R, ngroups=w.ngroups, heads=heads)
+        t_used += time.perf_counter() - t0
+        n_done += len(heads)
+        t += 1
+    return n_done / t_used, n_done, t
+
+
+def head_bits_of(w: W.Workload, rsq=None):
+    if w.state == "mixed":
+        score = W.mean_alpha_per_head(w)
+        n_hi = int(w.H * w.high_frac)
+        if rsq is not None:
+            return rsq.rsq_allocate_bits(score, n_hi)
+        import oracle
+        return oracle.allocate_bits(score, n_hi)
+    return W.head_bits_for(w)
+
+
+def run_reference(args, w: W.Workload):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    bits = head_bits_of(w)
+    # time one oracle head to size the per-step sample so the whole run stays within minutes
+    rate, _, _ = oracle_rate(w, bits, 0.5, heads_per_call=1)
+    per_head = 1.0 / rate
+    total_budget = 180.0
+    n_heads = int(max(1, min(w.B * w.H, total_budget / max(1, args.steps + args.warmup) / per_head)))
+    import oracle
+    R = 8 if w.dk <= 128 else 16
+    rounding = oracle.SR if w.rounding == "sr" else oracle.RTN
+    nb = max(1, min(w.B, (n_heads + w.H - 1) // w.H))
+    heads = [(b, h) for b in range(nb) for h in range(w.H)][:n_heads]
+    st = oracle.zero_state(nb, w.H, w.dk, w.dv, fp32=w.state == "fp32")
+    inp_cache = [W.inputs(w, t, B=nb) for t in range(4)]
+    elapsed = 0.0
+    for t in range(args.warmup + args.steps):
+        inp = inp_cache[t % 4]
+        t0 = time.perf_counter()
+        if w.family == "gdn":
+            st, _ = oracle.gdn_step(st, inp, bits, rounding=rounding, seed=w.sr_seed, step=t, R=R,
+                                    heads=heads)
+        else:
+            st, _ = oracle.mamba2_step(st, inp, bits, rounding=rounding, seed=w.sr_seed, step=t,
+                                       R=R, ngroups=w.ngroups, heads=heads)
+        dt = time.perf_counter() - t0
+        if t >= args.warmup:
+            elapsed += dt
+    value = n_heads * args.steps / elapsed
+    line = {
+        "impl": "reference", "metric": "head-updates/s", "value": value, "unit": "head-updates/s",
+        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * elapsed / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.B, "heads": w.H, "dk": w.dk, "dv": w.dv,
+                   "state": w.state, "rounding": w.rounding, "parallelism": "cpu"},
+        "cpu_baseline": {"value": value, "unit": "head-updates/s", "cores": 1, "kind": "oracle",
+                         "sample": "%d heads of one layer per step, single-threaded C oracle" % n_heads},
+        "e2e": {"value": value, "unit": "head-updates/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def run_ours(args, w: W.Workload):
+    import torch
+    import torch.distributed as dist
+
+    import ssm_decode_02_b200 as rsq
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    props = torch.cuda.get_device_properties(dev)
+    l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
+
+    bits = np.asarray(head_bits_of(w, rsq), np.int8)
+    fam = rsq.RSQ_GDN if w.family == "gdn" else rsq.RSQ_MAMBA2
+    ctx = rsq.Context(fam, w.B, w.H, w.dk, w.dv, head_bits=bits,
+                      rounding=rsq.RSQ_SR if w.rounding == "sr" else rsq.RSQ_RTN,
+                      in_dtype=rsq.RSQ_BF16 if w.in_dtype == "bf16" else rsq.RSQ_F32,
+                      seed=w.sr_seed + 7919 * rank, ngroups=w.ngroups)
+    state_bytes = ctx.code_bytes + ctx.scale_bytes
+    layers = max(2, -(-3 * l2 // state_bytes))
+    if args.layers:
+        layers = args.layers
+    # independent layer states, initialised from random full-precision states
+    states = []
+    S0 = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(1234 + rank)
+    for _ in range(layers):
+        st = ctx.alloc_state(dev)
+        S0.normal_(0.0, 0.05, generator=g)
+        ctx.quantize(S0, st, step=0)
+        states.append(st)
+    del S0
+    # input sets (seeded host generation, uploaded once)
+    inp_bytes = None
+    n_sets = max(8, min(256, -(-3 * l2 // max(1, step_input_bytes(w)))))
+    sets = []
+    for t in range(n_sets):
+        host = W.inputs(w, t + 100000 * rank)
+        d = {k: _to_dev(v, dev) for k, v in host.items()}
+        sets.append(d)
+    inp_bytes = step_input_bytes(w)
+    outs = [torch.empty((w.B, w.H, w.dv), dtype=torch.float32, device=dev) for _ in range(layers)]
+    structs = [_inputs_struct(rsq, w, s) for s in sets]
+    stream = torch.cuda.Stream(device=dev)
+
+    def launch(t):
+        li = t % layers
+        ctx.decode_step(states[li], states[li], structs[t % n_sets], outs[li], t, stream.cuda_stream)
+
+    # CUDA graphs of up to CH consecutive steps (launch-bound inner loop); CH is a
+    # multiple of the layer count so the rotation continues across graph replays
+    CH = max(1, 2048 // layers) * layers
+
+    def capture(t0, n):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(stream):
+            with torch.cuda.graph(gr, stream=stream):
+                for t in range(t0, t0 + n):
+                    launch(t)
+        return gr
+
+    with torch.cuda.stream(stream):
+        for t in range(min(8, args.warmup)):
+            launch(t)
+    stream.synchronize()
+    if ctx.check_flags(stream.cuda_stream):
+        raise RuntimeError("non-finite state during warm-up")
+
+    def plan(total):
+        chunks, t = [], 0
+        while t < total:
+            n = min(CH, total - t)
+            chunks.append((t, n))
+            t += n
+        return chunks
+
+    warm_graphs = [capture(t0, n) for t0, n in plan(args.warmup)]
+    timed_plan = plan(args.steps)
+    # distinct graphs for distinct chunk sizes; step numbers only matter for the SR counter
+    graph_cache = {}
+    for t0, n in timed_plan:
+        if n not in graph_cache:
+            graph_cache[n] = capture(args.warmup, n)
+    uuid = str(getattr(props, "uuid", ""))
+    clocks = ClockSampler(("GPU-" + uuid) if uuid and not uuid.startswith("GPU-") else (uuid or str(local)))
+    clocks.start()
+    time.sleep(0.3)
+    for gr in warm_graphs:
+        gr.replay()
+    stream.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for t0, n in timed_plan:
+        graph_cache[n].replay()
+    ev1.record(stream)
+    ev1.synchronize()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    time.sleep(0.15)
+    clk = clocks.stop()
+    elapsed = ev0.elapsed_time(ev1) / 1e3
+    if world > 1:
+        tt = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed = float(tt.item())
+    flag = ctx.check_flags(stream.cuda_stream)
+
+    # end-to-end through the public API with host buffers (pinned), per step:
+    # H2D of that step's inputs, the decode step, D2H of its output
+    n_e2e = max(1, min(args.steps, 500))
+    pinned = [{k: _to_pinned(v) for k, v in W.inputs(w, 200000 + t + 1000 * rank).items()}
+              for t in range(4)]
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in pinned[0].items()}
+    e2e_struct = _inputs_struct(rsq, w, dev_in)
+    out_host = torch.empty((w.B, w.H, w.dv), dtype=torch.float32, pin_memory=True)
+    h2d = sum(v.numel() * v.element_size() for v in pinned[0].values())
+    d2h = out_host.numel() * 4
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for t in range(n_e2e):
+            src = pinned[t % 4]
+            for k, v in src.items():
+                dev_in[k].copy_(v, non_blocking=True)
+            ctx.decode_step(states[0], states[0], e2e_struct, outs[0], args.warmup + args.steps + t,
+                            stream.cuda_stream)
+            out_host.copy_(outs[0], non_blocking=True)
+        e1.record(stream)
+    e1.synchronize()
+    e2e_elapsed = e0.elapsed_time(e1) / 1e3
+    if world > 1:
+        tt = torch.tensor([e2e_elapsed], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_elapsed = float(tt.item())
+
+    hu_step = w.B * w.H
+    value = world * hu_step * args.steps / elapsed
+    e2e_value = world * hu_step * n_e2e / e2e_elapsed
+    per_launch = elapsed / args.steps
+    alg = step_bytes(w, bits)
+    peak, peak_kind = measured_peak_gbs()
+    achieved = alg / per_launch / 1e9
+    kernel_tag = "rsq_decode_kernel<%s,%d,%d>" % (w.family, w.dk, min(64, w.dv))
+    line = {
+        "metric": "head-updates/s", "value": value, "unit": "head-updates/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * per_launch,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic",
+        "config": {"workload": w.name, "global_batch": w.B * world, "heads": w.H, "dk": w.dk,
+                   "dv": w.dv, "state": w.state, "rounding": w.rounding, "inputs": w.in_dtype,
+                   "parallelism": "dp%d" % world, "layers_rotated": layers,
+                   "l2": "inputs larger than L2: %d layer states + %d input sets = %.0f MB per "
+                         "rotation (L2 %.0f MB)" % (layers, n_sets,
+                                                    (layers * state_bytes + n_sets * inp_bytes) / 1e6,
+                                                    l2 / 1e6),
+                   "graphs": "CUDA graphs of <= %d steps" % CH},
+        "hbm_gbs": achieved,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": profiled_traffic(kernel_tag),
+                     "algorithmic_bytes_per_launch": alg, "kernel": kernel_tag},
+        "frac_of_8tbs_datasheet": achieved / 8000.0,
+        "e2e": {"value": e2e_value, "unit": "head-updates/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "steps": n_e2e},
+        "gpu_launches": args.steps,
+        "clocks": clk,
+        "nonfinite_flag": flag,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, n, steps = oracle_rate(w, bits, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": "head-updates/s", "cores": 1, "kind": "oracle",
+                                "sample": "%d head updates (%d decode steps of the first requests) "
+                                          "in ~%.0f s, single-threaded C oracle" % (n, steps, args.cpu_seconds)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    for gr in list(graph_cache.values()) + warm_graphs:
+        del gr
+    graph_cache.clear()
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    ctx.close()
+    return 0
+
+
+def step_input_bytes(w: W.Workload) -> int:
+    esz = 2 if w.in_dtype == "bf16" else 4
+    if w.family == "gdn":
+        return w.B * w.H * (esz * (2 * w.dk + w.dv) + 8)
+    return w.B * w.H * (esz * w.dv + 4) + w.B * w.ngroups * 2 * w.dk * esz + 8 * w.H
+
+
+def _to_dev(a: np.ndarray, dev):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a.copy()).to(dev)
+
+
+def _to_pinned(a: np.ndarray):
+    import torch
+    a = np.ascontiguousarray(a)
+    if a.dtype == np.uint16:
+        a = a.view(np.int16)
+    return torch.from_numpy(a.copy()).pin_memory()
+
+
+def _inputs_struct(rsq, w: W.Workload, d: dict):
+    if w.family == "gdn":
+        return rsq.gdn_inputs(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+    return rsq.mamba2_inputs(d["x"], d["Bm"], d["Cm"], d["dt"], d["A"], d["D"], None)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20000)
+    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.BY_NAME))
+    ap.add_argument("--layers", type=int, default=0, help="override the number of rotated layer states")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    w = W.BY_NAME[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_ours(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

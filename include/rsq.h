@@ -1,0 +1,240 @@
+/*
+ * rsq.h -- quantized recurrent-state decode step for NVIDIA B200 (sm_100a).
+ *
+ * One decode step of a linear-attention / SSM layer whose recurrent state is
+ * stored in low precision between steps: the stored state is dequantized,
+ * advanced by one token with the layer's recurrence, read out, given fresh
+ * per-value-channel absmax scales and requantized, in one fused pass.
+ *
+ * Method sources (cited below by tag):
+ *   [LoReS] "Quantizing Recurrent Language Models Is Easier Than You Think"
+ *           (LoReS blog post): "LoReS: State Quantization" (full-precision
+ *           updates, quantized stored state), "(1/4) Scale grouping"
+ *           (value-axis scales, r = 2^(b-1) - 1), "(2/4) Mixed precision"
+ *           (more bits for the slowest-decaying heads), "(3/4) Rounding"
+ *           (stochastic rounding), "(4/4) Rotations" (noisy vs copy scale).
+ *   [LRB]   "Preserving Updates in Low-Bit Recurrent State Quantization",
+ *           abstract: the state is requantized after every update; Gated
+ *           DeltaNet, GLA, Mamba2 and RetNet recurrences.
+ *   [FEED]  "When Dynamic Scaling Fails: A Scale-State Feedback Governs
+ *           Recurrent-State Quantization ...", key points: the dynamic scale
+ *           is derived from the state it quantizes.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All buffers are caller-owned.  Pointers marked "device" must point to
+ *    CUDA device memory of the current device, 16-byte aligned.  Pointers
+ *    marked "host" are ordinary host memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *    stream).  Every call that takes a stream is asynchronous on that stream
+ *    and never synchronizes, except rsq_check_flags.  Calls may be captured
+ *    into CUDA graphs.
+ *  - Host-side validation happens before any CUDA call; a failing check
+ *    returns RSQ_E_INVAL or RSQ_E_UNSUPPORTED and touches no memory.  A
+ *    failed launch returns RSQ_E_CUDA.  rsq_last_error() then holds a
+ *    human-readable reason (thread-local).
+ *  - A context is immutable after rsq_create and may be used from several
+ *    host threads and streams at once.
+ *
+ * State orientation (both families)
+ * ---------------------------------
+ *  One head's state is a dk x dv matrix S with rows i (GDN key axis / Mamba-2
+ *  SSM state axis N) and columns j (GDN value axis / Mamba-2 head-dim axis P).
+ *  A value channel is a column: it has one scale s_j = max_i |S_ij| / r with
+ *  r = 2^(b-1) - 1 (127 for 8-bit, 7 for 4-bit) ([LoReS] (1/4)).  Codes are
+ *  symmetric integers in [-r, r].
+ *
+ * State storage format (rsq_state)
+ * --------------------------------
+ *  codes: device bytes [batch][row_bytes].  Within a batch row the heads are
+ *    concatenated in order; head h occupies dk*dv*bits_h/8 bytes.  A head's
+ *    columns are cut into blocks of CB = min(64, dv) columns; block cb
+ *    (cb = 0 .. dv/CB-1) stores rows i = 0..dk-1 of columns cb*CB..cb*CB+CB-1
+ *    row after row, so every block is one contiguous run of dk*CB*bits/8
+ *    bytes.  Inside a row segment:
+ *      8-bit : byte = c + 128                       (one per column)
+ *      4-bit : byte t = (c_{2t} + 8) | (c_{2t+1} + 8) << 4
+ *      32-bit: IEEE binary32 value of S_ij          (full-precision state)
+ *  scales: device float [batch][heads][dv], s_j per column (unused for 32-bit).
+ *  The all-zero state S_0 = 0 is codes "zero code" (128 / 0x88) with scales 0;
+ *  rsq_quantize of a zero tensor produces it.
+ *
+ * Arithmetic (binary32 throughout; fixed evaluation order, see rsq_decode_step)
+ * ------------------------------------------------------------------------
+ *  Sums over the key axis i use R = rsq_reduction_partials(dk) partial sums:
+ *  partial p accumulates rows i = p, p+R, p+2R, ... in increasing i with one
+ *  fused multiply-add per term; then for d = 1, 2, ..., R/2 every partial p
+ *  becomes P[p] + P[p^d]; the sum is P[0].
+ */
+#ifndef RSQ_H
+#define RSQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RSQ_MAX_HEADS 512
+
+typedef enum {
+    RSQ_OK = 0,
+    RSQ_E_INVAL = 1,       /* bad argument: null / misaligned pointer, bad size or enum */
+    RSQ_E_UNSUPPORTED = 2, /* valid but not built: a dk/dv/bit-width combination */
+    RSQ_E_CUDA = 3,        /* a CUDA runtime call or kernel launch failed */
+    RSQ_E_NOMEM = 4,       /* the context's own small allocation failed */
+    RSQ_E_NONFINITE = 5    /* rsq_check_flags: a non-finite state column was seen */
+} rsq_status;
+
+typedef enum { RSQ_GDN = 0, RSQ_MAMBA2 = 1 } rsq_family;
+typedef enum { RSQ_RTN = 0, RSQ_SR = 1 } rsq_rounding;
+typedef enum { RSQ_F32 = 0, RSQ_BF16 = 1 } rsq_dtype;
+
+/* Layer configuration, read once by rsq_create. */
+typedef struct {
+    int family;      /* rsq_family */
+    int batch;       /* B >= 1 independent requests */
+    int heads;       /* H, 1..RSQ_MAX_HEADS */
+    int dk;          /* rows: GDN key dim d_k / Mamba-2 state dim N; one of 16,32,64,128,256 */
+    int dv;          /* columns: GDN value dim d_v / Mamba-2 head dim P; one of 16,32,64,128,256 */
+    int ngroups;     /* Mamba-2 B/C groups (divides heads); ignored for GDN */
+    const int8_t* head_bits; /* host [heads]: each 4 or 8, or every entry 32 (full-precision
+                                state).  NULL = all 8.  Copied by rsq_create. */
+    int rounding;    /* rsq_rounding: requantization rule */
+    int in_dtype;    /* rsq_dtype of the vector inputs (q, k, v / x, B, C) */
+    uint64_t seed;   /* stochastic-rounding key */
+} rsq_config;
+
+typedef struct rsq_ctx rsq_ctx;
+
+/* A stored state (device, caller-owned; format above). */
+typedef struct {
+    void* codes;     /* device [batch][row_bytes] */
+    float* scales;   /* device [batch][heads][dv] (may be NULL when every head is 32-bit) */
+} rsq_state;
+
+/* Gated DeltaNet step inputs (device).  q, k: [B][H][dk]; v: [B][H][dv], in
+ * in_dtype; alpha (decay gate in (0,1)), beta (write strength): float [B][H]. */
+typedef struct {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* alpha;
+    const float* beta;
+} rsq_gdn_inputs;
+
+/* Mamba-2 step inputs (device).  x: [B][H][dv]; Bm, Cm: [B][ngroups][dk], in
+ * in_dtype; dt: float [B][H]; A, D: float [H]; decay: float [B][H] or NULL.
+ * When decay is non-NULL it replaces exp(dt*A) (a caller that already holds
+ * the decay, or a test that needs a decay value fixed bit for bit). */
+typedef struct {
+    const void* x;
+    const void* Bm;
+    const void* Cm;
+    const float* dt;
+    const float* A;
+    const float* D;
+    const float* decay;
+} rsq_mamba2_inputs;
+
+/* Create a context for one layer configuration.  Validates the configuration
+ * (RSQ_E_INVAL / RSQ_E_UNSUPPORTED, nothing allocated), then allocates a
+ * 4-byte device flag word on the current device (RSQ_E_NOMEM / RSQ_E_CUDA on
+ * failure).  *out receives the context; release it with rsq_destroy. */
+rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out);
+
+/* Release a context (NULL is a no-op).  Not stream-ordered: call it only after
+ * every stream that used the context has finished with it. */
+void rsq_destroy(rsq_ctx* ctx);
+
+/* Bytes of the caller-owned state buffers: codes (batch * row_bytes) and
+ * scales (batch * heads * dv * 4). */
+rsq_status rsq_state_bytes(const rsq_ctx* ctx, size_t* code_bytes, size_t* scale_bytes);
+
+/* Per-head byte offset of head h inside a batch row of the code buffer. */
+rsq_status rsq_head_offset(const rsq_ctx* ctx, int h, size_t* offset);
+
+/* One decode step for every (request, head) of the layer.
+ *
+ * Per head, with the stored codes c and scales s of state_in:
+ *  GDN ([LRB] abstract, [LoReS] Table 1), state S_t = alpha (I - beta k k^T) S_{t-1} + beta k v^T:
+ *     u_j = s_j * sum_i c_ij k_i                 (= (S^_{t-1}^T k)_j, S^ = c*s)
+ *     w_j = beta * fma(-alpha, u_j, v_j)
+ *     S_ij = fma(c_ij, alpha*s_j, k_i*w_j)
+ *     out_j = sum_i S_ij q_i                     (readout from the full-precision S_t)
+ *  Mamba-2, state S_t = exp(dt A) S_{t-1} + dt B x^T:
+ *     a = decay ? decay : expf(dt*A);  S_ij = fma(c_ij, a*s_j, B_i*(dt*x_j))
+ *     out_j = fma(D, x_j, sum_i S_ij C_i)
+ *  then per column ([LoReS] (1/4), (3/4); noisy dynamic scale [FEED]):
+ *     m_j = max_i |S_ij|;  s'_j = m_j / r;  inv_j = r / m_j rounded toward zero
+ *     (inv_j = 0 when m_j = 0);
+ *     RTN: c'_ij = nearest integer (ties to even) of the exact S_ij * inv_j
+ *     SR : t = fma(S_ij, inv_j, o + u_ij/65536) in binary32, c'_ij = floor(t) - o,
+ *          o = 128 (8-bit) / 136 (4-bit); u_ij is a 16-bit uniform from
+ *          Philox4x32-10 (Salmon et al., SC'11) with key = seed and counter
+ *          { (i mod dk/2) | (j/4) << 16, h, b, step }; element (i, j) takes
+ *          16-bit chunk 4*[i >= dk/2] + (j mod 4) (word chunk/2, low half first).
+ *  32-bit heads skip the quantizer and store S_t; their update is
+ *     GDN: u_j = sum_i S_ij k_i, S_ij = fma(alpha, S_ij, k_i*w_j);
+ *     Mamba-2: S_ij = fma(a, S_ij, B_i*(dt*x_j)).
+ *  A column whose maximum is not finite keeps that scale (inf or NaN), gets
+ *  codes 0 and raises the context's non-finite flag (rsq_check_flags).
+ *
+ * Arguments: state_in / state_out: device states of this context's format;
+ *   state_out may equal state_in (in-place update; any other overlap is
+ *   invalid).  inputs: host pointer to rsq_gdn_inputs or rsq_mamba2_inputs
+ *   (family of the context) holding device pointers.  out: device float
+ *   [B][H][dv].  step: decode-step index (stochastic-rounding counter; keep it
+ *   across checkpoints for reproducible runs).
+ * Errors: RSQ_E_INVAL for null/misaligned pointers; RSQ_E_CUDA if the launch
+ *   fails.  No memory is written when an argument check fails. */
+rsq_status rsq_decode_step(const rsq_ctx* ctx, const rsq_state* state_in,
+                           const rsq_state* state_out, const void* inputs, float* out,
+                           uint32_t step, void* stream);
+
+/* Quantize a full-precision state (device float [B][H][dk][dv], row-major per
+ * head) into state_out with the same per-column scale and rounding as
+ * rsq_decode_step (RTN or SR with counter step).  32-bit heads are copied.
+ * Used to initialise and to load checkpoints. */
+rsq_status rsq_quantize(const rsq_ctx* ctx, const float* S, const rsq_state* state_out,
+                        uint32_t step, void* stream);
+
+/* Dequantize state_in into device float [B][H][dk][dv]: S^_ij = c_ij * s_j
+ * (32-bit heads: the stored value). */
+rsq_status rsq_dequantize(const rsq_ctx* ctx, const rsq_state* state_in, float* S_out,
+                          void* stream);
+
+/* Per-head sums for the relative state drift ||deq(Q) - F||_F / ||F||_F of a
+ * quantized trajectory Q against a full-precision trajectory F of the same
+ * shape (q_ctx: 4/8-bit heads; f_ctx: 32-bit heads).  sums: device double
+ * [B][H][2] receives { sum (S^_ij - F_ij)^2, sum F_ij^2 } per head. */
+rsq_status rsq_state_drift(const rsq_ctx* q_ctx, const rsq_state* q_state,
+                           const rsq_ctx* f_ctx, const rsq_state* f_state, double* sums,
+                           void* stream);
+
+/* Synchronize `stream`, then report (and clear) the context's non-finite
+ * flag: *seen = 1 if any decode step since the last check met a non-finite
+ * column.  Returns RSQ_E_NONFINITE when *seen = 1. */
+rsq_status rsq_check_flags(const rsq_ctx* ctx, int* seen, void* stream);
+
+/* Decay-based mixed precision ([LoReS] (2/4)): host-only.  score: host
+ * double [heads] (a decay statistic, e.g. the mean gate alpha; larger = slower
+ * decay).  The n_high heads with the largest score get high_bits, the others
+ * low_bits; ties go to the lower head index.  bits_out: host int8 [heads]. */
+rsq_status rsq_allocate_bits(const double* score, int heads, int n_high, int high_bits,
+                             int low_bits, int8_t* bits_out);
+
+/* Number of partial sums R of the key-axis reduction order for a given dk
+ * (host-only; 8 for dk <= 128, 16 for dk = 256). */
+int rsq_reduction_partials(int dk);
+
+const char* rsq_status_string(rsq_status s);
+const char* rsq_last_error(void);
+const char* rsq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RSQ_H */

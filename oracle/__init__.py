@@ -119,14 +119,21 @@ def rmax(bits: int) -> int:
 # ---------------------------------------------------------------------------
 # State containers
 # ---------------------------------------------------------------------------
-def zero_state(B: int, H: int, dk: int, dv: int) -> dict:
-    """S_0 = 0: all codes 0, all scales 0, full-precision part 0."""
+def zero_state(B: int, H: int, dk: int, dv: int, fp32: bool = True) -> dict:
+    """S_0 = 0: all codes 0, all scales 0; the full-precision part (used by 32-bit
+    heads) is allocated only when ``fp32``."""
     return {"codes": np.zeros((B, H, dk, dv), np.int8), "scales": np.zeros((B, H, dv), np.float32),
-            "f": np.zeros((B, H, dk, dv), np.float32)}
+            "f": np.zeros((B, H, dk, dv), np.float32) if fp32 else None}
 
 
 def copy_state(st: dict) -> dict:
-    return {k: v.copy() for k, v in st.items()}
+    return {k: (None if v is None else v.copy()) for k, v in st.items()}
+
+
+def _f_in(state, b, h, dk, dv):
+    if state["f"] is None:
+        return np.zeros((dk, dv), np.float32)
+    return _c(state["f"][b, h], np.float32)
 
 
 def _head(dk, dv, bits, rounding, mode, R, seed, b, h, step) -> _Head:
@@ -158,7 +165,7 @@ def gdn_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, ste
         bits = int(head_bits[h])
         hd = _head(dk, dv, bits, rounding, mode, R, seed, b, h, step)
         c_in, s_in, f_in = (_c(state["codes"][b, h], np.int8), _c(state["scales"][b, h], np.float32),
-                            _c(state["f"][b, h], np.float32))
+                            _f_in(state, b, h, dk, dv))
         c_out = np.zeros((dk, dv), np.int8)
         s_out = np.zeros(dv, np.float32)
         f_out = np.zeros((dk, dv), np.float32)
@@ -192,7 +199,7 @@ def mamba2_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, 
         g = h // heads_per_group
         hd = _head(dk, dv, bits, rounding, mode, R, seed, b, h, step)
         c_in, s_in, f_in = (_c(state["codes"][b, h], np.int8), _c(state["scales"][b, h], np.float32),
-                            _c(state["f"][b, h], np.float32))
+                            _f_in(state, b, h, dk, dv))
         c_out = np.zeros((dk, dv), np.int8)
         s_out = np.zeros(dv, np.float32)
         f_out = np.zeros((dk, dv), np.float32)
@@ -216,7 +223,7 @@ def quantize(S: np.ndarray, head_bits, *, rounding: int, seed: int, step: int,
              mode: int = CANONICAL) -> dict:
     """Quantize a full-precision state [B][H][dk][dv]; 32-bit heads are copied."""
     B, H, dk, dv = S.shape
-    st = zero_state(B, H, dk, dv)
+    st = zero_state(B, H, dk, dv, fp32=any(int(b) == 32 for b in head_bits))
     L = lib()
     for b in range(B):
         for h in range(H):
@@ -270,7 +277,7 @@ def pack_state(st: dict, head_bits) -> np.ndarray:
         for h in range(H):
             buf = np.zeros(sizes[h], np.uint8)
             c = _c(st["codes"][b, h], np.int8)
-            f = _c(st["f"][b, h], np.float32)
+            f = _f_in(st, b, h, dk, dv)
             L.orc_pack_head(dk, dv, int(head_bits[h]), _p(c), _p(f), _p(buf))
             out[b, off:off + sizes[h]] = buf
             off += sizes[h]
@@ -278,23 +285,23 @@ def pack_state(st: dict, head_bits) -> np.ndarray:
 
 
 def unpack_state(buf: np.ndarray, scales: np.ndarray, head_bits, B: int, H: int, dk: int,
-                 dv: int) -> dict:
-    """Library byte buffer [B][row_bytes] + scales [B][H][dv] -> logical state."""
+                 dv: int, heads=None) -> dict:
+    """Library byte buffer [B][row_bytes] + scales [B][H][dv] -> logical state
+    (only the listed (b, h) heads when ``heads`` is given; the others stay zero)."""
     sizes = [head_bytes(dk, dv, int(b)) for b in head_bits]
-    buf = _c(buf, np.uint8).reshape(B, sum(sizes))
-    st = zero_state(B, H, dk, dv)
+    offs = np.concatenate([[0], np.cumsum(sizes)]).astype(np.int64)
+    buf = _c(buf, np.uint8).reshape(B, int(offs[-1]))
+    st = zero_state(B, H, dk, dv, fp32=any(int(b) == 32 for b in head_bits))
     st["scales"] = _c(scales, np.float32).reshape(B, H, dv).copy()
     L = lib()
-    for b in range(B):
-        off = 0
-        for h in range(H):
-            src = _c(buf[b, off:off + sizes[h]], np.uint8)
-            c = np.zeros((dk, dv), np.int8)
-            f = np.zeros((dk, dv), np.float32)
-            L.orc_unpack_head(dk, dv, int(head_bits[h]), _p(src), _p(c), _p(f))
-            st["codes"][b, h] = c
+    for b, h in _heads(B, H, heads):
+        src = _c(buf[b, offs[h]:offs[h + 1]], np.uint8)
+        c = np.zeros((dk, dv), np.int8)
+        f = np.zeros((dk, dv), np.float32)
+        L.orc_unpack_head(dk, dv, int(head_bits[h]), _p(src), _p(c), _p(f))
+        st["codes"][b, h] = c
+        if st["f"] is not None:
             st["f"][b, h] = f
-            off += sizes[h]
     return st
 
 

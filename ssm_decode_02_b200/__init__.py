@@ -1,0 +1,270 @@
+"""Quantized recurrent-state decode step for B200 (sm_100a): Python binding.
+
+A thin ctypes layer over the C ABI of ``librsq.so`` (declared in include/rsq.h).
+The functions keep the C names (``rsq_create``, ``rsq_decode_step``, ...) and
+only marshal arguments: tensors become device pointers, streams become
+``cudaStream_t`` handles.  Every step of the decode path runs in the library's
+CUDA kernels; there is no fallback, and importing this package on a machine
+where the library cannot be loaded raises.
+
+PyTorch is used for device memory and streams only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "librsq.so")
+
+RSQ_GDN, RSQ_MAMBA2 = 0, 1
+RSQ_RTN, RSQ_SR = 0, 1
+RSQ_F32, RSQ_BF16 = 0, 1
+RSQ_OK, RSQ_E_INVAL, RSQ_E_UNSUPPORTED, RSQ_E_CUDA, RSQ_E_NOMEM, RSQ_E_NONFINITE = range(6)
+RSQ_MAX_HEADS = 512
+
+
+class RsqError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__("rsq status %d (%s): %s" % (status, _status_name(status), message))
+        self.status = status
+
+
+class rsq_config(ctypes.Structure):
+    _fields_ = [("family", ctypes.c_int), ("batch", ctypes.c_int), ("heads", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("ngroups", ctypes.c_int),
+                ("head_bits", ctypes.POINTER(ctypes.c_int8)), ("rounding", ctypes.c_int),
+                ("in_dtype", ctypes.c_int), ("seed", ctypes.c_uint64)]
+
+
+class rsq_state(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p)]
+
+
+class rsq_gdn_inputs(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("alpha", ctypes.c_void_p), ("beta", ctypes.c_void_p)]
+
+
+class rsq_mamba2_inputs(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("Bm", ctypes.c_void_p), ("Cm", ctypes.c_void_p),
+                ("dt", ctypes.c_void_p), ("A", ctypes.c_void_p), ("D", ctypes.c_void_p),
+                ("decay", ctypes.c_void_p)]
+
+
+_EXPORTS = ["rsq_create", "rsq_destroy", "rsq_state_bytes", "rsq_head_offset", "rsq_decode_step",
+            "rsq_quantize", "rsq_dequantize", "rsq_state_drift", "rsq_check_flags",
+            "rsq_allocate_bits", "rsq_reduction_partials", "rsq_status_string", "rsq_last_error",
+            "rsq_version"]
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError("librsq.so not built (run python -m ssm_decode_02_b200.build): %s" % LIB_PATH)
+    L = ctypes.CDLL(LIB_PATH)
+    P, C = ctypes.c_void_p, ctypes.c_int
+    sig = {
+        "rsq_create": ([ctypes.POINTER(rsq_config), ctypes.POINTER(P)], C),
+        "rsq_destroy": ([P], None),
+        "rsq_state_bytes": ([P, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t)], C),
+        "rsq_head_offset": ([P, C, ctypes.POINTER(ctypes.c_size_t)], C),
+        "rsq_decode_step": ([P, ctypes.POINTER(rsq_state), ctypes.POINTER(rsq_state), P, P,
+                             ctypes.c_uint32, P], C),
+        "rsq_quantize": ([P, P, ctypes.POINTER(rsq_state), ctypes.c_uint32, P], C),
+        "rsq_dequantize": ([P, ctypes.POINTER(rsq_state), P, P], C),
+        "rsq_state_drift": ([P, ctypes.POINTER(rsq_state), P, ctypes.POINTER(rsq_state), P, P], C),
+        "rsq_check_flags": ([P, ctypes.POINTER(C), P], C),
+        "rsq_allocate_bits": ([P, C, C, C, C, P], C),
+        "rsq_reduction_partials": ([C], C),
+        "rsq_status_string": ([C], ctypes.c_char_p),
+        "rsq_last_error": ([], ctypes.c_char_p),
+        "rsq_version": ([], ctypes.c_char_p),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(L, name)
+        f.argtypes = args
+        f.restype = res
+    return L
+
+
+lib = _load()
+
+
+def _status_name(s: int) -> str:
+    return lib.rsq_status_string(int(s)).decode()
+
+
+def _check(status: int) -> int:
+    if status != RSQ_OK:
+        raise RsqError(status, lib.rsq_last_error().decode())
+    return status
+
+
+def _ptr(t) -> int | None:
+    """Device (or host) address of a tensor / buffer; ints pass through; None stays None."""
+    if t is None:
+        return None
+    if isinstance(t, int):
+        return t
+    if hasattr(t, "data_ptr"):
+        return int(t.data_ptr())
+    if isinstance(t, np.ndarray):
+        return int(t.ctypes.data)
+    raise TypeError("cannot take the address of %r" % type(t))
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        import torch
+        return int(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return stream
+    return int(stream.cuda_stream)
+
+
+# ---------------------------------------------------------------------------
+# C functions under their own names (argument marshalling only)
+# ---------------------------------------------------------------------------
+def rsq_create(family: int, batch: int, heads: int, dk: int, dv: int, *, head_bits=None,
+               rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0,
+               ngroups: int = 1) -> int:
+    bits_arr = None
+    if head_bits is not None:
+        bits_arr = (ctypes.c_int8 * heads)(*[int(b) for b in head_bits])
+    cfg = rsq_config(int(family), int(batch), int(heads), int(dk), int(dv), int(ngroups),
+                     ctypes.cast(bits_arr, ctypes.POINTER(ctypes.c_int8)) if bits_arr else None,
+                     int(rounding), int(in_dtype), int(seed) & (2 ** 64 - 1))
+    out = ctypes.c_void_p()
+    _check(lib.rsq_create(ctypes.byref(cfg), ctypes.byref(out)))
+    return int(out.value)
+
+
+def rsq_destroy(ctx: int) -> None:
+    lib.rsq_destroy(ctx)
+
+
+def rsq_state_bytes(ctx: int) -> tuple[int, int]:
+    a, b = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib.rsq_state_bytes(ctx, ctypes.byref(a), ctypes.byref(b)))
+    return int(a.value), int(b.value)
+
+
+def rsq_head_offset(ctx: int, h: int) -> int:
+    o = ctypes.c_size_t()
+    _check(lib.rsq_head_offset(ctx, int(h), ctypes.byref(o)))
+    return int(o.value)
+
+
+def _state(st) -> rsq_state:
+    return rsq_state(_ptr(st.codes), _ptr(st.scales))
+
+
+def rsq_decode_step(ctx: int, state_in, state_out, inputs, out, step: int, stream=None) -> None:
+    """inputs: rsq_gdn_inputs / rsq_mamba2_inputs (see gdn_inputs / mamba2_inputs)."""
+    si, so = _state(state_in), _state(state_out)
+    _check(lib.rsq_decode_step(ctx, ctypes.byref(si), ctypes.byref(so), ctypes.byref(inputs),
+                               _ptr(out), int(step) & 0xFFFFFFFF, _stream(stream)))
+
+
+def rsq_quantize(ctx: int, S, state_out, step: int, stream=None) -> None:
+    so = _state(state_out)
+    _check(lib.rsq_quantize(ctx, _ptr(S), ctypes.byref(so), int(step) & 0xFFFFFFFF, _stream(stream)))
+
+
+def rsq_dequantize(ctx: int, state_in, S_out, stream=None) -> None:
+    si = _state(state_in)
+    _check(lib.rsq_dequantize(ctx, ctypes.byref(si), _ptr(S_out), _stream(stream)))
+
+
+def rsq_state_drift(q_ctx: int, q_state, f_ctx: int, f_state, sums, stream=None) -> None:
+    a, b = _state(q_state), _state(f_state)
+    _check(lib.rsq_state_drift(q_ctx, ctypes.byref(a), f_ctx, ctypes.byref(b), _ptr(sums),
+                               _stream(stream)))
+
+
+def rsq_check_flags(ctx: int, stream=None) -> int:
+    """Returns 1 if a non-finite column was seen since the last check (and clears it)."""
+    seen = ctypes.c_int(0)
+    st = lib.rsq_check_flags(ctx, ctypes.byref(seen), _stream(stream))
+    if st not in (RSQ_OK, RSQ_E_NONFINITE):
+        _check(st)
+    return int(seen.value)
+
+
+def rsq_allocate_bits(score, n_high: int, high_bits: int = 8, low_bits: int = 4) -> np.ndarray:
+    s = np.ascontiguousarray(score, dtype=np.float64)
+    out = np.zeros(s.shape[0], dtype=np.int8)
+    _check(lib.rsq_allocate_bits(_ptr(s), s.shape[0], int(n_high), int(high_bits), int(low_bits),
+                                 _ptr(out)))
+    return out
+
+
+def rsq_reduction_partials(dk: int) -> int:
+    return int(lib.rsq_reduction_partials(int(dk)))
+
+
+def rsq_version() -> str:
+    return lib.rsq_version().decode()
+
+
+# ---------------------------------------------------------------------------
+# Convenience containers (torch tensors for device memory)
+# ---------------------------------------------------------------------------
+class State:
+    """A stored state: codes uint8 [B][row_bytes] and scales float32 [B][H][dv] (device)."""
+
+    def __init__(self, codes, scales):
+        self.codes = codes
+        self.scales = scales
+
+
+def gdn_inputs(q, k, v, alpha, beta) -> rsq_gdn_inputs:
+    return rsq_gdn_inputs(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta))
+
+
+def mamba2_inputs(x, Bm, Cm, dt, A, D, decay=None) -> rsq_mamba2_inputs:
+    return rsq_mamba2_inputs(_ptr(x), _ptr(Bm), _ptr(Cm), _ptr(dt), _ptr(A), _ptr(D), _ptr(decay))
+
+
+class Context:
+    """Owns one rsq_ctx (one layer configuration)."""
+
+    def __init__(self, family: int, batch: int, heads: int, dk: int, dv: int, *, head_bits=None,
+                 rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0, ngroups: int = 1):
+        self.family, self.batch, self.heads, self.dk, self.dv = family, batch, heads, dk, dv
+        self.head_bits = None if head_bits is None else np.asarray(head_bits, np.int8)
+        self.rounding, self.in_dtype, self.seed, self.ngroups = rounding, in_dtype, seed, ngroups
+        self.ctx = rsq_create(family, batch, heads, dk, dv, head_bits=head_bits, rounding=rounding,
+                              in_dtype=in_dtype, seed=seed, ngroups=ngroups)
+        self.code_bytes, self.scale_bytes = rsq_state_bytes(self.ctx)
+
+    def close(self):
+        if getattr(self, "ctx", None):
+            rsq_destroy(self.ctx)
+            self.ctx = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def alloc_state(self, device="cuda") -> State:
+        import torch
+        codes = torch.empty((self.batch, self.code_bytes // self.batch), dtype=torch.uint8, device=device)
+        scales = torch.empty((self.batch, self.heads, self.dv), dtype=torch.float32, device=device)
+        return State(codes, scales)
+
+    def decode_step(self, state_in: State, state_out: State, inputs, out, step: int, stream=None):
+        rsq_decode_step(self.ctx, state_in, state_out, inputs, out, step, stream)
+
+    def quantize(self, S, state_out: State, step: int = 0, stream=None):
+        rsq_quantize(self.ctx, S, state_out, step, stream)
+
+    def dequantize(self, state_in: State, S_out, stream=None):
+        rsq_dequantize(self.ctx, state_in, S_out, stream)
+
+    def check_flags(self, stream=None) -> int:
+        return rsq_check_flags(self.ctx, stream)

@@ -1,0 +1,336 @@
+// rsq_api.cu -- the C ABI declared in include/rsq.h: validation, context
+// bookkeeping (per-head bit widths and offsets, launch geometry) and launches.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "rsq_internal.h"
+
+struct rsq_ctx {
+    rsq_config cfg;
+    int8_t bits[RSQ_MAX_HEADS];
+    uint32_t head_off[RSQ_MAX_HEADS];
+    long long row_bytes;
+    bool f32state;
+    int cb, ncb, units;
+    int grid;        // persistent decode grid
+    int device;
+    unsigned* flag;  // device word: rsq::kFlag* bits
+};
+
+namespace {
+
+thread_local char g_err[512] = "";
+
+rsq_status fail(rsq_status s, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+    return s;
+}
+
+rsq_status cuda_fail(int err, const char* what) {
+    return fail(RSQ_E_CUDA, "%s: %s", what, cudaGetErrorString(static_cast<cudaError_t>(err)));
+}
+
+bool pow2_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <class P>
+void fill_heads(const rsq_ctx* c, P& p) {
+    for (int h = 0; h < c->cfg.heads; ++h) {
+        p.head_off[h] = c->head_off[h];
+        p.head_bits[h] = static_cast<uint8_t>(c->bits[h]);
+    }
+}
+
+rsq_status check_state(const rsq_ctx* c, const rsq_state* s, const char* name) {
+    if (!s || !s->codes) return fail(RSQ_E_INVAL, "%s: null state or codes", name);
+    if (!aligned16(s->codes)) return fail(RSQ_E_INVAL, "%s: codes not 16-byte aligned", name);
+    if (!c->f32state) {
+        if (!s->scales) return fail(RSQ_E_INVAL, "%s: null scales", name);
+        if (!aligned16(s->scales)) return fail(RSQ_E_INVAL, "%s: scales not 16-byte aligned", name);
+    }
+    return RSQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rsq_last_error(void) { return g_err; }
+
+const char* rsq_version(void) { return "rsq 0.1 (sm_100a)"; }
+
+const char* rsq_status_string(rsq_status s) {
+    switch (s) {
+        case RSQ_OK: return "ok";
+        case RSQ_E_INVAL: return "invalid argument";
+        case RSQ_E_UNSUPPORTED: return "unsupported configuration";
+        case RSQ_E_CUDA: return "CUDA error";
+        case RSQ_E_NOMEM: return "out of memory";
+        case RSQ_E_NONFINITE: return "non-finite state column seen";
+    }
+    return "unknown status";
+}
+
+int rsq_reduction_partials(int dk) { return dk <= 128 ? 8 : 16; }
+
+rsq_status rsq_allocate_bits(const double* score, int heads, int n_high, int high_bits,
+                             int low_bits, int8_t* bits_out) {
+    if (!score || !bits_out) return fail(RSQ_E_INVAL, "allocate_bits: null pointer");
+    if (heads < 1 || heads > RSQ_MAX_HEADS) return fail(RSQ_E_INVAL, "allocate_bits: heads out of range");
+    if (n_high < 0 || n_high > heads) return fail(RSQ_E_INVAL, "allocate_bits: n_high out of range");
+    auto ok_bits = [](int b) { return b == 4 || b == 8; };
+    if (!ok_bits(high_bits) || !ok_bits(low_bits)) return fail(RSQ_E_INVAL, "allocate_bits: bits must be 4 or 8");
+    std::vector<int> order(static_cast<size_t>(heads));
+    for (int h = 0; h < heads; ++h) order[h] = h;
+    // slowest decay first; equal scores keep head order
+    std::stable_sort(order.begin(), order.end(),
+                     [&](int a, int b) { return score[a] > score[b]; });
+    for (int h = 0; h < heads; ++h) bits_out[h] = static_cast<int8_t>(low_bits);
+    for (int t = 0; t < n_high; ++t) bits_out[order[t]] = static_cast<int8_t>(high_bits);
+    return RSQ_OK;
+}
+
+rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
+    if (!cfg || !out) return fail(RSQ_E_INVAL, "create: null argument");
+    *out = nullptr;
+    const rsq_config& c = *cfg;
+    if (c.family != RSQ_GDN && c.family != RSQ_MAMBA2) return fail(RSQ_E_INVAL, "create: bad family %d", c.family);
+    if (c.batch < 1) return fail(RSQ_E_INVAL, "create: batch must be >= 1");
+    if (c.heads < 1 || c.heads > RSQ_MAX_HEADS) return fail(RSQ_E_INVAL, "create: heads must be in [1, %d]", RSQ_MAX_HEADS);
+    if (!pow2_dim(c.dk) || !pow2_dim(c.dv))
+        return fail(RSQ_E_UNSUPPORTED, "create: dk and dv must be one of 16, 32, 64, 128, 256 (got %d, %d)", c.dk, c.dv);
+    if (c.rounding != RSQ_RTN && c.rounding != RSQ_SR) return fail(RSQ_E_INVAL, "create: bad rounding %d", c.rounding);
+    if (c.in_dtype != RSQ_F32 && c.in_dtype != RSQ_BF16) return fail(RSQ_E_INVAL, "create: bad in_dtype %d", c.in_dtype);
+    if (c.family == RSQ_MAMBA2 && (c.ngroups < 1 || c.heads % c.ngroups != 0))
+        return fail(RSQ_E_INVAL, "create: ngroups must divide heads");
+
+    rsq_ctx* ctx = new (std::nothrow) rsq_ctx();
+    if (!ctx) return fail(RSQ_E_NOMEM, "create: host allocation failed");
+    ctx->cfg = c;
+    ctx->cfg.head_bits = nullptr;
+    int n32 = 0;
+    for (int h = 0; h < c.heads; ++h) {
+        const int b = c.head_bits ? c.head_bits[h] : 8;
+        if (b != 4 && b != 8 && b != 32) {
+            delete ctx;
+            return fail(RSQ_E_INVAL, "create: head %d has %d bits (4, 8 or 32)", h, b);
+        }
+        n32 += (b == 32);
+        ctx->bits[h] = static_cast<int8_t>(b);
+    }
+    if (n32 != 0 && n32 != c.heads) {
+        delete ctx;
+        return fail(RSQ_E_UNSUPPORTED, "create: 32-bit heads cannot be mixed with 4/8-bit heads");
+    }
+    ctx->f32state = (n32 == c.heads);
+    long long off = 0;
+    for (int h = 0; h < c.heads; ++h) {
+        ctx->head_off[h] = static_cast<uint32_t>(off);
+        off += static_cast<long long>(c.dk) * c.dv * ctx->bits[h] / 8;
+    }
+    ctx->row_bytes = off;
+    ctx->cb = std::min(c.dv, 64);
+    ctx->ncb = c.dv / ctx->cb;
+    const long long units = static_cast<long long>(c.batch) * c.heads * ctx->ncb;
+    if (units > (1LL << 30)) {
+        delete ctx;
+        return fail(RSQ_E_UNSUPPORTED, "create: too many work units");
+    }
+    ctx->units = static_cast<int>(units);
+
+    // launch geometry: persistent grid of every resident CTA
+    int threads = 0;
+    size_t smem = 0;
+    const void* func = nullptr;
+    if (rsq::decode_kernel_info(c.family, c.dk, ctx->cb, ctx->f32state, &threads, &smem, &func) != 0) {
+        delete ctx;
+        return fail(RSQ_E_UNSUPPORTED, "create: no kernel for dk=%d dv=%d", c.dk, c.dv);
+    }
+    int err = cudaGetDevice(&ctx->device);
+    int sms = 0, per_sm = 0;
+    if (!err) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, ctx->device);
+    if (!err) err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (!err) err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, func, threads, smem);
+    if (!err && per_sm < 1) err = cudaErrorInvalidConfiguration;
+    if (!err) err = cudaMalloc(&ctx->flag, sizeof(unsigned));
+    if (!err) err = cudaMemset(ctx->flag, 0, sizeof(unsigned));
+    if (err) {
+        if (ctx->flag) cudaFree(ctx->flag);
+        delete ctx;
+        if (err == cudaErrorMemoryAllocation) return fail(RSQ_E_NOMEM, "create: flag allocation failed");
+        return cuda_fail(err, "create");
+    }
+    ctx->grid = static_cast<int>(std::min<long long>(units, static_cast<long long>(sms) * per_sm));
+    *out = ctx;
+    return RSQ_OK;
+}
+
+void rsq_destroy(rsq_ctx* ctx) {
+    if (!ctx) return;
+    if (ctx->flag) cudaFree(ctx->flag);
+    delete ctx;
+}
+
+rsq_status rsq_state_bytes(const rsq_ctx* ctx, size_t* code_bytes, size_t* scale_bytes) {
+    if (!ctx || !code_bytes || !scale_bytes) return fail(RSQ_E_INVAL, "state_bytes: null argument");
+    *code_bytes = static_cast<size_t>(ctx->row_bytes) * ctx->cfg.batch;
+    *scale_bytes = static_cast<size_t>(ctx->cfg.batch) * ctx->cfg.heads * ctx->cfg.dv * sizeof(float);
+    return RSQ_OK;
+}
+
+rsq_status rsq_head_offset(const rsq_ctx* ctx, int h, size_t* offset) {
+    if (!ctx || !offset) return fail(RSQ_E_INVAL, "head_offset: null argument");
+    if (h < 0 || h >= ctx->cfg.heads) return fail(RSQ_E_INVAL, "head_offset: head out of range");
+    *offset = ctx->head_off[h];
+    return RSQ_OK;
+}
+
+rsq_status rsq_decode_step(const rsq_ctx* ctx, const rsq_state* state_in, const rsq_state* state_out,
+                           const void* inputs, float* out, uint32_t step, void* stream) {
+    if (!ctx) return fail(RSQ_E_INVAL, "decode_step: null context");
+    rsq_status s = check_state(ctx, state_in, "decode_step(state_in)");
+    if (s) return s;
+    if ((s = check_state(ctx, state_out, "decode_step(state_out)"))) return s;
+    if (!inputs) return fail(RSQ_E_INVAL, "decode_step: null inputs");
+    if (!out || !aligned16(out)) return fail(RSQ_E_INVAL, "decode_step: out null or not 16-byte aligned");
+    const rsq_config& c = ctx->cfg;
+    rsq::DecodeParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = c.batch; p.H = c.heads; p.dk = c.dk; p.dv = c.dv; p.ncb = ctx->ncb; p.units = ctx->units;
+    p.in_bf16 = (c.in_dtype == RSQ_BF16);
+    p.sr = (c.rounding == RSQ_SR);
+    p.row_bytes = ctx->row_bytes;
+    p.codes_in = static_cast<const uint8_t*>(state_in->codes);
+    p.codes_out = static_cast<uint8_t*>(state_out->codes);
+    p.scales_in = state_in->scales;
+    p.scales_out = state_out->scales;
+    p.out = out;
+    p.flag = ctx->flag;
+    p.step = step;
+    p.key0 = static_cast<uint32_t>(c.seed);
+    p.key1 = static_cast<uint32_t>(c.seed >> 32);
+    if (c.family == RSQ_GDN) {
+        const rsq_gdn_inputs* in = static_cast<const rsq_gdn_inputs*>(inputs);
+        if (!in->q || !in->k || !in->v || !in->alpha || !in->beta)
+            return fail(RSQ_E_INVAL, "decode_step: null GDN input");
+        if (!aligned16(in->q) || !aligned16(in->k) || !aligned16(in->v))
+            return fail(RSQ_E_INVAL, "decode_step: q/k/v not 16-byte aligned");
+        p.vA = in->q; p.vB = in->k; p.vC = in->v; p.g0 = in->alpha; p.g1 = in->beta;
+        p.ngroups = 1; p.heads_per_group = c.heads;
+    } else {
+        const rsq_mamba2_inputs* in = static_cast<const rsq_mamba2_inputs*>(inputs);
+        if (!in->x || !in->Bm || !in->Cm || !in->dt || !in->A || !in->D)
+            return fail(RSQ_E_INVAL, "decode_step: null Mamba-2 input");
+        if (!aligned16(in->x) || !aligned16(in->Bm) || !aligned16(in->Cm))
+            return fail(RSQ_E_INVAL, "decode_step: x/B/C not 16-byte aligned");
+        p.vA = in->Cm; p.vB = in->Bm; p.vC = in->x; p.g0 = in->dt; p.g1 = in->decay;
+        p.A = in->A; p.D = in->D;
+        p.ngroups = c.ngroups; p.heads_per_group = c.heads / c.ngroups;
+    }
+    fill_heads(ctx, p);
+    const int err = rsq::launch_decode(c.family, c.dk, ctx->cb, ctx->f32state, p, ctx->grid, stream);
+    if (err) return cuda_fail(err, "decode_step launch");
+    return RSQ_OK;
+}
+
+rsq_status rsq_quantize(const rsq_ctx* ctx, const float* S, const rsq_state* state_out, uint32_t step,
+                        void* stream) {
+    if (!ctx) return fail(RSQ_E_INVAL, "quantize: null context");
+    if (!S || !aligned16(S)) return fail(RSQ_E_INVAL, "quantize: S null or not 16-byte aligned");
+    rsq_status s = check_state(ctx, state_out, "quantize(state_out)");
+    if (s) return s;
+    const rsq_config& c = ctx->cfg;
+    rsq::QuantParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = c.batch; p.H = c.heads; p.dk = c.dk; p.dv = c.dv; p.ncb = ctx->ncb; p.units = ctx->units;
+    p.sr = (c.rounding == RSQ_SR);
+    p.row_bytes = ctx->row_bytes;
+    p.S = S;
+    p.codes = static_cast<uint8_t*>(state_out->codes);
+    p.scales = state_out->scales;
+    p.flag = ctx->flag;
+    p.step = step;
+    p.key0 = static_cast<uint32_t>(c.seed);
+    p.key1 = static_cast<uint32_t>(c.seed >> 32);
+    fill_heads(ctx, p);
+    const int err = rsq::launch_quantize(c.dk, ctx->cb, p, stream);
+    if (err) return cuda_fail(err, "quantize launch");
+    return RSQ_OK;
+}
+
+rsq_status rsq_dequantize(const rsq_ctx* ctx, const rsq_state* state_in, float* S_out, void* stream) {
+    if (!ctx) return fail(RSQ_E_INVAL, "dequantize: null context");
+    if (!S_out || !aligned16(S_out)) return fail(RSQ_E_INVAL, "dequantize: S_out null or not 16-byte aligned");
+    rsq_status s = check_state(ctx, state_in, "dequantize(state_in)");
+    if (s) return s;
+    const rsq_config& c = ctx->cfg;
+    rsq::DequantParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = c.batch; p.H = c.heads; p.dk = c.dk; p.dv = c.dv; p.ncb = ctx->ncb;
+    p.row_bytes = ctx->row_bytes;
+    p.codes = static_cast<const uint8_t*>(state_in->codes);
+    p.scales = state_in->scales;
+    p.S = S_out;
+    fill_heads(ctx, p);
+    const int err = rsq::launch_dequantize(c.dk, ctx->cb, p, stream);
+    if (err) return cuda_fail(err, "dequantize launch");
+    return RSQ_OK;
+}
+
+rsq_status rsq_state_drift(const rsq_ctx* q_ctx, const rsq_state* q_state, const rsq_ctx* f_ctx,
+                           const rsq_state* f_state, double* sums, void* stream) {
+    if (!q_ctx || !f_ctx || !sums) return fail(RSQ_E_INVAL, "state_drift: null argument");
+    if (q_ctx->f32state || !f_ctx->f32state)
+        return fail(RSQ_E_INVAL, "state_drift: need a quantized and a full-precision context");
+    const rsq_config& a = q_ctx->cfg;
+    const rsq_config& b = f_ctx->cfg;
+    if (a.batch != b.batch || a.heads != b.heads || a.dk != b.dk || a.dv != b.dv)
+        return fail(RSQ_E_INVAL, "state_drift: shapes differ");
+    rsq_status s = check_state(q_ctx, q_state, "state_drift(q)");
+    if (s) return s;
+    if ((s = check_state(f_ctx, f_state, "state_drift(f)"))) return s;
+    if (reinterpret_cast<uintptr_t>(sums) & 7u) return fail(RSQ_E_INVAL, "state_drift: sums not 8-byte aligned");
+    rsq::DriftParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = a.batch; p.H = a.heads; p.dk = a.dk; p.dv = a.dv; p.ncb = q_ctx->ncb;
+    p.q_row_bytes = q_ctx->row_bytes;
+    p.f_row_bytes = f_ctx->row_bytes;
+    p.q_codes = static_cast<const uint8_t*>(q_state->codes);
+    p.q_scales = q_state->scales;
+    p.f_codes = static_cast<const uint8_t*>(f_state->codes);
+    p.sums = sums;
+    for (int h = 0; h < a.heads; ++h) {
+        p.q_head_off[h] = q_ctx->head_off[h];
+        p.q_head_bits[h] = static_cast<uint8_t>(q_ctx->bits[h]);
+    }
+    const int err = rsq::launch_drift(p, stream);
+    if (err) return cuda_fail(err, "state_drift launch");
+    return RSQ_OK;
+}
+
+rsq_status rsq_check_flags(const rsq_ctx* ctx, int* seen, void* stream) {
+    if (!ctx || !seen) return fail(RSQ_E_INVAL, "check_flags: null argument");
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    unsigned h = 0;
+    int err = cudaStreamSynchronize(st);
+    if (!err) err = cudaMemcpyAsync(&h, ctx->flag, sizeof(unsigned), cudaMemcpyDeviceToHost, st);
+    if (!err) err = cudaMemsetAsync(ctx->flag, 0, sizeof(unsigned), st);
+    if (!err) err = cudaStreamSynchronize(st);
+    if (err) return cuda_fail(err, "check_flags");
+    *seen = (h & rsq::kFlagNonFinite) ? 1 : 0;
+    if (h & rsq::kFlagTimeout) return fail(RSQ_E_CUDA, "check_flags: a kernel barrier wait timed out");
+    if (*seen) return fail(RSQ_E_NONFINITE, "check_flags: non-finite state column seen");
+    return RSQ_OK;
+}
+
+}  // extern "C"

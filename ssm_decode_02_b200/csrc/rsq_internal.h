@@ -1,0 +1,82 @@
+// rsq_internal.h -- parameter blocks shared by the host API and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+
+#include "../../include/rsq.h"
+
+namespace rsq {
+
+constexpr unsigned kFlagNonFinite = 1u;  // a column's absmax was inf or NaN
+constexpr unsigned kFlagTimeout = 2u;    // a bounded barrier wait ran out
+
+// Everything one decode launch needs, passed by value as a __grid_constant__.
+struct DecodeParams {
+    int B, H, dk, dv, ncb, units;  // units = B * H * ncb column blocks
+    int ngroups, heads_per_group;
+    int in_bf16;                   // vector inputs are bf16 (else float)
+    int sr;                        // stochastic rounding (else round-to-nearest)
+    long long row_bytes;           // code bytes per batch row
+    const uint8_t* codes_in;
+    uint8_t* codes_out;
+    const float* scales_in;
+    float* scales_out;
+    const void* vA;                // GDN q      | Mamba-2 C
+    const void* vB;                // GDN k      | Mamba-2 B
+    const void* vC;                // GDN v      | Mamba-2 x
+    const float* g0;               // GDN alpha  | Mamba-2 dt
+    const float* g1;               // GDN beta   | Mamba-2 decay override (may be null)
+    const float* A;                // Mamba-2 A [H]
+    const float* D;                // Mamba-2 D [H]
+    float* out;                    // [B][H][dv]
+    unsigned* flag;
+    uint32_t step, key0, key1;
+    uint32_t head_off[RSQ_MAX_HEADS];  // byte offset of each head in a batch row
+    uint8_t head_bits[RSQ_MAX_HEADS];
+};
+
+struct QuantParams {
+    int B, H, dk, dv, ncb, units;
+    int sr;
+    long long row_bytes;
+    const float* S;                // natural [B][H][dk][dv]
+    uint8_t* codes;
+    float* scales;
+    unsigned* flag;
+    uint32_t step, key0, key1;
+    uint32_t head_off[RSQ_MAX_HEADS];
+    uint8_t head_bits[RSQ_MAX_HEADS];
+};
+
+struct DequantParams {
+    int B, H, dk, dv, ncb;
+    long long row_bytes;
+    const uint8_t* codes;
+    const float* scales;
+    float* S;                      // natural [B][H][dk][dv]
+    uint32_t head_off[RSQ_MAX_HEADS];
+    uint8_t head_bits[RSQ_MAX_HEADS];
+};
+
+struct DriftParams {
+    int B, H, dk, dv, ncb;
+    long long q_row_bytes, f_row_bytes;
+    const uint8_t* q_codes;
+    const float* q_scales;
+    const uint8_t* f_codes;
+    double* sums;                  // [B][H][2]
+    uint32_t q_head_off[RSQ_MAX_HEADS];
+    uint8_t q_head_bits[RSQ_MAX_HEADS];
+};
+
+// Launchers (defined in the .cu files).  Return a cudaError_t value.
+int launch_decode(int family, int dk, int cb, bool f32state, const DecodeParams& p, int grid,
+                  void* stream);
+int decode_kernel_info(int family, int dk, int cb, bool f32state, int* threads, size_t* smem,
+                       const void** func);
+int launch_quantize(int dk, int cb, const QuantParams& p, void* stream);
+int launch_dequantize(int dk, int cb, const DequantParams& p, void* stream);
+int launch_drift(const DriftParams& p, void* stream);
+
+}  // namespace rsq

@@ -8,7 +8,17 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def _build_libraries():
+    """Build the oracle and the CUDA library in-tree when missing or stale (nvcc
+    cross-compiles for sm_100a without a GPU)."""
+    from oracle import build as obuild
+    from ssm_decode_02_b200 import build as lbuild
+    obuild.build()
+    lbuild.build()
+
+
 def pytest_configure(config):
+    _build_libraries()
     config.addinivalue_line("markers", "gpu: needs a CUDA GPU (B200, sm_100a)")
     config.addinivalue_line("markers", "slow: long CPU statistical test")
 
