@@ -48,10 +48,9 @@
  * --------------------------------
  *  codes: device bytes [batch][row_bytes].  Within a batch row the heads are
  *    concatenated in order; head h occupies dk*dv*bits_h/8 bytes.  A head's
- *    columns are cut into blocks of CB = min(64, dv) columns; block cb
- *    (cb = 0 .. dv/CB-1) stores rows i = 0..dk-1 of columns cb*CB..cb*CB+CB-1
- *    row after row, so every block is one contiguous run of dk*CB*bits/8
- *    bytes.  Inside a row segment:
+ *    columns are cut into blocks of 16 columns; block cb (cb = 0 .. dv/16-1)
+ *    stores rows i = 0..dk-1 of columns 16cb..16cb+15 row after row, so every
+ *    block is one contiguous run of dk*16*bits/8 bytes.  Inside a row segment:
  *      8-bit : byte = c + 128                       (one per column)
  *      4-bit : byte t = (c_{2t} + 8) | (c_{2t+1} + 8) << 4
  *      32-bit: IEEE binary32 value of S_ij          (full-precision state)
@@ -61,9 +60,9 @@
  *
  * Arithmetic (binary32 throughout; fixed evaluation order, see rsq_decode_step)
  * ------------------------------------------------------------------------
- *  Sums over the key axis i use R = rsq_reduction_partials(dk) partial sums:
- *  partial p accumulates rows i = p, p+R, p+2R, ... in increasing i with one
- *  fused multiply-add per term; then for d = 1, 2, ..., R/2 every partial p
+ *  Sums over the key axis i use R = rsq_reduction_partials(dk) = 8 partial
+ *  sums: partial p accumulates rows i = p, p+R, p+2R, ... in increasing i with
+ *  one fused multiply-add per term; then for d = 1, 2, ..., R/2 every partial p
  *  becomes P[p] + P[p^d]; the sum is P[0].
  */
 #ifndef RSQ_H
@@ -96,7 +95,7 @@ typedef struct {
     int family;      /* rsq_family */
     int batch;       /* B >= 1 independent requests */
     int heads;       /* H, 1..RSQ_MAX_HEADS */
-    int dk;          /* rows: GDN key dim d_k / Mamba-2 state dim N; one of 16,32,64,128,256 */
+    int dk;          /* rows: GDN key dim d_k / Mamba-2 state dim N; one of 16, 32, 64, 128 */
     int dv;          /* columns: GDN value dim d_v / Mamba-2 head dim P; one of 16,32,64,128,256 */
     int ngroups;     /* Mamba-2 B/C groups (divides heads); ignored for GDN */
     const int8_t* head_bits; /* host [heads]: each 4 or 8, or every entry 32 (full-precision
@@ -226,7 +225,7 @@ rsq_status rsq_allocate_bits(const double* score, int heads, int n_high, int hig
                              int low_bits, int8_t* bits_out);
 
 /* Number of partial sums R of the key-axis reduction order for a given dk
- * (host-only; 8 for dk <= 128, 16 for dk = 256). */
+ * (host-only; 8 for every supported dk). */
 int rsq_reduction_partials(int dk);
 
 const char* rsq_status_string(rsq_status s);

@@ -368,14 +368,13 @@ void orc_dequantize_head(int dk, int dv, const int8_t* c, const float* s, float*
 
 /* ------------------------------------------------------------------------- */
 /* Storage format of the library, written out independently.                 */
-/*   A head's dv columns are cut into blocks of CB = min(64, dv) columns.     */
-/*   Block cb holds rows i = 0..dk-1 of columns cb*CB .. cb*CB+CB-1, row by   */
-/*   row.  8-bit code c is stored as the byte c + 128; 4-bit codes as the     */
+/*   A head's dv columns are cut into blocks of CB = 16 columns.  Block cb     */
+/*   holds rows i = 0..dk-1 of columns cb*CB .. cb*CB+CB-1, row by row.  8-bit code c is stored as the byte c + 128; 4-bit codes as the     */
 /*   nibble c + 8, column 2t in the low nibble of byte t of the row segment   */
 /*   and column 2t+1 in the high nibble.  32-bit heads store binary32 values  */
 /*   in the same block order.                                                 */
 /* ------------------------------------------------------------------------- */
-static int orc_cb(int dv) { return dv < 64 ? dv : 64; }
+static int orc_cb(int dv) { (void)dv; return 16; }
 
 int64_t orc_head_bytes(int dk, int dv, int bits) { return (int64_t)dk * dv * bits / 8; }
 

@@ -20,7 +20,7 @@ BUILD = os.path.join(ROOT, "_build")
 NVCC = os.environ.get("NVCC", "nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ARCH + ["-O3", "-lineinfo", "--fmad=false", "-std=c++17", "-Xcompiler", "-fPIC",
-                "-I", os.path.join(ROOT, "include")]
+                "-I", os.path.join(ROOT, "include")] + os.environ.get("RSQ_NVCC_FLAGS", "").split()
 
 
 def _sources():

@@ -1,0 +1,414 @@
+// decode_kernel.cuh -- fused quantized recurrent-state decode step (sm_100a).
+//
+// A work unit is one to four 16-column blocks of one head (all dk rows); the
+// CTA has one warp per block, and each warp owns its block's columns outright,
+// so every reduction over the key axis stays inside the warp and the loop has
+// no CTA-wide barrier.  Persistent CTAs walk the units with a grid stride.
+// Units arrive in an NS-stage shared-memory ring filled by bulk asynchronous
+// (TMA) copies; the last warp to finish with a stage refills it with the unit
+// NS ahead.  Per block a warp:
+//   1. decodes the codes to exact floats (packed pairs),
+//   2. (Gated DeltaNet) forms u = S^T k as s_j * sum_i c_ij k_i,
+//   3. updates the state in registers (full precision, packed f32x2),
+//   4. reads out o = S^T q (GDN) or y = S^T C + D x (Mamba-2) from that state,
+//   5. takes each column's absmax as its new scale (the dynamic "noisy" scale),
+//   6. requantizes (round-to-nearest or Philox stochastic rounding) and stores.
+// Method: LoReS ("Quantizing Recurrent Language Models Is Easier Than You
+// Think", sections "LoReS: State Quantization", "(1/4) Scale grouping", "(3/4)
+// Rounding"); recurrences as named in "Preserving Updates in Low-Bit Recurrent
+// State Quantization" (abstract).  No tensor cores: per head this is two
+// matrix-vector products over a state read once from HBM.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "rsq_internal.h"
+#include "rsq_tile.cuh"
+
+namespace rsq {
+
+constexpr uint32_t kWaitIters = 1u << 22;  // bounded mbarrier waits (error flag on expiry)
+
+template <int FAM, int DK, int UB, bool F32STATE>
+struct DecodeCfg {
+    using L = Layout<DK>;
+    static constexpr int NT = 32 * UB;         // one warp per 16-column block
+    static constexpr int UCOLS = 16 * UB;      // columns per unit
+    static constexpr int NS = F32STATE ? 2 : 3;  // pipeline stages
+    static constexpr int CODE_BYTES = F32STATE ? DK * UCOLS * 4 : DK * UCOLS;  // largest tile (8-bit)
+    static constexpr int OFF_SCALES = CODE_BYTES;
+    static constexpr int OFF_VA = OFF_SCALES + UCOLS * 4;  // GDN q / Mamba-2 C   (<= DK floats)
+    static constexpr int OFF_VB = OFF_VA + DK * 4;         // GDN k / Mamba-2 B
+    static constexpr int OFF_VC = OFF_VB + DK * 4;         // GDN v / Mamba-2 x   (<= UCOLS floats)
+    static constexpr int STAGE = (OFF_VC + UCOLS * 4 + 127) / 128 * 128;
+    // per warp: the two key-axis vectors as duplicated pairs (x, x), one row of
+    // PST pairs per row group (padded so the row groups hit different banks)
+    static constexpr int PST = L::RPT + 2;
+    static constexpr int P_WARP = 2 * kR * PST * 8;
+    static constexpr int OFF_P = NS * STAGE;
+    static constexpr int OFF_CNT = OFF_P + UB * P_WARP;  // NS release counters
+    static constexpr int OFF_BAR = OFF_CNT + 16;
+    static constexpr int SMEM = OFF_BAR + NS * 8;
+    // resident CTAs per SM the register budget is sized for (GDN keeps more live
+    // values across its extra reduction than Mamba-2)
+    static constexpr int MINB = F32STATE ? 1 : (NT < 128 ? 8 : (FAM == RSQ_GDN ? 4 : 5));
+};
+
+// Grid-stride walk over units without divisions: (b, h, cb) advance by the
+// grid size G, precomputed by the host as (gb, gh, gcb).
+struct UnitIt {
+    int u, b, h, cb;
+    __device__ __forceinline__ void init(int u0, const DecodeParams& p) {
+        u = u0;
+        const int hu = u0 / p.ncb;
+        cb = u0 - hu * p.ncb;
+        b = hu / p.H;
+        h = hu - b * p.H;
+    }
+    __device__ __forceinline__ void advance(const DecodeParams& p) {
+        u += p.grid;
+        cb += p.gcb;
+        h += p.gh;
+        b += p.gb;
+        if (cb >= p.ncb) { cb -= p.ncb; ++h; }
+        if (h >= p.H) { h -= p.H; ++b; }
+    }
+    __device__ __forceinline__ int hu(const DecodeParams& p) const { return b * p.H + h; }
+};
+
+// Issue the bulk copies of one unit into a stage (one thread).
+template <int FAM, int DK, int UB, bool F32STATE>
+__device__ __forceinline__ void issue_unit(const DecodeParams& p, const UnitIt& un, uint8_t* stage,
+                                           uint32_t bar) {
+    using C = DecodeCfg<FAM, DK, UB, F32STATE>;
+    constexpr int UCOLS = C::UCOLS;
+    const int bits = F32STATE ? 32 : p.head_bits[un.h];
+    const int hu = un.hu(p);
+    const uint32_t code_bytes = static_cast<uint32_t>(DK * UCOLS * bits / 8);
+    const uint32_t esz = p.in_bf16 ? 2u : 4u;
+    const uint32_t total = code_bytes + (F32STATE ? 0u : UCOLS * 4u) + 2u * DK * esz + UCOLS * esz;
+    const uint8_t* codes = p.codes_in + (long long)un.b * p.row_bytes + p.head_off[un.h] +
+                           (long long)un.cb * code_bytes;
+    const uint32_t s = smem_u32(stage);
+    mbar_arrive_expect_tx(bar, total);
+    bulk_g2s(s, codes, code_bytes, bar);
+    if (!F32STATE)
+        bulk_g2s(s + C::OFF_SCALES, p.scales_in + (long long)hu * p.dv + un.cb * UCOLS, UCOLS * 4u, bar);
+    const char* vA = static_cast<const char*>(p.vA);
+    const char* vB = static_cast<const char*>(p.vB);
+    const char* vC = static_cast<const char*>(p.vC);
+    const long long rowA = (FAM == RSQ_GDN)
+                               ? (long long)hu * DK  // q and k of this head
+                               : ((long long)un.b * p.ngroups + un.h / p.heads_per_group) * DK;
+    bulk_g2s(s + C::OFF_VA, vA + rowA * esz, DK * esz, bar);
+    bulk_g2s(s + C::OFF_VB, vB + rowA * esz, DK * esz, bar);
+    bulk_g2s(s + C::OFF_VC, vC + ((long long)hu * p.dv + un.cb * UCOLS) * esz, UCOLS * esz, bar);
+}
+
+__device__ __forceinline__ float ld_vec(const uint8_t* base, int e, bool bf16) {
+    if (bf16) return bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(base)[e]);
+    return reinterpret_cast<const float*>(base)[e];
+}
+
+// Four consecutive elements e..e+3 of a vector in the stage, widened.
+__device__ __forceinline__ float4 ld_vec4(const uint8_t* base, int e, bool bf16) {
+    if (bf16) {
+        const uint2 w = *reinterpret_cast<const uint2*>(base + 2 * e);
+        return make_float4(__uint_as_float(w.x << 16), __uint_as_float(w.x & 0xFFFF0000u),
+                           __uint_as_float(w.y << 16), __uint_as_float(w.y & 0xFFFF0000u));
+    }
+    return *reinterpret_cast<const float4*>(base + 4 * e);
+}
+
+// Per-unit scalars fetched one unit ahead.
+struct Gates {
+    float g0, g1, A, D;
+};
+
+template <int FAM>
+__device__ __forceinline__ Gates load_gates(const DecodeParams& p, const UnitIt& un) {
+    Gates g;
+    const int hu = un.hu(p);
+    g.g0 = __ldg(p.g0 + hu);
+    g.g1 = p.g1 ? __ldg(p.g1 + hu) : 0.f;
+    g.A = (FAM == RSQ_MAMBA2) ? __ldg(p.A + un.h) : 0.f;
+    g.D = (FAM == RSQ_MAMBA2) ? __ldg(p.D + un.h) : 0.f;
+    return g;
+}
+
+// One 16-column block of one unit, processed by warp w.
+template <int FAM, int DK, int UB, bool F32STATE, bool SR, int BITS>
+__device__ __forceinline__ void process_block(const DecodeParams& p, const UnitIt& un, uint8_t* stage,
+                                              uint8_t* smem, int stage_idx, uint32_t bar,
+                                              const Gates& gt, int w, int lane, int g, int cw) {
+    using L = Layout<DK>;
+    using C = DecodeCfg<FAM, DK, UB, F32STATE>;
+    constexpr int RPT = L::RPT;
+    constexpr int BLOCK_BYTES = DK * kBlockCols * BITS / 8;
+    const bool bf16 = p.in_bf16 != 0;
+    const int hu = un.hu(p);
+    const int blk = un.cb * UB + w;  // block index within the head
+    const int j0 = blk * kBlockCols;  // its first column
+
+    // ---- this warp's copy of the key-axis vectors as duplicated pairs --------
+    uint64_t* pa = reinterpret_cast<uint64_t*>(smem + C::OFF_P + w * C::P_WARP);
+    uint64_t* pb = pa + kR * C::PST;
+#pragma unroll
+    for (int i = lane; i < DK; i += 32) {
+        const float a = ld_vec(stage + C::OFF_VA, i, bf16);
+        const float b = ld_vec(stage + C::OFF_VB, i, bf16);
+        const int pos = (i & (kR - 1)) * C::PST + i / kR;
+        pa[pos] = pk(a, a);
+        pb[pos] = pk(b, b);
+    }
+    __syncwarp();
+    const uint64_t* qa = pa + g * C::PST;  // q (GDN) / C (Mamba-2) of rows g + 8k
+    const uint64_t* kb = pb + g * C::PST;  // k (GDN) / B (Mamba-2)
+
+    // ---- state block -> registers (packed pairs) ------------------------------
+    const uint8_t* tile = stage + w * BLOCK_BYTES;
+    uint64_t S2[RPT][2];
+    if constexpr (BITS == 32) {
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            const ulonglong2 t = *reinterpret_cast<const ulonglong2*>(tile + ((g + kR * k) * 16 + 4 * cw) * 4);
+            S2[k][0] = t.x;
+            S2[k][1] = t.y;
+        }
+    } else {
+        load_codes<BITS, RPT>(tile, g, cw, S2);  // exact float codes c
+    }
+    // scales and v (GDN) / x (Mamba-2) of this lane's columns, read where needed
+    // (keeping them live across the reductions costs registers)
+    auto load_s4 = [&]() {
+        if constexpr (BITS != 32)
+            return *reinterpret_cast<const float4*>(stage + C::OFF_SCALES + (16 * w + 4 * cw) * 4);
+        else
+            return make_float4(1.f, 1.f, 1.f, 1.f);
+    };
+    auto load_vc = [&]() { return ld_vec4(stage + C::OFF_VC, 16 * w + 4 * cw, bf16); };
+
+    // ---- state update ---------------------------------------------------------
+    if constexpr (FAM == RSQ_GDN) {
+        const float alpha = gt.g0, beta = gt.g1;
+        uint64_t a01 = pk(0.f, 0.f), a23 = pk(0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < RPT; k += 2) {
+            const ulonglong2 kk = *reinterpret_cast<const ulonglong2*>(kb + k);
+            a01 = fma2(S2[k][0], kk.x, a01);
+            a23 = fma2(S2[k][1], kk.x, a23);
+            a01 = fma2(S2[k + 1][0], kk.y, a01);
+            a23 = fma2(S2[k + 1][1], kk.y, a23);
+        }
+        float4 ck = unpk4(a01, a23);
+        warp_sum4(ck);
+        // reload the k pairs below instead of keeping 16 of them live across the
+        // reduction (register pressure)
+        asm volatile("" ::: "memory");
+        // u = s*ck, w = beta*(v - alpha*u), a = alpha*s  (full-precision state: u = ck, a = alpha)
+        const float4 s4 = load_s4();
+        const float4 vc = load_vc();
+        const float ckv[4] = {ck.x, ck.y, ck.z, ck.w};
+        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+        const float vv[4] = {vc.x, vc.y, vc.z, vc.w};
+        float wj[4], aj[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float u = (BITS == 32) ? ckv[j] : __fmul_rn(sv[j], ckv[j]);
+            wj[j] = __fmul_rn(beta, __fmaf_rn(-alpha, u, vv[j]));
+            aj[j] = (BITS == 32) ? alpha : __fmul_rn(alpha, sv[j]);
+        }
+        const uint64_t W01 = pk(wj[0], wj[1]), W23 = pk(wj[2], wj[3]);
+        const uint64_t A01 = pk(aj[0], aj[1]), A23 = pk(aj[2], aj[3]);
+#pragma unroll
+        for (int k = 0; k < RPT; k += 2) {
+            const ulonglong2 kk = *reinterpret_cast<const ulonglong2*>(kb + k);
+            // S = c*(alpha s) + k*w   (full-precision state: alpha*S + k*w)
+            S2[k][0] = fma2(S2[k][0], A01, mul2(kk.x, W01));
+            S2[k][1] = fma2(S2[k][1], A23, mul2(kk.x, W23));
+            S2[k + 1][0] = fma2(S2[k + 1][0], A01, mul2(kk.y, W01));
+            S2[k + 1][1] = fma2(S2[k + 1][1], A23, mul2(kk.y, W23));
+        }
+    } else {
+        const float dt = gt.g0;
+        const float a = (p.g1 != nullptr) ? gt.g1 : expf(__fmul_rn(dt, gt.A));
+        const float4 s4 = load_s4();
+        const float4 vc = load_vc();
+        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+        const float xv[4] = {vc.x, vc.y, vc.z, vc.w};
+        float xd[4], gj[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            xd[j] = __fmul_rn(dt, xv[j]);
+            gj[j] = (BITS == 32) ? a : __fmul_rn(a, sv[j]);
+        }
+        const uint64_t X01 = pk(xd[0], xd[1]), X23 = pk(xd[2], xd[3]);
+        const uint64_t G01 = pk(gj[0], gj[1]), G23 = pk(gj[2], gj[3]);
+#pragma unroll
+        for (int k = 0; k < RPT; k += 2) {
+            const ulonglong2 bb = *reinterpret_cast<const ulonglong2*>(kb + k);
+            // S = c*(a s) + B*(dt x)   (full-precision state: a*S + B*(dt x))
+            S2[k][0] = fma2(S2[k][0], G01, mul2(bb.x, X01));
+            S2[k][1] = fma2(S2[k][1], G23, mul2(bb.x, X23));
+            S2[k + 1][0] = fma2(S2[k + 1][0], G01, mul2(bb.y, X01));
+            S2[k + 1][1] = fma2(S2[k + 1][1], G23, mul2(bb.y, X23));
+        }
+    }
+
+    // ---- readout and column absmax ----------------------------------------------
+    uint64_t o01 = pk(0.f, 0.f), o23 = pk(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < RPT; k += 2) {
+        const ulonglong2 qq = *reinterpret_cast<const ulonglong2*>(qa + k);
+        o01 = fma2(S2[k][0], qq.x, o01);
+        o23 = fma2(S2[k][1], qq.x, o23);
+        o01 = fma2(S2[k + 1][0], qq.y, o01);
+        o23 = fma2(S2[k + 1][1], qq.y, o23);
+    }
+    float4 o4 = unpk4(o01, o23);
+    warp_sum4(o4);
+    const long long col = (long long)hu * p.dv + j0 + 4 * cw;  // this lane's first column
+    if (g < 4) {
+        float o = pick4(o4, g);
+        if constexpr (FAM == RSQ_MAMBA2) o = __fmaf_rn(gt.D, ld_vec(stage + C::OFF_VC, 16 * w + 4 * cw + g, bf16), o);
+        p.out[col + g] = o;
+    }
+    float4 iv = make_float4(0.f, 0.f, 0.f, 0.f);
+    if constexpr (BITS != 32) {
+        float m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
+#pragma unroll
+        for (int k = 0; k < RPT; k += 2) {
+            const float4 x = unpk4(S2[k][0], S2[k][1]);
+            const float4 y = unpk4(S2[k + 1][0], S2[k + 1][1]);
+            m0 = max3_nan(m0, fabsf(x.x), fabsf(y.x));
+            m1 = max3_nan(m1, fabsf(x.y), fabsf(y.y));
+            m2 = max3_nan(m2, fabsf(x.z), fabsf(y.z));
+            m3 = max3_nan(m3, fabsf(x.w), fabsf(y.w));
+        }
+        float4 m4 = make_float4(m0, m1, m2, m3);
+        warp_max4(m4);
+        bool nonfinite;
+        const float mine = scale_or_inv<BITS>(m4, g, nonfinite);
+        if (g < 4) {
+            p.scales_out[col + g] = mine;
+            if (nonfinite) atomicOr(p.flag, kFlagNonFinite);
+        }
+        iv = gather_inv(mine, cw);
+    }
+
+    // ---- release the stage; the last warp refills it with the unit NS ahead ----
+    __syncwarp();
+    if (lane == 0) {
+        uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + C::OFF_CNT) + stage_idx;
+        if (atomicAdd(cnt, 1u) == UB - 1) {
+            *cnt = 0u;
+            UnitIt refill = un;  // the unit NS ahead of this one
+#pragma unroll
+            for (int s = 0; s < C::NS; ++s) refill.advance(p);
+            if (refill.u < p.units) {
+                asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+                issue_unit<FAM, DK, UB, F32STATE>(p, refill, stage, bar);
+            }
+        }
+    }
+
+    // ---- store ------------------------------------------------------------------
+    uint8_t* dst = p.codes_out + (long long)un.b * p.row_bytes + p.head_off[un.h] +
+                   (long long)blk * BLOCK_BYTES;
+    if constexpr (BITS == 32) {
+#pragma unroll
+        for (int k = 0; k < RPT; ++k)
+            *reinterpret_cast<ulonglong2*>(dst + ((g + kR * k) * 16 + 4 * cw) * 4) =
+                make_ulonglong2(S2[k][0], S2[k][1]);
+    } else {
+        clear_zero_inv_columns<RPT>(S2, iv);
+        requantize_store<BITS, SR, RPT>(S2, iv, dst, g, cw, static_cast<uint32_t>(j0 / 4 + cw), un.h,
+                                        un.b, p.step, p.rk);
+    }
+}
+
+template <int FAM, int DK, int UB, bool F32STATE, bool SR>
+__global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (DecodeCfg<FAM, DK, UB, F32STATE>::MINB))
+    rsq_decode_kernel(const __grid_constant__ DecodeParams p) {
+    using C = DecodeCfg<FAM, DK, UB, F32STATE>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, w = tid >> 5;
+    const int g = lane >> 2, cw = lane & 3;
+    const uint32_t bar0 = smem_u32(smem + C::OFF_BAR);
+
+    if (tid == 0) {
+        uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + C::OFF_CNT);
+        for (int s = 0; s < C::NS; ++s) {
+            mbar_init(bar0 + 8 * s, 1);
+            cnt[s] = 0u;
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+    UnitIt cur;
+    cur.init(blockIdx.x, p);
+    if (tid == 0) {
+        UnitIt it = cur;
+        for (int s = 0; s < C::NS; ++s) {
+            if (it.u < p.units) issue_unit<FAM, DK, UB, F32STATE>(p, it, smem + s * C::STAGE, bar0 + 8 * s);
+            it.advance(p);
+        }
+    }
+    Gates gt = {0.f, 0.f, 0.f, 0.f};
+    if (cur.u < p.units) gt = load_gates<FAM>(p, cur);
+    for (int n = 0; cur.u < p.units; ++n) {
+        UnitIt nxt = cur;
+        nxt.advance(p);
+        Gates ng = gt;
+        if (nxt.u < p.units) ng = load_gates<FAM>(p, nxt);
+        const int stage = n % C::NS;
+        const uint32_t bar = bar0 + 8 * stage;
+        const bool ok = mbar_wait(bar, (n / C::NS) & 1, kWaitIters);
+        if (__any_sync(0xffffffffu, !ok)) {
+            if (lane == 0) atomicOr(p.flag, kFlagTimeout);
+            return;  // this warp stops; the others see their own waits expire
+        }
+        uint8_t* st = smem + stage * C::STAGE;
+        if constexpr (F32STATE) {
+            process_block<FAM, DK, UB, true, false, 32>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
+        } else {
+            if (p.head_bits[cur.h] == 8)
+                process_block<FAM, DK, UB, false, SR, 8>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
+            else
+                process_block<FAM, DK, UB, false, SR, 4>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
+        }
+        cur = nxt;
+        gt = ng;
+    }
+}
+
+// Kernel attributes for one instantiation.
+template <int FAM, int DK, int UB, bool F32, bool SR>
+int decode_info_one(int* threads, size_t* smem, const void** func) {
+    using C = DecodeCfg<FAM, DK, UB, F32>;
+    *threads = C::NT;
+    *smem = C::SMEM;
+    *func = reinterpret_cast<const void*>(&rsq_decode_kernel<FAM, DK, UB, F32, SR>);
+    return 0;
+}
+
+// All (dk, blocks per unit) instantiations of one family.
+template <int FAM>
+int decode_info_family(int dk, int ub, bool f32state, bool sr, int* threads, size_t* smem,
+                       const void** func) {
+#define RSQ_CASE(DK_, UB_)                                                                   \
+    if (dk == DK_ && ub == UB_) {                                                             \
+        if (f32state) return decode_info_one<FAM, DK_, UB_, true, false>(threads, smem, func); \
+        if (sr) return decode_info_one<FAM, DK_, UB_, false, true>(threads, smem, func);      \
+        return decode_info_one<FAM, DK_, UB_, false, false>(threads, smem, func);             \
+    }
+    RSQ_CASE(16, 1) RSQ_CASE(16, 2) RSQ_CASE(16, 4)
+    RSQ_CASE(32, 1) RSQ_CASE(32, 2) RSQ_CASE(32, 4)
+    RSQ_CASE(64, 1) RSQ_CASE(64, 2) RSQ_CASE(64, 4)
+    RSQ_CASE(128, 1) RSQ_CASE(128, 2) RSQ_CASE(128, 4)
+#undef RSQ_CASE
+    return -1;
+}
+
+}  // namespace rsq

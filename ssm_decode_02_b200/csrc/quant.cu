@@ -4,7 +4,8 @@
 // same per-column absmax scale and rounding as the decode step (initialisation,
 // checkpoint load).  rsq_dequantize expands codes * scales back to floats.
 // rsq_state_drift accumulates the per-head squared error of a quantized state
-// against a full-precision trajectory (relative state drift).
+// against a full-precision trajectory (relative state drift).  All three walk
+// the stored 16-column blocks with one warp per block.
 #include <cuda_runtime.h>
 
 #include "rsq_internal.h"
@@ -12,111 +13,125 @@
 
 namespace rsq {
 
-template <int DK, int CB, int BITS>
-__device__ __forceinline__ void quantize_unit(const QuantParams& p, int hu, int cb, int b, int h,
-                                              float* red, int warp, int rgl, int cw, int rho) {
-    using L = Layout<DK, CB>;
-    constexpr int R = L::R, RPT = L::RPT;
-    const float* src = p.S + (long long)hu * DK * p.dv + cb * CB + 4 * cw;
-    float S[RPT][4];
+constexpr int kWarpsPerCta = 4;
+
+struct BlockIdx {
+    int b, h, hu, blk;
+};
+
+__device__ __forceinline__ BlockIdx block_of(long long gb, int H, int nblk) {
+    BlockIdx r;
+    r.hu = static_cast<int>(gb / nblk);
+    r.blk = static_cast<int>(gb - (long long)r.hu * nblk);
+    r.b = r.hu / H;
+    r.h = r.hu - r.b * H;
+    return r;
+}
+
+template <int DK, int BITS>
+__device__ __forceinline__ void quantize_block(const QuantParams& p, const BlockIdx& bi, int lane, int g,
+                                               int cw) {
+    constexpr int RPT = Layout<DK>::RPT;
+    const int j0 = bi.blk * kBlockCols;
+    const float* src = p.S + (long long)bi.hu * DK * p.dv + j0 + 4 * cw;
+    uint64_t S2[RPT][2];
 #pragma unroll
     for (int k = 0; k < RPT; ++k) {
-        const float4 t = __ldg(reinterpret_cast<const float4*>(src + (long long)(rho + R * k) * p.dv));
-        S[k][0] = t.x; S[k][1] = t.y; S[k][2] = t.z; S[k][3] = t.w;
+        const ulonglong2 t = __ldg(reinterpret_cast<const ulonglong2*>(src + (long long)(g + kR * k) * p.dv));
+        S2[k][0] = t.x;
+        S2[k][1] = t.y;
     }
-    const uint32_t code_bytes = static_cast<uint32_t>(DK * CB * BITS / 8);
-    uint8_t* dst = p.codes + (long long)b * p.row_bytes + p.head_off[h] + (long long)cb * code_bytes;
+    constexpr int BLOCK_BYTES = DK * kBlockCols * BITS / 8;
+    uint8_t* dst = p.codes + (long long)bi.b * p.row_bytes + p.head_off[bi.h] + (long long)bi.blk * BLOCK_BYTES;
     if constexpr (BITS == 32) {
 #pragma unroll
         for (int k = 0; k < RPT; ++k)
-            *reinterpret_cast<float4*>(dst + ((rho + R * k) * CB + 4 * cw) * 4) =
-                make_float4(S[k][0], S[k][1], S[k][2], S[k][3]);
-        return;
+            *reinterpret_cast<ulonglong2*>(dst + ((g + kR * k) * 16 + 4 * cw) * 4) = make_ulonglong2(S2[k][0], S2[k][1]);
     } else {
-        float m[4] = {0.f, 0.f, 0.f, 0.f};
+        float4 m4 = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-        for (int k = 0; k + 1 < RPT; k += 2)
-#pragma unroll
-            for (int j = 0; j < 4; ++j) m[j] = max3_nan(m[j], fabsf(S[k][j]), fabsf(S[k + 1][j]));
-        const float4 m4 = colmax<L::LPR, L::W, CB>(make_float4(m[0], m[1], m[2], m[3]), red, warp, rgl, cw);
-        const float mv[4] = {m4.x, m4.y, m4.z, m4.w};
-        float sn[4], inv[4];
-        unsigned bad = 0;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) scale_and_inv<BITS>(mv[j], sn[j], inv[j], bad, j);
-        const long long col0 = (long long)hu * p.dv + cb * CB + 4 * cw;
-        if (rho == 0) *reinterpret_cast<float4*>(p.scales + col0) = make_float4(sn[0], sn[1], sn[2], sn[3]);
-        if (bad && rho == 0) atomicOr(p.flag, kFlagNonFinite);
-        const uint32_t g = static_cast<uint32_t>(cb * (CB / 4) + cw);
+        for (int k = 0; k < RPT; ++k) {
+            const float4 s = unpk4(S2[k][0], S2[k][1]);
+            m4.x = max_nan(m4.x, fabsf(s.x));
+            m4.y = max_nan(m4.y, fabsf(s.y));
+            m4.z = max_nan(m4.z, fabsf(s.z));
+            m4.w = max_nan(m4.w, fabsf(s.w));
+        }
+        warp_max4(m4);
+        bool nonfinite;
+        const float mine = scale_or_inv<BITS>(m4, g, nonfinite);
+        const long long col = (long long)bi.hu * p.dv + j0 + 4 * cw;
+        if (g < 4) {
+            p.scales[col + g] = mine;
+            if (nonfinite) atomicOr(p.flag, kFlagNonFinite);
+        }
+        const float4 iv = gather_inv(mine, cw);
+        clear_zero_inv_columns<RPT>(S2, iv);
+        const uint32_t gcol = static_cast<uint32_t>(j0 / 4 + cw);
         if (p.sr)
-            requantize_store<BITS, true, R, RPT, CB>(S, inv, dst, rho, cw, g, h, b, p.step, p.key0,
-                                                     p.key1, bad);
+            requantize_store<BITS, true, RPT>(S2, iv, dst, g, cw, gcol, bi.h, bi.b, p.step, p.rk);
         else
-            requantize_store<BITS, false, R, RPT, CB>(S, inv, dst, rho, cw, g, h, b, p.step,
-                                                      p.key0, p.key1, bad);
+            requantize_store<BITS, false, RPT>(S2, iv, dst, g, cw, gcol, bi.h, bi.b, p.step, p.rk);
     }
 }
 
-template <int DK, int CB>
-__global__ void __launch_bounds__(Layout<DK, CB>::NT) rsq_quantize_kernel(const __grid_constant__ QuantParams p) {
-    using L = Layout<DK, CB>;
-    __shared__ __align__(16) float red[L::W * CB];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int cw = lane % L::LPR, rgl = lane / L::LPR, rho = warp * L::RPW + rgl;
-    for (int u = blockIdx.x; u < p.units; u += gridDim.x) {
-        const int hu = u / p.ncb, cb = u - hu * p.ncb, b = hu / p.H, h = hu - b * p.H;
-        const int bits = p.head_bits[h];
-        if (bits == 8) quantize_unit<DK, CB, 8>(p, hu, cb, b, h, red, warp, rgl, cw, rho);
-        else if (bits == 4) quantize_unit<DK, CB, 4>(p, hu, cb, b, h, red, warp, rgl, cw, rho);
-        else quantize_unit<DK, CB, 32>(p, hu, cb, b, h, red, warp, rgl, cw, rho);
-        __syncthreads();
+template <int DK>
+__global__ void __launch_bounds__(32 * kWarpsPerCta) rsq_quantize_kernel(const __grid_constant__ QuantParams p) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int g = lane >> 2, cw = lane & 3;
+    const int nblk = p.dv / kBlockCols;
+    const long long total = (long long)p.B * p.H * nblk;
+    for (long long gb = (long long)blockIdx.x * kWarpsPerCta + w; gb < total; gb += (long long)gridDim.x * kWarpsPerCta) {
+        const BlockIdx bi = block_of(gb, p.H, nblk);
+        const int bits = p.head_bits[bi.h];
+        if (bits == 8) quantize_block<DK, 8>(p, bi, lane, g, cw);
+        else if (bits == 4) quantize_block<DK, 4>(p, bi, lane, g, cw);
+        else quantize_block<DK, 32>(p, bi, lane, g, cw);
     }
 }
 
-template <int DK, int CB, int BITS>
-__device__ __forceinline__ void dequantize_unit(const DequantParams& p, int hu, int cb, int b, int h,
-                                                int cw, int rho) {
-    using L = Layout<DK, CB>;
-    constexpr int R = L::R, RPT = L::RPT;
-    const uint32_t code_bytes = static_cast<uint32_t>(DK * CB * BITS / 8);
-    const uint8_t* src = p.codes + (long long)b * p.row_bytes + p.head_off[h] + (long long)cb * code_bytes;
-    float* dst = p.S + (long long)hu * DK * p.dv + cb * CB + 4 * cw;
-    float S[RPT][4];
+template <int DK, int BITS>
+__device__ __forceinline__ void dequantize_block(const DequantParams& p, const BlockIdx& bi, int g, int cw) {
+    constexpr int RPT = Layout<DK>::RPT;
+    constexpr int BLOCK_BYTES = DK * kBlockCols * BITS / 8;
+    const int j0 = bi.blk * kBlockCols;
+    const uint8_t* src = p.codes + (long long)bi.b * p.row_bytes + p.head_off[bi.h] + (long long)bi.blk * BLOCK_BYTES;
+    float* dst = p.S + (long long)bi.hu * DK * p.dv + j0 + 4 * cw;
+    uint64_t S2[RPT][2];
     if constexpr (BITS == 32) {
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
-            const float4 t = *reinterpret_cast<const float4*>(src + ((rho + R * k) * CB + 4 * cw) * 4);
-            S[k][0] = t.x; S[k][1] = t.y; S[k][2] = t.z; S[k][3] = t.w;
+            const ulonglong2 t = *reinterpret_cast<const ulonglong2*>(src + ((g + kR * k) * 16 + 4 * cw) * 4);
+            S2[k][0] = t.x;
+            S2[k][1] = t.y;
         }
     } else {
-        load_codes<BITS, R, RPT, CB>(src, rho, cw, S);
-        const float4 s = *reinterpret_cast<const float4*>(p.scales + (long long)hu * p.dv + cb * CB + 4 * cw);
+        load_codes<BITS, RPT>(src, g, cw, S2);
+        const float4 s = *reinterpret_cast<const float4*>(p.scales + (long long)bi.hu * p.dv + j0 + 4 * cw);
+        const uint64_t s01 = pk(s.x, s.y), s23 = pk(s.z, s.w);
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
-            S[k][0] = __fmul_rn(S[k][0], s.x);
-            S[k][1] = __fmul_rn(S[k][1], s.y);
-            S[k][2] = __fmul_rn(S[k][2], s.z);
-            S[k][3] = __fmul_rn(S[k][3], s.w);
+            S2[k][0] = mul2(S2[k][0], s01);
+            S2[k][1] = mul2(S2[k][1], s23);
         }
     }
 #pragma unroll
     for (int k = 0; k < RPT; ++k)
-        *reinterpret_cast<float4*>(dst + (long long)(rho + R * k) * p.dv) =
-            make_float4(S[k][0], S[k][1], S[k][2], S[k][3]);
+        *reinterpret_cast<ulonglong2*>(dst + (long long)(g + kR * k) * p.dv) = make_ulonglong2(S2[k][0], S2[k][1]);
 }
 
-template <int DK, int CB>
-__global__ void __launch_bounds__(Layout<DK, CB>::NT) rsq_dequantize_kernel(const __grid_constant__ DequantParams p) {
-    using L = Layout<DK, CB>;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int cw = lane % L::LPR, rgl = lane / L::LPR, rho = warp * L::RPW + rgl;
-    const int units = p.B * p.H * p.ncb;
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
-        const int hu = u / p.ncb, cb = u - hu * p.ncb, b = hu / p.H, h = hu - b * p.H;
-        const int bits = p.head_bits[h];
-        if (bits == 8) dequantize_unit<DK, CB, 8>(p, hu, cb, b, h, cw, rho);
-        else if (bits == 4) dequantize_unit<DK, CB, 4>(p, hu, cb, b, h, cw, rho);
-        else dequantize_unit<DK, CB, 32>(p, hu, cb, b, h, cw, rho);
+template <int DK>
+__global__ void __launch_bounds__(32 * kWarpsPerCta) rsq_dequantize_kernel(const __grid_constant__ DequantParams p) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int g = lane >> 2, cw = lane & 3;
+    const int nblk = p.dv / kBlockCols;
+    const long long total = (long long)p.B * p.H * nblk;
+    for (long long gb = (long long)blockIdx.x * kWarpsPerCta + w; gb < total; gb += (long long)gridDim.x * kWarpsPerCta) {
+        const BlockIdx bi = block_of(gb, p.H, nblk);
+        const int bits = p.head_bits[bi.h];
+        if (bits == 8) dequantize_block<DK, 8>(p, bi, g, cw);
+        else if (bits == 4) dequantize_block<DK, 4>(p, bi, g, cw);
+        else dequantize_block<DK, 32>(p, bi, g, cw);
     }
 }
 
@@ -126,7 +141,6 @@ __global__ void __launch_bounds__(256) rsq_drift_kernel(const __grid_constant__ 
     const int hu = blockIdx.x;
     const int b = hu / p.H, h = hu - b * p.H;
     const int bits = p.q_head_bits[h];
-    const int CB = p.dv < 64 ? p.dv : 64;
     const long long n = (long long)p.dk * p.dv;
     const uint8_t* q = p.q_codes + (long long)b * p.q_row_bytes + p.q_head_off[h];
     const float* f = reinterpret_cast<const float*>(p.f_codes + (long long)b * p.f_row_bytes +
@@ -134,11 +148,10 @@ __global__ void __launch_bounds__(256) rsq_drift_kernel(const __grid_constant__ 
     const float* sc = p.q_scales + (long long)hu * p.dv;
     double e2 = 0.0, f2 = 0.0;
     for (long long e = threadIdx.x; e < n; e += blockDim.x) {
-        // e walks the stored (column-block) order: block, row, column within block
-        const long long cb = e / ((long long)p.dk * CB);
-        const long long rem = e - cb * p.dk * CB;
-        const int jj = static_cast<int>(rem % CB);
-        const int j = static_cast<int>(cb) * CB + jj;
+        // e walks the stored order: block of 16 columns, row, column within block
+        const long long blk = e / ((long long)p.dk * kBlockCols);
+        const int jj = static_cast<int>(e % kBlockCols);
+        const int j = static_cast<int>(blk) * kBlockCols + jj;
         int c;
         if (bits == 8) {
             c = static_cast<int>(q[e]) - 128;
@@ -173,35 +186,36 @@ __global__ void __launch_bounds__(256) rsq_drift_kernel(const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------------------
-template <int DK, int CB>
-static int launch_q(const QuantParams& p, void* stream) {
-    const int grid = p.units < 148 * 16 ? p.units : 148 * 16;
-    rsq_quantize_kernel<DK, CB><<<grid, Layout<DK, CB>::NT, 0, static_cast<cudaStream_t>(stream)>>>(p);
-    return static_cast<int>(cudaGetLastError());
-}
-template <int DK, int CB>
-static int launch_dq(const DequantParams& p, void* stream) {
-    const int units = p.B * p.H * p.ncb;
-    const int grid = units < 148 * 16 ? units : 148 * 16;
-    rsq_dequantize_kernel<DK, CB><<<grid, Layout<DK, CB>::NT, 0, static_cast<cudaStream_t>(stream)>>>(p);
-    return static_cast<int>(cudaGetLastError());
+static int grid_for(long long blocks) {
+    const long long ctas = (blocks + kWarpsPerCta - 1) / kWarpsPerCta;
+    return static_cast<int>(ctas < 148 * 16 ? ctas : 148 * 16);
 }
 
-#define RSQ_DISPATCH(FN, P)                                                                   \
-    switch (dk * 1000 + cb) {                                                                \
-        case 16016: return FN<16, 16>(P, stream);   case 16032: return FN<16, 32>(P, stream);   \
-        case 16064: return FN<16, 64>(P, stream);   case 32016: return FN<32, 16>(P, stream);   \
-        case 32032: return FN<32, 32>(P, stream);   case 32064: return FN<32, 64>(P, stream);   \
-        case 64016: return FN<64, 16>(P, stream);   case 64032: return FN<64, 32>(P, stream);   \
-        case 64064: return FN<64, 64>(P, stream);   case 128016: return FN<128, 16>(P, stream); \
-        case 128032: return FN<128, 32>(P, stream); case 128064: return FN<128, 64>(P, stream); \
-        case 256016: return FN<256, 16>(P, stream); case 256032: return FN<256, 32>(P, stream); \
-        case 256064: return FN<256, 64>(P, stream);                                          \
-        default: return static_cast<int>(cudaErrorInvalidValue);                               \
+int launch_quantize(int dk, const QuantParams& p, void* stream) {
+    const int grid = grid_for((long long)p.B * p.H * (p.dv / kBlockCols));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (dk) {
+        case 16: rsq_quantize_kernel<16><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
+        case 32: rsq_quantize_kernel<32><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
+        case 64: rsq_quantize_kernel<64><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
+        case 128: rsq_quantize_kernel<128><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
+        default: return static_cast<int>(cudaErrorInvalidValue);
     }
+    return static_cast<int>(cudaGetLastError());
+}
 
-int launch_quantize(int dk, int cb, const QuantParams& p, void* stream) { RSQ_DISPATCH(launch_q, p) }
-int launch_dequantize(int dk, int cb, const DequantParams& p, void* stream) { RSQ_DISPATCH(launch_dq, p) }
+int launch_dequantize(int dk, const DequantParams& p, void* stream) {
+    const int grid = grid_for((long long)p.B * p.H * (p.dv / kBlockCols));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    switch (dk) {
+        case 16: rsq_dequantize_kernel<16><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
+        case 32: rsq_dequantize_kernel<32><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
+        case 64: rsq_dequantize_kernel<64><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
+        case 128: rsq_dequantize_kernel<128><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
+        default: return static_cast<int>(cudaErrorInvalidValue);
+    }
+    return static_cast<int>(cudaGetLastError());
+}
 
 int launch_drift(const DriftParams& p, void* stream) {
     rsq_drift_kernel<<<p.B * p.H, 256, 0, static_cast<cudaStream_t>(stream)>>>(p);

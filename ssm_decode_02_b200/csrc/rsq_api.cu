@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "rsq_internal.h"
+#include "rsq_tile.cuh"
 
 struct rsq_ctx {
     rsq_config cfg;
@@ -17,7 +18,7 @@ struct rsq_ctx {
     uint32_t head_off[RSQ_MAX_HEADS];
     long long row_bytes;
     bool f32state;
-    int cb, ncb, units;
+    int ub, ncb, units;   // 16-column blocks per unit, units per head, units per step
     int grid;        // persistent decode grid
     int device;
     unsigned* flag;  // device word: rsq::kFlag* bits
@@ -39,7 +40,8 @@ rsq_status cuda_fail(int err, const char* what) {
     return fail(RSQ_E_CUDA, "%s: %s", what, cudaGetErrorString(static_cast<cudaError_t>(err)));
 }
 
-bool pow2_dim(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
+bool dk_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool dv_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
@@ -81,7 +83,10 @@ const char* rsq_status_string(rsq_status s) {
     return "unknown status";
 }
 
-int rsq_reduction_partials(int dk) { return dk <= 128 ? 8 : 16; }
+int rsq_reduction_partials(int dk) {
+    (void)dk;
+    return rsq::kR;  // one partial per row group of a warp tile (rsq_tile.cuh)
+}
 
 rsq_status rsq_allocate_bits(const double* score, int heads, int n_high, int high_bits,
                              int low_bits, int8_t* bits_out) {
@@ -107,8 +112,8 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
     if (c.family != RSQ_GDN && c.family != RSQ_MAMBA2) return fail(RSQ_E_INVAL, "create: bad family %d", c.family);
     if (c.batch < 1) return fail(RSQ_E_INVAL, "create: batch must be >= 1");
     if (c.heads < 1 || c.heads > RSQ_MAX_HEADS) return fail(RSQ_E_INVAL, "create: heads must be in [1, %d]", RSQ_MAX_HEADS);
-    if (!pow2_dim(c.dk) || !pow2_dim(c.dv))
-        return fail(RSQ_E_UNSUPPORTED, "create: dk and dv must be one of 16, 32, 64, 128, 256 (got %d, %d)", c.dk, c.dv);
+    if (!dk_ok(c.dk) || !dv_ok(c.dv))
+        return fail(RSQ_E_UNSUPPORTED, "create: dk must be one of 16, 32, 64, 128 and dv one of 16, 32, 64, 128, 256 (got %d, %d)", c.dk, c.dv);
     if (c.rounding != RSQ_RTN && c.rounding != RSQ_SR) return fail(RSQ_E_INVAL, "create: bad rounding %d", c.rounding);
     if (c.in_dtype != RSQ_F32 && c.in_dtype != RSQ_BF16) return fail(RSQ_E_INVAL, "create: bad in_dtype %d", c.in_dtype);
     if (c.family == RSQ_MAMBA2 && (c.ngroups < 1 || c.heads % c.ngroups != 0))
@@ -139,8 +144,8 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
         off += static_cast<long long>(c.dk) * c.dv * ctx->bits[h] / 8;
     }
     ctx->row_bytes = off;
-    ctx->cb = std::min(c.dv, 64);
-    ctx->ncb = c.dv / ctx->cb;
+    ctx->ub = std::min(c.dv / rsq::kBlockCols, 4);
+    ctx->ncb = c.dv / (rsq::kBlockCols * ctx->ub);
     const long long units = static_cast<long long>(c.batch) * c.heads * ctx->ncb;
     if (units > (1LL << 30)) {
         delete ctx;
@@ -152,7 +157,8 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
     int threads = 0;
     size_t smem = 0;
     const void* func = nullptr;
-    if (rsq::decode_kernel_info(c.family, c.dk, ctx->cb, ctx->f32state, &threads, &smem, &func) != 0) {
+    if (rsq::decode_kernel_info(c.family, c.dk, ctx->ub, ctx->f32state, c.rounding == RSQ_SR, &threads,
+                                &smem, &func) != 0) {
         delete ctx;
         return fail(RSQ_E_UNSUPPORTED, "create: no kernel for dk=%d dv=%d", c.dk, c.dv);
     }
@@ -219,6 +225,7 @@ rsq_status rsq_decode_step(const rsq_ctx* ctx, const rsq_state* state_in, const 
     p.step = step;
     p.key0 = static_cast<uint32_t>(c.seed);
     p.key1 = static_cast<uint32_t>(c.seed >> 32);
+    p.rk = rsq::philox_round_keys(p.key0, p.key1);
     if (c.family == RSQ_GDN) {
         const rsq_gdn_inputs* in = static_cast<const rsq_gdn_inputs*>(inputs);
         if (!in->q || !in->k || !in->v || !in->alpha || !in->beta)
@@ -238,7 +245,13 @@ rsq_status rsq_decode_step(const rsq_ctx* ctx, const rsq_state* state_in, const 
         p.ngroups = c.ngroups; p.heads_per_group = c.heads / c.ngroups;
     }
     fill_heads(ctx, p);
-    const int err = rsq::launch_decode(c.family, c.dk, ctx->cb, ctx->f32state, p, ctx->grid, stream);
+    p.grid = ctx->grid;
+    p.gcb = ctx->grid % ctx->ncb;
+    const int ghu = ctx->grid / ctx->ncb;
+    p.gh = ghu % c.heads;
+    p.gb = ghu / c.heads;
+    const int err = rsq::launch_decode(c.family, c.dk, ctx->ub, ctx->f32state, c.rounding == RSQ_SR, p,
+                                       stream);
     if (err) return cuda_fail(err, "decode_step launch");
     return RSQ_OK;
 }
@@ -262,8 +275,9 @@ rsq_status rsq_quantize(const rsq_ctx* ctx, const float* S, const rsq_state* sta
     p.step = step;
     p.key0 = static_cast<uint32_t>(c.seed);
     p.key1 = static_cast<uint32_t>(c.seed >> 32);
+    p.rk = rsq::philox_round_keys(p.key0, p.key1);
     fill_heads(ctx, p);
-    const int err = rsq::launch_quantize(c.dk, ctx->cb, p, stream);
+    const int err = rsq::launch_quantize(c.dk, p, stream);
     if (err) return cuda_fail(err, "quantize launch");
     return RSQ_OK;
 }
@@ -282,7 +296,7 @@ rsq_status rsq_dequantize(const rsq_ctx* ctx, const rsq_state* state_in, float* 
     p.scales = state_in->scales;
     p.S = S_out;
     fill_heads(ctx, p);
-    const int err = rsq::launch_dequantize(c.dk, ctx->cb, p, stream);
+    const int err = rsq::launch_dequantize(c.dk, p, stream);
     if (err) return cuda_fail(err, "dequantize launch");
     return RSQ_OK;
 }

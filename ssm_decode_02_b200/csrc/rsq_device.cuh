@@ -127,16 +127,14 @@ struct U4 {
     uint32_t x, y, z, w;
 };
 
-__device__ __forceinline__ U4 philox4x32_10(U4 c, uint32_t k0, uint32_t k1) {
+// Round keys rk0[r], rk1[r] are the key advanced r times by the Weyl increments.
+__device__ __forceinline__ U4 philox4x32_10(U4 c, const uint32_t (&rk0)[10], const uint32_t (&rk1)[10]) {
     constexpr uint32_t kMulA = 0xD2511F53u, kMulB = 0xCD9E8D57u;
-    constexpr uint32_t kWeylA = 0x9E3779B9u, kWeylB = 0xBB67AE85u;
 #pragma unroll
     for (int round = 0; round < 10; ++round) {
         const uint32_t hiA = __umulhi(kMulA, c.x), loA = kMulA * c.x;
         const uint32_t hiB = __umulhi(kMulB, c.z), loB = kMulB * c.z;
-        c = U4{hiB ^ c.y ^ k0, loB, hiA ^ c.w ^ k1, loA};
-        k0 += kWeylA;
-        k1 += kWeylB;
+        c = U4{hiB ^ c.y ^ rk0[round], loB, hiA ^ c.w ^ rk1[round], loA};
     }
     return c;
 }

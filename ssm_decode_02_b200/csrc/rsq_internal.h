@@ -11,9 +11,28 @@ namespace rsq {
 constexpr unsigned kFlagNonFinite = 1u;  // a column's absmax was inf or NaN
 constexpr unsigned kFlagTimeout = 2u;    // a bounded barrier wait ran out
 
+// The ten round keys of Philox4x32-10 for one (key0, key1): round r uses
+// key0 + r * 0x9E3779B9 and key1 + r * 0xBB67AE85 (mod 2^32).  Computed once on
+// the host so the kernel reads them as constants.
+struct PhiloxKeys {
+    uint32_t k0[10];
+    uint32_t k1[10];
+};
+
+inline PhiloxKeys philox_round_keys(uint32_t key0, uint32_t key1) {
+    PhiloxKeys r;
+    for (int i = 0; i < 10; ++i) {
+        r.k0[i] = key0 + static_cast<uint32_t>(i) * 0x9E3779B9u;
+        r.k1[i] = key1 + static_cast<uint32_t>(i) * 0xBB67AE85u;
+    }
+    return r;
+}
+
 // Everything one decode launch needs, passed by value as a __grid_constant__.
 struct DecodeParams {
     int B, H, dk, dv, ncb, units;  // units = B * H * ncb column blocks
+    int grid;                      // persistent grid size G
+    int gcb, gh, gb;               // G decomposed as (batch, head, column block) steps
     int ngroups, heads_per_group;
     int in_bf16;                   // vector inputs are bf16 (else float)
     int sr;                        // stochastic rounding (else round-to-nearest)
@@ -32,6 +51,7 @@ struct DecodeParams {
     float* out;                    // [B][H][dv]
     unsigned* flag;
     uint32_t step, key0, key1;
+    PhiloxKeys rk;                 // Philox round keys of (key0, key1)
     uint32_t head_off[RSQ_MAX_HEADS];  // byte offset of each head in a batch row
     uint8_t head_bits[RSQ_MAX_HEADS];
 };
@@ -45,6 +65,7 @@ struct QuantParams {
     float* scales;
     unsigned* flag;
     uint32_t step, key0, key1;
+    PhiloxKeys rk;
     uint32_t head_off[RSQ_MAX_HEADS];
     uint8_t head_bits[RSQ_MAX_HEADS];
 };
@@ -71,12 +92,13 @@ struct DriftParams {
 };
 
 // Launchers (defined in the .cu files).  Return a cudaError_t value.
-int launch_decode(int family, int dk, int cb, bool f32state, const DecodeParams& p, int grid,
+// ub = 16-column blocks per decode work unit (1, 2 or 4)
+int launch_decode(int family, int dk, int ub, bool f32state, bool sr, const DecodeParams& p,
                   void* stream);
-int decode_kernel_info(int family, int dk, int cb, bool f32state, int* threads, size_t* smem,
+int decode_kernel_info(int family, int dk, int ub, bool f32state, bool sr, int* threads, size_t* smem,
                        const void** func);
-int launch_quantize(int dk, int cb, const QuantParams& p, void* stream);
-int launch_dequantize(int dk, int cb, const DequantParams& p, void* stream);
+int launch_quantize(int dk, const QuantParams& p, void* stream);
+int launch_dequantize(int dk, const DequantParams& p, void* stream);
 int launch_drift(const DriftParams& p, void* stream);
 
 }  // namespace rsq

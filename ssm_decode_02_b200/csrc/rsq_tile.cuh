@@ -1,14 +1,15 @@
-// rsq_tile.cuh -- thread layout, column reductions and the requantizer shared by
-// the decode, quantize and dequantize kernels.
+// rsq_tile.cuh -- warp tile layout, in-warp column reductions and the
+// requantizer shared by the decode, quantize and dequantize kernels.
 //
-// Work unit: one column block of one head, i.e. all dk rows of CB = min(64, dv)
-// consecutive value columns (the scale groups of the value-axis grouping are
-// columns, so a unit's reductions never leave the unit).  Thread layout inside
-// a unit: a thread owns 4 consecutive columns (4*cw .. 4*cw+3) of the rows
-// i = rho, rho + R, rho + 2R, ... (RPT rows), where R = 8 (dk <= 128) or 16.
-// Lanes of a warp cover LPR = CB/4 column groups of RPW = 32/LPR consecutive
-// rho, so every warp-wide shared-memory access reads consecutive rows without
-// bank conflicts.
+// A head's value columns are stored in blocks of 16 (the scale groups of the
+// value-axis grouping are columns, so a block carries everything its
+// reductions need).  One warp owns one block: all dk rows x 16 columns.  Lane
+// (cw, g) with cw = lane % 4 and g = lane / 4 holds columns 4cw..4cw+3 of the
+// rows i = g, g+8, g+16, ... (RPT = dk/8 rows).  Sums over the key axis are
+// therefore R = 8 partials p = i mod 8 (the lane's row group), each
+// accumulated in increasing i, then combined by the XOR butterfly over p with
+// d = 1, 2, 4 -- shuffles across lanes 4, 8, 16 apart.  A warp-wide shared load
+// of one row per lane group reads 8 consecutive rows: no bank conflicts.
 #pragma once
 
 #include "rsq_device.cuh"
@@ -20,167 +21,107 @@ constexpr uint32_t kMagicBits = 0x4B400000u;
 constexpr uint32_t kSrBits8 = 0x43000000u;  // 128.0f: SR offset of 8-bit codes
 constexpr uint32_t kSrBits4 = 0x43080000u;  // 136.0f: SR offset of 4-bit codes
 
-template <int DK, int CB>
+constexpr int kBlockCols = 16;  // columns per stored block (one warp)
+constexpr int kR = 8;           // partial sums over the key axis (row groups)
+
+template <int DK>
 struct Layout {
-    static constexpr int R = DK <= 128 ? 8 : 16;  // partial sums over the key axis
-    static constexpr int RPT = DK / R;            // rows per thread (even)
-    static constexpr int LPR = CB / 4;            // lanes per row
-    static constexpr int RPW = 32 / LPR;          // rows per warp instruction
-    static constexpr int NT = LPR * R;            // threads per unit
-    static constexpr int W = NT / 32;             // warps per unit
-    static_assert(RPT % 2 == 0, "rows per thread must pair up for the SR counter");
-    static_assert(W * RPW == R, "layout");
+    static constexpr int R = kR;
+    static constexpr int RPT = DK / kR;  // rows per lane
+    static_assert(RPT >= 2 && RPT % 2 == 0, "rows per lane must pair up for the SR counter");
 };
 
-__device__ __forceinline__ float4 add4(float4 a, float4 b) {
-    return make_float4(__fadd_rn(a.x, b.x), __fadd_rn(a.y, b.y), __fadd_rn(a.z, b.z),
-                       __fadd_rn(a.w, b.w));
-}
-__device__ __forceinline__ float4 max4(float4 a, float4 b) {
-    return make_float4(max_nan(a.x, b.x), max_nan(a.y, b.y), max_nan(a.z, b.z), max_nan(a.w, b.w));
+__device__ __forceinline__ float4 unpk4(uint64_t a, uint64_t b) {
+    float4 r;
+    upk(a, r.x, r.y);
+    upk(b, r.z, r.w);
+    return r;
 }
 
-// Sum of a per-thread partial over the R partials (rho), in the fixed order:
-// XOR butterfly over rho with d = 1, 2, ..., R/2.  Low rho bits live in the
-// lanes (shuffles), high bits in the warps (shared memory `red`, [W][CB]).
-// Every thread returns the full sum for its 4 columns.  Contains one
-// __syncthreads when W > 1.
-template <int LPR, int W, int CB>
-__device__ __forceinline__ float4 colsum(float4 v, float* red, int warp, int rgl, int cw) {
+// Butterfly over the 8 row groups (lanes 4, 8, 16 apart) in the order d = 1, 2, 4.
+__device__ __forceinline__ void warp_sum4(float4& v) {
 #pragma unroll
-    for (int off = LPR; off < 32; off <<= 1) {
+    for (int off = 4; off < 32; off <<= 1) {
         v.x = __fadd_rn(v.x, __shfl_xor_sync(0xffffffffu, v.x, off));
         v.y = __fadd_rn(v.y, __shfl_xor_sync(0xffffffffu, v.y, off));
         v.z = __fadd_rn(v.z, __shfl_xor_sync(0xffffffffu, v.z, off));
         v.w = __fadd_rn(v.w, __shfl_xor_sync(0xffffffffu, v.w, off));
     }
-    if constexpr (W > 1) {
-        if (rgl == 0) *reinterpret_cast<float4*>(red + warp * CB + 4 * cw) = v;
-        __syncthreads();
-        float4 P[W];
-#pragma unroll
-        for (int w = 0; w < W; ++w) P[w] = *reinterpret_cast<const float4*>(red + w * CB + 4 * cw);
-#pragma unroll
-        for (int d = 1; d < W; d <<= 1)
-#pragma unroll
-            for (int w = 0; w < W; w += 2 * d) P[w] = add4(P[w], P[w + d]);
-        v = P[0];
-    }
-    return v;
 }
-
-// Column sum and column max together (one barrier).
-template <int LPR, int W, int CB>
-__device__ __forceinline__ void colsum_max(float4& v, float4& m, float* red_s, float* red_m,
-                                           int warp, int rgl, int cw) {
+__device__ __forceinline__ void warp_max4(float4& m) {
 #pragma unroll
-    for (int off = LPR; off < 32; off <<= 1) {
-        v.x = __fadd_rn(v.x, __shfl_xor_sync(0xffffffffu, v.x, off));
-        v.y = __fadd_rn(v.y, __shfl_xor_sync(0xffffffffu, v.y, off));
-        v.z = __fadd_rn(v.z, __shfl_xor_sync(0xffffffffu, v.z, off));
-        v.w = __fadd_rn(v.w, __shfl_xor_sync(0xffffffffu, v.w, off));
+    for (int off = 4; off < 32; off <<= 1) {
         m.x = max_nan(m.x, __shfl_xor_sync(0xffffffffu, m.x, off));
         m.y = max_nan(m.y, __shfl_xor_sync(0xffffffffu, m.y, off));
         m.z = max_nan(m.z, __shfl_xor_sync(0xffffffffu, m.z, off));
         m.w = max_nan(m.w, __shfl_xor_sync(0xffffffffu, m.w, off));
     }
-    if constexpr (W > 1) {
-        if (rgl == 0) {
-            *reinterpret_cast<float4*>(red_s + warp * CB + 4 * cw) = v;
-            *reinterpret_cast<float4*>(red_m + warp * CB + 4 * cw) = m;
-        }
-        __syncthreads();
-        float4 P[W], Q[W];
-#pragma unroll
-        for (int w = 0; w < W; ++w) {
-            P[w] = *reinterpret_cast<const float4*>(red_s + w * CB + 4 * cw);
-            Q[w] = *reinterpret_cast<const float4*>(red_m + w * CB + 4 * cw);
-        }
-#pragma unroll
-        for (int d = 1; d < W; d <<= 1)
-#pragma unroll
-            for (int w = 0; w < W; w += 2 * d) {
-                P[w] = add4(P[w], P[w + d]);
-                Q[w] = max4(Q[w], Q[w + d]);
-            }
-        v = P[0];
-        m = Q[0];
-    }
 }
 
-// Column max only.
-template <int LPR, int W, int CB>
-__device__ __forceinline__ float4 colmax(float4 m, float* red_m, int warp, int rgl, int cw) {
-#pragma unroll
-    for (int off = LPR; off < 32; off <<= 1) {
-        m.x = max_nan(m.x, __shfl_xor_sync(0xffffffffu, m.x, off));
-        m.y = max_nan(m.y, __shfl_xor_sync(0xffffffffu, m.y, off));
-        m.z = max_nan(m.z, __shfl_xor_sync(0xffffffffu, m.z, off));
-        m.w = max_nan(m.w, __shfl_xor_sync(0xffffffffu, m.w, off));
-    }
-    if constexpr (W > 1) {
-        if (rgl == 0) *reinterpret_cast<float4*>(red_m + warp * CB + 4 * cw) = m;
-        __syncthreads();
-        float4 Q[W];
-#pragma unroll
-        for (int w = 0; w < W; ++w) Q[w] = *reinterpret_cast<const float4*>(red_m + w * CB + 4 * cw);
-#pragma unroll
-        for (int d = 1; d < W; d <<= 1)
-#pragma unroll
-            for (int w = 0; w < W; w += 2 * d) Q[w] = max4(Q[w], Q[w + d]);
-        m = Q[0];
-    }
-    return m;
+__device__ __forceinline__ float pick4(const float4& v, int j) {
+    return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
 }
 
-// Per-column scale s = m / r and multiplier inv = r / m rounded toward zero
-// (0 for an all-zero or non-finite column).  Sets bit j of `bad` for a
-// non-finite column.
+// Column finalisation after the butterflies (every lane of a column group holds
+// the column's absmax m): lanes g < 4 own column 4cw + g for the scale
+// s = m / r, lanes g >= 4 own column 4cw + g - 4 for the multiplier
+// inv = r / m rounded toward zero (0 for an all-zero or non-finite column).
+// Returns this lane's value (s or inv); the caller gathers the multipliers.
 template <int BITS>
-__device__ __forceinline__ void scale_and_inv(float m, float& s, float& inv, unsigned& bad, int j) {
+__device__ __forceinline__ float scale_or_inv(const float4& m4, int g, bool& nonfinite) {
     constexpr float r = float((1 << (BITS - 1)) - 1);
-    s = __fdiv_rn(m, r);
-    const bool finite = isfinite(m);
-    inv = (m > 0.0f && finite) ? __fdiv_rz(r, m) : 0.0f;
-    if (!finite) bad |= 1u << j;
+    const float m = pick4(m4, g & 3);
+    nonfinite = !isfinite(m);
+    if (g < 4) return __fdiv_rn(m, r);
+    return (m > 0.0f && !nonfinite) ? __fdiv_rz(r, m) : 0.0f;
 }
 
-// Decode RPT rows of 4 codes (this thread's part of a unit tile in shared
-// memory) into exact float codes c.
-template <int BITS, int R, int RPT, int CB>
-__device__ __forceinline__ void load_codes(const uint8_t* tile, int rho, int cw, float (&c)[RPT][4]) {
+// Multipliers of this lane's 4 columns, from the lanes g = 4..7 of its column group.
+__device__ __forceinline__ float4 gather_inv(float mine, int cw) {
+    float4 iv;
+    iv.x = __shfl_sync(0xffffffffu, mine, cw + 16);
+    iv.y = __shfl_sync(0xffffffffu, mine, cw + 20);
+    iv.z = __shfl_sync(0xffffffffu, mine, cw + 24);
+    iv.w = __shfl_sync(0xffffffffu, mine, cw + 28);
+    return iv;
+}
+
+// Decode this lane's RPT rows of 4 codes of a stored block into exact float
+// codes, kept as packed pairs: S2[k][0] = columns 0,1 and S2[k][1] = columns
+// 2,3 of row g + 8k.
+template <int BITS, int RPT>
+__device__ __forceinline__ void load_codes(const uint8_t* blk, int g, int cw, uint64_t (&S2)[RPT][2]) {
     if constexpr (BITS == 8) {
         const uint64_t off = pk(-(kMagic + 128.0f), -(kMagic + 128.0f));
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(tile + (rho + R * k) * CB + 4 * cw);
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(blk + (g + kR * k) * 16 + 4 * cw);
             const uint64_t f01 = pk(__uint_as_float(prmt(w, kMagicBits, 0x7650u)),
                                     __uint_as_float(prmt(w, kMagicBits, 0x7651u)));
             const uint64_t f23 = pk(__uint_as_float(prmt(w, kMagicBits, 0x7652u)),
                                     __uint_as_float(prmt(w, kMagicBits, 0x7653u)));
-            upk(add2(f01, off), c[k][0], c[k][1]);
-            upk(add2(f23, off), c[k][2], c[k][3]);
+            S2[k][0] = add2(f01, off);
+            S2[k][1] = add2(f23, off);
         }
     } else {
         const uint64_t off = pk(-(kMagic + 8.0f), -(kMagic + 8.0f));
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
-            const uint32_t h16 =
-                *reinterpret_cast<const uint16_t*>(tile + (rho + R * k) * (CB / 2) + 2 * cw);
+            const uint32_t h16 = *reinterpret_cast<const uint16_t*>(blk + (g + kR * k) * 8 + 2 * cw);
             const uint32_t lo = h16 & 0x0F0Fu;         // columns 0 and 2
             const uint32_t hi = (h16 >> 4) & 0x0F0Fu;  // columns 1 and 3
             const uint64_t f01 = pk(__uint_as_float(prmt(lo, kMagicBits, 0x7650u)),
                                     __uint_as_float(prmt(hi, kMagicBits, 0x7650u)));
             const uint64_t f23 = pk(__uint_as_float(prmt(lo, kMagicBits, 0x7651u)),
                                     __uint_as_float(prmt(hi, kMagicBits, 0x7651u)));
-            upk(add2(f01, off), c[k][0], c[k][1]);
-            upk(add2(f23, off), c[k][2], c[k][3]);
+            S2[k][0] = add2(f01, off);
+            S2[k][1] = add2(f23, off);
         }
     }
 }
 
-// Pack the 4 codes of one row held in the low byte (fill=0) or byte 2 of
-// four floats into the stored representation.
+// Pack the 4 codes of one row held in the low byte (RTN) or byte 2 (4-bit SR)
+// of four floats into the stored representation.
 template <int BITS>
 __device__ __forceinline__ uint32_t pack_row(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3,
                                              bool byte2) {
@@ -198,40 +139,38 @@ __device__ __forceinline__ uint32_t pack_row(uint32_t t0, uint32_t t1, uint32_t 
     }
 }
 
-// Requantize this thread's RPT x 4 block of the full-precision state S and
-// store it to the unit tile `dst` in global memory.
-//   RTN: nearest integer of the exact S*inv (fma with a magic offset).
-//   SR : t = fma(S, inv, o + u/2^16), c = floor(t) - o, u from Philox4x32-10.
-// Columns flagged in `bad` get the zero code.
-template <int BITS, bool SR, int R, int RPT, int CB>
-__device__ __forceinline__ void requantize_store(const float (&S)[RPT][4], const float (&inv)[4],
-                                                 uint8_t* dst, int rho, int cw, uint32_t g,
-                                                 uint32_t h, uint32_t b, uint32_t step,
-                                                 uint32_t key0, uint32_t key1, unsigned bad) {
-    const uint64_t inv01 = pk(inv[0], inv[1]);
-    const uint64_t inv23 = pk(inv[2], inv[3]);
-    // stored-code masks for non-finite columns: keep good columns, fill bad ones with zero code
-    uint32_t keep = 0xFFFFFFFFu, fill = 0u;
-    if (bad) {
+// Columns whose multiplier is 0 (all-zero or non-finite) must come out as the
+// zero code; a non-finite state value would not, so clear those columns.
+template <int RPT>
+__device__ __forceinline__ void clear_zero_inv_columns(uint64_t (&S2)[RPT][2], const float4& iv) {
+    if (__builtin_expect(iv.x == 0.0f || iv.y == 0.0f || iv.z == 0.0f || iv.w == 0.0f, 0)) {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-            if (bad & (1u << j)) {
-                if constexpr (BITS == 8) {
-                    keep &= ~(0xFFu << (8 * j));
-                    fill |= 0x80u << (8 * j);
-                } else {
-                    keep &= ~(0xFu << (4 * j));
-                    fill |= 0x8u << (4 * j);
-                }
-            }
+        for (int k = 0; k < RPT; ++k) {
+            const float4 s = unpk4(S2[k][0], S2[k][1]);
+            S2[k][0] = pk(iv.x == 0.0f ? 0.0f : s.x, iv.y == 0.0f ? 0.0f : s.y);
+            S2[k][1] = pk(iv.z == 0.0f ? 0.0f : s.z, iv.w == 0.0f ? 0.0f : s.w);
+        }
     }
+}
+
+// Requantize this lane's RPT x 4 part of the full-precision state and store it
+// to the block `dst` (global memory).
+//   RTN: nearest integer of the exact S*inv (fma with a magic offset).
+//   SR : t = fma(S, inv, o + u/2^16), c = floor(t) - o, u a 16-bit uniform from
+//        Philox4x32-10 with counter {i mod dk/2 | (j/4) << 16, h, b, step}.
+// `gcol` is j/4 of this lane's first column.
+template <int BITS, bool SR, int RPT, class PhiloxKeysT>
+__device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], const float4& iv,
+                                                 uint8_t* dst, int g, int cw, uint32_t gcol,
+                                                 uint32_t h, uint32_t b, uint32_t step,
+                                                 const PhiloxKeysT& rk) {
+    const uint64_t inv01 = pk(iv.x, iv.y), inv23 = pk(iv.z, iv.w);
     auto store_row = [&](int k, uint32_t word) {
-        word = (word & keep) | fill;
-        const int i = rho + R * k;
+        const int i = g + kR * k;
         if constexpr (BITS == 8)
-            *reinterpret_cast<uint32_t*>(dst + i * CB + 4 * cw) = word;
+            *reinterpret_cast<uint32_t*>(dst + i * 16 + 4 * cw) = word;
         else
-            *reinterpret_cast<uint16_t*>(dst + i * (CB / 2) + 2 * cw) = static_cast<uint16_t>(word);
+            *reinterpret_cast<uint16_t*>(dst + i * 8 + 2 * cw) = static_cast<uint16_t>(word);
     };
     if constexpr (!SR) {
         const float o = (BITS == 8) ? kMagic + 128.0f : kMagic + 8.0f;
@@ -239,8 +178,8 @@ __device__ __forceinline__ void requantize_store(const float (&S)[RPT][4], const
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
             float t0, t1, t2, t3;
-            upk(fma2(pk(S[k][0], S[k][1]), inv01, oo), t0, t1);
-            upk(fma2(pk(S[k][2], S[k][3]), inv23, oo), t2, t3);
+            upk(fma2(S2[k][0], inv01, oo), t0, t1);
+            upk(fma2(S2[k][1], inv23, oo), t2, t3);
             store_row(k, pack_row<BITS>(__float_as_uint(t0), __float_as_uint(t1),
                                         __float_as_uint(t2), __float_as_uint(t3), false));
         }
@@ -249,8 +188,8 @@ __device__ __forceinline__ void requantize_store(const float (&S)[RPT][4], const
         const uint64_t mm = pk(kMagic, kMagic);
 #pragma unroll
         for (int k = 0; k < RPT / 2; ++k) {
-            const uint32_t i = static_cast<uint32_t>(rho + R * k);  // i < dk/2; partner i + dk/2
-            const U4 rnd = philox4x32_10(U4{i | (g << 16), h, b, step}, key0, key1);
+            const uint32_t i = static_cast<uint32_t>(g + kR * k);  // i < dk/2; partner i + dk/2
+            const U4 rnd = philox4x32_10(U4{i | (gcol << 16), h, b, step}, rk.k0, rk.k1);
             const uint32_t u[2][2] = {{rnd.x, rnd.y}, {rnd.z, rnd.w}};
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
@@ -258,8 +197,8 @@ __device__ __forceinline__ void requantize_store(const float (&S)[RPT][4], const
                 const uint32_t w0 = u[half][0], w1 = u[half][1];
                 const uint64_t V01 = pk(__uint_as_float(vb | (w0 & 0xFFFFu)), __uint_as_float(vb | (w0 >> 16)));
                 const uint64_t V23 = pk(__uint_as_float(vb | (w1 & 0xFFFFu)), __uint_as_float(vb | (w1 >> 16)));
-                uint64_t t01 = fma2(pk(S[kk][0], S[kk][1]), inv01, V01);
-                uint64_t t23 = fma2(pk(S[kk][2], S[kk][3]), inv23, V23);
+                uint64_t t01 = fma2(S2[kk][0], inv01, V01);
+                uint64_t t23 = fma2(S2[kk][1], inv23, V23);
                 if constexpr (BITS == 8) {
                     // floor(t) + magic: byte 0 = floor(t) = c + 128
                     t01 = add2_rm(t01, mm);

@@ -8,13 +8,20 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 
+def _load_by_path(name, path):
+    import importlib.util
+    spec = importlib.util.spec_from_file_location(name, path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
+
+
 def _build_libraries():
     """Build the oracle and the CUDA library in-tree when missing or stale (nvcc
-    cross-compiles for sm_100a without a GPU)."""
-    from oracle import build as obuild
-    from ssm_decode_02_b200 import build as lbuild
-    obuild.build()
-    lbuild.build()
+    cross-compiles for sm_100a without a GPU).  The build scripts are loaded by
+    path: importing the packages would load the libraries they build."""
+    _load_by_path("_rsq_oracle_build", os.path.join(ROOT, "oracle", "build.py")).build()
+    _load_by_path("_rsq_lib_build", os.path.join(ROOT, "ssm_decode_02_b200", "build.py")).build()
 
 
 def pytest_configure(config):
