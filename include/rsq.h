@@ -228,6 +228,28 @@ rsq_status rsq_allocate_bits(const double* score, int heads, int n_high, int hig
  * (host-only; 8 for every supported dk). */
 int rsq_reduction_partials(int dk);
 
+/* Decode step that allocates nothing (no counterpart in the method's pages).
+ *
+ * Same computation, arguments and results as rsq_decode_step, but without a
+ * context: the configuration is passed directly and nothing is allocated.
+ * rsq_create allocates a 4-byte device flag word with cudaMalloc; callers that
+ * may not allocate device memory -- code running inside CUDA stream capture
+ * (allocation calls are not capturable) or a runtime whose device memory is
+ * owned entirely by its own pool allocator -- use this entry point instead.
+ *
+ * Its scratch (the decode kernel's flag word) lives in a statically allocated
+ * device array of 64 words (256 bytes) that every GPU loading the library
+ * holds until the process exits; a call needing more scratch than that is
+ * rejected with RSQ_E_UNSUPPORTED.  All calls share the array: the flag word is
+ * cleared at the start of every call, the flags it collects are not reported
+ * (use a context and rsq_check_flags for that), and calls that overlap on the
+ * GPU race on it.  The first call on a device looks up the array's device
+ * address (and sets kernel attributes) for that device; make that first call
+ * before any stream capture.  Errors as rsq_create plus rsq_decode_step. */
+rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_state* state_in,
+                                   const rsq_state* state_out, const void* inputs, float* out,
+                                   uint32_t step, void* stream);
+
 const char* rsq_status_string(rsq_status s);
 const char* rsq_last_error(void);
 const char* rsq_version(void);

@@ -57,7 +57,7 @@ class rsq_mamba2_inputs(ctypes.Structure):
 _EXPORTS = ["rsq_create", "rsq_destroy", "rsq_state_bytes", "rsq_head_offset", "rsq_decode_step",
             "rsq_quantize", "rsq_dequantize", "rsq_state_drift", "rsq_check_flags",
             "rsq_allocate_bits", "rsq_reduction_partials", "rsq_status_string", "rsq_last_error",
-            "rsq_version"]
+            "rsq_version", "rsq_decode_step_noalloc"]
 
 
 def _load():
@@ -81,6 +81,8 @@ def _load():
         "rsq_status_string": ([C], ctypes.c_char_p),
         "rsq_last_error": ([], ctypes.c_char_p),
         "rsq_version": ([], ctypes.c_char_p),
+        "rsq_decode_step_noalloc": ([ctypes.POINTER(rsq_config), ctypes.POINTER(rsq_state),
+                                     ctypes.POINTER(rsq_state), P, P, ctypes.c_uint32, P], C),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -139,6 +141,30 @@ def rsq_create(family: int, batch: int, heads: int, dk: int, dv: int, *, head_bi
     out = ctypes.c_void_p()
     _check(lib.rsq_create(ctypes.byref(cfg), ctypes.byref(out)))
     return int(out.value)
+
+
+def _config(family, batch, heads, dk, dv, head_bits, rounding, in_dtype, seed, ngroups):
+    bits_arr = None
+    if head_bits is not None:
+        bits_arr = (ctypes.c_int8 * heads)(*[int(b) for b in head_bits])
+    cfg = rsq_config(int(family), int(batch), int(heads), int(dk), int(dv), int(ngroups),
+                     ctypes.cast(bits_arr, ctypes.POINTER(ctypes.c_int8)) if bits_arr else None,
+                     int(rounding), int(in_dtype), int(seed) & (2 ** 64 - 1))
+    return cfg, bits_arr
+
+
+def rsq_decode_step_noalloc(family: int, batch: int, heads: int, dk: int, dv: int, state_in,
+                            state_out, inputs, out, step: int, *, head_bits=None,
+                            rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0,
+                            ngroups: int = 1, stream=None) -> None:
+    """Decode step without a context and without any device allocation (the
+    kernel's flag word lives in a static device array; see include/rsq.h)."""
+    cfg, keep = _config(family, batch, heads, dk, dv, head_bits, rounding, in_dtype, seed, ngroups)
+    si, so = _state(state_in), _state(state_out)
+    _check(lib.rsq_decode_step_noalloc(ctypes.byref(cfg), ctypes.byref(si), ctypes.byref(so),
+                                       ctypes.byref(inputs), _ptr(out), int(step) & 0xFFFFFFFF,
+                                       _stream(stream)))
+    del keep
 
 
 def rsq_destroy(ctx: int) -> None:

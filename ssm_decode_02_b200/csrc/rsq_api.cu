@@ -6,6 +6,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -348,3 +349,119 @@ rsq_status rsq_check_flags(const rsq_ctx* ctx, int* seen, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode step without any allocation.
+//
+// rsq_create allocates the context's 4-byte device flag word with cudaMalloc.
+// This entry point instead keeps that word in a small statically allocated
+// device array, so a caller that may not allocate device memory can still run
+// a decode step: code inside stream capture, where allocation calls are not
+// allowed, or a runtime whose memory is owned entirely by its own pool
+// allocator.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kNoallocScratchWords = 64;   // 256 bytes on every device that loads the library
+constexpr int kNoallocWordsNeeded = 1;     // the decode kernel's flag word
+constexpr int kNoallocMaxDevices = 64;
+
+// In host code this name is only a stand-in for the device array; its device
+// address comes from cudaGetSymbolAddress (per device) below.
+static __device__ __align__(256) unsigned g_noalloc_scratch[kNoallocScratchWords];
+
+std::mutex g_noalloc_mu;
+unsigned* g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+// Device address of the scratch array for the current device (resolved once
+// per device, with that device current).
+rsq_status noalloc_scratch(int device, unsigned** out) {
+    if (device < 0 || device >= kNoallocMaxDevices)
+        return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: device index %d out of range", device);
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (!g_noalloc_ptr[device]) {
+        void* ptr = nullptr;
+        const int err = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (err) return cuda_fail(err, "decode_step_noalloc: cudaGetSymbolAddress");
+        g_noalloc_ptr[device] = static_cast<unsigned*>(ptr);
+    }
+    *out = g_noalloc_ptr[device];
+    return RSQ_OK;
+}
+
+}  // namespace
+
+extern "C" rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_state* state_in,
+                                              const rsq_state* state_out, const void* inputs,
+                                              float* out, uint32_t step, void* stream) {
+    if (!cfg) return fail(RSQ_E_INVAL, "decode_step_noalloc: null config");
+    const rsq_config& c = *cfg;
+    if (c.family != RSQ_GDN && c.family != RSQ_MAMBA2)
+        return fail(RSQ_E_INVAL, "decode_step_noalloc: bad family %d", c.family);
+    if (c.batch < 1) return fail(RSQ_E_INVAL, "decode_step_noalloc: batch must be >= 1");
+    if (c.heads < 1 || c.heads > RSQ_MAX_HEADS)
+        return fail(RSQ_E_INVAL, "decode_step_noalloc: heads must be in [1, %d]", RSQ_MAX_HEADS);
+    if (!dk_ok(c.dk) || !dv_ok(c.dv))
+        return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: unsupported dk=%d dv=%d", c.dk, c.dv);
+    if (c.rounding != RSQ_RTN && c.rounding != RSQ_SR)
+        return fail(RSQ_E_INVAL, "decode_step_noalloc: bad rounding %d", c.rounding);
+    if (c.in_dtype != RSQ_F32 && c.in_dtype != RSQ_BF16)
+        return fail(RSQ_E_INVAL, "decode_step_noalloc: bad in_dtype %d", c.in_dtype);
+    if (c.family == RSQ_MAMBA2 && (c.ngroups < 1 || c.heads % c.ngroups != 0))
+        return fail(RSQ_E_INVAL, "decode_step_noalloc: ngroups must divide heads");
+    if (kNoallocWordsNeeded > kNoallocScratchWords)
+        return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: needs %d scratch words, the static array holds %d",
+                    kNoallocWordsNeeded, kNoallocScratchWords);
+
+    // the context lives on the stack: bit widths, offsets and launch geometry
+    rsq_ctx ctx;
+    std::memset(&ctx, 0, sizeof(ctx));
+    ctx.cfg = c;
+    ctx.cfg.head_bits = nullptr;
+    int n32 = 0;
+    for (int h = 0; h < c.heads; ++h) {
+        const int b = c.head_bits ? c.head_bits[h] : 8;
+        if (b != 4 && b != 8 && b != 32)
+            return fail(RSQ_E_INVAL, "decode_step_noalloc: head %d has %d bits (4, 8 or 32)", h, b);
+        n32 += (b == 32);
+        ctx.bits[h] = static_cast<int8_t>(b);
+    }
+    if (n32 != 0 && n32 != c.heads)
+        return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: 32-bit heads cannot be mixed with 4/8-bit heads");
+    ctx.f32state = (n32 == c.heads);
+    long long off = 0;
+    for (int h = 0; h < c.heads; ++h) {
+        ctx.head_off[h] = static_cast<uint32_t>(off);
+        off += static_cast<long long>(c.dk) * c.dv * ctx.bits[h] / 8;
+    }
+    ctx.row_bytes = off;
+    ctx.ub = std::min(c.dv / rsq::kBlockCols, 4);
+    ctx.ncb = c.dv / (rsq::kBlockCols * ctx.ub);
+    const long long units = static_cast<long long>(c.batch) * c.heads * ctx.ncb;
+    if (units > (1LL << 30)) return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: too many work units");
+    ctx.units = static_cast<int>(units);
+
+    int threads = 0;
+    size_t smem = 0;
+    const void* func = nullptr;
+    if (rsq::decode_kernel_info(c.family, c.dk, ctx.ub, ctx.f32state, c.rounding == RSQ_SR, &threads, &smem,
+                                &func) != 0)
+        return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: no kernel for dk=%d dv=%d", c.dk, c.dv);
+    int err = cudaGetDevice(&ctx.device);
+    int sms = 0, per_sm = 0;
+    if (!err) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, ctx.device);
+    if (!err) err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (!err) err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, func, threads, smem);
+    if (!err && per_sm < 1) err = cudaErrorInvalidConfiguration;
+    if (err) return cuda_fail(err, "decode_step_noalloc: launch geometry");
+    ctx.grid = static_cast<int>(std::min<long long>(units, static_cast<long long>(sms) * per_sm));
+
+    unsigned* scratch = nullptr;
+    rsq_status s = noalloc_scratch(ctx.device, &scratch);
+    if (s) return s;
+    // the flag word starts each call at zero (every call shares the array)
+    err = cudaMemsetAsync(scratch, 0, kNoallocWordsNeeded * sizeof(unsigned), static_cast<cudaStream_t>(stream));
+    if (err) return cuda_fail(err, "decode_step_noalloc: clear scratch");
+    ctx.flag = scratch;
+    return rsq_decode_step(&ctx, state_in, state_out, inputs, out, step, stream);
+}
