@@ -34,7 +34,7 @@ struct DecodeCfg {
     using L = Layout<DK>;
     static constexpr int NT = 32 * UB;         // one warp per 16-column block
     static constexpr int UCOLS = 16 * UB;      // columns per unit
-    static constexpr int NS = F32STATE ? 2 : 3;  // pipeline stages
+    static constexpr int NS = F32STATE ? 2 : 4;  // pipeline stages
     static constexpr int CODE_BYTES = F32STATE ? DK * UCOLS * 4 : DK * UCOLS;  // largest tile (8-bit)
     static constexpr int OFF_SCALES = CODE_BYTES;
     static constexpr int OFF_VA = OFF_SCALES + UCOLS * 4;  // GDN q / Mamba-2 C   (<= DK floats)
@@ -357,14 +357,15 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (DecodeC
     }
     Gates gt = {0.f, 0.f, 0.f, 0.f};
     if (cur.u < p.units) gt = load_gates<FAM>(p, cur);
-    for (int n = 0; cur.u < p.units; ++n) {
+    int stage = 0;
+    uint32_t parity = 0;
+    while (cur.u < p.units) {
         UnitIt nxt = cur;
         nxt.advance(p);
         Gates ng = gt;
         if (nxt.u < p.units) ng = load_gates<FAM>(p, nxt);
-        const int stage = n % C::NS;
         const uint32_t bar = bar0 + 8 * stage;
-        const bool ok = mbar_wait(bar, (n / C::NS) & 1, kWaitIters);
+        const bool ok = mbar_wait(bar, parity, kWaitIters);
         if (__any_sync(0xffffffffu, !ok)) {
             if (lane == 0) atomicOr(p.flag, kFlagTimeout);
             return;  // this warp stops; the others see their own waits expire
@@ -380,6 +381,10 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (DecodeC
         }
         cur = nxt;
         gt = ng;
+        if (++stage == C::NS) {
+            stage = 0;
+            parity ^= 1u;
+        }
     }
 }
 

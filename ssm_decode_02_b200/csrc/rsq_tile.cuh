@@ -66,14 +66,21 @@ __device__ __forceinline__ float pick4(const float4& v, int j) {
 // the column's absmax m): lanes g < 4 own column 4cw + g for the scale
 // s = m / r, lanes g >= 4 own column 4cw + g - 4 for the multiplier
 // inv = r / m rounded toward zero (0 for an all-zero or non-finite column).
-// Returns this lane's value (s or inv); the caller gathers the multipliers.
+// Every lane performs one round-to-nearest division (no divergence); the
+// multiplier lanes then step the quotient toward zero when it was rounded up,
+// which the exact sign of fma(q, m, -r) = q*m - r tells.  Returns this lane's
+// value (s or inv); the caller gathers the multipliers.
 template <int BITS>
 __device__ __forceinline__ float scale_or_inv(const float4& m4, int g, bool& nonfinite) {
     constexpr float r = float((1 << (BITS - 1)) - 1);
     const float m = pick4(m4, g & 3);
     nonfinite = !isfinite(m);
-    if (g < 4) return __fdiv_rn(m, r);
-    return (m > 0.0f && !nonfinite) ? __fdiv_rz(r, m) : 0.0f;
+    const bool scale_lane = g < 4;
+    const float q = __fdiv_rn(scale_lane ? m : r, scale_lane ? r : m);
+    const bool rounded_up = __fmaf_rn(q, m, -r) > 0.0f;
+    const float q_rz = rounded_up ? __uint_as_float(__float_as_uint(q) - 1u) : q;
+    const float inv = (m > 0.0f && !nonfinite) ? q_rz : 0.0f;
+    return scale_lane ? q : inv;
 }
 
 // Multipliers of this lane's 4 columns, from the lanes g = 4..7 of its column group.
@@ -126,9 +133,11 @@ template <int BITS>
 __device__ __forceinline__ uint32_t pack_row(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3,
                                              bool byte2) {
     if constexpr (BITS == 8) {
-        // byte 0 of each float holds c + 128
-        const uint32_t a = prmt(t0, t1, 0x0040u);
-        const uint32_t b = prmt(t2, t3, 0x0040u);
+        // Byte 0 of each float holds c + 128 and byte 1 is zero, so t1*256 + t0
+        // (mod 2^32) carries (byte0(t1), byte0(t0)) in its low 16 bits without any
+        // carry between them; one byte permute joins the two halves.
+        const uint32_t a = t1 * 256u + t0;
+        const uint32_t b = t3 * 256u + t2;
         return prmt(a, b, 0x5410u);
     } else {
         // the code nibble c + 8 sits in byte 0 (RTN) or byte 2 (SR)
@@ -165,12 +174,13 @@ __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], c
                                                  uint32_t h, uint32_t b, uint32_t step,
                                                  const PhiloxKeysT& rk) {
     const uint64_t inv01 = pk(iv.x, iv.y), inv23 = pk(iv.z, iv.w);
+    // this lane's first row; row k sits k * 8 rows further
+    uint8_t* const row0 = dst + (BITS == 8 ? g * 16 + 4 * cw : g * 8 + 2 * cw);
     auto store_row = [&](int k, uint32_t word) {
-        const int i = g + kR * k;
         if constexpr (BITS == 8)
-            *reinterpret_cast<uint32_t*>(dst + i * 16 + 4 * cw) = word;
+            *reinterpret_cast<uint32_t*>(row0 + k * (kR * 16)) = word;
         else
-            *reinterpret_cast<uint16_t*>(dst + i * 8 + 2 * cw) = static_cast<uint16_t>(word);
+            *reinterpret_cast<uint16_t*>(row0 + k * (kR * 8)) = static_cast<uint16_t>(word);
     };
     if constexpr (!SR) {
         const float o = (BITS == 8) ? kMagic + 128.0f : kMagic + 8.0f;
@@ -195,8 +205,10 @@ __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], c
             for (int half = 0; half < 2; ++half) {
                 const int kk = k + half * (RPT / 2);
                 const uint32_t w0 = u[half][0], w1 = u[half][1];
-                const uint64_t V01 = pk(__uint_as_float(vb | (w0 & 0xFFFFu)), __uint_as_float(vb | (w0 >> 16)));
-                const uint64_t V23 = pk(__uint_as_float(vb | (w1 & 0xFFFFu)), __uint_as_float(vb | (w1 >> 16)));
+                // offset + u/2^16: the low half by a mask, the high half as
+                // hi(w * 2^16) + offset bits (a multiply-add, off the logic pipe)
+                const uint64_t V01 = pk(__uint_as_float(vb | (w0 & 0xFFFFu)), __uint_as_float(umulhi_add(w0, 0x10000u, vb)));
+                const uint64_t V23 = pk(__uint_as_float(vb | (w1 & 0xFFFFu)), __uint_as_float(umulhi_add(w1, 0x10000u, vb)));
                 uint64_t t01 = fma2(S2[kk][0], inv01, V01);
                 uint64_t t23 = fma2(S2[kk][1], inv23, V23);
                 if constexpr (BITS == 8) {
