@@ -122,6 +122,23 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(x: float, dist=None, device=None) -> float:
+    """The maximum of a per-rank scalar over all ranks (the timed interval of a
+    multi-GPU run is the slowest rank's); identity without a process group."""
+    if dist is None or not dist.is_available() or not dist.is_initialized():
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_input_step(t: int, rank: int) -> int:
+    """Input-generator step index of local step t on a rank: every rank serves its
+    own requests (independent shards, no exchange), so the draws must differ."""
+    return t + 100000 * rank
+
+
 def measured_peak_gbs():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -281,7 +298,7 @@ def run_ours(args, w: W.Workload):
     n_sets = max(8, min(256, -(-3 * l2 // max(1, step_input_bytes(w)))))
     sets = []
     for t in range(n_sets):
-        host = W.inputs(w, t + 100000 * rank)
+        host = W.inputs(w, rank_input_step(t, rank))
         d = {k: _to_dev(v, dev) for k, v in host.items()}
         sets.append(d)
     inp_bytes = step_input_bytes(w)
@@ -353,17 +370,13 @@ def run_ours(args, w: W.Workload):
         dist.barrier()
     time.sleep(0.15)
     clk = clocks.stop()
-    elapsed = ev0.elapsed_time(ev1) / 1e3
-    if world > 1:
-        tt = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed = float(tt.item())
+    elapsed = max_over_ranks(ev0.elapsed_time(ev1) / 1e3, dist if world > 1 else None, dev)
     flag = ctx.check_flags(stream.cuda_stream)
 
     # end-to-end through the public API with host buffers (pinned), per step:
     # H2D of that step's inputs, the decode step, D2H of its output
     n_e2e = max(1, min(args.steps, 500))
-    pinned = [{k: _to_pinned(v) for k, v in W.inputs(w, 200000 + t + 1000 * rank).items()}
+    pinned = [{k: _to_pinned(v) for k, v in W.inputs(w, rank_input_step(200000 + t, rank)).items()}
               for t in range(4)]
     dev_in = {k: torch.empty_like(v, device=dev) for k, v in pinned[0].items()}
     e2e_struct = _inputs_struct(rsq, w, dev_in)
@@ -385,11 +398,7 @@ def run_ours(args, w: W.Workload):
             out_host.copy_(outs[0], non_blocking=True)
         e1.record(stream)
     e1.synchronize()
-    e2e_elapsed = e0.elapsed_time(e1) / 1e3
-    if world > 1:
-        tt = torch.tensor([e2e_elapsed], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_elapsed = float(tt.item())
+    e2e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist if world > 1 else None, dev)
 
     hu_step = w.B * w.H
     value = world * hu_step * args.steps / elapsed
@@ -398,7 +407,8 @@ def run_ours(args, w: W.Workload):
     alg = step_bytes(w, bits)
     peak, peak_kind = measured_peak_gbs()
     achieved = alg / per_launch / 1e9
-    kernel_tag = "rsq_decode_kernel<%s,%d,%d>" % (w.family, w.dk, min(64, w.dv))
+    kernel_tag = "rsq_decode_kernel<%s,dk=%d,blocks=%d,%s>" % (w.family, w.dk, min(4, w.dv // 16),
+                                                                 "fp32" if w.state == "fp32" else w.rounding)
     line = {
         "metric": "head-updates/s", "value": value, "unit": "head-updates/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * per_launch,

@@ -1,0 +1,87 @@
+"""Multi-process host logic of the N-GPU benchmark path, on CPU with gloo.
+
+Requests and heads are independent, so N GPUs run N independent shards with
+no exchange on the data path; the only collectives are the barrier and the
+maximum of the timed interval over ranks.  These tests run two gloo ranks.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, values, out_q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    sys.path.insert(0, ROOT)
+    import bench
+    from datetime import timedelta
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        got = bench.max_over_ranks(values[rank], dist)
+        dist.barrier()
+        out_q.put((rank, got))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_two_gloo_ranks():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    values = [0.125, 0.5]
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, values, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    res = dict(q.get(timeout=10) for _ in range(2))
+    assert res == {0: 0.5, 1: 0.5}
+
+
+def test_max_over_ranks_without_process_group_is_identity():
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.5) == 3.5
+
+
+def test_ranks_serve_independent_requests():
+    """Weak scaling: each rank draws its own requests (different inputs)."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    w = W.WORKLOADS[1]
+    a = W.gdn_inputs(w, bench.rank_input_step(3, 0), B=2)
+    b = W.gdn_inputs(w, bench.rank_input_step(3, 1), B=2)
+    assert not np.array_equal(a["v"], b["v"])
+    assert len({bench.rank_input_step(t, r) for t in range(1000) for r in range(8)}) == 8000
+
+
+@pytest.mark.slow
+def test_reference_arm_under_torchrun_prints_one_line():
+    """`bench.py --impl reference` launched like the multi-GPU run: rank 0 alone
+    times the oracle and prints one JSON line; rank 1 exits 0 without work."""
+    port = _free_port()
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node=2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--impl",
+           "reference", "--gpus", "2", "--steps", "2", "--warmup", "1"]
+    res = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=900)
+    assert res.returncode == 0, res.stderr[-3000:]
+    lines = [l for l in res.stdout.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
