@@ -200,8 +200,7 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
             a01 = fma2(S2[k + 1][0], kk.y, a01);
             a23 = fma2(S2[k + 1][1], kk.y, a23);
         }
-        float4 ck = unpk4(a01, a23);
-        warp_sum4(ck);
+        const float4 ck = gather_cols(reduce_scatter4(unpk4(a01, a23), g, AddOp()), cw, 0);
         // reload the k pairs below instead of keeping 16 of them live across the
         // reduction (register pressure)
         asm volatile("" ::: "memory");
@@ -256,6 +255,8 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
     }
 
     // ---- readout and column absmax ----------------------------------------------
+    // From here to the code stores the block is branch-free, so the compiler can
+    // overlap the reductions' shuffle and division latency with Philox work.
     uint64_t o01 = pk(0.f, 0.f), o23 = pk(0.f, 0.f);
 #pragma unroll
     for (int k = 0; k < RPT; k += 2) {
@@ -265,14 +266,11 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
         o01 = fma2(S2[k + 1][0], qq.y, o01);
         o23 = fma2(S2[k + 1][1], qq.y, o23);
     }
-    float4 o4 = unpk4(o01, o23);
-    warp_sum4(o4);
-    const long long col = (long long)hu * p.dv + j0 + 4 * cw;  // this lane's first column
-    if (g < 4) {
-        float o = pick4(o4, g);
-        if constexpr (FAM == RSQ_MAMBA2) o = __fmaf_rn(gt.D, ld_vec(stage + C::OFF_VC, 16 * w + 4 * cw + g, bf16), o);
-        p.out[col + g] = o;
-    }
+    const int c = col_of(g);  // the column this lane finalises
+    float o = reduce_scatter4(unpk4(o01, o23), g, AddOp());
+    if constexpr (FAM == RSQ_MAMBA2) o = __fmaf_rn(gt.D, ld_vec(stage + C::OFF_VC, 16 * w + 4 * cw + c, bf16), o);
+    const long long col = (long long)hu * p.dv + j0 + 4 * cw + c;
+    if (g < 4) p.out[col] = o;
     float4 iv = make_float4(0.f, 0.f, 0.f, 0.f);
     if constexpr (BITS != 32) {
         float m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
@@ -285,15 +283,29 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
             m2 = max3_nan(m2, fabsf(x.z), fabsf(y.z));
             m3 = max3_nan(m3, fabsf(x.w), fabsf(y.w));
         }
-        float4 m4 = make_float4(m0, m1, m2, m3);
-        warp_max4(m4);
-        bool nonfinite;
-        const float mine = scale_or_inv<BITS>(m4, g, nonfinite);
-        if (g < 4) {
-            p.scales_out[col + g] = mine;
-            if (nonfinite) atomicOr(p.flag, kFlagNonFinite);
+        const float m = reduce_scatter4(make_float4(m0, m1, m2, m3), g, MaxOp());
+        const float mine = scale_or_inv<BITS>(m, g);
+        if (g < 4) p.scales_out[col] = mine;
+        iv = gather_cols(mine, cw, 16);
+    }
+
+    // ---- store ------------------------------------------------------------------
+    uint8_t* dst = p.codes_out + (long long)un.b * p.row_bytes + p.head_off[un.h] +
+                   (long long)blk * BLOCK_BYTES;
+    const uint32_t gcol = static_cast<uint32_t>(j0 / 4 + cw);
+    if constexpr (BITS == 32) {
+#pragma unroll
+        for (int k = 0; k < RPT; ++k)
+            *reinterpret_cast<ulonglong2*>(dst + ((g + kR * k) * 16 + 4 * cw) * 4) =
+                make_ulonglong2(S2[k][0], S2[k][1]);
+    } else {
+        requantize_store<BITS, SR, RPT>(S2, iv, dst, g, cw, gcol, un.h, un.b, p.step, p.rk);
+        // rare: a non-finite column (multiplier -0.0) is stored as the zero code
+        if (is_neg_zero(iv.x) || is_neg_zero(iv.y) || is_neg_zero(iv.z) || is_neg_zero(iv.w)) {
+            atomicOr(p.flag, kFlagNonFinite);
+            clear_nonfinite_columns<RPT>(S2, iv);
+            requantize_store<BITS, SR, RPT>(S2, iv, dst, g, cw, gcol, un.h, un.b, p.step, p.rk);
         }
-        iv = gather_inv(mine, cw);
     }
 
     // ---- release the stage; the last warp refills it with the unit NS ahead ----
@@ -310,20 +322,6 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
                 issue_unit<FAM, DK, UB, F32STATE>(p, refill, stage, bar);
             }
         }
-    }
-
-    // ---- store ------------------------------------------------------------------
-    uint8_t* dst = p.codes_out + (long long)un.b * p.row_bytes + p.head_off[un.h] +
-                   (long long)blk * BLOCK_BYTES;
-    if constexpr (BITS == 32) {
-#pragma unroll
-        for (int k = 0; k < RPT; ++k)
-            *reinterpret_cast<ulonglong2*>(dst + ((g + kR * k) * 16 + 4 * cw) * 4) =
-                make_ulonglong2(S2[k][0], S2[k][1]);
-    } else {
-        clear_zero_inv_columns<RPT>(S2, iv);
-        requantize_store<BITS, SR, RPT>(S2, iv, dst, g, cw, static_cast<uint32_t>(j0 / 4 + cw), un.h,
-                                        un.b, p.step, p.rk);
     }
 }
 

@@ -57,16 +57,16 @@ __device__ __forceinline__ void quantize_block(const QuantParams& p, const Block
             m4.z = max_nan(m4.z, fabsf(s.z));
             m4.w = max_nan(m4.w, fabsf(s.w));
         }
-        warp_max4(m4);
-        bool nonfinite;
-        const float mine = scale_or_inv<BITS>(m4, g, nonfinite);
-        const long long col = (long long)bi.hu * p.dv + j0 + 4 * cw;
-        if (g < 4) {
-            p.scales[col + g] = mine;
-            if (nonfinite) atomicOr(p.flag, kFlagNonFinite);
+        const float m = reduce_scatter4(m4, g, MaxOp());
+        const float mine = scale_or_inv<BITS>(m, g);
+        const long long col = (long long)bi.hu * p.dv + j0 + 4 * cw + col_of(g);
+        if (g < 4) p.scales[col] = mine;
+        const float4 iv = gather_cols(mine, cw, 16);
+        const bool any_nonfinite = is_neg_zero(iv.x) || is_neg_zero(iv.y) || is_neg_zero(iv.z) || is_neg_zero(iv.w);
+        if (any_nonfinite) {
+            atomicOr(p.flag, kFlagNonFinite);
+            clear_nonfinite_columns<RPT>(S2, iv);
         }
-        const float4 iv = gather_inv(mine, cw);
-        clear_zero_inv_columns<RPT>(S2, iv);
         const uint32_t gcol = static_cast<uint32_t>(j0 / 4 + cw);
         if (p.sr)
             requantize_store<BITS, true, RPT>(S2, iv, dst, g, cw, gcol, bi.h, bi.b, p.step, p.rk);

@@ -58,40 +58,69 @@ __device__ __forceinline__ void warp_max4(float4& m) {
     }
 }
 
+// Reduce-scatter over the 8 row groups of a column group.  Afterwards lane
+// (cw, g) holds the total of column 4cw + col_of(g), col_of(g) = 2*(g&1) +
+// ((g>>1)&1); lanes g and g^4 hold the same column.  Every addition pairs the
+// same two partials as the butterfly d = 1, 2, 4 (floating-point addition is
+// commutative), so each column total is bit-identical to the butterfly's.
+__device__ __forceinline__ int col_of(int g) { return 2 * (g & 1) + ((g >> 1) & 1); }
+
+template <class Op>
+__device__ __forceinline__ float reduce_scatter4(const float4& v, int g, Op op) {
+    const bool b0 = (g & 1) != 0, b1 = (g & 2) != 0;
+    // d = 1 (lanes 4 apart): keep columns {0,1} (b0 = 0) or {2,3} (b0 = 1)
+    const float send0 = b0 ? v.x : v.z, send1 = b0 ? v.y : v.w;
+    const float keep0 = b0 ? v.z : v.x, keep1 = b0 ? v.w : v.y;
+    const float a0 = op(keep0, __shfl_xor_sync(0xffffffffu, send0, 4));
+    const float a1 = op(keep1, __shfl_xor_sync(0xffffffffu, send1, 4));
+    // d = 2 (lanes 8 apart): keep column 2*b0 (b1 = 0) or 2*b0 + 1 (b1 = 1)
+    const float send = b1 ? a0 : a1, keep = b1 ? a1 : a0;
+    const float c = op(keep, __shfl_xor_sync(0xffffffffu, send, 8));
+    // d = 4 (lanes 16 apart): both hold the same column
+    return op(c, __shfl_xor_sync(0xffffffffu, c, 16));
+}
+struct AddOp {
+    __device__ __forceinline__ float operator()(float a, float b) const { return __fadd_rn(a, b); }
+};
+struct MaxOp {
+    __device__ __forceinline__ float operator()(float a, float b) const { return max_nan(a, b); }
+};
+
+// Values of this lane's 4 columns 4cw..4cw+3 after a reduce-scatter: column j
+// sits on the lanes with col_of(g) = j, i.e. g = 0, 2, 1, 3 (+ base).
+__device__ __forceinline__ float4 gather_cols(float mine, int cw, int base) {
+    float4 r;
+    r.x = __shfl_sync(0xffffffffu, mine, base + cw);
+    r.y = __shfl_sync(0xffffffffu, mine, base + cw + 8);
+    r.z = __shfl_sync(0xffffffffu, mine, base + cw + 4);
+    r.w = __shfl_sync(0xffffffffu, mine, base + cw + 12);
+    return r;
+}
+
 __device__ __forceinline__ float pick4(const float4& v, int j) {
     return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
 }
 
-// Column finalisation after the butterflies (every lane of a column group holds
-// the column's absmax m): lanes g < 4 own column 4cw + g for the scale
-// s = m / r, lanes g >= 4 own column 4cw + g - 4 for the multiplier
-// inv = r / m rounded toward zero (0 for an all-zero or non-finite column).
-// Every lane performs one round-to-nearest division (no divergence); the
-// multiplier lanes then step the quotient toward zero when it was rounded up,
-// which the exact sign of fma(q, m, -r) = q*m - r tells.  Returns this lane's
-// value (s or inv); the caller gathers the multipliers.
+// Column finalisation after the reduce-scatter (m = absmax of this lane's
+// column): lanes g < 4 compute the scale s = m / r, lanes g >= 4 the multiplier
+// inv = r / m rounded toward zero -- 0 for an all-zero column and -0.0 for a
+// non-finite one (so the caller can find non-finite columns from the
+// multipliers alone).  Every lane performs one round-to-nearest division (no
+// divergence); the multiplier lanes then step the quotient toward zero when it
+// was rounded up, which the exact sign of fma(q, m, -r) = q*m - r tells.
 template <int BITS>
-__device__ __forceinline__ float scale_or_inv(const float4& m4, int g, bool& nonfinite) {
+__device__ __forceinline__ float scale_or_inv(float m, int g) {
     constexpr float r = float((1 << (BITS - 1)) - 1);
-    const float m = pick4(m4, g & 3);
-    nonfinite = !isfinite(m);
+    const bool finite = isfinite(m);
     const bool scale_lane = g < 4;
     const float q = __fdiv_rn(scale_lane ? m : r, scale_lane ? r : m);
     const bool rounded_up = __fmaf_rn(q, m, -r) > 0.0f;
     const float q_rz = rounded_up ? __uint_as_float(__float_as_uint(q) - 1u) : q;
-    const float inv = (m > 0.0f && !nonfinite) ? q_rz : 0.0f;
+    const float inv = !finite ? -0.0f : (m > 0.0f ? q_rz : 0.0f);
     return scale_lane ? q : inv;
 }
 
-// Multipliers of this lane's 4 columns, from the lanes g = 4..7 of its column group.
-__device__ __forceinline__ float4 gather_inv(float mine, int cw) {
-    float4 iv;
-    iv.x = __shfl_sync(0xffffffffu, mine, cw + 16);
-    iv.y = __shfl_sync(0xffffffffu, mine, cw + 20);
-    iv.z = __shfl_sync(0xffffffffu, mine, cw + 24);
-    iv.w = __shfl_sync(0xffffffffu, mine, cw + 28);
-    return iv;
-}
+__device__ __forceinline__ bool is_neg_zero(float x) { return __float_as_uint(x) == 0x80000000u; }
 
 // Decode this lane's RPT rows of 4 codes of a stored block into exact float
 // codes, kept as packed pairs: S2[k][0] = columns 0,1 and S2[k][1] = columns
@@ -148,17 +177,16 @@ __device__ __forceinline__ uint32_t pack_row(uint32_t t0, uint32_t t1, uint32_t 
     }
 }
 
-// Columns whose multiplier is 0 (all-zero or non-finite) must come out as the
-// zero code; a non-finite state value would not, so clear those columns.
+// Non-finite columns (multiplier -0.0) must come out as the zero code; their
+// state values would not, so clear them (used on the rare path only).
 template <int RPT>
-__device__ __forceinline__ void clear_zero_inv_columns(uint64_t (&S2)[RPT][2], const float4& iv) {
-    if (__builtin_expect(iv.x == 0.0f || iv.y == 0.0f || iv.z == 0.0f || iv.w == 0.0f, 0)) {
+__device__ __forceinline__ void clear_nonfinite_columns(uint64_t (&S2)[RPT][2], const float4& iv) {
+    const bool b0 = is_neg_zero(iv.x), b1 = is_neg_zero(iv.y), b2 = is_neg_zero(iv.z), b3 = is_neg_zero(iv.w);
 #pragma unroll
-        for (int k = 0; k < RPT; ++k) {
-            const float4 s = unpk4(S2[k][0], S2[k][1]);
-            S2[k][0] = pk(iv.x == 0.0f ? 0.0f : s.x, iv.y == 0.0f ? 0.0f : s.y);
-            S2[k][1] = pk(iv.z == 0.0f ? 0.0f : s.z, iv.w == 0.0f ? 0.0f : s.w);
-        }
+    for (int k = 0; k < RPT; ++k) {
+        const float4 s = unpk4(S2[k][0], S2[k][1]);
+        S2[k][0] = pk(b0 ? 0.0f : s.x, b1 ? 0.0f : s.y);
+        S2[k][1] = pk(b2 ? 0.0f : s.z, b3 ? 0.0f : s.w);
     }
 }
 
