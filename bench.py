@@ -9,10 +9,15 @@ quoted on).  Consecutive steps cycle through enough independent layer states
 model do, so every step reads its state from HBM.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+  python bench.py --drift [--workload W] [--drift-steps T] [--drift-every E]
 
 N > 1 is launched by torchrun (one process per GPU); every rank runs its own
 requests (weak scaling, no collective on the data path); the time is the max
 over ranks.  --impl reference times the CPU oracle on the host cores instead.
+--drift runs the long-horizon study instead (default: Gated DeltaNet B=1024,
+H=16, d=128, 4096 steps): the relative state drift of INT4/INT8 trajectories
+with stochastic and nearest rounding against the FP32 trajectory, every 256
+steps, as one JSON line.
 """
 from __future__ import annotations
 
@@ -34,6 +39,7 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 DEFAULT_WORKLOAD = "gdn_b64_h16_d128_int8_sr"
+DRIFT_WORKLOAD = "gdn_b1024_h16_d128_int4_sr_long"
 
 
 def algorithmic_bytes_per_head(w: W.Workload, bits: int) -> int:
@@ -373,6 +379,24 @@ def run_ours(args, w: W.Workload):
     elapsed = max_over_ranks(ev0.elapsed_time(ev1) / 1e3, dist if world > 1 else None, dev)
     flag = ctx.check_flags(stream.cuda_stream)
 
+    # L2-hot reference point (labelled, not the headline): one layer state and one
+    # input set, so the whole step's working set stays in L2
+    n_hot = max(1, min(args.steps, 2000))
+    hot = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(stream):
+        with torch.cuda.graph(hot, stream=stream):
+            for t in range(n_hot):
+                ctx.decode_step(states[0], states[0], structs[0], outs[0], args.warmup + t,
+                                stream.cuda_stream)
+        hot.replay()
+        h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        h0.record(stream)
+        hot.replay()
+        h1.record(stream)
+    h1.synchronize()
+    hot_ms = h0.elapsed_time(h1) / n_hot
+    del hot
+
     # end-to-end through the public API with host buffers (pinned), per step:
     # H2D of that step's inputs, the decode step, D2H of its output
     n_e2e = max(1, min(args.steps, 500))
@@ -430,6 +454,8 @@ def run_ours(args, w: W.Workload):
         "frac_of_8tbs_datasheet": achieved / 8000.0,
         "e2e": {"value": e2e_value, "unit": "head-updates/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "steps": n_e2e},
+        "l2_hot": {"ms_per_step": hot_ms, "steps": n_hot,
+                   "setup": "one layer state and one input set, resident in L2 (not the headline)"},
         "gpu_launches": args.steps,
         "wall_s_timed_region": wall,
         "clocks": clk,
@@ -449,6 +475,91 @@ def run_ours(args, w: W.Workload):
         dist.barrier()
         dist.destroy_process_group()
     ctx.close()
+    return 0
+
+
+# ---------------------------------------------------------------------------
+# Long-horizon state drift (quantized trajectories against the FP32 trajectory)
+# ---------------------------------------------------------------------------
+DRIFT_VARIANTS = (("int4_sr", 4, "sr"), ("int4_rtn", 4, "rtn"), ("int8_sr", 8, "sr"),
+                  ("int8_rtn", 8, "rtn"))
+
+
+def _drift_inputs(job):
+    w, B, t = job
+    return t, W.inputs(w, t, B=B)
+
+
+def drift_series(w: W.Workload, steps: int, every: int, B: int | None = None, variants=DRIFT_VARIANTS,
+                 pool=None, device="cuda") -> dict:
+    """Relative state drift ||deq(S_q) - S_fp32||_F / ||S_fp32||_F of quantized
+    trajectories against the full-precision trajectory run by the same kernel
+    with 32-bit heads, all from S_0 = 0 on identical inputs, sampled every
+    `every` steps.  Also the relative error of the readout at those steps.
+
+    Returns {label: [[t, global drift, max per-head drift, readout error], ...]}."""
+    import torch
+
+    import ssm_decode_02_b200 as rsq
+
+    B = w.B if B is None else B
+    fam = rsq.RSQ_GDN if w.family == "gdn" else rsq.RSQ_MAMBA2
+    in_dtype = rsq.RSQ_BF16 if w.in_dtype == "bf16" else rsq.RSQ_F32
+
+    def make(bits, rounding):
+        ctx = rsq.Context(fam, B, w.H, w.dk, w.dv, head_bits=np.full(w.H, bits, np.int8),
+                          rounding=rsq.RSQ_SR if rounding == "sr" else rsq.RSQ_RTN,
+                          in_dtype=in_dtype, seed=w.sr_seed, ngroups=w.ngroups)
+        st = ctx.alloc_state(device)
+        ctx.quantize(torch.zeros((B, w.H, w.dk, w.dv), dtype=torch.float32, device=device), st)
+        out = torch.empty((B, w.H, w.dv), dtype=torch.float32, device=device)
+        return ctx, st, out
+
+    ref = make(32, "rtn")
+    runs = {label: make(bits, rnd) for label, bits, rnd in variants}
+    sums = torch.empty((B, w.H, 2), dtype=torch.float64, device=device)
+    series = {label: [] for label, _, _ in variants}
+    jobs = [(w, B, t) for t in range(steps)]
+    it = pool.imap(_drift_inputs, jobs, chunksize=2) if pool is not None else map(_drift_inputs, jobs)
+    for t, host in it:
+        d = {k: _to_dev(v, device) for k, v in host.items()}
+        ins = _inputs_struct(rsq, w, d)
+        for ctx, st, out in [ref] + list(runs.values()):
+            ctx.decode_step(st, st, ins, out, t)
+        if (t + 1) % every == 0:
+            o_ref = ref[2].double()
+            for label, (ctx, st, out) in runs.items():
+                rsq.rsq_state_drift(ctx.ctx, st, ref[0].ctx, ref[1], sums)
+                s = sums.cpu().numpy()
+                num, den = s[..., 0], s[..., 1]
+                per_head = np.sqrt(num[den > 0] / den[den > 0])
+                o_err = float(torch.linalg.vector_norm(out.double() - o_ref) /
+                              torch.linalg.vector_norm(o_ref))
+                series[label].append([t + 1, float(np.sqrt(num.sum() / den.sum())),
+                                      float(per_head.max()) if per_head.size else 0.0, o_err])
+    for ctx, _, _ in [ref] + list(runs.values()):
+        if ctx.check_flags():
+            raise RuntimeError("non-finite state in the drift study")
+        ctx.close()
+    return series
+
+
+def run_drift(args, w: W.Workload, pool) -> int:
+    import torch
+    torch.cuda.set_device(0)
+    steps = args.drift_steps or w.steps
+    t0 = time.perf_counter()
+    series = drift_series(w, steps, args.drift_every, pool=pool)
+    line = {
+        "metric": "relative state drift ||deq(S_q) - S_fp32||_F / ||S_fp32||_F",
+        "workload": w.name, "batch": w.B, "heads": w.H, "dk": w.dk, "dv": w.dv, "steps": steps,
+        "every": args.drift_every, "start": "S_0 = 0",
+        "reference": "FP32 trajectory: the same kernel with 32-bit heads, identical inputs",
+        "columns": ["step", "global drift", "max per-head drift", "readout relative error"],
+        "series": series, "input_workers": getattr(pool, "_processes", 0),
+        "wall_s": time.perf_counter() - t0,
+    }
+    print(json.dumps(line), flush=True)
     return 0
 
 
@@ -491,8 +602,18 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="override the number of rotated layer states")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--drift", action="store_true",
+                    help="run the long-horizon state drift study instead of the throughput bench")
+    ap.add_argument("--drift-steps", type=int, default=0, help="horizon (default: the workload's)")
+    ap.add_argument("--drift-every", type=int, default=256)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.drift:
+        w = W.BY_NAME[args.workload if args.workload != DEFAULT_WORKLOAD else DRIFT_WORKLOAD]
+        # the input generator pool starts before the first CUDA call
+        import multiprocessing as mp
+        with mp.get_context("spawn").Pool(max(1, min(32, (os.cpu_count() or 2) - 1))) as pool:
+            return run_drift(args, w, pool)
     w = W.BY_NAME[args.workload]
     if args.impl == "reference":
         return run_reference(args, w)
