@@ -22,6 +22,7 @@ from . import build as _build
 
 PLAIN, CANONICAL = 0, 1
 RTN, SR = 0, 1
+BDR, SR_BDR = 2, 3      # nearest / stochastic base rounding + Bounded Directional Rounding
 
 
 class _Head(ctypes.Structure):
@@ -62,6 +63,9 @@ def lib():
         L.orc_quantize_scalar.argtypes = [ctypes.c_float, ctypes.c_float, ctypes.c_int,
                                           ctypes.c_int, ctypes.c_int, ctypes.c_uint32]
         L.orc_quantize_scalar.restype = ctypes.c_int
+        L.orc_bdr_adjust.argtypes = [ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_float,
+                                     ctypes.c_int, ctypes.c_int]
+        L.orc_bdr_adjust.restype = ctypes.c_int
         L.orc_allocate_bits.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, P]
         _lib = L
@@ -100,6 +104,12 @@ def quantize_scalar(S: float, m: float, bits: int, rounding: int, mode: int, u: 
     """Code of one element S of a column with absolute maximum m (> 0), given its uniform u."""
     return int(lib().orc_quantize_scalar(float(S), float(m), int(bits), int(rounding), int(mode),
                                          int(u)))
+
+
+def bdr_adjust(c: int, S: float, prev: float, m: float, bits: int, mode: int = CANONICAL) -> int:
+    """Bounded Directional Rounding of one element: base code c of S (column
+    maximum m), previous dequantized value prev."""
+    return int(lib().orc_bdr_adjust(int(c), float(S), float(prev), float(m), int(bits), int(mode)))
 
 
 def widen(x: np.ndarray) -> np.ndarray:

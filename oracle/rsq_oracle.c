@@ -14,6 +14,10 @@
  *            abstract (state requantized after every update).
  *   [FEED]   "When Dynamic Scaling Fails: A Scale-State Feedback Governs
  *            Recurrent-State Quantization ...", key points (dynamic scale).
+ *   [BDR]    "Preserving Updates in Low-Bit Recurrent State Quantization",
+ *            abstract: Bounded Directional Rounding -- an element whose
+ *            rounding moves it opposite to its update is rounded toward the
+ *            update instead, with no extra storage.
  *   [PHILOX] Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as
  *            1, 2, 3", SC'11 -- Philox4x32-10 block function.
  *   Recurrences: gated delta rule and Mamba-2 scalar-decay SSM as named in
@@ -45,8 +49,13 @@
 
 #define ORC_PLAIN 0
 #define ORC_CANONICAL 1
+/* Rounding: bit 0 selects the base rounding (0 nearest, 1 stochastic); bit 1
+ * adds the directional correction of [BDR] on top of it.                    */
 #define ORC_RTN 0
 #define ORC_SR 1
+#define ORC_BDR 2
+#define ORC_SR_BASE(rnd) ((rnd) & 1)
+#define ORC_HAS_BDR(rnd) (((rnd) & 2) != 0)
 
 /* ------------------------------------------------------------------------- */
 /* Philox4x32-10 [PHILOX]: 10 rounds of two 32x32->64 multiplies; the key is
@@ -165,7 +174,7 @@ int orc_quantize_scalar(float S, float m, int bits, int rounding, int mode, uint
     if (mode == ORC_PLAIN) {
         const float s = m / rf;
         const float x = S / s;
-        if (rounding == ORC_RTN)
+        if (!ORC_SR_BASE(rounding))
             c = (int)rintf(x);
         else
             c = (int)floor((double)x + (double)u / 65536.0);
@@ -173,7 +182,7 @@ int orc_quantize_scalar(float S, float m, int bits, int rounding, int mode, uint
         if (c < -r) c = -r;
     } else {
         const float inv = orc_inv_rz(rf, m);
-        if (rounding == ORC_RTN) {
+        if (!ORC_SR_BASE(rounding)) {
             c = (int)rint((double)S * (double)inv);
         } else {
             const float off = (bits == 8) ? 128.0f : 136.0f;
@@ -185,12 +194,36 @@ int orc_quantize_scalar(float S, float m, int bits, int rounding, int mode, uint
     return c;
 }
 
+/* Bounded Directional Rounding [BDR].  c is the base code of S (column maximum
+ * m, stored scale s_new = m / r); prev is the element's previous dequantized
+ * value c_{t-1} * s_{t-1}.  The update moves the element from prev to S; when
+ * the rounded value c * s_new lies strictly on the other side of prev (a
+ * reversal), the code becomes the integer next to x on the update's side:
+ * ceil(x) for an upward update, floor(x) for a downward one, so the rounding
+ * error stays below one step ("bounded").  x is S / s (plain) or the exact
+ * product S * inv (canonical), as in the base rounding.                     */
+int orc_bdr_adjust(int c, float S, float prev, float m, int bits, int mode)
+{
+    const float rf = (float)orc_rmax(bits);
+    const float s_new = m / rf;
+    const float now = (float)c * s_new;
+    const int up = (S > prev) && (now < prev);
+    const int down = (S < prev) && (now > prev);
+    if (!up && !down) return c;
+    const double x = (mode == ORC_PLAIN) ? (double)(S / s_new) : (double)S * (double)orc_inv_rz(rf, m);
+    int d = up ? (int)ceil(x) : (int)floor(x);
+    const int r = orc_rmax(bits);
+    if (d > r) d = r;
+    if (d < -r) d = -r;
+    return d;
+}
+
 /* Quantize column j of the full-precision state S (dk x dv, row-major) with
  * the dynamic scale computed from S itself: the "noisy" scale of [LoReS]
  * (4/4), through which earlier errors feed back [FEED].                     */
-static void orc_quantize_column(const float* S, int dk, int dv, int j, int bits, int rounding,
-                                int mode, uint64_t seed, uint32_t b, uint32_t h,
-                                uint32_t step, int8_t* codes, float* scale_out)
+static void orc_quantize_column(const float* S, const float* prev, int dk, int dv, int j,
+                                int bits, int rounding, int mode, uint64_t seed, uint32_t b,
+                                uint32_t h, uint32_t step, int8_t* codes, float* scale_out)
 {
     const float rf = (float)orc_rmax(bits);
     /* m_j = max_i |S_ij|; a NaN anywhere in the column makes m NaN. */
@@ -209,8 +242,13 @@ static void orc_quantize_column(const float* S, int dk, int dv, int j, int bits,
     for (int i = 0; i < dk; ++i) {
         int c = 0;
         if (usable) {
-            uint32_t u = (rounding == ORC_SR) ? orc_sr_uniform16(seed, b, h, step, dk, i, j) : 0u;
+            uint32_t u = ORC_SR_BASE(rounding) ? orc_sr_uniform16(seed, b, h, step, dk, i, j) : 0u;
             c = orc_quantize_scalar(S[(int64_t)i * dv + j], m, bits, rounding, mode, u);
+            /* without a previous state (initial quantization) there is no
+             * update direction and the base rounding stands */
+            if (ORC_HAS_BDR(rounding) && prev)
+                c = orc_bdr_adjust(c, S[(int64_t)i * dv + j], prev[(int64_t)i * dv + j], m, bits,
+                                   mode);
         }
         codes[(int64_t)i * dv + j] = (int8_t)c;
     }
@@ -222,7 +260,7 @@ static void orc_quantize_column(const float* S, int dk, int dv, int j, int bits,
 typedef struct {
     int dk, dv;       /* rows (key / SSM-state axis) and columns (value / head-dim axis) */
     int bits;         /* 4, 8 (quantized) or 32 (full-precision state) */
-    int rounding;     /* ORC_RTN or ORC_SR */
+    int rounding;     /* ORC_RTN or ORC_SR, optionally | ORC_BDR */
     int mode;         /* ORC_PLAIN or ORC_CANONICAL */
     int R;            /* canonical partial-sum count (power of two, <= 64); 1 = sequential */
     uint64_t seed;    /* stochastic-rounding key */
@@ -286,8 +324,12 @@ int orc_gdn_head_step(const orc_head* hd, const int8_t* c_in, const float* s_in,
     if (hd->bits == 32) {
         for (int64_t t = 0; t < (int64_t)dk * dv; ++t) f_out[t] = S[t];
     } else {
+        /* previous dequantized values c_{t-1} s_{t-1} (the directional rounding's reference) */
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j)
+                Sh[(int64_t)i * dv + j] = (float)c_in[(int64_t)i * dv + j] * s_in[j];
         for (int j = 0; j < dv; ++j)
-            orc_quantize_column(S, dk, dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
+            orc_quantize_column(S, Sh, dk, dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
                                 hd->b, hd->h, hd->step, c_out, &s_out[j]);
     }
     free(S); free(Sh); free(cf);
@@ -306,7 +348,8 @@ int orc_mamba2_head_step(const orc_head* hd, const int8_t* c_in, const float* s_
     const int R = (hd->mode == ORC_PLAIN) ? 1 : hd->R;
     float* S = (float*)malloc(sizeof(float) * (size_t)dk * (size_t)dv);
     float* cf = (float*)malloc(sizeof(float) * (size_t)dk * (size_t)dv);
-    if (!S || !cf) { free(S); free(cf); return 1; }
+    float* Sh = (float*)malloc(sizeof(float) * (size_t)dk * (size_t)dv);
+    if (!S || !cf || !Sh) { free(S); free(cf); free(Sh); return 1; }
     const float a = (decay >= 0.0f) ? decay : expf(dt * A);
 
     if (hd->bits == 32) {
@@ -339,11 +382,14 @@ int orc_mamba2_head_step(const orc_head* hd, const int8_t* c_in, const float* s_
     if (hd->bits == 32) {
         for (int64_t t = 0; t < (int64_t)dk * dv; ++t) f_out[t] = S[t];
     } else {
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j)
+                Sh[(int64_t)i * dv + j] = (float)c_in[(int64_t)i * dv + j] * s_in[j];
         for (int j = 0; j < dv; ++j)
-            orc_quantize_column(S, dk, dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
+            orc_quantize_column(S, Sh, dk, dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
                                 hd->b, hd->h, hd->step, c_out, &s_out[j]);
     }
-    free(S); free(cf);
+    free(S); free(cf); free(Sh);
     return 0;
 }
 
@@ -353,8 +399,8 @@ int orc_quantize_head(const orc_head* hd, const float* S, int8_t* c_out, float* 
 {
     if (hd->bits != 4 && hd->bits != 8) return 1;
     for (int j = 0; j < hd->dv; ++j)
-        orc_quantize_column(S, hd->dk, hd->dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
-                            hd->b, hd->h, hd->step, c_out, &s_out[j]);
+        orc_quantize_column(S, NULL, hd->dk, hd->dv, j, hd->bits, hd->rounding, hd->mode,
+                            hd->seed, hd->b, hd->h, hd->step, c_out, &s_out[j]);
     return 0;
 }
 

@@ -511,3 +511,82 @@ def test_pack_roundtrip_mixed():
     back = oracle.unpack_state(buf, st["scales"], hb, B, H, dk, dv)
     assert np.array_equal(back["codes"][:, :2], st["codes"][:, :2])
     assert np.array_equal(back["f"][:, 2], st["f"][:, 2])
+
+
+# ---------------------------------------------------------------------------
+# Bounded Directional Rounding ("Preserving Updates in Low-Bit Recurrent State
+# Quantization", abstract): an element whose rounding moves it opposite to its
+# update is rounded toward the update instead; the error stays below one step.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
+def test_bdr_worked_scalar_cases(mode):
+    """Column maximum 127 at 8 bits: scale 1, so x = S.  Hand-derived cases."""
+    m = 127.0
+    rtn = lambda S: oracle.quantize_scalar(S, m, 8, oracle.RTN, mode)
+    # update +0.1 from 0.3 to 0.4: nearest rounding gives 0, below the old value -> reversed -> 1
+    assert rtn(0.4) == 0 and oracle.bdr_adjust(0, 0.4, 0.3, m, 8, mode) == 1
+    # the mirror image: from -0.3 down to -0.4
+    assert oracle.bdr_adjust(0, -0.4, -0.3, m, 8, mode) == -1
+    # update from 0.5 down to 0.4: rounding to 0 moves down as well -> kept
+    assert oracle.bdr_adjust(0, 0.4, 0.5, m, 8, mode) == 0
+    # a lost update (0.0 -> 0.4 rounds back to 0.0) is not a reversal -> kept
+    assert oracle.bdr_adjust(0, 0.4, 0.0, m, 8, mode) == 0
+    # no update: kept whatever the code
+    assert oracle.bdr_adjust(3, 2.6, 2.6, m, 8, mode) == 3
+    # next to the column maximum the corrected code is still within [-r, r]
+    assert oracle.bdr_adjust(126, 126.4, 126.3, m, 8, mode) == 127
+
+
+def _one_step_f64(st, inp, b, h):
+    """Full-precision update of the previous dequantized state, in float64 (the
+    gated delta rule written out: S = alpha S^ + k (beta (v - alpha S^T k))^T)."""
+    Sh = (st["codes"][b, h].astype(np.float64) * st["scales"][b, h].astype(np.float64))
+    k = oracle.widen(inp["k"])[b, h].astype(np.float64)
+    v = oracle.widen(inp["v"])[b, h].astype(np.float64)
+    a, be = float(inp["alpha"][b, h]), float(inp["beta"][b, h])
+    w = be * (v - a * (Sh.T @ k))
+    return a * Sh + np.outer(k, w), Sh
+
+
+@pytest.mark.parametrize("base", [oracle.RTN, oracle.SR])
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
+def test_bdr_properties_on_trajectories(base, bits, mode):
+    """On free-running trajectories, against the base rounding from the same state:
+    (1) scales are unchanged and codes move by at most one step (bounded);
+    (2) no element is left moving opposite to its update (checked against a
+        float64 update, away from ties);
+    (3) where the base rounding had no reversal the code is the base code;
+    (4) reversals of the base rounding occur and every one is corrected."""
+    w = dataclasses.replace(TINY, B=2, H=2, dk=16, dv=16)
+    hb = np.full(w.H, bits, np.int8)
+    st = oracle.zero_state(w.B, w.H, w.dk, w.dv)
+    n_rev = n_fixed = 0
+    for t in range(40):
+        inp = W.gdn_inputs(w, t)
+        kw = dict(seed=91, step=t, mode=mode)
+        nb, _ = oracle.gdn_step(st, inp, hb, rounding=base, **kw)
+        nd, _ = oracle.gdn_step(st, inp, hb, rounding=base | oracle.BDR, **kw)
+        assert np.array_equal(nb["scales"], nd["scales"])
+        dc = nd["codes"].astype(int) - nb["codes"].astype(int)
+        assert np.abs(dc).max() <= 1
+        for b in range(w.B):
+            for h in range(w.H):
+                S, prev = _one_step_f64(st, inp, b, h)
+                s = nd["scales"][b, h].astype(np.float64)
+                scale = np.abs(S).max()
+                tol = 1e-5 * max(scale, 1e-30)
+                clear = (np.abs(S - prev) > tol)
+                up, down = clear & (S > prev), clear & (S < prev)
+                base_now = nb["codes"][b, h] * s
+                bdr_now = nd["codes"][b, h] * s
+                far = lambda now: np.abs(now - prev) > tol
+                rev_base = (up & (base_now < prev) & far(base_now)) | (down & (base_now > prev) & far(base_now))
+                rev_bdr = (up & (bdr_now < prev) & far(bdr_now)) | (down & (bdr_now > prev) & far(bdr_now))
+                assert not rev_bdr.any()
+                ok_base = clear & ~rev_base & ~(np.abs(base_now - prev) <= tol)
+                assert np.array_equal(nd["codes"][b, h][ok_base], nb["codes"][b, h][ok_base])
+                n_rev += int(rev_base.sum())
+                n_fixed += int((rev_base & (dc[b, h] != 0)).sum())
+        st = nd
+    assert n_rev > 0 and n_fixed == n_rev
