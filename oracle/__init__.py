@@ -53,6 +53,9 @@ def lib():
                                            ctypes.c_float, ctypes.c_float, ctypes.c_float, P, P,
                                            P, P]
         L.orc_mamba2_head_step.restype = ctypes.c_int
+        L.orc_diag_head_step.argtypes = [ctypes.POINTER(_Head), ctypes.c_int, P, P, P, P, P, P, P,
+                                         ctypes.c_float, P, P, P, P]
+        L.orc_diag_head_step.restype = ctypes.c_int
         L.orc_quantize_head.argtypes = [ctypes.POINTER(_Head), P, P, P]
         L.orc_quantize_head.restype = ctypes.c_int
         L.orc_dequantize_head.argtypes = [ctypes.c_int, ctypes.c_int, P, P, P]
@@ -227,6 +230,50 @@ def mamba2_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, 
             new["scales"][b, h] = s_out
         y[b, h] = y_h
     return new, y
+
+
+def _diag_step(delta: int, state: dict, inp: dict, head_bits, rounding, seed, step, mode, R, heads):
+    B, H, dk, dv = state["codes"].shape
+    q, k, v = widen(inp["q"]), widen(inp["k"]), widen(inp["v"])
+    alpha = _c(inp["alpha"], np.float32)            # [B][H][dk]
+    beta = _c(inp["beta"], np.float32) if delta else np.zeros((B, H), np.float32)
+    new = copy_state(state)
+    o = np.zeros((B, H, dv), np.float32)
+    L = lib()
+    for b, h in _heads(B, H, heads):
+        bits = int(head_bits[h])
+        hd = _head(dk, dv, bits, rounding, mode, R, seed, b, h, step)
+        c_in, s_in, f_in = (_c(state["codes"][b, h], np.int8), _c(state["scales"][b, h], np.float32),
+                            _f_in(state, b, h, dk, dv))
+        c_out = np.zeros((dk, dv), np.int8)
+        s_out = np.zeros(dv, np.float32)
+        f_out = np.zeros((dk, dv), np.float32)
+        o_h = np.zeros(dv, np.float32)
+        qh, kh, vh = _c(q[b, h], np.float32), _c(k[b, h], np.float32), _c(v[b, h], np.float32)
+        ah = _c(alpha[b, h], np.float32)
+        rc = L.orc_diag_head_step(ctypes.byref(hd), int(delta), _p(c_in), _p(s_in), _p(f_in), _p(qh),
+                                  _p(kh), _p(vh), _p(ah), float(beta[b, h]), _p(c_out), _p(s_out),
+                                  _p(f_out), _p(o_h))
+        assert rc == 0
+        if bits == 32:
+            new["f"][b, h] = f_out
+        else:
+            new["codes"][b, h] = c_out
+            new["scales"][b, h] = s_out
+        o[b, h] = o_h
+    return new, o
+
+
+def gla_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, step: int,
+             mode: int = CANONICAL, R: int = 8, heads=None):
+    """One GLA decode step (decay vector alpha [B][H][dk] over the key axis, no delta rule)."""
+    return _diag_step(0, state, inp, head_bits, rounding, seed, step, mode, R, heads)
+
+
+def kda_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, step: int,
+             mode: int = CANONICAL, R: int = 8, heads=None):
+    """One KDA decode step (delta rule with a decay vector alpha [B][H][dk] and gate beta [B][H])."""
+    return _diag_step(1, state, inp, head_bits, rounding, seed, step, mode, R, heads)
 
 
 def quantize(S: np.ndarray, head_bits, *, rounding: int, seed: int, step: int,

@@ -21,7 +21,11 @@
  *   [PHILOX] Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as
  *            1, 2, 3", SC'11 -- Philox4x32-10 block function.
  *   Recurrences: gated delta rule and Mamba-2 scalar-decay SSM as named in
- *   [LRB] abstract and [LoReS] Table 1.
+ *   [LRB] abstract and [LoReS] Table 1; GLA (gated linear attention, a decay
+ *   per key channel) and KDA (the delta rule with a decay per key channel),
+ *   the diagonal-decay mixers of [LoReS] Table 1 / "Decayed recurrences are
+ *   robust" (RetNet and plain linear attention are the Mamba-2 step with a
+ *   constant decay, dt = 1 and D = 0).
  *
  * Orientation.  The state of one head is stored with the key / SSM-state axis i
  * as rows (dk rows) and the value / head-dim axis j as columns (dv columns):
@@ -390,6 +394,80 @@ int orc_mamba2_head_step(const orc_head* hd, const int8_t* c_in, const float* s_
                                 hd->b, hd->h, hd->step, c_out, &s_out[j]);
     }
     free(S); free(cf); free(Sh);
+    return 0;
+}
+
+/* Diagonal-decay recurrences ([LoReS] Table 1: GLA, KDA).  alpha is the decay
+ * vector over the key axis (dk entries in (0, 1)).
+ *   GLA:  S_t = diag(alpha) S_{t-1} + k v^T,                         o = S_t^T q
+ *   KDA:  S_t = (I - beta k k^T) diag(alpha) S_{t-1} + beta k v^T,    o = S_t^T q
+ * KDA in steps: D = diag(alpha) S^, u = D^T k, w = beta (v - u), S = D + k w^T.
+ * Canonical c-form (s_j = 1 for a full-precision state):
+ *   GLA  S_ij = fma(c_ij, alpha_i s_j, k_i v_j)
+ *   KDA  u_j = s_j * sum_i c_ij (alpha_i k_i),  w_j = beta (v_j - u_j),
+ *        S_ij = fma(c_ij, alpha_i s_j, k_i w_j)
+ * Plain: dequantize S^ = c s, then D_ij = alpha_i S^_ij, sequential sums,
+ * S_ij = fma(k_i, w_j, D_ij).                                              */
+int orc_diag_head_step(const orc_head* hd, int delta, const int8_t* c_in, const float* s_in,
+                       const float* f_in, const float* q, const float* k, const float* v,
+                       const float* alpha, float beta, int8_t* c_out, float* s_out,
+                       float* f_out, float* o)
+{
+    const int dk = hd->dk, dv = hd->dv;
+    const int R = (hd->mode == ORC_PLAIN) ? 1 : hd->R;
+    const size_t n = (size_t)dk * (size_t)dv;
+    float* S = (float*)malloc(sizeof(float) * n);
+    float* Sh = (float*)malloc(sizeof(float) * n);
+    float* cf = (float*)malloc(sizeof(float) * n);
+    float* ak = (float*)malloc(sizeof(float) * (size_t)dk);
+    if (!S || !Sh || !cf || !ak) { free(S); free(Sh); free(cf); free(ak); return 1; }
+    for (int i = 0; i < dk; ++i) ak[i] = alpha[i] * k[i];
+
+    if (hd->bits != 32 && hd->mode == ORC_PLAIN) {
+        /* dequantize, decay, then the (delta) update in the literal order */
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j)
+                Sh[(int64_t)i * dv + j] = alpha[i] * ((float)c_in[(int64_t)i * dv + j] * s_in[j]);
+        for (int j = 0; j < dv; ++j) {
+            float w = v[j];
+            if (delta) {
+                const float u = orc_dot_rows(Sh + j, dv, k, dk, 1); /* u = D^T k */
+                w = beta * (v[j] - u);
+            }
+            for (int i = 0; i < dk; ++i)
+                S[(int64_t)i * dv + j] = fmaf(k[i], w, Sh[(int64_t)i * dv + j]);
+        }
+    } else {
+        /* canonical c-form; a full-precision state is its own "code" with s = 1 */
+        for (size_t t = 0; t < n; ++t) cf[t] = (hd->bits == 32) ? f_in[t] : (float)c_in[t];
+        for (int j = 0; j < dv; ++j) {
+            const float sj = (hd->bits == 32) ? 1.0f : s_in[j];
+            float w = v[j];
+            if (delta) {
+                const float ck = orc_dot_rows(cf + j, dv, ak, dk, R);
+                const float u = (hd->bits == 32) ? ck : sj * ck;
+                w = beta * (v[j] - u);
+            }
+            for (int i = 0; i < dk; ++i) {
+                const float a = (hd->bits == 32) ? alpha[i] : alpha[i] * sj;
+                S[(int64_t)i * dv + j] = fmaf(cf[(int64_t)i * dv + j], a, k[i] * w);
+            }
+        }
+    }
+    for (int j = 0; j < dv; ++j)
+        o[j] = orc_dot_rows(S + j, dv, q, dk, R);
+
+    if (hd->bits == 32) {
+        for (size_t t = 0; t < n; ++t) f_out[t] = S[t];
+    } else {
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j)
+                Sh[(int64_t)i * dv + j] = (float)c_in[(int64_t)i * dv + j] * s_in[j];
+        for (int j = 0; j < dv; ++j)
+            orc_quantize_column(S, Sh, dk, dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
+                                hd->b, hd->h, hd->step, c_out, &s_out[j]);
+    }
+    free(S); free(Sh); free(cf); free(ak);
     return 0;
 }
 

@@ -590,3 +590,81 @@ def test_bdr_properties_on_trajectories(base, bits, mode):
                 n_fixed += int((rev_base & (dc[b, h] != 0)).sum())
         st = nd
     assert n_rev > 0 and n_fixed == n_rev
+
+
+# ---------------------------------------------------------------------------
+# Diagonal-decay recurrences of the mixer zoo (LoReS Table 1: GLA, KDA)
+# ---------------------------------------------------------------------------
+TINY_GLA = dataclasses.replace(W.BY_NAME["gla_b64_h16_d128_int8_sr"], B=1, H=2, dk=16, dv=16,
+                               in_dtype="f32")
+TINY_KDA = dataclasses.replace(W.BY_NAME["kda_b64_h16_d128_int8_sr"], B=1, H=2, dk=16, dv=16,
+                               in_dtype="f32")
+
+
+def _gla_closed_form(ins, t_end, b, h):
+    """S_t = sum_tau diag(prod_{s=tau+1..t} alpha_s) k_tau v_tau^T (cumulative decay products)."""
+    S = 0.0
+    for tau in range(t_end):
+        decay = np.ones(ins[0]["alpha"].shape[-1])
+        for s in range(tau + 1, t_end):
+            decay *= np.asarray(ins[s]["alpha"][b, h], np.float64)
+        S = S + np.outer(decay * np.asarray(ins[tau]["k"][b, h], np.float64),
+                         np.asarray(ins[tau]["v"][b, h], np.float64))
+    return S
+
+
+def _kda_closed_form(ins, t_end, b, h):
+    """S_t = sum_tau [prod_{s=tau+1..t} (I - beta_s k_s k_s^T) diag(alpha_s)] beta_tau k_tau v_tau^T."""
+    S = 0.0
+    for tau in range(t_end):
+        k0 = np.asarray(ins[tau]["k"][b, h], np.float64)
+        M = float(ins[tau]["beta"][b, h]) * np.outer(k0, np.asarray(ins[tau]["v"][b, h], np.float64))
+        for s in range(tau + 1, t_end):
+            a = np.asarray(ins[s]["alpha"][b, h], np.float64)
+            ks = np.asarray(ins[s]["k"][b, h], np.float64)
+            Dm = a[:, None] * M
+            M = Dm - float(ins[s]["beta"][b, h]) * np.outer(ks, ks @ Dm)
+        S = S + M
+    return S
+
+
+@pytest.mark.parametrize("family", ["gla", "kda"])
+@pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
+def test_diag_decay_fp32_state_matches_closed_form(family, mode):
+    """(a) for the diagonal-decay mixers: with quantization disabled the state and
+    readout equal the unrolled sums of decayed outer products."""
+    w = TINY_GLA if family == "gla" else TINY_KDA
+    step = oracle.gla_step if family == "gla" else oracle.kda_step
+    close = _gla_closed_form if family == "gla" else _kda_closed_form
+    T = 48
+    ins = [W.inputs(w, t) for t in range(T)]
+    hb = np.full(w.H, 32, np.int8)
+    st = oracle.zero_state(w.B, w.H, w.dk, w.dv)
+    for t in range(T):
+        st, o = step(st, ins[t], hb, rounding=0, seed=0, step=t, mode=mode)
+        if (t + 1) % 8 == 0:
+            for h in range(w.H):
+                ref = close(ins, t + 1, 0, h)
+                assert _rel(st["f"][0, h], ref) <= 1e-5
+                assert _rel(o[0, h], ref.T @ np.asarray(ins[t]["q"][0, h], np.float64)) <= 1e-5
+
+
+def test_gla_constant_decay_is_the_scalar_decay_step():
+    """GLA with the same decay on every key channel is RetNet's recurrence, i.e.
+    the Mamba-2 step with B = k, C = q, x = v, dt = 1, decay = gamma and D = 0:
+    both evaluation orders reduce to the same operations, state for state."""
+    w = dataclasses.replace(TINY_GLA, B=2, H=3)
+    hb = np.array([8, 4, 32], np.int8)
+    a = oracle.zero_state(w.B, w.H, w.dk, w.dv)
+    m = oracle.zero_state(w.B, w.H, w.dk, w.dv)
+    for t in range(12):
+        inp = W.inputs(w, t)
+        gamma = inp["alpha"][:, :, 0].copy()
+        inp["alpha"] = np.repeat(gamma[:, :, None], w.dk, axis=2)
+        a, o_a = oracle.gla_step(a, inp, hb, rounding=oracle.SR, seed=5, step=t)
+        mi = {"x": inp["v"], "Bm": inp["k"], "Cm": inp["q"], "dt": np.ones((w.B, w.H), np.float32),
+              "A": np.zeros(w.H, np.float32), "D": np.zeros(w.H, np.float32)}
+        m, o_m = oracle.mamba2_step(m, mi, hb, rounding=oracle.SR, seed=5, step=t, ngroups=w.H,
+                                    decay=gamma)
+        assert np.array_equal(a["codes"], m["codes"]) and np.array_equal(a["scales"], m["scales"])
+        assert np.array_equal(a["f"], m["f"]) and np.array_equal(o_a, o_m)

@@ -12,6 +12,9 @@ Input distributions follow the five workloads the method is evaluated on:
   v ~ N(0, 1), alpha = sigmoid(N(3, 1)), beta = sigmoid(N(0, 1)).
 * Mamba-2: A_h = -exp(U(0, 2.8)), dt = softplus(N(-2, 1)), x, B, C ~ N(0, 1),
   D_h ~ N(1, 0.1).
+* GLA / KDA (diagonal decay): q, k, v as for Gated DeltaNet, a decay per key
+  channel alpha_i = sigmoid(N(3, 1)) (the GDN gate law per channel), and for
+  KDA beta = sigmoid(N(0, 1)).
 
 Every quantity of every decode step is drawn from its own numpy stream keyed
 on (input_seed, step, quantity), so any step can be regenerated alone and any
@@ -32,7 +35,7 @@ class Workload:
     """One decode workload: family, shapes, horizon, state format, input law."""
 
     name: str
-    family: str          # "gdn" or "mamba2"
+    family: str          # "gdn", "mamba2", "gla" or "kda"
     B: int               # batch (independent requests)
     H: int               # heads
     dk: int              # GDN key dim d_k; Mamba-2 state dim N (rows of the stored state)
@@ -65,7 +68,14 @@ WORKLOADS = [
     Workload("gdn_b1024_h16_d128_int4_sr_long", "gdn", 1024, 16, 128, 128, 4096, "int4", "sr",
              "bf16", input_seed=4, sr_seed=1004),
 ]
-BY_NAME = {w.name: w for w in WORKLOADS}
+# Further recurrence families on the decode shape of the benchmark workload.
+EXTRA_WORKLOADS = [
+    Workload("gla_b64_h16_d128_int8_sr", "gla", 64, 16, 128, 128, 1024, "int8", "sr", "bf16",
+             input_seed=5, sr_seed=1005),
+    Workload("kda_b64_h16_d128_int8_sr", "kda", 64, 16, 128, 128, 1024, "int8", "sr", "bf16",
+             input_seed=6, sr_seed=1006),
+]
+BY_NAME = {w.name: w for w in WORKLOADS + EXTRA_WORKLOADS}
 
 
 def _rng(seed: int, step: int, qty: int) -> np.random.Generator:
@@ -129,6 +139,24 @@ def gdn_inputs(w: Workload, step: int, B: int | None = None) -> dict:
     }
 
 
+def diag_inputs(w: Workload, step: int, B: int | None = None) -> dict:
+    """Inputs of one GLA / KDA decode step: q, k: [B][H][dk], v: [B][H][dv]
+    (float32 or bf16 bits), alpha: [B][H][dk] float32 (decay per key channel),
+    beta: [B][H] float32 (KDA only)."""
+    assert w.family in ("gla", "kda")
+    B = w.B if B is None else B
+    s = w.input_seed
+    q = _rng(s, step, _Q).standard_normal((w.B, w.H, w.dk), dtype=np.float32)[:B]
+    k = _rng(s, step, _K).standard_normal((w.B, w.H, w.dk), dtype=np.float32)[:B]
+    v = _rng(s, step, _V).standard_normal((w.B, w.H, w.dv), dtype=np.float32)[:B]
+    alpha = _sigmoid(_rng(s, step, _ALPHA).normal(3.0, 1.0, (w.B, w.H, w.dk)))[:B]
+    out = {"q": _vec(w, _l2_normalise(q)), "k": _vec(w, _l2_normalise(k)), "v": _vec(w, v),
+           "alpha": np.ascontiguousarray(alpha)}
+    if w.family == "kda":
+        out["beta"] = np.ascontiguousarray(_sigmoid(_rng(s, step, _BETA).normal(0.0, 1.0, (w.B, w.H)))[:B])
+    return out
+
+
 def gdn_alpha(w: Workload, step: int) -> np.ndarray:
     """Only the alpha gates of one GDN step ([B][H] float32), same values as gdn_inputs."""
     return _sigmoid(_rng(w.input_seed, step, _ALPHA).normal(3.0, 1.0, (w.B, w.H)))
@@ -162,7 +190,11 @@ def mamba2_inputs(w: Workload, step: int, B: int | None = None) -> dict:
 
 
 def inputs(w: Workload, step: int, B: int | None = None) -> dict:
-    return gdn_inputs(w, step, B) if w.family == "gdn" else mamba2_inputs(w, step, B)
+    if w.family == "gdn":
+        return gdn_inputs(w, step, B)
+    if w.family == "mamba2":
+        return mamba2_inputs(w, step, B)
+    return diag_inputs(w, step, B)
 
 
 def mean_alpha_per_head(w: Workload, steps: int | None = None) -> np.ndarray:
