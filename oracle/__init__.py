@@ -29,7 +29,7 @@ class _Head(ctypes.Structure):
     _fields_ = [("dk", ctypes.c_int), ("dv", ctypes.c_int), ("bits", ctypes.c_int),
                 ("rounding", ctypes.c_int), ("mode", ctypes.c_int), ("R", ctypes.c_int),
                 ("seed", ctypes.c_uint64), ("b", ctypes.c_uint32), ("h", ctypes.c_uint32),
-                ("step", ctypes.c_uint32)]
+                ("step", ctypes.c_uint32), ("m_copy", ctypes.c_void_p)]
 
 
 _lib = None
@@ -162,11 +162,12 @@ def _heads(B, H, heads):
 # Decode steps
 # ---------------------------------------------------------------------------
 def gdn_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, step: int,
-             mode: int = CANONICAL, R: int = 8, heads=None):
+             mode: int = CANONICAL, R: int = 8, heads=None, copy_absmax=None):
     """One Gated DeltaNet decode step over the given (b, h) heads (default: all).
 
     Returns (new_state, o) with o float32 [B][H][dv]; heads not processed keep
-    their old state and a zero output.
+    their old state and a zero output.  ``copy_absmax`` ([B][H][dv] float32)
+    switches to the copy scale: the column maxima of an unquantized copy.
     """
     B, H, dk, dv = state["codes"].shape
     q, k, v = widen(inp["q"]), widen(inp["k"]), widen(inp["v"])
@@ -177,6 +178,10 @@ def gdn_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, ste
     for b, h in _heads(B, H, heads):
         bits = int(head_bits[h])
         hd = _head(dk, dv, bits, rounding, mode, R, seed, b, h, step)
+        mc = None
+        if copy_absmax is not None:
+            mc = _c(copy_absmax[b, h], np.float32)
+            hd.m_copy = mc.ctypes.data
         c_in, s_in, f_in = (_c(state["codes"][b, h], np.int8), _c(state["scales"][b, h], np.float32),
                             _f_in(state, b, h, dk, dv))
         c_out = np.zeros((dk, dv), np.int8)
@@ -198,7 +203,8 @@ def gdn_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, ste
 
 
 def mamba2_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, step: int,
-                mode: int = CANONICAL, R: int = 8, ngroups: int = 1, decay=None, heads=None):
+                mode: int = CANONICAL, R: int = 8, ngroups: int = 1, decay=None, heads=None,
+                copy_absmax=None):
     """One Mamba-2 decode step.  ``decay`` ([B][H] float32) replaces exp(dt*A) when given."""
     B, H, dk, dv = state["codes"].shape
     x, Bm, Cm = widen(inp["x"]), widen(inp["Bm"]), widen(inp["Cm"])
@@ -211,6 +217,10 @@ def mamba2_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, 
         bits = int(head_bits[h])
         g = h // heads_per_group
         hd = _head(dk, dv, bits, rounding, mode, R, seed, b, h, step)
+        mc = None
+        if copy_absmax is not None:
+            mc = _c(copy_absmax[b, h], np.float32)
+            hd.m_copy = mc.ctypes.data
         c_in, s_in, f_in = (_c(state["codes"][b, h], np.int8), _c(state["scales"][b, h], np.float32),
                             _f_in(state, b, h, dk, dv))
         c_out = np.zeros((dk, dv), np.int8)
@@ -232,7 +242,8 @@ def mamba2_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, 
     return new, y
 
 
-def _diag_step(delta: int, state: dict, inp: dict, head_bits, rounding, seed, step, mode, R, heads):
+def _diag_step(delta: int, state: dict, inp: dict, head_bits, rounding, seed, step, mode, R, heads,
+               copy_absmax=None):
     B, H, dk, dv = state["codes"].shape
     q, k, v = widen(inp["q"]), widen(inp["k"]), widen(inp["v"])
     alpha = _c(inp["alpha"], np.float32)            # [B][H][dk]
@@ -243,6 +254,10 @@ def _diag_step(delta: int, state: dict, inp: dict, head_bits, rounding, seed, st
     for b, h in _heads(B, H, heads):
         bits = int(head_bits[h])
         hd = _head(dk, dv, bits, rounding, mode, R, seed, b, h, step)
+        mc = None
+        if copy_absmax is not None:
+            mc = _c(copy_absmax[b, h], np.float32)
+            hd.m_copy = mc.ctypes.data
         c_in, s_in, f_in = (_c(state["codes"][b, h], np.int8), _c(state["scales"][b, h], np.float32),
                             _f_in(state, b, h, dk, dv))
         c_out = np.zeros((dk, dv), np.int8)
@@ -265,20 +280,21 @@ def _diag_step(delta: int, state: dict, inp: dict, head_bits, rounding, seed, st
 
 
 def gla_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, step: int,
-             mode: int = CANONICAL, R: int = 8, heads=None):
+             mode: int = CANONICAL, R: int = 8, heads=None, copy_absmax=None):
     """One GLA decode step (decay vector alpha [B][H][dk] over the key axis, no delta rule)."""
-    return _diag_step(0, state, inp, head_bits, rounding, seed, step, mode, R, heads)
+    return _diag_step(0, state, inp, head_bits, rounding, seed, step, mode, R, heads, copy_absmax)
 
 
 def kda_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, step: int,
-             mode: int = CANONICAL, R: int = 8, heads=None):
+             mode: int = CANONICAL, R: int = 8, heads=None, copy_absmax=None):
     """One KDA decode step (delta rule with a decay vector alpha [B][H][dk] and gate beta [B][H])."""
-    return _diag_step(1, state, inp, head_bits, rounding, seed, step, mode, R, heads)
+    return _diag_step(1, state, inp, head_bits, rounding, seed, step, mode, R, heads, copy_absmax)
 
 
 def quantize(S: np.ndarray, head_bits, *, rounding: int, seed: int, step: int,
-             mode: int = CANONICAL) -> dict:
-    """Quantize a full-precision state [B][H][dk][dv]; 32-bit heads are copied."""
+             mode: int = CANONICAL, copy_absmax=None) -> dict:
+    """Quantize a full-precision state [B][H][dk][dv]; 32-bit heads are copied.
+    ``copy_absmax`` ([B][H][dv]) replaces each column's own maximum in the scale."""
     B, H, dk, dv = S.shape
     st = zero_state(B, H, dk, dv, fp32=any(int(b) == 32 for b in head_bits))
     L = lib()
@@ -289,6 +305,10 @@ def quantize(S: np.ndarray, head_bits, *, rounding: int, seed: int, step: int,
                 st["f"][b, h] = S[b, h]
                 continue
             hd = _head(dk, dv, bits, rounding, mode, 1, seed, b, h, step)
+            mc = None
+            if copy_absmax is not None:
+                mc = _c(copy_absmax[b, h], np.float32)
+                hd.m_copy = mc.ctypes.data
             src = _c(S[b, h], np.float32)
             c_out = np.zeros((dk, dv), np.int8)
             s_out = np.zeros(dv, np.float32)

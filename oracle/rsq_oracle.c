@@ -224,10 +224,16 @@ int orc_bdr_adjust(int c, float S, float prev, float m, int bits, int mode)
 
 /* Quantize column j of the full-precision state S (dk x dv, row-major) with
  * the dynamic scale computed from S itself: the "noisy" scale of [LoReS]
- * (4/4), through which earlier errors feed back [FEED].                     */
-static void orc_quantize_column(const float* S, const float* prev, int dk, int dv, int j,
-                                int bits, int rounding, int mode, uint64_t seed, uint32_t b,
-                                uint32_t h, uint32_t step, int8_t* codes, float* scale_out)
+ * (4/4), through which earlier errors feed back [FEED].
+ * Copy scale ([LoReS] (4/4), animation details; the ablation of [FEED]): when
+ * m_copy is given, the scale is *m_copy / r, the column maximum of an
+ * unquantized copy of the state, instead; the state is first clipped to
+ * [-m_copy, m_copy], so elements beyond it get the codes +-r.  The column's
+ * own maximum still decides whether it is finite.                          */
+static void orc_quantize_column(const float* S, const float* prev, const float* m_copy, int dk,
+                                int dv, int j, int bits, int rounding, int mode, uint64_t seed,
+                                uint32_t b, uint32_t h, uint32_t step, int8_t* codes,
+                                float* scale_out)
 {
     const float rf = (float)orc_rmax(bits);
     /* m_j = max_i |S_ij|; a NaN anywhere in the column makes m NaN. */
@@ -239,20 +245,25 @@ static void orc_quantize_column(const float* S, const float* prev, int dk, int d
         else if (a > m)
             m = a;
     }
-    *scale_out = m / rf; /* s_j = max_i |S_ij| / r */
+    const float ms = m_copy ? *m_copy : m; /* the maximum the scale is taken from */
+    *scale_out = ms / rf;                  /* s_j = max_i |S_ij| / r */
     /* An all-zero column has scale 0 and codes 0; a non-finite column keeps
      * its non-finite scale and gets codes 0.                                */
-    const int usable = (m > 0.0f) && isfinite(m);
+    const int usable = (ms > 0.0f) && isfinite(ms) && isfinite(m);
+    const int r = orc_rmax(bits);
     for (int i = 0; i < dk; ++i) {
         int c = 0;
         if (usable) {
+            float x = S[(int64_t)i * dv + j];
+            if (m_copy) x = fminf(fmaxf(x, -ms), ms); /* clip to the copy's range */
             uint32_t u = ORC_SR_BASE(rounding) ? orc_sr_uniform16(seed, b, h, step, dk, i, j) : 0u;
-            c = orc_quantize_scalar(S[(int64_t)i * dv + j], m, bits, rounding, mode, u);
+            c = orc_quantize_scalar(x, ms, bits, rounding, mode, u);
             /* without a previous state (initial quantization) there is no
              * update direction and the base rounding stands */
             if (ORC_HAS_BDR(rounding) && prev)
-                c = orc_bdr_adjust(c, S[(int64_t)i * dv + j], prev[(int64_t)i * dv + j], m, bits,
-                                   mode);
+                c = orc_bdr_adjust(c, x, prev[(int64_t)i * dv + j], ms, bits, mode);
+            if (c > r) c = r; /* plain order: S/s may exceed r by a rounding */
+            if (c < -r) c = -r;
         }
         codes[(int64_t)i * dv + j] = (int8_t)c;
     }
@@ -269,6 +280,7 @@ typedef struct {
     int R;            /* canonical partial-sum count (power of two, <= 64); 1 = sequential */
     uint64_t seed;    /* stochastic-rounding key */
     uint32_t b, h, step;
+    const float* m_copy; /* copy scale: dv column maxima of an unquantized copy, or NULL */
 } orc_head;
 
 /* Gated delta rule decode step ([LRB] abstract: Gated DeltaNet; the LoReS
@@ -333,7 +345,8 @@ int orc_gdn_head_step(const orc_head* hd, const int8_t* c_in, const float* s_in,
             for (int j = 0; j < dv; ++j)
                 Sh[(int64_t)i * dv + j] = (float)c_in[(int64_t)i * dv + j] * s_in[j];
         for (int j = 0; j < dv; ++j)
-            orc_quantize_column(S, Sh, dk, dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
+            orc_quantize_column(S, Sh, hd->m_copy ? hd->m_copy + j : NULL, dk, dv, j, hd->bits,
+                                hd->rounding, hd->mode, hd->seed,
                                 hd->b, hd->h, hd->step, c_out, &s_out[j]);
     }
     free(S); free(Sh); free(cf);
@@ -390,7 +403,8 @@ int orc_mamba2_head_step(const orc_head* hd, const int8_t* c_in, const float* s_
             for (int j = 0; j < dv; ++j)
                 Sh[(int64_t)i * dv + j] = (float)c_in[(int64_t)i * dv + j] * s_in[j];
         for (int j = 0; j < dv; ++j)
-            orc_quantize_column(S, Sh, dk, dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
+            orc_quantize_column(S, Sh, hd->m_copy ? hd->m_copy + j : NULL, dk, dv, j, hd->bits,
+                                hd->rounding, hd->mode, hd->seed,
                                 hd->b, hd->h, hd->step, c_out, &s_out[j]);
     }
     free(S); free(cf); free(Sh);
@@ -464,7 +478,8 @@ int orc_diag_head_step(const orc_head* hd, int delta, const int8_t* c_in, const 
             for (int j = 0; j < dv; ++j)
                 Sh[(int64_t)i * dv + j] = (float)c_in[(int64_t)i * dv + j] * s_in[j];
         for (int j = 0; j < dv; ++j)
-            orc_quantize_column(S, Sh, dk, dv, j, hd->bits, hd->rounding, hd->mode, hd->seed,
+            orc_quantize_column(S, Sh, hd->m_copy ? hd->m_copy + j : NULL, dk, dv, j, hd->bits,
+                                hd->rounding, hd->mode, hd->seed,
                                 hd->b, hd->h, hd->step, c_out, &s_out[j]);
     }
     free(S); free(Sh); free(cf); free(ak);
@@ -477,8 +492,9 @@ int orc_quantize_head(const orc_head* hd, const float* S, int8_t* c_out, float* 
 {
     if (hd->bits != 4 && hd->bits != 8) return 1;
     for (int j = 0; j < hd->dv; ++j)
-        orc_quantize_column(S, NULL, hd->dk, hd->dv, j, hd->bits, hd->rounding, hd->mode,
-                            hd->seed, hd->b, hd->h, hd->step, c_out, &s_out[j]);
+        orc_quantize_column(S, NULL, hd->m_copy ? hd->m_copy + j : NULL, hd->dk, hd->dv, j,
+                            hd->bits, hd->rounding, hd->mode, hd->seed, hd->b, hd->h, hd->step,
+                            c_out, &s_out[j]);
     return 0;
 }
 

@@ -668,3 +668,63 @@ def test_gla_constant_decay_is_the_scalar_decay_step():
                                     decay=gamma)
         assert np.array_equal(a["codes"], m["codes"]) and np.array_equal(a["scales"], m["scales"])
         assert np.array_equal(a["f"], m["f"]) and np.array_equal(o_a, o_m)
+
+
+# ---------------------------------------------------------------------------
+# Copy scale (LoReS (4/4), animation details: the scale taken from an
+# unquantized copy of the state; "When Dynamic Scaling Fails", key points: the
+# dynamic scale feeds back on the state it is derived from)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("rounding", [oracle.RTN, oracle.SR])
+@pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
+def test_copy_scale_equal_to_own_maximum_is_the_noisy_quantizer(rounding, mode):
+    rng = np.random.default_rng(3)
+    S = (rng.standard_normal((2, 3, 16, 32)) * 0.3).astype(np.float32)
+    hb = np.array([8, 4, 8], np.int8)
+    own = np.abs(S).max(axis=2)                      # exact column maxima
+    a = oracle.quantize(S, hb, rounding=rounding, seed=4, step=2, mode=mode)
+    b = oracle.quantize(S, hb, rounding=rounding, seed=4, step=2, mode=mode, copy_absmax=own)
+    assert np.array_equal(a["codes"], b["codes"]) and np.array_equal(a["scales"], b["scales"])
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_copy_scale_clips_beyond_the_copy_maximum(bits):
+    """A copy maximum below the column's own: elements beyond it clip to +-r, the
+    others keep the half-step bound of nearest rounding."""
+    rng = np.random.default_rng(bits)
+    S = rng.standard_normal((1, 2, 32, 16)).astype(np.float32)
+    hb = np.full(2, bits, np.int8)
+    mc = (np.abs(S).max(axis=2) * 0.5).astype(np.float32)
+    st = oracle.quantize(S, hb, rounding=oracle.RTN, seed=0, step=0, copy_absmax=mc)
+    r = oracle.rmax(bits)
+    s = st["scales"].astype(np.float64)[:, :, None, :]
+    c = st["codes"].astype(np.float64)
+    assert np.abs(c).max() == r
+    inside = np.abs(S) <= mc[:, :, None, :]
+    err = np.abs(c * s - S)
+    assert np.all(err[inside] <= (s / 2 * (1 + 1e-6) + 0 * err)[inside])
+    assert np.array_equal(c[~inside], r * np.sign(S[~inside]))
+
+
+def test_copy_scale_removes_the_error_dependence_of_the_scale():
+    """With the copy scale the scales follow the unquantized trajectory whatever
+    the rounding draws; with the state's own (noisy) scale they do not."""
+    w = dataclasses.replace(TINY, B=1, H=2)
+    hb4 = np.full(w.H, 4, np.int8)
+    hb32 = np.full(w.H, 32, np.int8)
+    ref = oracle.zero_state(w.B, w.H, w.dk, w.dv)
+    cp = {s: oracle.zero_state(w.B, w.H, w.dk, w.dv) for s in (1, 2)}
+    ny = {s: oracle.zero_state(w.B, w.H, w.dk, w.dv) for s in (1, 2)}
+    noisy_differ = False
+    for t in range(24):
+        inp = W.gdn_inputs(w, t)
+        ref, _ = oracle.gdn_step(ref, inp, hb32, rounding=0, seed=0, step=t)
+        m = np.abs(ref["f"]).max(axis=2)
+        for seed in (1, 2):
+            cp[seed], _ = oracle.gdn_step(cp[seed], inp, hb4, rounding=oracle.SR, seed=seed, step=t,
+                                          copy_absmax=m)
+            ny[seed], _ = oracle.gdn_step(ny[seed], inp, hb4, rounding=oracle.SR, seed=seed, step=t)
+        assert np.array_equal(cp[1]["scales"], cp[2]["scales"])
+        assert np.array_equal(cp[1]["scales"], (m / np.float32(7)).astype(np.float32))
+        noisy_differ |= not np.array_equal(ny[1]["scales"], ny[2]["scales"])
+    assert noisy_differ
