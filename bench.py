@@ -51,6 +51,8 @@ def algorithmic_bytes_per_head(w: W.Workload, bits: int) -> int:
     out = 4 * w.dv
     if w.family == "gdn":
         vecs = esz * (2 * w.dk + w.dv) + 8          # q, k, v, alpha, beta
+    elif w.family in ("gla", "kda"):
+        vecs = esz * (2 * w.dk + w.dv) + 4 * w.dk + (4 if w.family == "kda" else 0)  # + decay vector
     else:
         vecs = esz * w.dv + 4                       # x, dt (B, C, A, D added per request / head)
     return 2 * codes + 2 * scales + vecs + out
@@ -177,7 +179,7 @@ def oracle_rate(w: W.Workload, head_bits, budget_s: float, heads_per_call: int =
     of the workload (the first requests of a few steps, from the zero state)."""
     import oracle
     R = 8 if w.dk <= 128 else 16
-    rounding = oracle.SR if w.rounding == "sr" else oracle.RTN
+    rounding = ROUNDING[w.rounding]
     n_done, t_used, t = 0, 0.0, 0
     nb = max(1, min(w.B, heads_per_call // w.H + 1))
     st = oracle.zero_state(nb, w.H, w.dk, w.dv, fp32=w.state == "fp32")
@@ -185,16 +187,25 @@ def oracle_rate(w: W.Workload, head_bits, budget_s: float, heads_per_call: int =
         inp = W.inputs(w, t, B=nb)
         heads = [(b, h) for b in range(nb) for h in range(w.H)][:heads_per_call]
         t0 = time.perf_counter()
-        if w.family == "gdn":
-            st, _ = oracle.gdn_step(st, inp, head_bits, rounding=rounding, seed=w.sr_seed, step=t,
-                                    R=R, heads=heads)
-        else:
-            st, _ = oracle.mamba2_step(st, inp, head_bits, rounding=rounding, seed=w.sr_seed,
-                                       step=t, R=R, ngroups=w.ngroups, heads=heads)
+        st, _ = _oracle_step(oracle, w, st, inp, head_bits, rounding, t, R, heads)
         t_used += time.perf_counter() - t0
         n_done += len(heads)
         t += 1
     return n_done / t_used, n_done, t
+
+
+def _oracle_step(oracle, w: W.Workload, st, inp, bits, rounding, t, R, heads):
+    kw = dict(rounding=rounding, seed=w.sr_seed, step=t, R=R, heads=heads)
+    if w.family == "gdn":
+        return oracle.gdn_step(st, inp, bits, **kw)
+    if w.family == "gla":
+        return oracle.gla_step(st, inp, bits, **kw)
+    if w.family == "kda":
+        return oracle.kda_step(st, inp, bits, **kw)
+    return oracle.mamba2_step(st, inp, bits, ngroups=w.ngroups, **kw)
+
+
+FAMILY = {"gdn": 0, "mamba2": 1, "gla": 2, "kda": 3}   # rsq_family values
 
 
 def head_bits_of(w: W.Workload, rsq=None):
@@ -220,7 +231,7 @@ def run_reference(args, w: W.Workload):
     n_heads = int(max(1, min(w.B * w.H, total_budget / max(1, args.steps + args.warmup) / per_head)))
     import oracle
     R = 8 if w.dk <= 128 else 16
-    rounding = oracle.SR if w.rounding == "sr" else oracle.RTN
+    rounding = ROUNDING[w.rounding]
     nb = max(1, min(w.B, (n_heads + w.H - 1) // w.H))
     heads = [(b, h) for b in range(nb) for h in range(w.H)][:n_heads]
     st = oracle.zero_state(nb, w.H, w.dk, w.dv, fp32=w.state == "fp32")
@@ -229,12 +240,7 @@ def run_reference(args, w: W.Workload):
     for t in range(args.warmup + args.steps):
         inp = inp_cache[t % 4]
         t0 = time.perf_counter()
-        if w.family == "gdn":
-            st, _ = oracle.gdn_step(st, inp, bits, rounding=rounding, seed=w.sr_seed, step=t, R=R,
-                                    heads=heads)
-        else:
-            st, _ = oracle.mamba2_step(st, inp, bits, rounding=rounding, seed=w.sr_seed, step=t,
-                                       R=R, ngroups=w.ngroups, heads=heads)
+        st, _ = _oracle_step(oracle, w, st, inp, bits, rounding, t, R, heads)
         dt = time.perf_counter() - t0
         if t >= args.warmup:
             elapsed += dt
@@ -279,9 +285,9 @@ def run_ours(args, w: W.Workload):
     l2 = int(getattr(props, "L2_cache_size", 126 * 2 ** 20))
 
     bits = np.asarray(head_bits_of(w, rsq), np.int8)
-    fam = rsq.RSQ_GDN if w.family == "gdn" else rsq.RSQ_MAMBA2
+    fam = FAMILY[w.family]
     ctx = rsq.Context(fam, w.B, w.H, w.dk, w.dv, head_bits=bits,
-                      rounding=rsq.RSQ_SR if w.rounding == "sr" else rsq.RSQ_RTN,
+                      rounding=ROUNDING[w.rounding],
                       in_dtype=rsq.RSQ_BF16 if w.in_dtype == "bf16" else rsq.RSQ_F32,
                       seed=w.sr_seed + 7919 * rank, ngroups=w.ngroups)
     state_bytes = ctx.code_bytes + ctx.scale_bytes
@@ -481,8 +487,14 @@ def run_ours(args, w: W.Workload):
 # ---------------------------------------------------------------------------
 # Long-horizon state drift (quantized trajectories against the FP32 trajectory)
 # ---------------------------------------------------------------------------
-DRIFT_VARIANTS = (("int4_sr", 4, "sr"), ("int4_rtn", 4, "rtn"), ("int8_sr", 8, "sr"),
-                  ("int8_rtn", 8, "rtn"))
+# (label, bits, rounding, scale source): "noisy" = the quantized state's own
+# column maxima, "copy" = the column maxima of the FP32 trajectory
+DRIFT_VARIANTS = (("int4_sr", 4, "sr", "noisy"), ("int4_rtn", 4, "rtn", "noisy"),
+                  ("int4_bdr", 4, "bdr", "noisy"), ("int4_sr_bdr", 4, "sr_bdr", "noisy"),
+                  ("int4_sr_copy", 4, "sr", "copy"), ("int4_rtn_copy", 4, "rtn", "copy"),
+                  ("int8_sr", 8, "sr", "noisy"), ("int8_rtn", 8, "rtn", "noisy"),
+                  ("int8_bdr", 8, "bdr", "noisy"), ("int8_sr_copy", 8, "sr", "copy"))
+ROUNDING = {"rtn": 0, "sr": 1, "bdr": 2, "sr_bdr": 3}   # rsq_rounding values
 
 
 def _drift_inputs(job):
@@ -496,6 +508,8 @@ def drift_series(w: W.Workload, steps: int, every: int, B: int | None = None, va
     trajectories against the full-precision trajectory run by the same kernel
     with 32-bit heads, all from S_0 = 0 on identical inputs, sampled every
     `every` steps.  Also the relative error of the readout at those steps.
+    Variants with the "copy" scale source take each step's scales from the
+    FP32 trajectory's column maxima instead of their own state.
 
     Returns {label: [[t, global drift, max per-head drift, readout error], ...]}."""
     import torch
@@ -503,12 +517,12 @@ def drift_series(w: W.Workload, steps: int, every: int, B: int | None = None, va
     import ssm_decode_02_b200 as rsq
 
     B = w.B if B is None else B
-    fam = rsq.RSQ_GDN if w.family == "gdn" else rsq.RSQ_MAMBA2
+    fam = FAMILY[w.family]
     in_dtype = rsq.RSQ_BF16 if w.in_dtype == "bf16" else rsq.RSQ_F32
 
     def make(bits, rounding):
         ctx = rsq.Context(fam, B, w.H, w.dk, w.dv, head_bits=np.full(w.H, bits, np.int8),
-                          rounding=rsq.RSQ_SR if rounding == "sr" else rsq.RSQ_RTN,
+                          rounding=ROUNDING[rounding],
                           in_dtype=in_dtype, seed=w.sr_seed, ngroups=w.ngroups)
         st = ctx.alloc_state(device)
         ctx.quantize(torch.zeros((B, w.H, w.dk, w.dv), dtype=torch.float32, device=device), st)
@@ -516,16 +530,23 @@ def drift_series(w: W.Workload, steps: int, every: int, B: int | None = None, va
         return ctx, st, out
 
     ref = make(32, "rtn")
-    runs = {label: make(bits, rnd) for label, bits, rnd in variants}
+    runs = {label: make(bits, rnd) for label, bits, rnd, _ in variants}
+    source = {label: src for label, _, _, src in variants}
+    copy_max = torch.empty((B, w.H, w.dv), dtype=torch.float32, device=device)
     sums = torch.empty((B, w.H, 2), dtype=torch.float64, device=device)
-    series = {label: [] for label, _, _ in variants}
+    series = {label: [] for label, _, _, _ in variants}
     jobs = [(w, B, t) for t in range(steps)]
     it = pool.imap(_drift_inputs, jobs, chunksize=2) if pool is not None else map(_drift_inputs, jobs)
     for t, host in it:
         d = {k: _to_dev(v, device) for k, v in host.items()}
         ins = _inputs_struct(rsq, w, d)
-        for ctx, st, out in [ref] + list(runs.values()):
-            ctx.decode_step(st, st, ins, out, t)
+        ref[0].decode_step(ref[1], ref[1], ins, ref[2], t)
+        ref[0].column_absmax(ref[1], copy_max)
+        for label, (ctx, st, out) in runs.items():
+            if source[label] == "copy":
+                ctx.decode_step_copy_scale(st, st, ins, copy_max, out, t)
+            else:
+                ctx.decode_step(st, st, ins, out, t)
         if (t + 1) % every == 0:
             o_ref = ref[2].double()
             for label, (ctx, st, out) in runs.items():
@@ -567,6 +588,8 @@ def step_input_bytes(w: W.Workload) -> int:
     esz = 2 if w.in_dtype == "bf16" else 4
     if w.family == "gdn":
         return w.B * w.H * (esz * (2 * w.dk + w.dv) + 8)
+    if w.family in ("gla", "kda"):
+        return w.B * w.H * (esz * (2 * w.dk + w.dv) + 4 * w.dk + (4 if w.family == "kda" else 0))
     return w.B * w.H * (esz * w.dv + 4) + w.B * w.ngroups * 2 * w.dk * esz + 8 * w.H
 
 
@@ -589,6 +612,8 @@ def _to_pinned(a: np.ndarray):
 def _inputs_struct(rsq, w: W.Workload, d: dict):
     if w.family == "gdn":
         return rsq.gdn_inputs(d["q"], d["k"], d["v"], d["alpha"], d["beta"])
+    if w.family in ("gla", "kda"):
+        return rsq.diag_inputs(d["q"], d["k"], d["v"], d["alpha"], d.get("beta"))
     return rsq.mamba2_inputs(d["x"], d["Bm"], d["Cm"], d["dt"], d["A"], d["D"], None)
 
 
@@ -602,6 +627,8 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="override the number of rotated layer states")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--rounding", choices=sorted(ROUNDING), default=None,
+                    help="override the workload's requantization rule")
     ap.add_argument("--drift", action="store_true",
                     help="run the long-horizon state drift study instead of the throughput bench")
     ap.add_argument("--drift-steps", type=int, default=0, help="horizon (default: the workload's)")
@@ -615,6 +642,9 @@ def main():
         with mp.get_context("spawn").Pool(max(1, min(32, (os.cpu_count() or 2) - 1))) as pool:
             return run_drift(args, w, pool)
     w = W.BY_NAME[args.workload]
+    if args.rounding:
+        import dataclasses
+        w = dataclasses.replace(w, rounding=args.rounding)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)

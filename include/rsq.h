@@ -86,8 +86,24 @@ typedef enum {
     RSQ_E_NONFINITE = 5    /* rsq_check_flags: a non-finite state column was seen */
 } rsq_status;
 
-typedef enum { RSQ_GDN = 0, RSQ_MAMBA2 = 1 } rsq_family;
-typedef enum { RSQ_RTN = 0, RSQ_SR = 1 } rsq_rounding;
+/* Recurrence of the layer.  RSQ_GDN: gated delta rule; RSQ_MAMBA2: scalar
+ * decay (RetNet and plain linear attention are this step with B = k, C = q,
+ * x = v, dt = 1, decay = gamma (resp. 1), D = 0 and ngroups = heads);
+ * RSQ_GLA: S_t = diag(alpha) S_{t-1} + k v^T with a decay per key channel;
+ * RSQ_KDA: S_t = (I - beta k k^T) diag(alpha) S_{t-1} + beta k v^T.  GLA and
+ * KDA are the diagonal-decay mixers of [LoReS] Table 1. */
+typedef enum { RSQ_GDN = 0, RSQ_MAMBA2 = 1, RSQ_GLA = 2, RSQ_KDA = 3 } rsq_family;
+/* Requantization rule.  RSQ_RTN: nearest code (ties to even).  RSQ_SR:
+ * stochastic rounding with a 16-bit Philox uniform per element ([LoReS] (3/4)).
+ * RSQ_BDR / RSQ_SR_BDR: the same base rounding followed by Bounded Directional
+ * Rounding ("Preserving Updates in Low-Bit Recurrent State Quantization",
+ * abstract): when the rounded value c_t s_t lies strictly on the other side of
+ * the previous value c_{t-1} s_{t-1} than the updated state S_t does (the
+ * element moved against its update), the code becomes the integer next to
+ * S_t / s_t on the update's side (ceil for an upward update, floor for a
+ * downward one), so the error stays below one step.  No extra storage.
+ * rsq_quantize has no previous state and applies the base rounding. */
+typedef enum { RSQ_RTN = 0, RSQ_SR = 1, RSQ_BDR = 2, RSQ_SR_BDR = 3 } rsq_rounding;
 typedef enum { RSQ_F32 = 0, RSQ_BF16 = 1 } rsq_dtype;
 
 /* Layer configuration, read once by rsq_create. */
@@ -137,6 +153,21 @@ typedef struct {
     const float* decay;
 } rsq_mamba2_inputs;
 
+/* GLA / KDA step inputs (device).  q, k: [B][H][dk], v: [B][H][dv] in
+ * in_dtype; alpha: float [B][H][dk], the decay of each key channel; beta:
+ * float [B][H] (KDA; ignored and may be NULL for GLA).
+ *   GLA:  S_ij = alpha_i S^_ij + k_i v_j
+ *   KDA:  u_j = sum_i alpha_i S^_ij k_i,  w_j = beta (v_j - u_j),
+ *         S_ij = alpha_i S^_ij + k_i w_j
+ * with S^ the dequantized previous state; readout o_j = sum_i S_ij q_i. */
+typedef struct {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* alpha;
+    const float* beta;
+} rsq_diag_inputs;
+
 /* Create a context for one layer configuration.  Validates the configuration
  * (RSQ_E_INVAL / RSQ_E_UNSUPPORTED, nothing allocated), then allocates a
  * 4-byte device flag word on the current device (RSQ_E_NOMEM / RSQ_E_CUDA on
@@ -182,8 +213,9 @@ rsq_status rsq_head_offset(const rsq_ctx* ctx, int h, size_t* offset);
  *
  * Arguments: state_in / state_out: device states of this context's format;
  *   state_out may equal state_in (in-place update; any other overlap is
- *   invalid).  inputs: host pointer to rsq_gdn_inputs or rsq_mamba2_inputs
- *   (family of the context) holding device pointers.  out: device float
+ *   invalid).  inputs: host pointer to rsq_gdn_inputs, rsq_mamba2_inputs or
+ *   rsq_diag_inputs (GLA, KDA) -- the context's family -- holding device
+ *   pointers.  out: device float
  *   [B][H][dv].  step: decode-step index (stochastic-rounding counter; keep it
  *   across checkpoints for reproducible runs).
  * Errors: RSQ_E_INVAL for null/misaligned pointers; RSQ_E_CUDA if the launch
@@ -211,6 +243,25 @@ rsq_status rsq_dequantize(const rsq_ctx* ctx, const rsq_state* state_in, float* 
 rsq_status rsq_state_drift(const rsq_ctx* q_ctx, const rsq_state* q_state,
                            const rsq_ctx* f_ctx, const rsq_state* f_state, double* sums,
                            void* stream);
+
+/* Decode step with the copy scale ([LoReS] (4/4), animation details; the
+ * ablation of [FEED]): identical to rsq_decode_step except that each column's
+ * new scale is copy_absmax[b][h][j] / r, the maximum of |S_t| of an
+ * unquantized copy of the state (e.g. a full-precision trajectory run on the
+ * same inputs, read with rsq_column_absmax), instead of the maximum of the
+ * column itself; codes beyond it clip to +-r.  This removes the feedback of
+ * earlier quantization errors into the scale.  copy_absmax: device float
+ * [B][H][dv].  A column whose own values are non-finite is still flagged and
+ * stored as zero codes.  RSQ_E_UNSUPPORTED for a full-precision context. */
+rsq_status rsq_decode_step_copy_scale(const rsq_ctx* ctx, const rsq_state* state_in,
+                                      const rsq_state* state_out, const void* inputs,
+                                      const float* copy_absmax, float* out, uint32_t step,
+                                      void* stream);
+
+/* Column maxima max_i |S^_ij| of a stored state (dequantized values; the
+ * stored values for 32-bit heads), NaN-propagating.  absmax: device float
+ * [B][H][dv]. */
+rsq_status rsq_column_absmax(const rsq_ctx* ctx, const rsq_state* state, float* absmax, void* stream);
 
 /* Synchronize `stream`, then report (and clear) the context's non-finite
  * flag: *seen = 1 if any decode step since the last check met a non-finite

@@ -19,8 +19,8 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "librsq.so")
 
-RSQ_GDN, RSQ_MAMBA2 = 0, 1
-RSQ_RTN, RSQ_SR = 0, 1
+RSQ_GDN, RSQ_MAMBA2, RSQ_GLA, RSQ_KDA = 0, 1, 2, 3
+RSQ_RTN, RSQ_SR, RSQ_BDR, RSQ_SR_BDR = 0, 1, 2, 3
 RSQ_F32, RSQ_BF16 = 0, 1
 RSQ_OK, RSQ_E_INVAL, RSQ_E_UNSUPPORTED, RSQ_E_CUDA, RSQ_E_NOMEM, RSQ_E_NONFINITE = range(6)
 RSQ_MAX_HEADS = 512
@@ -54,10 +54,16 @@ class rsq_mamba2_inputs(ctypes.Structure):
                 ("decay", ctypes.c_void_p)]
 
 
+class rsq_diag_inputs(ctypes.Structure):
+    _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
+                ("alpha", ctypes.c_void_p), ("beta", ctypes.c_void_p)]
+
+
 _EXPORTS = ["rsq_create", "rsq_destroy", "rsq_state_bytes", "rsq_head_offset", "rsq_decode_step",
             "rsq_quantize", "rsq_dequantize", "rsq_state_drift", "rsq_check_flags",
             "rsq_allocate_bits", "rsq_reduction_partials", "rsq_status_string", "rsq_last_error",
-            "rsq_version", "rsq_decode_step_noalloc"]
+            "rsq_version", "rsq_decode_step_noalloc", "rsq_decode_step_copy_scale",
+            "rsq_column_absmax"]
 
 
 def _load():
@@ -83,6 +89,9 @@ def _load():
         "rsq_version": ([], ctypes.c_char_p),
         "rsq_decode_step_noalloc": ([ctypes.POINTER(rsq_config), ctypes.POINTER(rsq_state),
                                      ctypes.POINTER(rsq_state), P, P, ctypes.c_uint32, P], C),
+        "rsq_decode_step_copy_scale": ([P, ctypes.POINTER(rsq_state), ctypes.POINTER(rsq_state), P, P,
+                                        P, ctypes.c_uint32, P], C),
+        "rsq_column_absmax": ([P, ctypes.POINTER(rsq_state), P, P], C),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -188,10 +197,27 @@ def _state(st) -> rsq_state:
 
 
 def rsq_decode_step(ctx: int, state_in, state_out, inputs, out, step: int, stream=None) -> None:
-    """inputs: rsq_gdn_inputs / rsq_mamba2_inputs (see gdn_inputs / mamba2_inputs)."""
+    """inputs: rsq_gdn_inputs / rsq_mamba2_inputs / rsq_diag_inputs (see gdn_inputs,
+    mamba2_inputs, diag_inputs)."""
     si, so = _state(state_in), _state(state_out)
     _check(lib.rsq_decode_step(ctx, ctypes.byref(si), ctypes.byref(so), ctypes.byref(inputs),
                                _ptr(out), int(step) & 0xFFFFFFFF, _stream(stream)))
+
+
+def rsq_decode_step_copy_scale(ctx: int, state_in, state_out, inputs, copy_absmax, out, step: int,
+                               stream=None) -> None:
+    """Decode step whose scales come from copy_absmax ([B][H][dv], column maxima of an
+    unquantized copy of the state) instead of the state's own columns."""
+    si, so = _state(state_in), _state(state_out)
+    _check(lib.rsq_decode_step_copy_scale(ctx, ctypes.byref(si), ctypes.byref(so), ctypes.byref(inputs),
+                                          _ptr(copy_absmax), _ptr(out), int(step) & 0xFFFFFFFF,
+                                          _stream(stream)))
+
+
+def rsq_column_absmax(ctx: int, state, absmax, stream=None) -> None:
+    """Column maxima of |S^| of a stored state into absmax ([B][H][dv] float32, device)."""
+    si = _state(state)
+    _check(lib.rsq_column_absmax(ctx, ctypes.byref(si), _ptr(absmax), _stream(stream)))
 
 
 def rsq_quantize(ctx: int, S, state_out, step: int, stream=None) -> None:
@@ -250,6 +276,11 @@ def gdn_inputs(q, k, v, alpha, beta) -> rsq_gdn_inputs:
     return rsq_gdn_inputs(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta))
 
 
+def diag_inputs(q, k, v, alpha, beta=None) -> rsq_diag_inputs:
+    """GLA / KDA inputs: alpha is the decay per key channel ([B][H][dk] float32)."""
+    return rsq_diag_inputs(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta))
+
+
 def mamba2_inputs(x, Bm, Cm, dt, A, D, decay=None) -> rsq_mamba2_inputs:
     return rsq_mamba2_inputs(_ptr(x), _ptr(Bm), _ptr(Cm), _ptr(dt), _ptr(A), _ptr(D), _ptr(decay))
 
@@ -285,6 +316,13 @@ class Context:
 
     def decode_step(self, state_in: State, state_out: State, inputs, out, step: int, stream=None):
         rsq_decode_step(self.ctx, state_in, state_out, inputs, out, step, stream)
+
+    def decode_step_copy_scale(self, state_in: State, state_out: State, inputs, copy_absmax, out,
+                               step: int, stream=None):
+        rsq_decode_step_copy_scale(self.ctx, state_in, state_out, inputs, copy_absmax, out, step, stream)
+
+    def column_absmax(self, state: State, absmax, stream=None):
+        rsq_column_absmax(self.ctx, state, absmax, stream)
 
     def quantize(self, S, state_out: State, step: int = 0, stream=None):
         rsq_quantize(self.ctx, S, state_out, step, stream)

@@ -1,0 +1,11 @@
+// decode_gdn_copy_bdr.cu -- Gated DeltaNet instantiations of the fused decode
+// kernel with the copy scale and Bounded Directional Rounding.
+#include "decode_kernel.cuh"
+
+namespace rsq {
+int decode_info_gdn_copy_bdr(int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
+                             const void** func) {
+    return decode_info_family<RSQ_GDN, kRndCopy | kRndBdr, kRndCopy | kRndBdr | kRndSr>(
+        dk, ub, f32state, rnd, threads, smem, func);
+}
+}  // namespace rsq

@@ -1,0 +1,12 @@
+// decode_kda_copy.cu -- KDA instantiations of the fused decode kernel
+// with the copy scale (scales from an unquantized copy's column maxima), with
+// nearest and stochastic rounding.
+#include "decode_kernel.cuh"
+
+namespace rsq {
+int decode_info_kda_copy(int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
+                         const void** func) {
+    return decode_info_family<RSQ_KDA, kRndCopy, kRndCopy | kRndSr>(dk, ub, f32state, rnd, threads,
+                                                                   smem, func);
+}
+}  // namespace rsq

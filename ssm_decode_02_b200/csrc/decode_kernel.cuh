@@ -34,24 +34,30 @@ struct DecodeCfg {
     using L = Layout<DK>;
     static constexpr int NT = 32 * UB;         // one warp per 16-column block
     static constexpr int UCOLS = 16 * UB;      // columns per unit
-    static constexpr int NS = F32STATE ? 2 : 4;  // pipeline stages
+    // pipeline stages (KDA's extra pair array leaves room for three)
+    static constexpr int NS = F32STATE ? 2 : (FAM == RSQ_KDA ? 3 : 4);
     static constexpr int CODE_BYTES = F32STATE ? DK * UCOLS * 4 : DK * UCOLS;  // largest tile (8-bit)
     static constexpr int OFF_SCALES = CODE_BYTES;
     static constexpr int OFF_VA = OFF_SCALES + UCOLS * 4;  // GDN q / Mamba-2 C   (<= DK floats)
     static constexpr int OFF_VB = OFF_VA + DK * 4;         // GDN k / Mamba-2 B
     static constexpr int OFF_VC = OFF_VB + DK * 4;         // GDN v / Mamba-2 x   (<= UCOLS floats)
-    static constexpr int STAGE = (OFF_VC + UCOLS * 4 + 127) / 128 * 128;
+    static constexpr int OFF_VD = OFF_VC + UCOLS * 4;      // GLA / KDA decay per key channel (DK floats)
+    static constexpr bool DIAG = (FAM == RSQ_GLA || FAM == RSQ_KDA);
+    static constexpr int STAGE = ((DIAG ? OFF_VD + DK * 4 : OFF_VD) + 127) / 128 * 128;
     // per warp: the two key-axis vectors as duplicated pairs (x, x), one row of
     // PST pairs per row group (padded so the row groups hit different banks)
     static constexpr int PST = L::RPT + 2;
-    static constexpr int P_WARP = 2 * kR * PST * 8;
+    // pair arrays: q, k (+ the decay per key channel for GLA, + decay and
+    // decay * k for KDA)
+    static constexpr int NPAIR = FAM == RSQ_KDA ? 4 : (DIAG ? 3 : 2);
+    static constexpr int P_WARP = NPAIR * kR * PST * 8;
     static constexpr int OFF_P = NS * STAGE;
     static constexpr int OFF_CNT = OFF_P + UB * P_WARP;  // NS release counters
     static constexpr int OFF_BAR = OFF_CNT + 16;
     static constexpr int SMEM = OFF_BAR + NS * 8;
-    // resident CTAs per SM the register budget is sized for (GDN keeps more live
-    // values across its extra reduction than Mamba-2)
-    static constexpr int MINB = F32STATE ? 1 : (NT < 128 ? 8 : (FAM == RSQ_GDN ? 4 : 5));
+    // resident CTAs per SM the register budget is sized for: shared memory holds
+    // four 128-thread CTAs per SM (4 x ~50 KB), so 128 registers per thread
+    static constexpr int MINB = F32STATE ? 1 : (NT < 128 ? 8 : 4);
 };
 
 // Grid-stride walk over units without divisions: (b, h, cb) advance by the
@@ -86,7 +92,8 @@ __device__ __forceinline__ void issue_unit(const DecodeParams& p, const UnitIt& 
     const int hu = un.hu(p);
     const uint32_t code_bytes = static_cast<uint32_t>(DK * UCOLS * bits / 8);
     const uint32_t esz = p.in_bf16 ? 2u : 4u;
-    const uint32_t total = code_bytes + (F32STATE ? 0u : UCOLS * 4u) + 2u * DK * esz + UCOLS * esz;
+    const uint32_t total = code_bytes + (F32STATE ? 0u : UCOLS * 4u) + 2u * DK * esz + UCOLS * esz +
+                           (C::DIAG ? DK * 4u : 0u);
     const uint8_t* codes = p.codes_in + (long long)un.b * p.row_bytes + p.head_off[un.h] +
                            (long long)un.cb * code_bytes;
     const uint32_t s = smem_u32(stage);
@@ -97,12 +104,13 @@ __device__ __forceinline__ void issue_unit(const DecodeParams& p, const UnitIt& 
     const char* vA = static_cast<const char*>(p.vA);
     const char* vB = static_cast<const char*>(p.vB);
     const char* vC = static_cast<const char*>(p.vC);
-    const long long rowA = (FAM == RSQ_GDN)
+    const long long rowA = (FAM != RSQ_MAMBA2)
                                ? (long long)hu * DK  // q and k of this head
                                : ((long long)un.b * p.ngroups + un.h / p.heads_per_group) * DK;
     bulk_g2s(s + C::OFF_VA, vA + rowA * esz, DK * esz, bar);
     bulk_g2s(s + C::OFF_VB, vB + rowA * esz, DK * esz, bar);
     bulk_g2s(s + C::OFF_VC, vC + ((long long)hu * p.dv + un.cb * UCOLS) * esz, UCOLS * esz, bar);
+    if constexpr (C::DIAG) bulk_g2s(s + C::OFF_VD, p.vD + (long long)hu * DK, DK * 4u, bar);
 }
 
 __device__ __forceinline__ float ld_vec(const uint8_t* base, int e, bool bf16) {
@@ -129,15 +137,15 @@ template <int FAM>
 __device__ __forceinline__ Gates load_gates(const DecodeParams& p, const UnitIt& un) {
     Gates g;
     const int hu = un.hu(p);
-    g.g0 = __ldg(p.g0 + hu);
-    g.g1 = p.g1 ? __ldg(p.g1 + hu) : 0.f;
+    g.g0 = (FAM == RSQ_GLA || FAM == RSQ_KDA) ? 0.f : __ldg(p.g0 + hu);
+    g.g1 = (FAM != RSQ_GLA && p.g1) ? __ldg(p.g1 + hu) : 0.f;
     g.A = (FAM == RSQ_MAMBA2) ? __ldg(p.A + un.h) : 0.f;
     g.D = (FAM == RSQ_MAMBA2) ? __ldg(p.D + un.h) : 0.f;
     return g;
 }
 
 // One 16-column block of one unit, processed by warp w.
-template <int FAM, int DK, int UB, bool F32STATE, bool SR, int BITS>
+template <int FAM, int DK, int UB, bool F32STATE, int RND, int BITS>
 __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitIt& un, uint8_t* stage,
                                               uint8_t* smem, int stage_idx, uint32_t bar,
                                               const Gates& gt, int w, int lane, int g, int cw) {
@@ -153,6 +161,8 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
     // ---- this warp's copy of the key-axis vectors as duplicated pairs --------
     uint64_t* pa = reinterpret_cast<uint64_t*>(smem + C::OFF_P + w * C::P_WARP);
     uint64_t* pb = pa + kR * C::PST;
+    uint64_t* pc = pb + kR * C::PST;  // GLA / KDA: decay alpha_i
+    uint64_t* pd = pc + kR * C::PST;  // KDA: alpha_i * k_i
 #pragma unroll
     for (int i = lane; i < DK; i += 32) {
         const float a = ld_vec(stage + C::OFF_VA, i, bf16);
@@ -160,10 +170,20 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
         const int pos = (i & (kR - 1)) * C::PST + i / kR;
         pa[pos] = pk(a, a);
         pb[pos] = pk(b, b);
+        if constexpr (C::DIAG) {
+            const float d = reinterpret_cast<const float*>(stage + C::OFF_VD)[i];
+            pc[pos] = pk(d, d);
+            if constexpr (FAM == RSQ_KDA) {
+                const float ak = __fmul_rn(d, b);
+                pd[pos] = pk(ak, ak);
+            }
+        }
     }
     __syncwarp();
-    const uint64_t* qa = pa + g * C::PST;  // q (GDN) / C (Mamba-2) of rows g + 8k
-    const uint64_t* kb = pb + g * C::PST;  // k (GDN) / B (Mamba-2)
+    const uint64_t* qa = pa + g * C::PST;  // q (GDN, GLA, KDA) / C (Mamba-2) of rows g + 8k
+    const uint64_t* kb = pb + g * C::PST;  // k / B
+    const uint64_t* ga = pc + g * C::PST;  // decay per key channel (GLA, KDA)
+    const uint64_t* gk = pd + g * C::PST;  // decay * k (KDA)
 
     // ---- state block -> registers (packed pairs) ------------------------------
     const uint8_t* tile = stage + w * BLOCK_BYTES;
@@ -228,6 +248,52 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
             S2[k + 1][0] = fma2(S2[k + 1][0], A01, mul2(kk.y, W01));
             S2[k + 1][1] = fma2(S2[k + 1][1], A23, mul2(kk.y, W23));
         }
+    } else if constexpr (C::DIAG) {
+        // GLA: w = v.  KDA: u = s * sum_i c_ij (alpha_i k_i), w = beta (v - u).
+        const float4 s4 = load_s4();
+        const float4 vc = load_vc();
+        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
+        const float vv[4] = {vc.x, vc.y, vc.z, vc.w};
+        float wj[4] = {vv[0], vv[1], vv[2], vv[3]};
+        if constexpr (FAM == RSQ_KDA) {
+            uint64_t a01 = pk(0.f, 0.f), a23 = pk(0.f, 0.f);
+#pragma unroll
+            for (int k = 0; k < RPT; k += 2) {
+                const ulonglong2 kk = *reinterpret_cast<const ulonglong2*>(gk + k);  // alpha_i k_i
+                a01 = fma2(S2[k][0], kk.x, a01);
+                a23 = fma2(S2[k][1], kk.x, a23);
+                a01 = fma2(S2[k + 1][0], kk.y, a01);
+                a23 = fma2(S2[k + 1][1], kk.y, a23);
+            }
+            const float4 ck = gather_cols(reduce_scatter4(unpk4(a01, a23), g, AddOp()), cw, 0);
+            asm volatile("" ::: "memory");
+            const float ckv[4] = {ck.x, ck.y, ck.z, ck.w};
+            const float beta = gt.g1;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const float u = (BITS == 32) ? ckv[j] : __fmul_rn(sv[j], ckv[j]);
+                wj[j] = __fmul_rn(beta, __fsub_rn(vv[j], u));
+            }
+        }
+        const uint64_t W01 = pk(wj[0], wj[1]), W23 = pk(wj[2], wj[3]);
+        const uint64_t S01 = pk(sv[0], sv[1]), S23 = pk(sv[2], sv[3]);
+#pragma unroll
+        for (int k = 0; k < RPT; k += 2) {
+            const ulonglong2 kk = *reinterpret_cast<const ulonglong2*>(kb + k);
+            const ulonglong2 aa = *reinterpret_cast<const ulonglong2*>(ga + k);
+            // S = c*(alpha_i s_j) + k_i w_j   (full-precision state: S*alpha_i + k_i w_j)
+            if constexpr (BITS == 32) {
+                S2[k][0] = fma2(S2[k][0], aa.x, mul2(kk.x, W01));
+                S2[k][1] = fma2(S2[k][1], aa.x, mul2(kk.x, W23));
+                S2[k + 1][0] = fma2(S2[k + 1][0], aa.y, mul2(kk.y, W01));
+                S2[k + 1][1] = fma2(S2[k + 1][1], aa.y, mul2(kk.y, W23));
+            } else {
+                S2[k][0] = fma2(S2[k][0], mul2(aa.x, S01), mul2(kk.x, W01));
+                S2[k][1] = fma2(S2[k][1], mul2(aa.x, S23), mul2(kk.x, W23));
+                S2[k + 1][0] = fma2(S2[k + 1][0], mul2(aa.y, S01), mul2(kk.y, W01));
+                S2[k + 1][1] = fma2(S2[k + 1][1], mul2(aa.y, S23), mul2(kk.y, W23));
+            }
+        }
     } else {
         const float dt = gt.g0;
         const float a = (p.g1 != nullptr) ? gt.g1 : expf(__fmul_rn(dt, gt.A));
@@ -272,6 +338,7 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
     const long long col = (long long)hu * p.dv + j0 + 4 * cw + c;
     if (g < 4) p.out[col] = o;
     float4 iv = make_float4(0.f, 0.f, 0.f, 0.f);
+    float mine_scale = 0.f;  // the scale (lanes g < 4) or multiplier (g >= 4) of this lane's column
     if constexpr (BITS != 32) {
         float m0 = 0.f, m1 = 0.f, m2 = 0.f, m3 = 0.f;
 #pragma unroll
@@ -284,9 +351,16 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
             m3 = max3_nan(m3, fabsf(x.w), fabsf(y.w));
         }
         const float m = reduce_scatter4(make_float4(m0, m1, m2, m3), g, MaxOp());
-        const float mine = scale_or_inv<BITS>(m, g);
-        if (g < 4) p.scales_out[col] = mine;
-        iv = gather_cols(mine, cw, 16);
+        if constexpr ((RND & kRndCopy) == 0) {
+            mine_scale = scale_or_inv<BITS>(m, g);
+        } else {
+            // copy scale: the column maximum of an unquantized copy of the state;
+            // the column's own maximum still decides whether it is finite
+            mine_scale = scale_or_inv<BITS>(__ldg(p.copy_absmax + col), g);
+            if (g >= 4 && !isfinite(m)) mine_scale = -0.0f;
+        }
+        if (g < 4) p.scales_out[col] = mine_scale;
+        iv = gather_cols(mine_scale, cw, 16);
     }
 
     // ---- store ------------------------------------------------------------------
@@ -299,12 +373,33 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
             *reinterpret_cast<ulonglong2*>(dst + ((g + kR * k) * 16 + 4 * cw) * 4) =
                 make_ulonglong2(S2[k][0], S2[k][1]);
     } else {
-        requantize_store<BITS, SR, RPT>(S2, iv, dst, g, cw, gcol, un.h, un.b, p.step, p.rk);
+        BdrRef bdr{};
+        if constexpr ((RND & kRndBdr) != 0) {
+            const float4 so = load_s4();
+            const float4 sn = gather_cols(mine_scale, cw, 0);
+            bdr.old_block = tile;
+            bdr.s_old01 = pk(so.x, so.y);
+            bdr.s_old23 = pk(so.z, so.w);
+            bdr.s_new01 = pk(sn.x, sn.y);
+            bdr.s_new23 = pk(sn.z, sn.w);
+        }
+        if constexpr ((RND & kRndCopy) != 0) {
+            // a copy scale can lie below the state's own maximum: the state is
+            // clipped to the copy's range first, so every code stays within +-r
+            const float4 mc = __ldg(reinterpret_cast<const float4*>(p.copy_absmax + (long long)hu * p.dv + j0 + 4 * cw));
+#pragma unroll
+            for (int k = 0; k < RPT; ++k) {
+                const float4 v = unpk4(S2[k][0], S2[k][1]);
+                S2[k][0] = pk(fminf(fmaxf(v.x, -mc.x), mc.x), fminf(fmaxf(v.y, -mc.y), mc.y));
+                S2[k][1] = pk(fminf(fmaxf(v.z, -mc.z), mc.z), fminf(fmaxf(v.w, -mc.w), mc.w));
+            }
+        }
+        requantize_store<BITS, RND, RPT>(S2, iv, dst, g, cw, gcol, un.h, un.b, p.step, p.rk, bdr);
         // rare: a non-finite column (multiplier -0.0) is stored as the zero code
         if (is_neg_zero(iv.x) || is_neg_zero(iv.y) || is_neg_zero(iv.z) || is_neg_zero(iv.w)) {
             atomicOr(p.flag, kFlagNonFinite);
             clear_nonfinite_columns<RPT>(S2, iv);
-            requantize_store<BITS, SR, RPT>(S2, iv, dst, g, cw, gcol, un.h, un.b, p.step, p.rk);
+            requantize_store<BITS, RND, RPT>(S2, iv, dst, g, cw, gcol, un.h, un.b, p.step, p.rk, bdr);
         }
     }
 
@@ -325,8 +420,18 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
     }
 }
 
-template <int FAM, int DK, int UB, bool F32STATE, bool SR>
-__global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (DecodeCfg<FAM, DK, UB, F32STATE>::MINB))
+// Resident CTAs per SM the register budget is sized for: Bounded Directional
+// Rounding re-decodes the previous codes while requantizing and needs more
+// registers than the plain rules.
+template <int FAM, int DK, int UB, bool F32STATE, int RND>
+constexpr int decode_min_blocks() {
+    using C = DecodeCfg<FAM, DK, UB, F32STATE>;
+    // BDR: about 168 registers per thread (65536 / (168 * 128) = 3 CTAs of 128 threads)
+    return (RND & kRndBdr) != 0 ? 384 / C::NT : C::MINB;
+}
+
+template <int FAM, int DK, int UB, bool F32STATE, int RND>
+__global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_min_blocks<FAM, DK, UB, F32STATE, RND>()))
     rsq_decode_kernel(const __grid_constant__ DecodeParams p) {
     using C = DecodeCfg<FAM, DK, UB, F32STATE>;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -370,12 +475,12 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (DecodeC
         }
         uint8_t* st = smem + stage * C::STAGE;
         if constexpr (F32STATE) {
-            process_block<FAM, DK, UB, true, false, 32>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
+            process_block<FAM, DK, UB, true, 0, 32>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
         } else {
             if (p.head_bits[cur.h] == 8)
-                process_block<FAM, DK, UB, false, SR, 8>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
+                process_block<FAM, DK, UB, false, RND, 8>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
             else
-                process_block<FAM, DK, UB, false, SR, 4>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
+                process_block<FAM, DK, UB, false, RND, 4>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
         }
         cur = nxt;
         gt = ng;
@@ -387,24 +492,33 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (DecodeC
 }
 
 // Kernel attributes for one instantiation.
-template <int FAM, int DK, int UB, bool F32, bool SR>
+template <int FAM, int DK, int UB, bool F32, int RND>
 int decode_info_one(int* threads, size_t* smem, const void** func) {
     using C = DecodeCfg<FAM, DK, UB, F32>;
     *threads = C::NT;
     *smem = C::SMEM;
-    *func = reinterpret_cast<const void*>(&rsq_decode_kernel<FAM, DK, UB, F32, SR>);
+    *func = reinterpret_cast<const void*>(&rsq_decode_kernel<FAM, DK, UB, F32, RND>);
     return 0;
 }
 
-// All (dk, blocks per unit) instantiations of one family.
-template <int FAM>
-int decode_info_family(int dk, int ub, bool f32state, bool sr, int* threads, size_t* smem,
+// All (dk, blocks per unit) instantiations of one family for the rounding
+// rules in RNDS (a full-precision state ignores the rounding: it is built with
+// the first rule only).  The rules are split over translation units so the
+// instantiations compile in parallel.
+template <int FAM, int RND0, int RND1>
+int decode_info_family(int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
                        const void** func) {
-#define RSQ_CASE(DK_, UB_)                                                                   \
-    if (dk == DK_ && ub == UB_) {                                                             \
-        if (f32state) return decode_info_one<FAM, DK_, UB_, true, false>(threads, smem, func); \
-        if (sr) return decode_info_one<FAM, DK_, UB_, false, true>(threads, smem, func);      \
-        return decode_info_one<FAM, DK_, UB_, false, false>(threads, smem, func);             \
+#define RSQ_CASE(DK_, UB_)                                                                      \
+    if (dk == DK_ && ub == UB_) {                                                                \
+        if (f32state) {                                                                          \
+            if constexpr (RND0 == 0)                                                             \
+                return decode_info_one<FAM, DK_, UB_, true, 0>(threads, smem, func);             \
+            else                                                                                 \
+                return -1;                                                                       \
+        }                                                                                        \
+        if (rnd == RND0) return decode_info_one<FAM, DK_, UB_, false, RND0>(threads, smem, func); \
+        if (rnd == RND1) return decode_info_one<FAM, DK_, UB_, false, RND1>(threads, smem, func); \
+        return -1;                                                                               \
     }
     RSQ_CASE(16, 1) RSQ_CASE(16, 2) RSQ_CASE(16, 4)
     RSQ_CASE(32, 1) RSQ_CASE(32, 2) RSQ_CASE(32, 4)

@@ -68,10 +68,12 @@ __device__ __forceinline__ void quantize_block(const QuantParams& p, const Block
             clear_nonfinite_columns<RPT>(S2, iv);
         }
         const uint32_t gcol = static_cast<uint32_t>(j0 / 4 + cw);
+        // no previous state: the base rounding of the context's rule
+        const BdrRef none{};
         if (p.sr)
-            requantize_store<BITS, true, RPT>(S2, iv, dst, g, cw, gcol, bi.h, bi.b, p.step, p.rk);
+            requantize_store<BITS, kRndSr, RPT>(S2, iv, dst, g, cw, gcol, bi.h, bi.b, p.step, p.rk, none);
         else
-            requantize_store<BITS, false, RPT>(S2, iv, dst, g, cw, gcol, bi.h, bi.b, p.step, p.rk);
+            requantize_store<BITS, 0, RPT>(S2, iv, dst, g, cw, gcol, bi.h, bi.b, p.step, p.rk, none);
     }
 }
 
@@ -114,6 +116,21 @@ __device__ __forceinline__ void dequantize_block(const DequantParams& p, const B
             S2[k][0] = mul2(S2[k][0], s01);
             S2[k][1] = mul2(S2[k][1], s23);
         }
+    }
+    if (p.absmax != nullptr) {
+        // column maxima of |S| (NaN-propagating), one lane per column after the reduce-scatter
+        float4 m4 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            const float4 v = unpk4(S2[k][0], S2[k][1]);
+            m4.x = max_nan(m4.x, fabsf(v.x));
+            m4.y = max_nan(m4.y, fabsf(v.y));
+            m4.z = max_nan(m4.z, fabsf(v.z));
+            m4.w = max_nan(m4.w, fabsf(v.w));
+        }
+        const float m = reduce_scatter4(m4, g, MaxOp());
+        if (g < 4) p.absmax[(long long)bi.hu * p.dv + j0 + 4 * cw + col_of(g)] = m;
+        return;
     }
 #pragma unroll
     for (int k = 0; k < RPT; ++k)

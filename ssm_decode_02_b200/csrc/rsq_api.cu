@@ -41,6 +41,9 @@ rsq_status cuda_fail(int err, const char* what) {
     return fail(RSQ_E_CUDA, "%s: %s", what, cudaGetErrorString(static_cast<cudaError_t>(err)));
 }
 
+constexpr int kCopyScaleBit = 4;  // kernel rule bit of the copy scale (beside the rsq_rounding bits)
+bool family_ok(int f) { return f == RSQ_GDN || f == RSQ_MAMBA2 || f == RSQ_GLA || f == RSQ_KDA; }
+bool rounding_ok(int r) { return r == RSQ_RTN || r == RSQ_SR || r == RSQ_BDR || r == RSQ_SR_BDR; }
 bool dk_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
 bool dv_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
 
@@ -110,12 +113,12 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
     if (!cfg || !out) return fail(RSQ_E_INVAL, "create: null argument");
     *out = nullptr;
     const rsq_config& c = *cfg;
-    if (c.family != RSQ_GDN && c.family != RSQ_MAMBA2) return fail(RSQ_E_INVAL, "create: bad family %d", c.family);
+    if (!family_ok(c.family)) return fail(RSQ_E_INVAL, "create: bad family %d", c.family);
     if (c.batch < 1) return fail(RSQ_E_INVAL, "create: batch must be >= 1");
     if (c.heads < 1 || c.heads > RSQ_MAX_HEADS) return fail(RSQ_E_INVAL, "create: heads must be in [1, %d]", RSQ_MAX_HEADS);
     if (!dk_ok(c.dk) || !dv_ok(c.dv))
         return fail(RSQ_E_UNSUPPORTED, "create: dk must be one of 16, 32, 64, 128 and dv one of 16, 32, 64, 128, 256 (got %d, %d)", c.dk, c.dv);
-    if (c.rounding != RSQ_RTN && c.rounding != RSQ_SR) return fail(RSQ_E_INVAL, "create: bad rounding %d", c.rounding);
+    if (!rounding_ok(c.rounding)) return fail(RSQ_E_INVAL, "create: bad rounding %d", c.rounding);
     if (c.in_dtype != RSQ_F32 && c.in_dtype != RSQ_BF16) return fail(RSQ_E_INVAL, "create: bad in_dtype %d", c.in_dtype);
     if (c.family == RSQ_MAMBA2 && (c.ngroups < 1 || c.heads % c.ngroups != 0))
         return fail(RSQ_E_INVAL, "create: ngroups must divide heads");
@@ -158,7 +161,7 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
     int threads = 0;
     size_t smem = 0;
     const void* func = nullptr;
-    if (rsq::decode_kernel_info(c.family, c.dk, ctx->ub, ctx->f32state, c.rounding == RSQ_SR, &threads,
+    if (rsq::decode_kernel_info(c.family, c.dk, ctx->ub, ctx->f32state, c.rounding, &threads,
                                 &smem, &func) != 0) {
         delete ctx;
         return fail(RSQ_E_UNSUPPORTED, "create: no kernel for dk=%d dv=%d", c.dk, c.dv);
@@ -169,6 +172,15 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
     if (!err) err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
     if (!err) err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, func, threads, smem);
     if (!err && per_sm < 1) err = cudaErrorInvalidConfiguration;
+    if (!err && !ctx->f32state) {
+        // the copy-scale instance of the same rule (rsq_decode_step_copy_scale)
+        int t2 = 0;
+        size_t sm2 = 0;
+        const void* f2 = nullptr;
+        if (rsq::decode_kernel_info(c.family, c.dk, ctx->ub, false, c.rounding | kCopyScaleBit, &t2, &sm2,
+                                    &f2) == 0)
+            err = cudaFuncSetAttribute(f2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2));
+    }
     if (!err) err = cudaMalloc(&ctx->flag, sizeof(unsigned));
     if (!err) err = cudaMemset(ctx->flag, 0, sizeof(unsigned));
     if (err) {
@@ -202,8 +214,52 @@ rsq_status rsq_head_offset(const rsq_ctx* ctx, int h, size_t* offset) {
     return RSQ_OK;
 }
 
+namespace {
+rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const rsq_state* state_out,
+                            const void* inputs, const float* copy_absmax, float* out, uint32_t step,
+                            void* stream);
+}
+
 rsq_status rsq_decode_step(const rsq_ctx* ctx, const rsq_state* state_in, const rsq_state* state_out,
                            const void* inputs, float* out, uint32_t step, void* stream) {
+    return decode_step_impl(ctx, state_in, state_out, inputs, nullptr, out, step, stream);
+}
+
+rsq_status rsq_decode_step_copy_scale(const rsq_ctx* ctx, const rsq_state* state_in,
+                                      const rsq_state* state_out, const void* inputs,
+                                      const float* copy_absmax, float* out, uint32_t step,
+                                      void* stream) {
+    if (!ctx) return fail(RSQ_E_INVAL, "decode_step_copy_scale: null context");
+    if (!copy_absmax || !aligned16(copy_absmax))
+        return fail(RSQ_E_INVAL, "decode_step_copy_scale: copy_absmax null or not 16-byte aligned");
+    if (ctx->f32state)
+        return fail(RSQ_E_UNSUPPORTED, "decode_step_copy_scale: a full-precision state has no scale");
+    return decode_step_impl(ctx, state_in, state_out, inputs, copy_absmax, out, step, stream);
+}
+
+rsq_status rsq_column_absmax(const rsq_ctx* ctx, const rsq_state* state, float* absmax, void* stream) {
+    if (!ctx) return fail(RSQ_E_INVAL, "column_absmax: null context");
+    if (!absmax || !aligned16(absmax)) return fail(RSQ_E_INVAL, "column_absmax: absmax null or not 16-byte aligned");
+    rsq_status s = check_state(ctx, state, "column_absmax(state)");
+    if (s) return s;
+    const rsq_config& c = ctx->cfg;
+    rsq::DequantParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.B = c.batch; p.H = c.heads; p.dk = c.dk; p.dv = c.dv; p.ncb = ctx->ncb;
+    p.row_bytes = ctx->row_bytes;
+    p.codes = static_cast<const uint8_t*>(state->codes);
+    p.scales = state->scales;
+    p.absmax = absmax;
+    fill_heads(ctx, p);
+    const int err = rsq::launch_dequantize(c.dk, p, stream);
+    if (err) return cuda_fail(err, "column_absmax launch");
+    return RSQ_OK;
+}
+
+namespace {
+rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const rsq_state* state_out,
+                            const void* inputs, const float* copy_absmax, float* out, uint32_t step,
+                            void* stream) {
     if (!ctx) return fail(RSQ_E_INVAL, "decode_step: null context");
     rsq_status s = check_state(ctx, state_in, "decode_step(state_in)");
     if (s) return s;
@@ -215,13 +271,14 @@ rsq_status rsq_decode_step(const rsq_ctx* ctx, const rsq_state* state_in, const 
     std::memset(&p, 0, sizeof(p));
     p.B = c.batch; p.H = c.heads; p.dk = c.dk; p.dv = c.dv; p.ncb = ctx->ncb; p.units = ctx->units;
     p.in_bf16 = (c.in_dtype == RSQ_BF16);
-    p.sr = (c.rounding == RSQ_SR);
+    p.sr = (c.rounding & RSQ_SR) != 0;
     p.row_bytes = ctx->row_bytes;
     p.codes_in = static_cast<const uint8_t*>(state_in->codes);
     p.codes_out = static_cast<uint8_t*>(state_out->codes);
     p.scales_in = state_in->scales;
     p.scales_out = state_out->scales;
     p.out = out;
+    p.copy_absmax = copy_absmax;
     p.flag = ctx->flag;
     p.step = step;
     p.key0 = static_cast<uint32_t>(c.seed);
@@ -234,6 +291,15 @@ rsq_status rsq_decode_step(const rsq_ctx* ctx, const rsq_state* state_in, const 
         if (!aligned16(in->q) || !aligned16(in->k) || !aligned16(in->v))
             return fail(RSQ_E_INVAL, "decode_step: q/k/v not 16-byte aligned");
         p.vA = in->q; p.vB = in->k; p.vC = in->v; p.g0 = in->alpha; p.g1 = in->beta;
+        p.ngroups = 1; p.heads_per_group = c.heads;
+    } else if (c.family == RSQ_GLA || c.family == RSQ_KDA) {
+        const rsq_diag_inputs* in = static_cast<const rsq_diag_inputs*>(inputs);
+        if (!in->q || !in->k || !in->v || !in->alpha || (c.family == RSQ_KDA && !in->beta))
+            return fail(RSQ_E_INVAL, "decode_step: null GLA/KDA input");
+        if (!aligned16(in->q) || !aligned16(in->k) || !aligned16(in->v) || !aligned16(in->alpha))
+            return fail(RSQ_E_INVAL, "decode_step: q/k/v/alpha not 16-byte aligned");
+        p.vA = in->q; p.vB = in->k; p.vC = in->v; p.vD = in->alpha;
+        p.g0 = nullptr; p.g1 = (c.family == RSQ_KDA) ? in->beta : nullptr;
         p.ngroups = 1; p.heads_per_group = c.heads;
     } else {
         const rsq_mamba2_inputs* in = static_cast<const rsq_mamba2_inputs*>(inputs);
@@ -251,11 +317,14 @@ rsq_status rsq_decode_step(const rsq_ctx* ctx, const rsq_state* state_in, const 
     const int ghu = ctx->grid / ctx->ncb;
     p.gh = ghu % c.heads;
     p.gb = ghu / c.heads;
-    const int err = rsq::launch_decode(c.family, c.dk, ctx->ub, ctx->f32state, c.rounding == RSQ_SR, p,
+    const int err = rsq::launch_decode(c.family, c.dk, ctx->ub, ctx->f32state,
+                                       c.rounding | (copy_absmax ? kCopyScaleBit : 0), p,
                                        stream);
     if (err) return cuda_fail(err, "decode_step launch");
     return RSQ_OK;
 }
+
+}  // namespace
 
 rsq_status rsq_quantize(const rsq_ctx* ctx, const float* S, const rsq_state* state_out, uint32_t step,
                         void* stream) {
@@ -267,7 +336,7 @@ rsq_status rsq_quantize(const rsq_ctx* ctx, const float* S, const rsq_state* sta
     rsq::QuantParams p;
     std::memset(&p, 0, sizeof(p));
     p.B = c.batch; p.H = c.heads; p.dk = c.dk; p.dv = c.dv; p.ncb = ctx->ncb; p.units = ctx->units;
-    p.sr = (c.rounding == RSQ_SR);
+    p.sr = (c.rounding & RSQ_SR) != 0;
     p.row_bytes = ctx->row_bytes;
     p.S = S;
     p.codes = static_cast<uint8_t*>(state_out->codes);
@@ -396,14 +465,14 @@ extern "C" rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_s
                                               float* out, uint32_t step, void* stream) {
     if (!cfg) return fail(RSQ_E_INVAL, "decode_step_noalloc: null config");
     const rsq_config& c = *cfg;
-    if (c.family != RSQ_GDN && c.family != RSQ_MAMBA2)
+    if (!family_ok(c.family))
         return fail(RSQ_E_INVAL, "decode_step_noalloc: bad family %d", c.family);
     if (c.batch < 1) return fail(RSQ_E_INVAL, "decode_step_noalloc: batch must be >= 1");
     if (c.heads < 1 || c.heads > RSQ_MAX_HEADS)
         return fail(RSQ_E_INVAL, "decode_step_noalloc: heads must be in [1, %d]", RSQ_MAX_HEADS);
     if (!dk_ok(c.dk) || !dv_ok(c.dv))
         return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: unsupported dk=%d dv=%d", c.dk, c.dv);
-    if (c.rounding != RSQ_RTN && c.rounding != RSQ_SR)
+    if (!rounding_ok(c.rounding))
         return fail(RSQ_E_INVAL, "decode_step_noalloc: bad rounding %d", c.rounding);
     if (c.in_dtype != RSQ_F32 && c.in_dtype != RSQ_BF16)
         return fail(RSQ_E_INVAL, "decode_step_noalloc: bad in_dtype %d", c.in_dtype);
@@ -444,7 +513,7 @@ extern "C" rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_s
     int threads = 0;
     size_t smem = 0;
     const void* func = nullptr;
-    if (rsq::decode_kernel_info(c.family, c.dk, ctx.ub, ctx.f32state, c.rounding == RSQ_SR, &threads, &smem,
+    if (rsq::decode_kernel_info(c.family, c.dk, ctx.ub, ctx.f32state, c.rounding, &threads, &smem,
                                 &func) != 0)
         return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: no kernel for dk=%d dv=%d", c.dk, c.dv);
     int err = cudaGetDevice(&ctx.device);

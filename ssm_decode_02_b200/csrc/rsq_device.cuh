@@ -96,6 +96,18 @@ __device__ __forceinline__ uint64_t add2_rm(uint64_t a, uint64_t b) {
     return d;
 }
 
+// d = a*b + c rounded toward plus / minus infinity (exact product, one rounding)
+__device__ __forceinline__ uint64_t fma2_rp(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rp.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t fma2_rm(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rm.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+
 // hi(a * b) + c (32-bit unsigned)
 __device__ __forceinline__ uint32_t umulhi_add(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;

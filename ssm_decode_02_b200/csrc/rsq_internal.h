@@ -44,11 +44,13 @@ struct DecodeParams {
     const void* vA;                // GDN q      | Mamba-2 C
     const void* vB;                // GDN k      | Mamba-2 B
     const void* vC;                // GDN v      | Mamba-2 x
-    const float* g0;               // GDN alpha  | Mamba-2 dt
-    const float* g1;               // GDN beta   | Mamba-2 decay override (may be null)
+    const float* vD;               // GLA / KDA decay per key channel [B][H][dk]
+    const float* g0;               // GDN alpha  | Mamba-2 dt                          | GLA, KDA: unused
+    const float* g1;               // GDN beta   | Mamba-2 decay override (may be null) | KDA beta
     const float* A;                // Mamba-2 A [H]
     const float* D;                // Mamba-2 D [H]
     float* out;                    // [B][H][dv]
+    const float* copy_absmax;      // copy scale: column maxima [B][H][dv] of an unquantized copy, or null
     unsigned* flag;
     uint32_t step, key0, key1;
     PhiloxKeys rk;                 // Philox round keys of (key0, key1)
@@ -75,7 +77,8 @@ struct DequantParams {
     long long row_bytes;
     const uint8_t* codes;
     const float* scales;
-    float* S;                      // natural [B][H][dk][dv]
+    float* S;                      // natural [B][H][dk][dv] (dequantize), or null
+    float* absmax;                 // [B][H][dv] column maxima of |S| (column_absmax), or null
     uint32_t head_off[RSQ_MAX_HEADS];
     uint8_t head_bits[RSQ_MAX_HEADS];
 };
@@ -93,9 +96,9 @@ struct DriftParams {
 
 // Launchers (defined in the .cu files).  Return a cudaError_t value.
 // ub = 16-column blocks per decode work unit (1, 2 or 4)
-int launch_decode(int family, int dk, int ub, bool f32state, bool sr, const DecodeParams& p,
+int launch_decode(int family, int dk, int ub, bool f32state, int rnd, const DecodeParams& p,
                   void* stream);
-int decode_kernel_info(int family, int dk, int ub, bool f32state, bool sr, int* threads, size_t* smem,
+int decode_kernel_info(int family, int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
                        const void** func);
 int launch_quantize(int dk, const QuantParams& p, void* stream);
 int launch_dequantize(int dk, const DequantParams& p, void* stream);

@@ -21,6 +21,13 @@ constexpr uint32_t kMagicBits = 0x4B400000u;
 constexpr uint32_t kSrBits8 = 0x43000000u;  // 128.0f: SR offset of 8-bit codes
 constexpr uint32_t kSrBits4 = 0x43080000u;  // 136.0f: SR offset of 4-bit codes
 
+// Requantization rule of a kernel instance: bit 0 = stochastic base rounding
+// (else nearest), bit 1 = Bounded Directional Rounding on top of it, bit 2 =
+// scales from the column maxima of an unquantized copy (copy scale).
+constexpr int kRndSr = 1;
+constexpr int kRndBdr = 2;
+constexpr int kRndCopy = 4;
+
 constexpr int kBlockCols = 16;  // columns per stored block (one warp)
 constexpr int kR = 8;           // partial sums over the key axis (row groups)
 
@@ -156,6 +163,19 @@ __device__ __forceinline__ void load_codes(const uint8_t* blk, int g, int cw, ui
     }
 }
 
+// Exact float codes of row g + 8k of a stored block (this lane's 4 columns).
+template <int BITS>
+__device__ __forceinline__ void load_code_row(const uint8_t* blk, int g, int cw, int k, uint64_t& c01,
+                                              uint64_t& c23) {
+    uint64_t S2[1][2];
+    if constexpr (BITS == 8)
+        load_codes<8, 1>(blk + kR * k * 16, g, cw, S2);
+    else
+        load_codes<4, 1>(blk + kR * k * 8, g, cw, S2);
+    c01 = S2[0][0];
+    c23 = S2[0][1];
+}
+
 // Pack the 4 codes of one row held in the low byte (RTN) or byte 2 (4-bit SR)
 // of four floats into the stored representation.
 template <int BITS>
@@ -190,17 +210,41 @@ __device__ __forceinline__ void clear_nonfinite_columns(uint64_t (&S2)[RPT][2], 
     }
 }
 
+// What Bounded Directional Rounding needs besides the new state: the previous
+// codes (the stage's copy of the stored block) and scales, and the new scales.
+struct BdrRef {
+    const uint8_t* old_block;  // stored block as loaded (shared memory)
+    uint64_t s_old01, s_old23;  // previous scales of this lane's 4 columns
+    uint64_t s_new01, s_new23;  // new scales of this lane's 4 columns
+};
+
+// Bounded Directional Rounding of one element, in the magic domain T = c + M
+// (M = 1.5 * 2^23 + code offset): the base code tb stands unless its value
+// c * s_new lies strictly on the other side of the previous value prev than
+// the new state S does; then the integer next to x = S * inv on the update's
+// side (tu = ceil, td = floor) replaces it.
+__device__ __forceinline__ float bdr_pick(float S, float prev, float now, float tb, float tu, float td) {
+    const bool up = (S > prev) && (now < prev);
+    const bool down = (S < prev) && (now > prev);
+    return up ? tu : (down ? td : tb);
+}
+
 // Requantize this lane's RPT x 4 part of the full-precision state and store it
 // to the block `dst` (global memory).
 //   RTN: nearest integer of the exact S*inv (fma with a magic offset).
 //   SR : t = fma(S, inv, o + u/2^16), c = floor(t) - o, u a 16-bit uniform from
 //        Philox4x32-10 with counter {i mod dk/2 | (j/4) << 16, h, b, step}.
+//   +BDR: the base code is replaced by ceil / floor of the exact S*inv when it
+//        moves the element opposite to its update (see bdr_pick).
 // `gcol` is j/4 of this lane's first column.
-template <int BITS, bool SR, int RPT, class PhiloxKeysT>
+template <int BITS, int RND, int RPT, class PhiloxKeysT>
 __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], const float4& iv,
                                                  uint8_t* dst, int g, int cw, uint32_t gcol,
                                                  uint32_t h, uint32_t b, uint32_t step,
-                                                 const PhiloxKeysT& rk) {
+                                                 const PhiloxKeysT& rk, const BdrRef& bdr) {
+    constexpr bool SR = (RND & kRndSr) != 0;
+    constexpr bool BDR = (RND & kRndBdr) != 0;
+    constexpr float kOff = (BITS == 8) ? 128.0f : 8.0f;  // stored code = c + kOff
     const uint64_t inv01 = pk(iv.x, iv.y), inv23 = pk(iv.z, iv.w);
     // this lane's first row; row k sits k * 8 rows further
     uint8_t* const row0 = dst + (BITS == 8 ? g * 16 + 4 * cw : g * 8 + 2 * cw);
@@ -210,17 +254,32 @@ __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], c
         else
             *reinterpret_cast<uint16_t*>(row0 + k * (kR * 8)) = static_cast<uint16_t>(word);
     };
-    if constexpr (!SR) {
-        const float o = (BITS == 8) ? kMagic + 128.0f : kMagic + 8.0f;
-        const uint64_t oo = pk(o, o);
-#pragma unroll
-        for (int k = 0; k < RPT; ++k) {
-            float t0, t1, t2, t3;
-            upk(fma2(S2[k][0], inv01, oo), t0, t1);
-            upk(fma2(S2[k][1], inv23, oo), t2, t3);
-            store_row(k, pack_row<BITS>(__float_as_uint(t0), __float_as_uint(t1),
-                                        __float_as_uint(t2), __float_as_uint(t3), false));
+    const uint64_t moff = pk(kMagic + kOff, kMagic + kOff);
+    // Row k with its base codes T = c + M + kOff (two packed pairs): apply the
+    // directional correction if enabled, then pack and store (low byte = c + kOff).
+    auto finish_row = [&](int k, uint64_t T01, uint64_t T23) {
+        if constexpr (BDR) {
+            const uint64_t nmoff = pk(-(kMagic + kOff), -(kMagic + kOff));
+            uint64_t c01, c23;
+            load_code_row<BITS>(bdr.old_block, g, cw, k, c01, c23);
+            const float4 prev = unpk4(mul2(c01, bdr.s_old01), mul2(c23, bdr.s_old23));
+            const float4 now = unpk4(mul2(add2(T01, nmoff), bdr.s_new01), mul2(add2(T23, nmoff), bdr.s_new23));
+            const float4 tu = unpk4(fma2_rp(S2[k][0], inv01, moff), fma2_rp(S2[k][1], inv23, moff));
+            const float4 td = unpk4(fma2_rm(S2[k][0], inv01, moff), fma2_rm(S2[k][1], inv23, moff));
+            const float4 S = unpk4(S2[k][0], S2[k][1]);
+            const float4 tb = unpk4(T01, T23);
+            T01 = pk(bdr_pick(S.x, prev.x, now.x, tb.x, tu.x, td.x), bdr_pick(S.y, prev.y, now.y, tb.y, tu.y, td.y));
+            T23 = pk(bdr_pick(S.z, prev.z, now.z, tb.z, tu.z, td.z), bdr_pick(S.w, prev.w, now.w, tb.w, tu.w, td.w));
         }
+        float t0, t1, t2, t3;
+        upk(T01, t0, t1);
+        upk(T23, t2, t3);
+        store_row(k, pack_row<BITS>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
+                                    __float_as_uint(t3), false));
+    };
+    if constexpr (!SR) {
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) finish_row(k, fma2(S2[k][0], inv01, moff), fma2(S2[k][1], inv23, moff));
     } else {
         constexpr uint32_t vb = (BITS == 8) ? kSrBits8 : kSrBits4;
         const uint64_t mm = pk(kMagic, kMagic);
@@ -239,17 +298,26 @@ __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], c
                 const uint64_t V23 = pk(__uint_as_float(vb | (w1 & 0xFFFFu)), __uint_as_float(umulhi_add(w1, 0x10000u, vb)));
                 uint64_t t01 = fma2(S2[kk][0], inv01, V01);
                 uint64_t t23 = fma2(S2[kk][1], inv23, V23);
-                if constexpr (BITS == 8) {
-                    // floor(t) + magic: byte 0 = floor(t) = c + 128
+                if constexpr (BITS == 8 || BDR) {
+                    // floor(t) + magic = c + o + magic
                     t01 = add2_rm(t01, mm);
                     t23 = add2_rm(t23, mm);
                 }
-                float t0, t1, t2, t3;
-                upk(t01, t0, t1);
-                upk(t23, t2, t3);
-                // 4-bit: t in [129, 144) so byte 2 of t is floor(t) - 128 = c + 8
-                store_row(kk, pack_row<BITS>(__float_as_uint(t0), __float_as_uint(t1),
-                                             __float_as_uint(t2), __float_as_uint(t3), BITS == 4));
+                if constexpr (BITS == 8) {
+                    // o = 128 = kOff: byte 0 already holds c + 128
+                    finish_row(kk, t01, t23);
+                } else if constexpr (BDR) {
+                    // o = 136 = kOff + 128
+                    const uint64_t m128 = pk(-128.0f, -128.0f);
+                    finish_row(kk, add2(t01, m128), add2(t23, m128));
+                } else {
+                    // 4-bit: t in [129, 144) so byte 2 of t is floor(t) - 128 = c + 8
+                    float t0, t1, t2, t3;
+                    upk(t01, t0, t1);
+                    upk(t23, t2, t3);
+                    store_row(kk, pack_row<BITS>(__float_as_uint(t0), __float_as_uint(t1),
+                                                 __float_as_uint(t2), __float_as_uint(t3), true));
+                }
             }
         }
     }

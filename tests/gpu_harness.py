@@ -41,7 +41,8 @@ class Run:
         self.rounding = {"rtn": rsq.RSQ_RTN, "sr": rsq.RSQ_SR}[w.rounding] if rounding is None else rounding
         self.seed = w.sr_seed if seed is None else seed
         self.in_dtype = {"f32": rsq.RSQ_F32, "bf16": rsq.RSQ_BF16}[w.in_dtype] if in_dtype is None else in_dtype
-        self.family = rsq.RSQ_GDN if w.family == "gdn" else rsq.RSQ_MAMBA2
+        self.family = {"gdn": rsq.RSQ_GDN, "mamba2": rsq.RSQ_MAMBA2, "gla": rsq.RSQ_GLA,
+                       "kda": rsq.RSQ_KDA}[w.family]
         self.ctx = rsq.Context(self.family, self.B, self.H, self.dk, self.dv, head_bits=self.head_bits,
                                rounding=self.rounding, in_dtype=self.in_dtype, seed=self.seed,
                                ngroups=w.ngroups)
@@ -80,6 +81,8 @@ class Run:
         keep = {k: dev(v) for k, v in inp.items()}
         if self.family == rsq.RSQ_GDN:
             s = rsq.gdn_inputs(keep["q"], keep["k"], keep["v"], keep["alpha"], keep["beta"])
+        elif self.family in (rsq.RSQ_GLA, rsq.RSQ_KDA):
+            s = rsq.diag_inputs(keep["q"], keep["k"], keep["v"], keep["alpha"], keep.get("beta"))
         else:
             dd = None if decay is None else dev(np.ascontiguousarray(decay, np.float32))
             keep["decay"] = dd
@@ -99,6 +102,10 @@ class Run:
         if self.family == rsq.RSQ_GDN:
             return oracle.gdn_step(st, inp, self.head_bits, rounding=self.rounding, seed=self.seed,
                                    step=t, mode=mode, R=self.R, heads=heads)
+        if self.family in (rsq.RSQ_GLA, rsq.RSQ_KDA):
+            step = oracle.gla_step if self.family == rsq.RSQ_GLA else oracle.kda_step
+            return step(st, inp, self.head_bits, rounding=self.rounding, seed=self.seed, step=t,
+                        mode=mode, R=self.R, heads=heads)
         return oracle.mamba2_step(st, inp, self.head_bits, rounding=self.rounding, seed=self.seed,
                                   step=t, mode=mode, R=self.R, ngroups=self.w.ngroups, decay=decay,
                                   heads=heads)

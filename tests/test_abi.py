@@ -55,7 +55,8 @@ def _create(**kw):
     (dict(dk=100), rsq.RSQ_E_UNSUPPORTED),
     (dict(dk=256), rsq.RSQ_E_UNSUPPORTED),
     (dict(dv=8), rsq.RSQ_E_UNSUPPORTED),
-    (dict(rounding=3), rsq.RSQ_E_INVAL),
+    (dict(rounding=4), rsq.RSQ_E_INVAL),
+    (dict(rounding=-1), rsq.RSQ_E_INVAL),
     (dict(in_dtype=9), rsq.RSQ_E_INVAL),
     (dict(head_bits=[8, 4, 2, 8]), rsq.RSQ_E_INVAL),
     (dict(head_bits=[8, 32, 32, 32]), rsq.RSQ_E_UNSUPPORTED),

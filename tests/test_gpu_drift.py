@@ -23,17 +23,19 @@ import bench  # noqa: E402
 
 
 def _oracle_series(w, steps, every, variants):
-    rnd = {"sr": oracle.SR, "rtn": oracle.RTN}
+    rnd = {"sr": oracle.SR, "rtn": oracle.RTN, "bdr": oracle.BDR, "sr_bdr": oracle.SR_BDR}
     ref = oracle.zero_state(w.B, w.H, w.dk, w.dv, fp32=True)
-    qs = {lab: oracle.zero_state(w.B, w.H, w.dk, w.dv, fp32=False) for lab, _, _ in variants}
-    out = {lab: [] for lab, _, _ in variants}
+    qs = {lab: oracle.zero_state(w.B, w.H, w.dk, w.dv, fp32=False) for lab, _, _, _ in variants}
+    out = {lab: [] for lab, _, _, _ in variants}
     f32 = np.full(w.H, 32, np.int8)
     for t in range(steps):
         inp = W.inputs(w, t)
         ref, o_ref = oracle.gdn_step(ref, inp, f32, rounding=oracle.RTN, seed=w.sr_seed, step=t)
-        for lab, bits, r in variants:
+        m = np.abs(ref["f"]).max(axis=2)
+        for lab, bits, r, src in variants:
             hb = np.full(w.H, bits, np.int8)
-            qs[lab], o = oracle.gdn_step(qs[lab], inp, hb, rounding=rnd[r], seed=w.sr_seed, step=t)
+            qs[lab], o = oracle.gdn_step(qs[lab], inp, hb, rounding=rnd[r], seed=w.sr_seed, step=t,
+                                         copy_absmax=m if src == "copy" else None)
             if (t + 1) % every == 0:
                 F = oracle.dequantize(ref, f32).astype(np.float64)
                 D = oracle.dequantize(qs[lab], hb).astype(np.float64)
@@ -50,7 +52,7 @@ def test_drift_series_matches_oracle():
     steps, every = 24, 8
     got = bench.drift_series(w, steps, every)
     want = _oracle_series(w, steps, every, bench.DRIFT_VARIANTS)
-    for lab, _, _ in bench.DRIFT_VARIANTS:
+    for lab, _, _, _ in bench.DRIFT_VARIANTS:
         g, e = np.array(got[lab]), np.array(want[lab])
         assert g.shape == e.shape == (steps // every, 4)
         assert np.array_equal(g[:, 0], e[:, 0])
