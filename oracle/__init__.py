@@ -69,6 +69,14 @@ def lib():
         L.orc_bdr_adjust.argtypes = [ctypes.c_int, ctypes.c_float, ctypes.c_float, ctypes.c_float,
                                      ctypes.c_int, ctypes.c_int]
         L.orc_bdr_adjust.restype = ctypes.c_int
+        L.orc_e4m3_encode.argtypes = [ctypes.c_float]
+        L.orc_e4m3_encode.restype = ctypes.c_uint8
+        L.orc_e4m3_decode.argtypes = [ctypes.c_uint8]
+        L.orc_e4m3_decode.restype = ctypes.c_float
+        L.orc_gdn_pw_head_step.argtypes = [ctypes.POINTER(_Head), ctypes.c_int, ctypes.c_int, P, P, P, P,
+                                           P, P, P, P, P, P, ctypes.c_float, ctypes.c_float, P, P, P,
+                                           P, P, P, P, P]
+        L.orc_gdn_pw_head_step.restype = ctypes.c_int
         L.orc_allocate_bits.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, P]
         _lib = L
@@ -289,6 +297,78 @@ def kda_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, ste
              mode: int = CANONICAL, R: int = 8, heads=None, copy_absmax=None):
     """One KDA decode step (delta rule with a decay vector alpha [B][H][dk] and gate beta [B][H])."""
     return _diag_step(1, state, inp, head_bits, rounding, seed, step, mode, R, heads, copy_absmax)
+
+
+def e4m3_encode(x: float) -> int:
+    """FP8 E4M3 code of x (round to nearest even, saturating to +-448)."""
+    return int(lib().orc_e4m3_encode(float(x)))
+
+
+def e4m3_decode(code: int) -> float:
+    return float(lib().orc_e4m3_decode(int(code)))
+
+
+def zero_window(B: int, H: int, W: int, dk: int, dv: int, fp32: bool = False) -> dict:
+    """An empty pure-write window (all slots zero): a [B][H][W][dk], b [B][H][W][dv]
+    as FP8 codes with scales as [B][H][W], bs [B][H][W] (binary32 vectors when fp32)."""
+    t = np.float32 if fp32 else np.uint8
+    return {"a": np.zeros((B, H, W, dk), t), "as": np.zeros((B, H, W), np.float32),
+            "b": np.zeros((B, H, W, dv), t), "bs": np.zeros((B, H, W), np.float32)}
+
+
+def gdn_pw_step(state: dict, window: dict, inp: dict, head_bits, *, rounding: int, seed: int,
+                step: int, mode: int = CANONICAL, R: int = 8, heads=None, fp32window: bool = False):
+    """One Gated DeltaNet decode step with a pure-write window (slot step % W is
+    merged into the history and takes the new write).  Returns (state, window, o)."""
+    B, H, dk, dv = state["codes"].shape
+    W = window["a"].shape[2]
+    q, k, v = widen(inp["q"]), widen(inp["k"]), widen(inp["v"])
+    alpha, beta = _c(inp["alpha"], np.float32), _c(inp["beta"], np.float32)
+    new = copy_state(state)
+    win = {key: val.copy() for key, val in window.items()}
+    o = np.zeros((B, H, dv), np.float32)
+    L = lib()
+    vt = np.float32 if fp32window else np.uint8
+    for b, h in _heads(B, H, heads):
+        bits = int(head_bits[h])
+        hd = _head(dk, dv, bits, rounding, mode, R, seed, b, h, step)
+        c_in, s_in, f_in = (_c(state["codes"][b, h], np.int8), _c(state["scales"][b, h], np.float32),
+                            _f_in(state, b, h, dk, dv))
+        a_in, as_in = _c(window["a"][b, h], vt), _c(window["as"][b, h], np.float32)
+        b_in, bs_in = _c(window["b"][b, h], vt), _c(window["bs"][b, h], np.float32)
+        c_out = np.zeros((dk, dv), np.int8)
+        s_out = np.zeros(dv, np.float32)
+        f_out = np.zeros((dk, dv), np.float32)
+        a_out, as_out = np.zeros_like(a_in), np.zeros_like(as_in)
+        b_out, bs_out = np.zeros_like(b_in), np.zeros_like(bs_in)
+        o_h = np.zeros(dv, np.float32)
+        qh, kh, vh = _c(q[b, h], np.float32), _c(k[b, h], np.float32), _c(v[b, h], np.float32)
+        rc = L.orc_gdn_pw_head_step(ctypes.byref(hd), int(W), int(fp32window), _p(c_in), _p(s_in),
+                                    _p(f_in), _p(a_in), _p(as_in), _p(b_in), _p(bs_in), _p(qh),
+                                    _p(kh), _p(vh), float(alpha[b, h]), float(beta[b, h]),
+                                    _p(c_out), _p(s_out), _p(f_out), _p(a_out), _p(as_out),
+                                    _p(b_out), _p(bs_out), _p(o_h))
+        assert rc == 0
+        if bits == 32:
+            new["f"][b, h] = f_out
+        else:
+            new["codes"][b, h] = c_out
+            new["scales"][b, h] = s_out
+        win["a"][b, h], win["as"][b, h], win["b"][b, h], win["bs"][b, h] = a_out, as_out, b_out, bs_out
+        o[b, h] = o_h
+    return new, win, o
+
+
+def window_full_state(state: dict, window: dict, head_bits, fp32window: bool = False) -> np.ndarray:
+    """The full state H + sum_w a_w b_w^T (float64) of a state with a pure-write window."""
+    Hs = dequantize(state, head_bits).astype(np.float64)
+    if fp32window:
+        a, b = window["a"].astype(np.float64), window["b"].astype(np.float64)
+    else:
+        dec = np.vectorize(e4m3_decode, otypes=[np.float32])
+        a = (dec(window["a"]) * window["as"][..., None]).astype(np.float64)
+        b = (dec(window["b"]) * window["bs"][..., None]).astype(np.float64)
+    return Hs + np.einsum("bhwi,bhwj->bhij", a, b)
 
 
 def quantize(S: np.ndarray, head_bits, *, rounding: int, seed: int, step: int,

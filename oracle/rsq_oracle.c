@@ -18,6 +18,13 @@
  *            abstract: Bounded Directional Rounding -- an element whose
  *            rounding moves it opposite to its update is rounded toward the
  *            update instead, with no extra storage.
+ *   [PW]     "Low-Bit GDN Recurrent-State Quantization: Global Gradient-aware
+ *            Allocation and Pure-Write Sliding Windows", abstract: recent pure
+ *            writes kept as FP8 vector pairs, propagated through the full GDN
+ *            transition, merged into the low-bit state when they leave the
+ *            window.
+ *   [OCP8]   OCP 8-bit floating point specification, E4M3 format (bias 7,
+ *            no infinities, max normal 448, subnormals m * 2^-9).
  *   [PHILOX] Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy as
  *            1, 2, 3", SC'11 -- Philox4x32-10 block function.
  *   Recurrences: gated delta rule and Mamba-2 scalar-decay SSM as named in
@@ -483,6 +490,172 @@ int orc_diag_head_step(const orc_head* hd, int delta, const int8_t* c_in, const 
                                 hd->b, hd->h, hd->step, c_out, &s_out[j]);
     }
     free(S); free(Sh); free(cf); free(ak);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* FP8 E4M3 [OCP8]: round to nearest even, saturating to +-448.              */
+/* ------------------------------------------------------------------------- */
+uint8_t orc_e4m3_encode(float x)
+{
+    if (isnan(x)) return 0x7F;
+    const uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (a >= 448.0) return sign | 0x7E;                  /* saturate */
+    if (a < 0.015625) {                                   /* below the smallest normal 2^-6 */
+        const double m = nearbyint(a * 512.0);            /* subnormal steps of 2^-9 */
+        return sign | (uint8_t)m;                         /* m = 8 is the smallest normal, 0x08 */
+    }
+    int e;
+    const double fr = frexp(a, &e);                       /* a = fr * 2^e, fr in [0.5, 1) */
+    int E = e - 1;                                        /* a = (2 fr) * 2^E, 2 fr in [1, 2) */
+    double m = nearbyint((2.0 * fr - 1.0) * 8.0);         /* 3 mantissa bits */
+    if (m == 8.0) { m = 0.0; E += 1; }
+    if (E > 8 || (E == 8 && m > 6.0)) return sign | 0x7E;
+    return sign | (uint8_t)(((E + 7) << 3) | (int)m);
+}
+
+float orc_e4m3_decode(uint8_t v)
+{
+    const int e = (v >> 3) & 15, m = v & 7;
+    if (e == 15 && m == 7) return NAN;
+    const double mag = (e == 0) ? ldexp((double)m, -9) : ldexp(1.0 + m / 8.0, e - 7);
+    return (float)((v & 0x80) ? -mag : mag);
+}
+
+/* FP8 vector with one scale [PW]: s = max|x| / 448, codes e4m3(x_i * (448 / max|x|)). */
+static void orc_fp8_vector_encode(const float* x, int n, uint8_t* q, float* scale)
+{
+    float m = 0.0f;
+    for (int i = 0; i < n; ++i) {
+        const float a = fabsf(x[i]);
+        if (isnan(a) || isnan(m)) m = NAN;
+        else if (a > m) m = a;
+    }
+    *scale = m / 448.0f;
+    const float inv = (m > 0.0f && isfinite(m)) ? 448.0f / m : 0.0f;
+    for (int i = 0; i < n; ++i) q[i] = orc_e4m3_encode(x[i] * inv);
+}
+
+/* Window dot product: 8 partials over contiguous chunks of n/8 entries, each
+ * summed in increasing index, then combined by the XOR butterfly d = 1, 2, 4. */
+static float orc_dot_chunks(const float* a, const float* b, int n)
+{
+    float part[8];
+    const int len = n / 8;
+    for (int p = 0; p < 8; ++p) {
+        float acc = 0.0f;
+        for (int t = 0; t < len; ++t) acc = fmaf(a[p * len + t], b[p * len + t], acc);
+        part[p] = acc;
+    }
+    for (int d = 1; d < 8; d <<= 1)
+        for (int p = 0; p < 8; ++p)
+            if ((p & d) == 0) part[p] = part[p] + part[p | d];
+    return part[0];
+}
+
+/* Gated DeltaNet decode step with a pure-write window [PW] of W slots.
+ *
+ * The full state is S_t = H_t + sum_w a_w b_w^T: H is the low-bit historical
+ * state, slot w holds a recent pure write beta v k^T as the pair (a = k
+ * propagated to the current step, b = beta v), each vector in FP8 with one
+ * scale (fp8 = 0) or in binary32 (fp8 = 1 keeps them exact for the pins).
+ * Step t uses slot p = t mod W: its write (from step t - W) leaves the window.
+ *   1. H: the GDN transition of the dequantized history (no new write):
+ *        u_j = s_j sum_i c_ij k_i,  w_j = beta * (-alpha u_j),
+ *        S_ij = fma(c_ij, alpha s_j, k_i w_j)          (c-form, as GDN)
+ *   2. every slot: a <- alpha (a - beta k (k^T a)):
+ *        g = beta * dot(k, a),  a'_i = alpha * fma(-g, k_i, a_i)
+ *   3. slot p leaves: S_ij = fma(a'_p,i, b_p,j, S_ij)
+ *   4. slot p takes the new write: a = k, b = beta v
+ *   5. readout from the full-precision state:
+ *        o_j = sum_i S_ij q_i, then for w = 0..W-1: o_j = fma(b_w,j, z_w, o_j)
+ *        with z_w = dot(a'_w, q) (slot p: dot(k, q))
+ *   6. requantize H (rounding as configured, no BDR), encode the window.
+ * Window layout: a [W][dk] codes + [W] scales, b [W][dv] codes + [W] scales
+ * (binary32 arrays when fp32window).  Dots over the window use
+ * orc_dot_chunks; sums over the state the canonical R-partial order.       */
+int orc_gdn_pw_head_step(const orc_head* hd, int W, int fp32window, const int8_t* c_in,
+                         const float* s_in, const float* f_in, const void* a_in,
+                         const float* as_in, const void* b_in, const float* bs_in,
+                         const float* q, const float* k, const float* v, float alpha, float beta,
+                         int8_t* c_out, float* s_out, float* f_out, void* a_out, float* as_out,
+                         void* b_out, float* bs_out, float* o)
+{
+    const int dk = hd->dk, dv = hd->dv;
+    const int R = (hd->mode == ORC_PLAIN) ? 1 : hd->R;
+    const int p = (int)(hd->step % (uint32_t)W);
+    const size_t n = (size_t)dk * (size_t)dv;
+    float* S = (float*)malloc(sizeof(float) * n);
+    float* cf = (float*)malloc(sizeof(float) * n);
+    float* A = (float*)malloc(sizeof(float) * (size_t)W * dk);   /* propagated a'_w */
+    float* Bv = (float*)malloc(sizeof(float) * (size_t)W * dv);  /* decoded b_w */
+    float* z = (float*)malloc(sizeof(float) * (size_t)W);
+    if (!S || !cf || !A || !Bv || !z) { free(S); free(cf); free(A); free(Bv); free(z); return 1; }
+
+    /* decode the window */
+    for (int w = 0; w < W; ++w) {
+        for (int i = 0; i < dk; ++i)
+            A[w * dk + i] = fp32window ? ((const float*)a_in)[w * dk + i]
+                                       : orc_e4m3_decode(((const uint8_t*)a_in)[w * dk + i]) * as_in[w];
+        for (int j = 0; j < dv; ++j)
+            Bv[w * dv + j] = fp32window ? ((const float*)b_in)[w * dv + j]
+                                        : orc_e4m3_decode(((const uint8_t*)b_in)[w * dv + j]) * bs_in[w];
+    }
+    /* 1. history: the GDN transition without a write */
+    for (size_t t = 0; t < n; ++t) cf[t] = (hd->bits == 32) ? f_in[t] : (float)c_in[t];
+    for (int j = 0; j < dv; ++j) {
+        const float sj = (hd->bits == 32) ? 1.0f : s_in[j];
+        const float ck = orc_dot_rows(cf + j, dv, k, dk, R);
+        const float u = (hd->bits == 32) ? ck : sj * ck;
+        const float wj = beta * fmaf(-alpha, u, 0.0f);
+        const float a = (hd->bits == 32) ? alpha : alpha * sj;
+        for (int i = 0; i < dk; ++i)
+            S[(int64_t)i * dv + j] = fmaf(cf[(int64_t)i * dv + j], a, k[i] * wj);
+    }
+    /* 2. propagate every slot through the transition */
+    for (int w = 0; w < W; ++w) {
+        const float g = beta * orc_dot_chunks(k, A + w * dk, dk);
+        for (int i = 0; i < dk; ++i) A[w * dk + i] = alpha * fmaf(-g, k[i], A[w * dk + i]);
+    }
+    /* 3. slot p leaves the window into the history */
+    for (int i = 0; i < dk; ++i)
+        for (int j = 0; j < dv; ++j)
+            S[(int64_t)i * dv + j] = fmaf(A[p * dk + i], Bv[p * dv + j], S[(int64_t)i * dv + j]);
+    /* 4. the new write takes slot p */
+    for (int i = 0; i < dk; ++i) A[p * dk + i] = k[i];
+    for (int j = 0; j < dv; ++j) Bv[p * dv + j] = beta * v[j];
+    /* 5. readout */
+    for (int w = 0; w < W; ++w) z[w] = orc_dot_chunks(A + w * dk, q, dk);
+    for (int j = 0; j < dv; ++j) {
+        float acc = orc_dot_rows(S + j, dv, q, dk, R);
+        for (int w = 0; w < W; ++w) acc = fmaf(Bv[w * dv + j], z[w], acc);
+        o[j] = acc;
+    }
+    /* 6. requantize the history, encode the window */
+    if (hd->bits == 32) {
+        for (size_t t = 0; t < n; ++t) f_out[t] = S[t];
+    } else {
+        for (int j = 0; j < dv; ++j)
+            orc_quantize_column(S, NULL, hd->m_copy ? hd->m_copy + j : NULL, dk, dv, j, hd->bits,
+                                hd->rounding & 1, hd->mode, hd->seed, hd->b, hd->h, hd->step,
+                                c_out, &s_out[j]);
+    }
+    for (int w = 0; w < W; ++w) {
+        if (fp32window) {
+            memcpy((float*)a_out + w * dk, A + w * dk, sizeof(float) * dk);
+            memcpy((float*)b_out + w * dv, Bv + w * dv, sizeof(float) * dv);
+            continue;
+        }
+        orc_fp8_vector_encode(A + w * dk, dk, (uint8_t*)a_out + w * dk, &as_out[w]);
+        if (w == p) {
+            orc_fp8_vector_encode(Bv + w * dv, dv, (uint8_t*)b_out + w * dv, &bs_out[w]);
+        } else {
+            memcpy((uint8_t*)b_out + w * dv, (const uint8_t*)b_in + w * dv, (size_t)dv);
+            bs_out[w] = bs_in[w];
+        }
+    }
+    free(S); free(cf); free(A); free(Bv); free(z);
     return 0;
 }
 

@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 import workloads as W
+import workloads as W_mod
 
 TINY = W.WORKLOADS[0]                      # GDN B=1 H=2 d=16, fp32 inputs, 64 steps
 TINY_M = dataclasses.replace(W.WORKLOADS[3], name="mamba2_tiny", B=1, H=2, dk=16, dv=16,
@@ -728,3 +729,69 @@ def test_copy_scale_removes_the_error_dependence_of_the_scale():
         assert np.array_equal(cp[1]["scales"], (m / np.float32(7)).astype(np.float32))
         noisy_differ |= not np.array_equal(ny[1]["scales"], ny[2]["scales"])
     assert noisy_differ
+
+
+# ---------------------------------------------------------------------------
+# Pure-write window ("Low-Bit GDN Recurrent-State Quantization: ... Pure-Write
+# Sliding Windows", abstract) and its FP8 E4M3 vectors
+# ---------------------------------------------------------------------------
+def test_e4m3_decode_table_matches_torch():
+    """All 256 codes against PyTorch's float8_e4m3fn (an independent implementation)."""
+    import torch
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).float().numpy()
+    got = np.array([oracle.e4m3_decode(c) for c in range(256)], np.float32)
+    assert np.array_equal(np.isnan(ref), np.isnan(got))
+    assert np.array_equal(ref[~np.isnan(ref)], got[~np.isnan(got)])
+
+
+def test_e4m3_encode_matches_torch_in_range_and_saturates():
+    """Round to nearest even against PyTorch on random values, every tie between
+    neighbouring codes and the subnormal range; beyond 448 the codec saturates."""
+    import torch
+    rng = np.random.default_rng(8)
+    x = np.concatenate([rng.standard_normal(4000) * 30, rng.uniform(-0.02, 0.02, 2000),
+                        rng.uniform(-463.9, 463.9, 2000)]).astype(np.float32)
+    vals = np.array([oracle.e4m3_decode(c) for c in range(127)], np.float64)
+    mids = ((vals[:-1] + vals[1:]) / 2).astype(np.float32)          # exact ties (binary32 holds them)
+    x = np.concatenate([x, mids, -mids])
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    got = np.array([oracle.e4m3_encode(v) for v in x], np.uint8)
+    assert np.array_equal(ref, got)
+    assert oracle.e4m3_encode(1e6) == 0x7E and oracle.e4m3_encode(-500.0) == 0xFE
+
+
+@pytest.mark.parametrize("W", [4, 8])
+def test_pure_write_window_decomposition_is_exact(W):
+    """With binary32 vectors and history, H + sum_w a_w b_w^T is the Gated DeltaNet
+    state (closed form in float64) at every step, before and after slots start to
+    merge, and the readout is S_t^T q."""
+    w = TINY
+    T = 3 * W + 5
+    ins = [W_inputs for W_inputs in (W_mod.gdn_inputs(w, t) for t in range(T))]
+    hb = np.full(w.H, 32, np.int8)
+    st = oracle.zero_state(w.B, w.H, w.dk, w.dv)
+    win = oracle.zero_window(w.B, w.H, W, w.dk, w.dv, fp32=True)
+    for t in range(T):
+        st, win, o = oracle.gdn_pw_step(st, win, ins[t], hb, rounding=0, seed=0, step=t,
+                                        fp32window=True)
+        full = oracle.window_full_state(st, win, hb, fp32window=True)
+        for h in range(w.H):
+            ref = _gdn_closed_form(ins, t + 1, 0, h)
+            assert _rel(full[0, h], ref) <= 1e-5
+            assert _rel(o[0, h], ref.T @ np.asarray(ins[t]["q"][0, h], np.float64)) <= 1e-5
+
+
+def test_pure_write_window_fp8_error_is_bounded():
+    """FP8 vectors (3 mantissa bits, one scale per vector) keep the full state
+    within a few percent of the exact one."""
+    w = TINY
+    T, W = 40, 8
+    ins = [W_mod.gdn_inputs(w, t) for t in range(T)]
+    hb = np.full(w.H, 32, np.int8)
+    st = oracle.zero_state(w.B, w.H, w.dk, w.dv)
+    win = oracle.zero_window(w.B, w.H, W, w.dk, w.dv)
+    for t in range(T):
+        st, win, _ = oracle.gdn_pw_step(st, win, ins[t], hb, rounding=0, seed=0, step=t)
+    full = oracle.window_full_state(st, win, hb)
+    for h in range(w.H):
+        assert _rel(full[0, h], _gdn_closed_form(ins, T, 0, h)) <= 0.08
