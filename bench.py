@@ -58,8 +58,15 @@ def algorithmic_bytes_per_head(w: W.Workload, bits: int) -> int:
     return 2 * codes + 2 * scales + vecs + out
 
 
-def step_bytes(w: W.Workload, head_bits) -> int:
-    per = sum(algorithmic_bytes_per_head(w, int(b)) for b in head_bits) * w.B
+def window_bytes_per_head(w: W.Workload, window: int) -> int:
+    """Pure-write window traffic per head update: the FP8 a and b vectors and
+    their scales, read and written."""
+    return 2 * (window * (w.dk + w.dv) + 2 * 4 * window) if window else 0
+
+
+def step_bytes(w: W.Workload, head_bits, window: int = 0) -> int:
+    per = sum(algorithmic_bytes_per_head(w, int(b)) + window_bytes_per_head(w, window)
+              for b in head_bits) * w.B
     if w.family == "mamba2":
         esz = 2 if w.in_dtype == "bf16" else 4
         per += w.B * w.ngroups * 2 * w.dk * esz + 8 * w.H   # B, C per request; A, D per head
@@ -289,7 +296,7 @@ def run_ours(args, w: W.Workload):
     ctx = rsq.Context(fam, w.B, w.H, w.dk, w.dv, head_bits=bits,
                       rounding=ROUNDING[w.rounding],
                       in_dtype=rsq.RSQ_BF16 if w.in_dtype == "bf16" else rsq.RSQ_F32,
-                      seed=w.sr_seed + 7919 * rank, ngroups=w.ngroups)
+                      seed=w.sr_seed + 7919 * rank, ngroups=w.ngroups, window=args.window)
     state_bytes = ctx.code_bytes + ctx.scale_bytes
     layers = max(2, -(-3 * l2 // state_bytes))
     if args.layers:
@@ -305,6 +312,8 @@ def run_ours(args, w: W.Workload):
         ctx.quantize(S0, st, step=0)
         states.append(st)
     del S0
+    # pure-write windows: a ping-pong pair per layer (the step reads one, writes the other)
+    wins = [(ctx.alloc_window(dev), ctx.alloc_window(dev)) for _ in range(layers)] if args.window else None
     # input sets (seeded host generation, uploaded once)
     inp_bytes = None
     n_sets = max(8, min(256, -(-3 * l2 // max(1, step_input_bytes(w)))))
@@ -318,13 +327,21 @@ def run_ours(args, w: W.Workload):
     structs = [_inputs_struct(rsq, w, s) for s in sets]
     stream = torch.cuda.Stream(device=dev)
 
+    def step_on(li, ins, t, visit):
+        """One decode step of layer li (its window ping-pong by visit parity)."""
+        if wins is None:
+            ctx.decode_step(states[li], states[li], ins, outs[li], t, stream.cuda_stream)
+        else:
+            ctx.decode_step_window(states[li], states[li], wins[li][visit % 2], wins[li][(visit + 1) % 2],
+                                   ins, outs[li], t, stream.cuda_stream)
+
     def launch(t):
-        li = t % layers
-        ctx.decode_step(states[li], states[li], structs[t % n_sets], outs[li], t, stream.cuda_stream)
+        step_on(t % layers, structs[t % n_sets], t, t // layers)
 
     # CUDA graphs of up to CH consecutive steps (launch-bound inner loop); CH is a
     # multiple of the layer count so the rotation continues across graph replays
-    CH = max(1, 2048 // layers) * layers
+    # (an even number of visits per layer, so the window ping-pong ends where it began)
+    CH = 2 * max(1, 1024 // layers) * layers
 
     def capture(t0, n):
         gr = torch.cuda.CUDAGraph()
@@ -387,13 +404,12 @@ def run_ours(args, w: W.Workload):
 
     # L2-hot reference point (labelled, not the headline): one layer state and one
     # input set, so the whole step's working set stays in L2
-    n_hot = max(1, min(args.steps, 2000))
+    n_hot = 2 * max(1, min(args.steps, 2000) // 2)
     hot = torch.cuda.CUDAGraph()
     with torch.cuda.stream(stream):
         with torch.cuda.graph(hot, stream=stream):
             for t in range(n_hot):
-                ctx.decode_step(states[0], states[0], structs[0], outs[0], args.warmup + t,
-                                stream.cuda_stream)
+                step_on(0, structs[0], args.warmup + t, t)
         hot.replay()
         h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         h0.record(stream)
@@ -423,8 +439,7 @@ def run_ours(args, w: W.Workload):
             src = pinned[t % 4]
             for k, v in src.items():
                 dev_in[k].copy_(v, non_blocking=True)
-            ctx.decode_step(states[0], states[0], e2e_struct, outs[0], args.warmup + args.steps + t,
-                            stream.cuda_stream)
+            step_on(0, e2e_struct, args.warmup + args.steps + t, t)
             out_host.copy_(outs[0], non_blocking=True)
         e1.record(stream)
     e1.synchronize()
@@ -434,7 +449,7 @@ def run_ours(args, w: W.Workload):
     value = world * hu_step * args.steps / elapsed
     e2e_value = world * hu_step * n_e2e / e2e_elapsed
     per_launch = elapsed / args.steps
-    alg = step_bytes(w, bits)
+    alg = step_bytes(w, bits, args.window)
     peak, peak_kind = measured_peak_gbs()
     achieved = alg / per_launch / 1e9
     kernel_tag = "rsq_decode_kernel<%s,dk=%d,blocks=%d,%s>" % (w.family, w.dk, min(4, w.dv // 16),
@@ -446,6 +461,7 @@ def run_ours(args, w: W.Workload):
         "data": "synthetic",
         "config": {"workload": w.name, "global_batch": w.B * world, "heads": w.H, "dk": w.dk,
                    "dv": w.dv, "state": w.state, "rounding": w.rounding, "inputs": w.in_dtype,
+                   "window": args.window,
                    "parallelism": "dp%d" % world, "layers_rotated": layers,
                    "l2": "inputs larger than L2: %d layer states + %d input sets = %.0f MB per "
                          "rotation (L2 %.0f MB)" % (layers, n_sets,
@@ -629,6 +645,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--rounding", choices=sorted(ROUNDING), default=None,
                     help="override the workload's requantization rule")
+    ap.add_argument("--window", type=int, default=0,
+                    help="pure-write window slots (Gated DeltaNet): 0, 4, 8 or 16")
     ap.add_argument("--drift", action="store_true",
                     help="run the long-horizon state drift study instead of the throughput bench")
     ap.add_argument("--drift-steps", type=int, default=0, help="horizon (default: the workload's)")

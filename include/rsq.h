@@ -19,6 +19,9 @@
  *   [FEED]  "When Dynamic Scaling Fails: A Scale-State Feedback Governs
  *           Recurrent-State Quantization ...", key points: the dynamic scale
  *           is derived from the state it quantizes.
+ *   [PW]    "Low-Bit GDN Recurrent-State Quantization: Global Gradient-aware
+ *           Allocation and Pure-Write Sliding Windows", abstract: recent pure
+ *           writes kept as FP8 vector pairs beside the low-bit state.
  *
  * Conventions shared by every entry point
  * ---------------------------------------
@@ -119,6 +122,8 @@ typedef struct {
     int rounding;    /* rsq_rounding: requantization rule */
     int in_dtype;    /* rsq_dtype of the vector inputs (q, k, v / x, B, C) */
     uint64_t seed;   /* stochastic-rounding key */
+    int window;      /* pure-write window slots W for Gated DeltaNet ([PW]): 0 (none), 4, 8
+                        or 16; needs RSQ_RTN or RSQ_SR and rsq_decode_step_window */
 } rsq_config;
 
 typedef struct rsq_ctx rsq_ctx;
@@ -262,6 +267,42 @@ rsq_status rsq_decode_step_copy_scale(const rsq_ctx* ctx, const rsq_state* state
  * stored values for 32-bit heads), NaN-propagating.  absmax: device float
  * [B][H][dv]. */
 rsq_status rsq_column_absmax(const rsq_ctx* ctx, const rsq_state* state, float* absmax, void* stream);
+
+/* Pure-write window of a Gated DeltaNet context with rsq_config.window = W > 0
+ * ([PW]).  The full state is the stored low-bit history H plus the W most
+ * recent pure writes a b^T: a = k propagated through every later transition
+ * a <- alpha (a - beta k (k.a)), b = beta v.  Each vector is FP8 E4M3 (round to
+ * nearest even, saturating) with one float scale max|x| / 448.  Device
+ * buffers, caller-owned, 16-byte aligned; an all-zero window is empty:
+ *   a        uint8 [B][H][W][dk]          codes of the a vectors
+ *   a_scale  float [B][H][W]
+ *   b        uint8 [B][H][dv/16][W][16]   codes of the b vectors, in 16-column
+ *                                          blocks like the state
+ *   b_scale  float [B][H][W] */
+typedef struct {
+    void* a;
+    float* a_scale;
+    void* b;
+    float* b_scale;
+} rsq_window;
+
+/* Bytes of the window buffers: a codes, b codes, and each scale array. */
+rsq_status rsq_window_bytes(const rsq_ctx* ctx, size_t* a_bytes, size_t* b_bytes,
+                            size_t* scale_bytes);
+
+/* Decode step of a context with a pure-write window.  Step t uses slot
+ * p = t mod W: its write (from step t - W) is propagated, merged into H, and
+ * the slot takes the new write (k, beta v).  H follows the GDN transition
+ * without the new write, is read out together with the window
+ * (o_j = sum_i H_ij q_i + sum_w b_w,j (a_w . q), window dots in 8 contiguous
+ * chunks combined by the XOR butterfly) and requantized as usual.  win_in and
+ * win_out must not share buffers (every column unit of a head reads the a
+ * vectors); states may be updated in place.  RSQ_E_INVAL for a context
+ * without a window. */
+rsq_status rsq_decode_step_window(const rsq_ctx* ctx, const rsq_state* state_in,
+                                  const rsq_state* state_out, const rsq_window* win_in,
+                                  const rsq_window* win_out, const void* inputs, float* out,
+                                  uint32_t step, void* stream);
 
 /* Synchronize `stream`, then report (and clear) the context's non-finite
  * flag: *seen = 1 if any decode step since the last check met a non-finite

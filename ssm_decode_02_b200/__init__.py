@@ -36,7 +36,7 @@ class rsq_config(ctypes.Structure):
     _fields_ = [("family", ctypes.c_int), ("batch", ctypes.c_int), ("heads", ctypes.c_int),
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("ngroups", ctypes.c_int),
                 ("head_bits", ctypes.POINTER(ctypes.c_int8)), ("rounding", ctypes.c_int),
-                ("in_dtype", ctypes.c_int), ("seed", ctypes.c_uint64)]
+                ("in_dtype", ctypes.c_int), ("seed", ctypes.c_uint64), ("window", ctypes.c_int)]
 
 
 class rsq_state(ctypes.Structure):
@@ -54,6 +54,11 @@ class rsq_mamba2_inputs(ctypes.Structure):
                 ("decay", ctypes.c_void_p)]
 
 
+class rsq_window(ctypes.Structure):
+    _fields_ = [("a", ctypes.c_void_p), ("a_scale", ctypes.c_void_p), ("b", ctypes.c_void_p),
+                ("b_scale", ctypes.c_void_p)]
+
+
 class rsq_diag_inputs(ctypes.Structure):
     _fields_ = [("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
                 ("alpha", ctypes.c_void_p), ("beta", ctypes.c_void_p)]
@@ -63,7 +68,7 @@ _EXPORTS = ["rsq_create", "rsq_destroy", "rsq_state_bytes", "rsq_head_offset", "
             "rsq_quantize", "rsq_dequantize", "rsq_state_drift", "rsq_check_flags",
             "rsq_allocate_bits", "rsq_reduction_partials", "rsq_status_string", "rsq_last_error",
             "rsq_version", "rsq_decode_step_noalloc", "rsq_decode_step_copy_scale",
-            "rsq_column_absmax"]
+            "rsq_column_absmax", "rsq_window_bytes", "rsq_decode_step_window"]
 
 
 def _load():
@@ -92,6 +97,11 @@ def _load():
         "rsq_decode_step_copy_scale": ([P, ctypes.POINTER(rsq_state), ctypes.POINTER(rsq_state), P, P,
                                         P, ctypes.c_uint32, P], C),
         "rsq_column_absmax": ([P, ctypes.POINTER(rsq_state), P, P], C),
+        "rsq_window_bytes": ([P, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t),
+                              ctypes.POINTER(ctypes.c_size_t)], C),
+        "rsq_decode_step_window": ([P, ctypes.POINTER(rsq_state), ctypes.POINTER(rsq_state),
+                                    ctypes.POINTER(rsq_window), ctypes.POINTER(rsq_window), P, P,
+                                    ctypes.c_uint32, P], C),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -140,25 +150,21 @@ def _stream(stream) -> int | None:
 # ---------------------------------------------------------------------------
 def rsq_create(family: int, batch: int, heads: int, dk: int, dv: int, *, head_bits=None,
                rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0,
-               ngroups: int = 1) -> int:
-    bits_arr = None
-    if head_bits is not None:
-        bits_arr = (ctypes.c_int8 * heads)(*[int(b) for b in head_bits])
-    cfg = rsq_config(int(family), int(batch), int(heads), int(dk), int(dv), int(ngroups),
-                     ctypes.cast(bits_arr, ctypes.POINTER(ctypes.c_int8)) if bits_arr else None,
-                     int(rounding), int(in_dtype), int(seed) & (2 ** 64 - 1))
+               ngroups: int = 1, window: int = 0) -> int:
+    cfg, bits_arr = _config(family, batch, heads, dk, dv, head_bits, rounding, in_dtype, seed, ngroups,
+                            window)
     out = ctypes.c_void_p()
     _check(lib.rsq_create(ctypes.byref(cfg), ctypes.byref(out)))
     return int(out.value)
 
 
-def _config(family, batch, heads, dk, dv, head_bits, rounding, in_dtype, seed, ngroups):
+def _config(family, batch, heads, dk, dv, head_bits, rounding, in_dtype, seed, ngroups, window=0):
     bits_arr = None
     if head_bits is not None:
         bits_arr = (ctypes.c_int8 * heads)(*[int(b) for b in head_bits])
     cfg = rsq_config(int(family), int(batch), int(heads), int(dk), int(dv), int(ngroups),
                      ctypes.cast(bits_arr, ctypes.POINTER(ctypes.c_int8)) if bits_arr else None,
-                     int(rounding), int(in_dtype), int(seed) & (2 ** 64 - 1))
+                     int(rounding), int(in_dtype), int(seed) & (2 ** 64 - 1), int(window))
     return cfg, bits_arr
 
 
@@ -220,6 +226,25 @@ def rsq_column_absmax(ctx: int, state, absmax, stream=None) -> None:
     _check(lib.rsq_column_absmax(ctx, ctypes.byref(si), _ptr(absmax), _stream(stream)))
 
 
+def rsq_window_bytes(ctx: int) -> tuple[int, int, int]:
+    a, b, sc = ctypes.c_size_t(), ctypes.c_size_t(), ctypes.c_size_t()
+    _check(lib.rsq_window_bytes(ctx, ctypes.byref(a), ctypes.byref(b), ctypes.byref(sc)))
+    return int(a.value), int(b.value), int(sc.value)
+
+
+def _window(win) -> rsq_window:
+    return rsq_window(_ptr(win.a), _ptr(win.a_scale), _ptr(win.b), _ptr(win.b_scale))
+
+
+def rsq_decode_step_window(ctx: int, state_in, state_out, win_in, win_out, inputs, out, step: int,
+                           stream=None) -> None:
+    si, so = _state(state_in), _state(state_out)
+    wi, wo = _window(win_in), _window(win_out)
+    _check(lib.rsq_decode_step_window(ctx, ctypes.byref(si), ctypes.byref(so), ctypes.byref(wi),
+                                      ctypes.byref(wo), ctypes.byref(inputs), _ptr(out),
+                                      int(step) & 0xFFFFFFFF, _stream(stream)))
+
+
 def rsq_quantize(ctx: int, S, state_out, step: int, stream=None) -> None:
     so = _state(state_out)
     _check(lib.rsq_quantize(ctx, _ptr(S), ctypes.byref(so), int(step) & 0xFFFFFFFF, _stream(stream)))
@@ -272,6 +297,14 @@ class State:
         self.scales = scales
 
 
+class Window:
+    """A pure-write window (device): a uint8 [B][H][W][dk], a_scale float [B][H][W],
+    b uint8 [B][H][dv/16][W][16], b_scale float [B][H][W]."""
+
+    def __init__(self, a, a_scale, b, b_scale):
+        self.a, self.a_scale, self.b, self.b_scale = a, a_scale, b, b_scale
+
+
 def gdn_inputs(q, k, v, alpha, beta) -> rsq_gdn_inputs:
     return rsq_gdn_inputs(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta))
 
@@ -289,12 +322,14 @@ class Context:
     """Owns one rsq_ctx (one layer configuration)."""
 
     def __init__(self, family: int, batch: int, heads: int, dk: int, dv: int, *, head_bits=None,
-                 rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0, ngroups: int = 1):
+                 rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0, ngroups: int = 1,
+                 window: int = 0):
         self.family, self.batch, self.heads, self.dk, self.dv = family, batch, heads, dk, dv
         self.head_bits = None if head_bits is None else np.asarray(head_bits, np.int8)
         self.rounding, self.in_dtype, self.seed, self.ngroups = rounding, in_dtype, seed, ngroups
+        self.window = window
         self.ctx = rsq_create(family, batch, heads, dk, dv, head_bits=head_bits, rounding=rounding,
-                              in_dtype=in_dtype, seed=seed, ngroups=ngroups)
+                              in_dtype=in_dtype, seed=seed, ngroups=ngroups, window=window)
         self.code_bytes, self.scale_bytes = rsq_state_bytes(self.ctx)
 
     def close(self):
@@ -316,6 +351,19 @@ class Context:
 
     def decode_step(self, state_in: State, state_out: State, inputs, out, step: int, stream=None):
         rsq_decode_step(self.ctx, state_in, state_out, inputs, out, step, stream)
+
+    def alloc_window(self, device="cuda") -> Window:
+        """An empty (all-zero) pure-write window."""
+        import torch
+        B, H, W = self.batch, self.heads, self.window
+        return Window(torch.zeros((B, H, W, self.dk), dtype=torch.uint8, device=device),
+                      torch.zeros((B, H, W), dtype=torch.float32, device=device),
+                      torch.zeros((B, H, self.dv // 16, W, 16), dtype=torch.uint8, device=device),
+                      torch.zeros((B, H, W), dtype=torch.float32, device=device))
+
+    def decode_step_window(self, state_in: State, state_out: State, win_in: Window, win_out: Window,
+                           inputs, out, step: int, stream=None):
+        rsq_decode_step_window(self.ctx, state_in, state_out, win_in, win_out, inputs, out, step, stream)
 
     def decode_step_copy_scale(self, state_in: State, state_out: State, inputs, copy_absmax, out,
                                step: int, stream=None):

@@ -27,6 +27,7 @@ RSQ_DECLARE(decode_info_gla_copy)
 RSQ_DECLARE(decode_info_gla_copy_bdr)
 RSQ_DECLARE(decode_info_kda_copy)
 RSQ_DECLARE(decode_info_kda_copy_bdr)
+RSQ_DECLARE(decode_info_gdn_pw)
 #undef RSQ_DECLARE
 
 int decode_kernel_info(int family, int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
@@ -37,8 +38,11 @@ int decode_kernel_info(int family, int dk, int ub, bool f32state, int rnd, int* 
         {decode_info_mamba2, decode_info_mamba2_bdr, decode_info_mamba2_copy, decode_info_mamba2_copy_bdr},
         {decode_info_gla, decode_info_gla_bdr, decode_info_gla_copy, decode_info_gla_copy_bdr},
         {decode_info_kda, decode_info_kda_bdr, decode_info_kda_copy, decode_info_kda_copy_bdr}};
-    if (family < 0 || family > 3 || rnd < 0 || rnd > 7) return -1;
+    if (rnd < 0 || rnd > 7) return -1;
     const int group = f32state ? 0 : (rnd >> 1);
+    if (family == kFamGdnPw)  // pure-write window: plain rules only
+        return group == 0 ? decode_info_gdn_pw(dk, ub, f32state, rnd, threads, smem, func) : -1;
+    if (family < 0 || family > 3) return -1;
     return table[family][group](dk, ub, f32state, rnd, threads, smem, func);
 }
 

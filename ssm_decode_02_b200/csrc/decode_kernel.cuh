@@ -35,7 +35,7 @@ struct DecodeCfg {
     static constexpr int NT = 32 * UB;         // one warp per 16-column block
     static constexpr int UCOLS = 16 * UB;      // columns per unit
     // pipeline stages (KDA's extra pair array leaves room for three)
-    static constexpr int NS = F32STATE ? 2 : (FAM == RSQ_KDA ? 3 : 4);
+    static constexpr int NS = F32STATE ? 2 : ((FAM == RSQ_KDA || FAM == kFamGdnPw) ? 3 : 4);
     static constexpr int CODE_BYTES = F32STATE ? DK * UCOLS * 4 : DK * UCOLS;  // largest tile (8-bit)
     static constexpr int OFF_SCALES = CODE_BYTES;
     static constexpr int OFF_VA = OFF_SCALES + UCOLS * 4;  // GDN q / Mamba-2 C   (<= DK floats)
@@ -43,14 +43,25 @@ struct DecodeCfg {
     static constexpr int OFF_VC = OFF_VB + DK * 4;         // GDN v / Mamba-2 x   (<= UCOLS floats)
     static constexpr int OFF_VD = OFF_VC + UCOLS * 4;      // GLA / KDA decay per key channel (DK floats)
     static constexpr bool DIAG = (FAM == RSQ_GLA || FAM == RSQ_KDA);
-    static constexpr int STAGE = ((DIAG ? OFF_VD + DK * 4 : OFF_VD) + 127) / 128 * 128;
+    // pure-write window: the whole v (<= 256 floats), the slots' a codes and
+    // scales, this unit's b codes (W x 16 per block) and the b scales
+    static constexpr bool PW = (FAM == kFamGdnPw);
+    static constexpr int OFF_VF = OFF_VD;
+    static constexpr int OFF_WA = OFF_VF + 256 * 4;
+    static constexpr int OFF_WAS = OFF_WA + kMaxWindow * DK;
+    static constexpr int OFF_WB = OFF_WAS + kMaxWindow * 4;
+    static constexpr int OFF_WBS = OFF_WB + UB * kMaxWindow * 16;
+    static constexpr int END_BASE = DIAG ? OFF_VD + DK * 4 : OFF_VD;
+    static constexpr int STAGE = ((PW ? OFF_WBS + kMaxWindow * 4 : END_BASE) + 127) / 128 * 128;
     // per warp: the two key-axis vectors as duplicated pairs (x, x), one row of
     // PST pairs per row group (padded so the row groups hit different banks)
     static constexpr int PST = L::RPT + 2;
     // pair arrays: q, k (+ the decay per key channel for GLA, + decay and
     // decay * k for KDA)
-    static constexpr int NPAIR = FAM == RSQ_KDA ? 4 : (DIAG ? 3 : 2);
-    static constexpr int P_WARP = NPAIR * kR * PST * 8;
+    static constexpr int NPAIR = FAM == RSQ_KDA ? 4 : ((DIAG || FAM == kFamGdnPw) ? 3 : 2);
+    // (+ the window's z_w = a_w . q for the pure-write window)
+    static constexpr int OFF_PZ = NPAIR * kR * PST * 8;
+    static constexpr int P_WARP = OFF_PZ + (FAM == kFamGdnPw ? kMaxWindow * 4 : 0);
     static constexpr int OFF_P = NS * STAGE;
     static constexpr int OFF_CNT = OFF_P + UB * P_WARP;  // NS release counters
     static constexpr int OFF_BAR = OFF_CNT + 16;
@@ -92,8 +103,10 @@ __device__ __forceinline__ void issue_unit(const DecodeParams& p, const UnitIt& 
     const int hu = un.hu(p);
     const uint32_t code_bytes = static_cast<uint32_t>(DK * UCOLS * bits / 8);
     const uint32_t esz = p.in_bf16 ? 2u : 4u;
+    const uint32_t W = static_cast<uint32_t>(p.W);
     const uint32_t total = code_bytes + (F32STATE ? 0u : UCOLS * 4u) + 2u * DK * esz + UCOLS * esz +
-                           (C::DIAG ? DK * 4u : 0u);
+                           (C::DIAG ? DK * 4u : 0u) +
+                           (C::PW ? p.dv * esz + W * DK + 2u * W * 4u + UB * W * 16u : 0u);
     const uint8_t* codes = p.codes_in + (long long)un.b * p.row_bytes + p.head_off[un.h] +
                            (long long)un.cb * code_bytes;
     const uint32_t s = smem_u32(stage);
@@ -111,6 +124,14 @@ __device__ __forceinline__ void issue_unit(const DecodeParams& p, const UnitIt& 
     bulk_g2s(s + C::OFF_VB, vB + rowA * esz, DK * esz, bar);
     bulk_g2s(s + C::OFF_VC, vC + ((long long)hu * p.dv + un.cb * UCOLS) * esz, UCOLS * esz, bar);
     if constexpr (C::DIAG) bulk_g2s(s + C::OFF_VD, p.vD + (long long)hu * DK, DK * 4u, bar);
+    if constexpr (C::PW) {
+        const long long nblk = p.dv / kBlockCols;
+        bulk_g2s(s + C::OFF_VF, vC + (long long)hu * p.dv * esz, p.dv * esz, bar);
+        bulk_g2s(s + C::OFF_WA, p.win_a_in + (long long)hu * W * DK, W * DK, bar);
+        bulk_g2s(s + C::OFF_WAS, p.win_as_in + (long long)hu * W, W * 4u, bar);
+        bulk_g2s(s + C::OFF_WB, p.win_b_in + ((long long)hu * nblk + (long long)un.cb * UB) * W * 16, UB * W * 16u, bar);
+        bulk_g2s(s + C::OFF_WBS, p.win_bs_in + (long long)hu * W, W * 4u, bar);
+    }
 }
 
 __device__ __forceinline__ float ld_vec(const uint8_t* base, int e, bool bf16) {
@@ -142,6 +163,81 @@ __device__ __forceinline__ Gates load_gates(const DecodeParams& p, const UnitIt&
     g.A = (FAM == RSQ_MAMBA2) ? __ldg(p.A + un.h) : 0.f;
     g.D = (FAM == RSQ_MAMBA2) ? __ldg(p.D + un.h) : 0.f;
     return g;
+}
+
+// Pure-write window ("Low-Bit GDN Recurrent-State Quantization: ... Pure-Write
+// Sliding Windows", abstract), per warp: every slot's a vector goes through
+// the step's transition a <- alpha (a - beta k (k.a)); the slot `ps` leaving
+// the window leaves its propagated a in the pair array `pm` (rows as
+// duplicated pairs) for the merge into the history; z_w = a_w . q (slot ps:
+// k . q, its new write) goes to `zs`.  Lane (slot group, chunk) handles rows
+// [chunk * DK/8, (chunk+1) * DK/8) of one slot; the dot products sum each
+// chunk in increasing row order and combine the 8 chunks by the XOR butterfly
+// d = 1, 2, 4.  The writer warp also encodes the new a vectors (FP8 E4M3, one
+// scale = max|a| / 448 per vector).
+template <int DK, int PST>
+__device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* stage, int off_wa,
+                                         int off_was, int off_va, int off_vb, int hu, int ps,
+                                         float alpha, float beta, bool writer, uint64_t* pm,
+                                         float* zs, int lane) {
+    constexpr int CH = DK / 8;
+    const bool bf16 = p.in_bf16 != 0;
+    const int sl = lane >> 3, chunk = lane & 7, i0 = chunk * CH;
+    for (int pass = 0; pass * 4 < p.W; ++pass) {
+        const int slot = pass * 4 + sl;
+        const bool merging = (slot == ps);
+        const float as = reinterpret_cast<const float*>(stage + off_was)[slot];
+        const uint16_t* ab = reinterpret_cast<const uint16_t*>(stage + off_wa + slot * DK + i0);
+        float a[CH], kk[CH];
+        float ka = 0.f;
+#pragma unroll
+        for (int t = 0; t < CH; t += 2) {
+            float lo, hi;
+            e4m3x2_to_f32(ab[t / 2], lo, hi);
+            a[t] = __fmul_rn(lo, as);
+            a[t + 1] = __fmul_rn(hi, as);
+            kk[t] = ld_vec(stage + off_vb, i0 + t, bf16);
+            kk[t + 1] = ld_vec(stage + off_vb, i0 + t + 1, bf16);
+        }
+#pragma unroll
+        for (int t = 0; t < CH; ++t) ka = __fmaf_rn(kk[t], a[t], ka);
+#pragma unroll
+        for (int d = 1; d < 8; d <<= 1) ka = __fadd_rn(ka, __shfl_xor_sync(0xffffffffu, ka, d));
+        const float gg = __fmul_rn(beta, ka);
+        float z = 0.f;
+#pragma unroll
+        for (int t = 0; t < CH; ++t) {
+            a[t] = __fmul_rn(alpha, __fmaf_rn(-gg, kk[t], a[t]));  // propagated a'
+            const float q = ld_vec(stage + off_va, i0 + t, bf16);
+            z = __fmaf_rn(merging ? kk[t] : a[t], q, z);
+            if (merging) {
+                const int i = i0 + t;
+                pm[(i & (kR - 1)) * PST + i / kR] = pk(a[t], a[t]);
+            }
+        }
+#pragma unroll
+        for (int d = 1; d < 8; d <<= 1) z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, d));
+        if (chunk == 0) zs[slot] = z;
+        if (writer) {
+            // the stored a: propagated for the slots that stay, k for the new write
+            float m = 0.f;
+#pragma unroll
+            for (int t = 0; t < CH; ++t) {
+                if (merging) a[t] = kk[t];
+                m = max_nan(m, fabsf(a[t]));
+            }
+#pragma unroll
+            for (int d = 1; d < 8; d <<= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, d));
+            const float inv = (m > 0.f && isfinite(m)) ? __fdiv_rn(448.f, m) : 0.f;
+            uint8_t* dst = p.win_a_out + ((long long)hu * p.W + slot) * DK + i0;
+#pragma unroll
+            for (int t = 0; t < CH; t += 2) {
+                const uint32_t two = e4m3x2_from_f32(__fmul_rn(a[t + 1], inv), __fmul_rn(a[t], inv));
+                *reinterpret_cast<uint16_t*>(dst + t) = static_cast<uint16_t>(two);
+            }
+            if (chunk == 0) p.win_as_out[(long long)hu * p.W + slot] = __fdiv_rn(m, 448.f);
+        }
+    }
 }
 
 // One 16-column block of one unit, processed by warp w.
@@ -180,6 +276,13 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
         }
     }
     __syncwarp();
+    float* zs = reinterpret_cast<float*>(smem + C::OFF_P + w * C::P_WARP + C::OFF_PZ);  // window z_w
+    const int ps = C::PW ? static_cast<int>(p.step % static_cast<uint32_t>(p.W)) : 0;  // slot leaving
+    if constexpr (C::PW) {
+        pw_slots<DK, C::PST>(p, stage, C::OFF_WA, C::OFF_WAS, C::OFF_VA, C::OFF_VB, hu, ps, gt.g0, gt.g1,
+                             un.cb == 0 && w == 0, pc, zs, lane);
+        __syncwarp();
+    }
     const uint64_t* qa = pa + g * C::PST;  // q (GDN, GLA, KDA) / C (Mamba-2) of rows g + 8k
     const uint64_t* kb = pb + g * C::PST;  // k / B
     const uint64_t* ga = pc + g * C::PST;  // decay per key channel (GLA, KDA)
@@ -209,7 +312,7 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
     auto load_vc = [&]() { return ld_vec4(stage + C::OFF_VC, 16 * w + 4 * cw, bf16); };
 
     // ---- state update ---------------------------------------------------------
-    if constexpr (FAM == RSQ_GDN) {
+    if constexpr (FAM == RSQ_GDN || C::PW) {
         const float alpha = gt.g0, beta = gt.g1;
         uint64_t a01 = pk(0.f, 0.f), a23 = pk(0.f, 0.f);
 #pragma unroll
@@ -229,7 +332,8 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
         const float4 vc = load_vc();
         const float ckv[4] = {ck.x, ck.y, ck.z, ck.w};
         const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-        const float vv[4] = {vc.x, vc.y, vc.z, vc.w};
+        // (with a pure-write window the new write goes to the window: v = 0 here)
+        const float vv[4] = {C::PW ? 0.f : vc.x, C::PW ? 0.f : vc.y, C::PW ? 0.f : vc.z, C::PW ? 0.f : vc.w};
         float wj[4], aj[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -247,6 +351,25 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
             S2[k][1] = fma2(S2[k][1], A23, mul2(kk.x, W23));
             S2[k + 1][0] = fma2(S2[k + 1][0], A01, mul2(kk.y, W01));
             S2[k + 1][1] = fma2(S2[k + 1][1], A23, mul2(kk.y, W23));
+        }
+        if constexpr (C::PW) {
+            // the slot leaving the window merges into the history: S += a'_ps b_ps^T
+            const float bsc = reinterpret_cast<const float*>(stage + C::OFF_WBS)[ps];
+            const uint32_t b4 = *reinterpret_cast<const uint32_t*>(stage + C::OFF_WB + (w * p.W + ps) * 16 + 4 * cw);
+            float b0, b1, b2, b3;
+            e4m3x2_to_f32(b4 & 0xFFFFu, b0, b1);
+            e4m3x2_to_f32(b4 >> 16, b2, b3);
+            const uint64_t B01 = pk(__fmul_rn(b0, bsc), __fmul_rn(b1, bsc));
+            const uint64_t B23 = pk(__fmul_rn(b2, bsc), __fmul_rn(b3, bsc));
+            const uint64_t* mg = pc + g * C::PST;
+#pragma unroll
+            for (int k = 0; k < RPT; k += 2) {
+                const ulonglong2 aa = *reinterpret_cast<const ulonglong2*>(mg + k);
+                S2[k][0] = fma2(aa.x, B01, S2[k][0]);
+                S2[k][1] = fma2(aa.x, B23, S2[k][1]);
+                S2[k + 1][0] = fma2(aa.y, B01, S2[k + 1][0]);
+                S2[k + 1][1] = fma2(aa.y, B23, S2[k + 1][1]);
+            }
         }
     } else if constexpr (C::DIAG) {
         // GLA: w = v.  KDA: u = s * sum_i c_ij (alpha_i k_i), w = beta (v - u).
@@ -335,6 +458,18 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
     const int c = col_of(g);  // the column this lane finalises
     float o = reduce_scatter4(unpk4(o01, o23), g, AddOp());
     if constexpr (FAM == RSQ_MAMBA2) o = __fmaf_rn(gt.D, ld_vec(stage + C::OFF_VC, 16 * w + 4 * cw + c, bf16), o);
+    if constexpr (C::PW) {
+        // the window's part of the readout: o_j += b_w,j z_w in slot order
+        const float vcol = ld_vec(stage + C::OFF_VC, 16 * w + 4 * cw + c, bf16);
+        const uint8_t* bcol = stage + C::OFF_WB + w * p.W * 16 + 4 * cw + c;
+        const float* bscale = reinterpret_cast<const float*>(stage + C::OFF_WBS);
+        for (int ws = 0; ws < p.W; ++ws) {
+            float bw, unused;
+            e4m3x2_to_f32(bcol[ws * 16], bw, unused);
+            bw = (ws == ps) ? __fmul_rn(gt.g1, vcol) : __fmul_rn(bw, bscale[ws]);
+            o = __fmaf_rn(bw, zs[ws], o);
+        }
+    }
     const long long col = (long long)hu * p.dv + j0 + 4 * cw + c;
     if (g < 4) p.out[col] = o;
     float4 iv = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -403,6 +538,41 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
         }
     }
 
+    if constexpr (C::PW) {
+        // window b codes of this block: the slots that stay are copied, the new
+        // write (slot ps) is encoded with one scale over the whole vector beta v
+        const float beta = gt.g1;
+        float mb = 0.f;
+        for (int j = lane; j < p.dv; j += 32)
+            mb = max_nan(mb, fabsf(__fmul_rn(beta, ld_vec(stage + C::OFF_VF, j, bf16))));
+#pragma unroll
+        for (int d = 16; d >= 1; d >>= 1) mb = max_nan(mb, __shfl_xor_sync(0xffffffffu, mb, d));
+        const float invb = (mb > 0.f && isfinite(mb)) ? __fdiv_rn(448.f, mb) : 0.f;
+        const long long nblk = p.dv / kBlockCols;
+        uint8_t* bdst = p.win_b_out + ((long long)hu * nblk + blk) * p.W * 16;
+        if (lane < p.W) {
+            uint4 row;
+            if (lane != ps) {
+                row = *reinterpret_cast<const uint4*>(stage + C::OFF_WB + (w * p.W + lane) * 16);
+            } else {
+                uint32_t wd[4];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    float x[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        x[e] = __fmul_rn(__fmul_rn(beta, ld_vec(stage + C::OFF_VF, j0 + 4 * q4 + e, bf16)), invb);
+                    wd[q4] = e4m3x2_from_f32(x[1], x[0]) | (e4m3x2_from_f32(x[3], x[2]) << 16);
+                }
+                row = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            }
+            *reinterpret_cast<uint4*>(bdst + lane * 16) = row;
+            if (un.cb == 0 && w == 0)
+                p.win_bs_out[(long long)hu * p.W + lane] =
+                    (lane == ps) ? __fdiv_rn(mb, 448.f) : reinterpret_cast<const float*>(stage + C::OFF_WBS)[lane];
+        }
+    }
+
     // ---- release the stage; the last warp refills it with the unit NS ahead ----
     __syncwarp();
     if (lane == 0) {
@@ -427,7 +597,8 @@ template <int FAM, int DK, int UB, bool F32STATE, int RND>
 constexpr int decode_min_blocks() {
     using C = DecodeCfg<FAM, DK, UB, F32STATE>;
     // BDR: about 168 registers per thread (65536 / (168 * 128) = 3 CTAs of 128 threads)
-    return (RND & kRndBdr) != 0 ? 384 / C::NT : C::MINB;
+    // (the pure-write window's slot pass needs as many)
+    return ((RND & kRndBdr) != 0 || FAM == kFamGdnPw) ? 384 / C::NT : C::MINB;
 }
 
 template <int FAM, int DK, int UB, bool F32STATE, int RND>

@@ -42,6 +42,8 @@ rsq_status cuda_fail(int err, const char* what) {
 }
 
 constexpr int kCopyScaleBit = 4;  // kernel rule bit of the copy scale (beside the rsq_rounding bits)
+// Kernel family of a configuration (Gated DeltaNet with a window has its own kernels).
+int kernel_family(const rsq_config& c) { return (c.family == RSQ_GDN && c.window > 0) ? rsq::kFamGdnPw : c.family; }
 bool family_ok(int f) { return f == RSQ_GDN || f == RSQ_MAMBA2 || f == RSQ_GLA || f == RSQ_KDA; }
 bool rounding_ok(int r) { return r == RSQ_RTN || r == RSQ_SR || r == RSQ_BDR || r == RSQ_SR_BDR; }
 bool dk_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
@@ -122,6 +124,12 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
     if (c.in_dtype != RSQ_F32 && c.in_dtype != RSQ_BF16) return fail(RSQ_E_INVAL, "create: bad in_dtype %d", c.in_dtype);
     if (c.family == RSQ_MAMBA2 && (c.ngroups < 1 || c.heads % c.ngroups != 0))
         return fail(RSQ_E_INVAL, "create: ngroups must divide heads");
+    if (c.window != 0 && c.window != 4 && c.window != 8 && c.window != 16)
+        return fail(RSQ_E_INVAL, "create: window must be 0, 4, 8 or 16 (got %d)", c.window);
+    if (c.window && c.family != RSQ_GDN)
+        return fail(RSQ_E_UNSUPPORTED, "create: the pure-write window is defined for Gated DeltaNet");
+    if (c.window && c.rounding != RSQ_RTN && c.rounding != RSQ_SR)
+        return fail(RSQ_E_UNSUPPORTED, "create: the pure-write window takes nearest or stochastic rounding");
 
     rsq_ctx* ctx = new (std::nothrow) rsq_ctx();
     if (!ctx) return fail(RSQ_E_NOMEM, "create: host allocation failed");
@@ -161,7 +169,7 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
     int threads = 0;
     size_t smem = 0;
     const void* func = nullptr;
-    if (rsq::decode_kernel_info(c.family, c.dk, ctx->ub, ctx->f32state, c.rounding, &threads,
+    if (rsq::decode_kernel_info(kernel_family(c), c.dk, ctx->ub, ctx->f32state, c.rounding, &threads,
                                 &smem, &func) != 0) {
         delete ctx;
         return fail(RSQ_E_UNSUPPORTED, "create: no kernel for dk=%d dv=%d", c.dk, c.dv);
@@ -177,7 +185,7 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
         int t2 = 0;
         size_t sm2 = 0;
         const void* f2 = nullptr;
-        if (rsq::decode_kernel_info(c.family, c.dk, ctx->ub, false, c.rounding | kCopyScaleBit, &t2, &sm2,
+        if (rsq::decode_kernel_info(kernel_family(c), c.dk, ctx->ub, false, c.rounding | kCopyScaleBit, &t2, &sm2,
                                     &f2) == 0)
             err = cudaFuncSetAttribute(f2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2));
     }
@@ -216,13 +224,39 @@ rsq_status rsq_head_offset(const rsq_ctx* ctx, int h, size_t* offset) {
 
 namespace {
 rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const rsq_state* state_out,
-                            const void* inputs, const float* copy_absmax, float* out, uint32_t step,
-                            void* stream);
+                            const void* inputs, const float* copy_absmax, const rsq_window* win_in,
+                            const rsq_window* win_out, float* out, uint32_t step, void* stream);
 }
 
 rsq_status rsq_decode_step(const rsq_ctx* ctx, const rsq_state* state_in, const rsq_state* state_out,
                            const void* inputs, float* out, uint32_t step, void* stream) {
-    return decode_step_impl(ctx, state_in, state_out, inputs, nullptr, out, step, stream);
+    return decode_step_impl(ctx, state_in, state_out, inputs, nullptr, nullptr, nullptr, out, step, stream);
+}
+
+rsq_status rsq_window_bytes(const rsq_ctx* ctx, size_t* a_bytes, size_t* b_bytes, size_t* scale_bytes) {
+    if (!ctx || !a_bytes || !b_bytes || !scale_bytes) return fail(RSQ_E_INVAL, "window_bytes: null argument");
+    const rsq_config& c = ctx->cfg;
+    const size_t bhw = static_cast<size_t>(c.batch) * c.heads * c.window;
+    *a_bytes = bhw * c.dk;
+    *b_bytes = bhw * c.dv;
+    *scale_bytes = bhw * sizeof(float);
+    return RSQ_OK;
+}
+
+rsq_status rsq_decode_step_window(const rsq_ctx* ctx, const rsq_state* state_in, const rsq_state* state_out,
+                                  const rsq_window* win_in, const rsq_window* win_out, const void* inputs,
+                                  float* out, uint32_t step, void* stream) {
+    if (!ctx) return fail(RSQ_E_INVAL, "decode_step_window: null context");
+    if (!win_in || !win_out) return fail(RSQ_E_INVAL, "decode_step_window: null window");
+    const rsq_window* ws[2] = {win_in, win_out};
+    for (const rsq_window* wv : ws)
+        if (!wv->a || !wv->a_scale || !wv->b || !wv->b_scale || !aligned16(wv->a) || !aligned16(wv->a_scale) ||
+            !aligned16(wv->b) || !aligned16(wv->b_scale))
+            return fail(RSQ_E_INVAL, "decode_step_window: window buffer null or not 16-byte aligned");
+    if (win_in->a == win_out->a || win_in->b == win_out->b || win_in->a_scale == win_out->a_scale ||
+        win_in->b_scale == win_out->b_scale)
+        return fail(RSQ_E_INVAL, "decode_step_window: win_in and win_out must be distinct buffers");
+    return decode_step_impl(ctx, state_in, state_out, inputs, nullptr, win_in, win_out, out, step, stream);
 }
 
 rsq_status rsq_decode_step_copy_scale(const rsq_ctx* ctx, const rsq_state* state_in,
@@ -234,7 +268,8 @@ rsq_status rsq_decode_step_copy_scale(const rsq_ctx* ctx, const rsq_state* state
         return fail(RSQ_E_INVAL, "decode_step_copy_scale: copy_absmax null or not 16-byte aligned");
     if (ctx->f32state)
         return fail(RSQ_E_UNSUPPORTED, "decode_step_copy_scale: a full-precision state has no scale");
-    return decode_step_impl(ctx, state_in, state_out, inputs, copy_absmax, out, step, stream);
+    if (ctx->cfg.window) return fail(RSQ_E_UNSUPPORTED, "decode_step_copy_scale: not with a pure-write window");
+    return decode_step_impl(ctx, state_in, state_out, inputs, copy_absmax, nullptr, nullptr, out, step, stream);
 }
 
 rsq_status rsq_column_absmax(const rsq_ctx* ctx, const rsq_state* state, float* absmax, void* stream) {
@@ -258,9 +293,12 @@ rsq_status rsq_column_absmax(const rsq_ctx* ctx, const rsq_state* state, float* 
 
 namespace {
 rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const rsq_state* state_out,
-                            const void* inputs, const float* copy_absmax, float* out, uint32_t step,
-                            void* stream) {
+                            const void* inputs, const float* copy_absmax, const rsq_window* win_in,
+                            const rsq_window* win_out, float* out, uint32_t step, void* stream) {
     if (!ctx) return fail(RSQ_E_INVAL, "decode_step: null context");
+    if ((ctx->cfg.window > 0) != (win_in != nullptr))
+        return fail(RSQ_E_INVAL, ctx->cfg.window ? "decode_step: this context has a pure-write window: use rsq_decode_step_window"
+                                                 : "decode_step_window: this context has no window");
     rsq_status s = check_state(ctx, state_in, "decode_step(state_in)");
     if (s) return s;
     if ((s = check_state(ctx, state_out, "decode_step(state_out)"))) return s;
@@ -279,6 +317,17 @@ rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const
     p.scales_out = state_out->scales;
     p.out = out;
     p.copy_absmax = copy_absmax;
+    if (win_in) {
+        p.W = c.window;
+        p.win_a_in = static_cast<const uint8_t*>(win_in->a);
+        p.win_as_in = win_in->a_scale;
+        p.win_b_in = static_cast<const uint8_t*>(win_in->b);
+        p.win_bs_in = win_in->b_scale;
+        p.win_a_out = static_cast<uint8_t*>(win_out->a);
+        p.win_as_out = win_out->a_scale;
+        p.win_b_out = static_cast<uint8_t*>(win_out->b);
+        p.win_bs_out = win_out->b_scale;
+    }
     p.flag = ctx->flag;
     p.step = step;
     p.key0 = static_cast<uint32_t>(c.seed);
@@ -317,7 +366,7 @@ rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const
     const int ghu = ctx->grid / ctx->ncb;
     p.gh = ghu % c.heads;
     p.gb = ghu / c.heads;
-    const int err = rsq::launch_decode(c.family, c.dk, ctx->ub, ctx->f32state,
+    const int err = rsq::launch_decode(kernel_family(c), c.dk, ctx->ub, ctx->f32state,
                                        c.rounding | (copy_absmax ? kCopyScaleBit : 0), p,
                                        stream);
     if (err) return cuda_fail(err, "decode_step launch");
@@ -478,6 +527,8 @@ extern "C" rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_s
         return fail(RSQ_E_INVAL, "decode_step_noalloc: bad in_dtype %d", c.in_dtype);
     if (c.family == RSQ_MAMBA2 && (c.ngroups < 1 || c.heads % c.ngroups != 0))
         return fail(RSQ_E_INVAL, "decode_step_noalloc: ngroups must divide heads");
+    if (c.window != 0)
+        return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: no pure-write window in this entry point");
     if (kNoallocWordsNeeded > kNoallocScratchWords)
         return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: needs %d scratch words, the static array holds %d",
                     kNoallocWordsNeeded, kNoallocScratchWords);
@@ -513,7 +564,7 @@ extern "C" rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_s
     int threads = 0;
     size_t smem = 0;
     const void* func = nullptr;
-    if (rsq::decode_kernel_info(c.family, c.dk, ctx.ub, ctx.f32state, c.rounding, &threads, &smem,
+    if (rsq::decode_kernel_info(kernel_family(c), c.dk, ctx.ub, ctx.f32state, c.rounding, &threads, &smem,
                                 &func) != 0)
         return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: no kernel for dk=%d dv=%d", c.dk, c.dv);
     int err = cudaGetDevice(&ctx.device);

@@ -108,6 +108,21 @@ __device__ __forceinline__ uint64_t fma2_rm(uint64_t a, uint64_t b, uint64_t c) 
     return d;
 }
 
+// FP8 E4M3: two codes from two floats (round to nearest even, saturating to
+// +-448); `hi` lands in the upper byte of the 16-bit result.
+__device__ __forceinline__ uint32_t e4m3x2_from_f32(float hi, float lo) {
+    uint16_t d;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+// Two E4M3 codes (low byte first) to two floats (exact, through f16).
+__device__ __forceinline__ void e4m3x2_to_f32(uint32_t two, float& lo, float& hi) {
+    uint32_t h2;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(two)));
+    asm("{ .reg .f16 a, b; mov.b32 {a, b}, %2; cvt.f32.f16 %0, a; cvt.f32.f16 %1, b; }"
+        : "=f"(lo), "=f"(hi) : "r"(h2));
+}
+
 // hi(a * b) + c (32-bit unsigned)
 __device__ __forceinline__ uint32_t umulhi_add(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;

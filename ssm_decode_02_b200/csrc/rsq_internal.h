@@ -8,6 +8,11 @@
 
 namespace rsq {
 
+// Internal family value of Gated DeltaNet with a pure-write window (the public
+// family is RSQ_GDN with rsq_config.window > 0).
+constexpr int kFamGdnPw = 4;
+constexpr int kMaxWindow = 16;
+
 constexpr unsigned kFlagNonFinite = 1u;  // a column's absmax was inf or NaN
 constexpr unsigned kFlagTimeout = 2u;    // a bounded barrier wait ran out
 
@@ -51,6 +56,17 @@ struct DecodeParams {
     const float* D;                // Mamba-2 D [H]
     float* out;                    // [B][H][dv]
     const float* copy_absmax;      // copy scale: column maxima [B][H][dv] of an unquantized copy, or null
+    // pure-write window (GDN): W slots; a [B][H][W][dk] FP8 + as [B][H][W],
+    // b [B][H][dv/16][W][16] FP8 + bs [B][H][W]; in and out buffers differ
+    int W;
+    const uint8_t* win_a_in;
+    const float* win_as_in;
+    const uint8_t* win_b_in;
+    const float* win_bs_in;
+    uint8_t* win_a_out;
+    float* win_as_out;
+    uint8_t* win_b_out;
+    float* win_bs_out;
     unsigned* flag;
     uint32_t step, key0, key1;
     PhiloxKeys rk;                 // Philox round keys of (key0, key1)

@@ -61,6 +61,9 @@ def _create(**kw):
     (dict(head_bits=[8, 4, 2, 8]), rsq.RSQ_E_INVAL),
     (dict(head_bits=[8, 32, 32, 32]), rsq.RSQ_E_UNSUPPORTED),
     (dict(family=rsq.RSQ_MAMBA2, ngroups=3), rsq.RSQ_E_INVAL),
+    (dict(window=3), rsq.RSQ_E_INVAL),
+    (dict(window=8, family=rsq.RSQ_MAMBA2), rsq.RSQ_E_UNSUPPORTED),
+    (dict(window=8, rounding=rsq.RSQ_BDR), rsq.RSQ_E_UNSUPPORTED),
 ])
 def test_create_rejects_bad_configs_on_host(kw, status):
     with pytest.raises(rsq.RsqError) as e:
