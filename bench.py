@@ -503,13 +503,16 @@ def run_ours(args, w: W.Workload):
 # ---------------------------------------------------------------------------
 # Long-horizon state drift (quantized trajectories against the FP32 trajectory)
 # ---------------------------------------------------------------------------
-# (label, bits, rounding, scale source): "noisy" = the quantized state's own
-# column maxima, "copy" = the column maxima of the FP32 trajectory
+# (label, bits, rounding, variant): "noisy" = the quantized state's own column
+# maxima as scales, "copy" = the column maxima of the FP32 trajectory, "wN" = a
+# pure-write window of N FP8 slots beside the low-bit history (GDN)
 DRIFT_VARIANTS = (("int4_sr", 4, "sr", "noisy"), ("int4_rtn", 4, "rtn", "noisy"),
                   ("int4_bdr", 4, "bdr", "noisy"), ("int4_sr_bdr", 4, "sr_bdr", "noisy"),
                   ("int4_sr_copy", 4, "sr", "copy"), ("int4_rtn_copy", 4, "rtn", "copy"),
+                  ("int4_sr_w8", 4, "sr", "w8"), ("int4_rtn_w8", 4, "rtn", "w8"),
                   ("int8_sr", 8, "sr", "noisy"), ("int8_rtn", 8, "rtn", "noisy"),
-                  ("int8_bdr", 8, "bdr", "noisy"), ("int8_sr_copy", 8, "sr", "copy"))
+                  ("int8_bdr", 8, "bdr", "noisy"), ("int8_sr_copy", 8, "sr", "copy"),
+                  ("int8_sr_w8", 8, "sr", "w8"))
 ROUNDING = {"rtn": 0, "sr": 1, "bdr": 2, "sr_bdr": 3}   # rsq_rounding values
 
 
@@ -536,18 +539,23 @@ def drift_series(w: W.Workload, steps: int, every: int, B: int | None = None, va
     fam = FAMILY[w.family]
     in_dtype = rsq.RSQ_BF16 if w.in_dtype == "bf16" else rsq.RSQ_F32
 
-    def make(bits, rounding):
+    def make(bits, rounding, window=0):
         ctx = rsq.Context(fam, B, w.H, w.dk, w.dv, head_bits=np.full(w.H, bits, np.int8),
                           rounding=ROUNDING[rounding],
-                          in_dtype=in_dtype, seed=w.sr_seed, ngroups=w.ngroups)
+                          in_dtype=in_dtype, seed=w.sr_seed, ngroups=w.ngroups, window=window)
         st = ctx.alloc_state(device)
         ctx.quantize(torch.zeros((B, w.H, w.dk, w.dv), dtype=torch.float32, device=device), st)
         out = torch.empty((B, w.H, w.dv), dtype=torch.float32, device=device)
         return ctx, st, out
 
+    def window_of(src):
+        return int(src[1:]) if src.startswith("w") else 0
+
     ref = make(32, "rtn")
-    runs = {label: make(bits, rnd) for label, bits, rnd, _ in variants}
+    runs = {label: make(bits, rnd, window_of(src)) for label, bits, rnd, src in variants}
     source = {label: src for label, _, _, src in variants}
+    wins = {label: [runs[label][0].alloc_window(device), runs[label][0].alloc_window(device)]
+            for label, _, _, src in variants if window_of(src)}
     copy_max = torch.empty((B, w.H, w.dv), dtype=torch.float32, device=device)
     sums = torch.empty((B, w.H, 2), dtype=torch.float64, device=device)
     series = {label: [] for label, _, _, _ in variants}
@@ -561,14 +569,19 @@ def drift_series(w: W.Workload, steps: int, every: int, B: int | None = None, va
         for label, (ctx, st, out) in runs.items():
             if source[label] == "copy":
                 ctx.decode_step_copy_scale(st, st, ins, copy_max, out, t)
+            elif label in wins:
+                ctx.decode_step_window(st, st, wins[label][t % 2], wins[label][(t + 1) % 2], ins, out, t)
             else:
                 ctx.decode_step(st, st, ins, out, t)
         if (t + 1) % every == 0:
             o_ref = ref[2].double()
             for label, (ctx, st, out) in runs.items():
-                rsq.rsq_state_drift(ctx.ctx, st, ref[0].ctx, ref[1], sums)
-                s = sums.cpu().numpy()
-                num, den = s[..., 0], s[..., 1]
+                if label in wins:
+                    num, den = _window_drift_sums(rsq, ctx, st, wins[label][(t + 1) % 2], ref, B, w, device)
+                else:
+                    rsq.rsq_state_drift(ctx.ctx, st, ref[0].ctx, ref[1], sums)
+                    s = sums.cpu().numpy()
+                    num, den = s[..., 0], s[..., 1]
                 per_head = np.sqrt(num[den > 0] / den[den > 0])
                 o_err = float(torch.linalg.vector_norm(out.double() - o_ref) /
                               torch.linalg.vector_norm(o_ref))
@@ -579,6 +592,25 @@ def drift_series(w: W.Workload, steps: int, every: int, B: int | None = None, va
             raise RuntimeError("non-finite state in the drift study")
         ctx.close()
     return series
+
+
+def _window_drift_sums(rsq, ctx, st, win, ref, B, w, device):
+    """Per-head sums of (full state - FP32 state)^2 and FP32 state^2 for a state
+    with a pure-write window: full state = dequantized history + sum_w a_w b_w^T."""
+    import torch
+    Hq = torch.empty((B, w.H, w.dk, w.dv), dtype=torch.float32, device=device)
+    F = torch.empty_like(Hq)
+    ctx.dequantize(st, Hq)
+    ref[0].dequantize(ref[1], F)
+    Wn = ctx.window
+    dec = lambda codes: codes.view(torch.float8_e4m3fn).to(torch.float32)
+    a = dec(win.a) * win.a_scale[..., None]                                   # [B][H][W][dk]
+    b = dec(win.b).permute(0, 1, 3, 2, 4).reshape(B, w.H, Wn, w.dv) * win.b_scale[..., None]
+    full = Hq.double() + torch.einsum("bhwi,bhwj->bhij", a.double(), b.double())
+    F = F.double()
+    num = ((full - F) ** 2).sum(dim=(2, 3)).cpu().numpy()
+    den = (F ** 2).sum(dim=(2, 3)).cpu().numpy()
+    return num, den
 
 
 def run_drift(args, w: W.Workload, pool) -> int:

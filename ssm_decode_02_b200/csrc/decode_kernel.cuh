@@ -175,6 +175,63 @@ __device__ __forceinline__ Gates load_gates(const DecodeParams& p, const UnitIt&
 // chunk in increasing row order and combine the 8 chunks by the XOR butterfly
 // d = 1, 2, 4.  The writer warp also encodes the new a vectors (FP8 E4M3, one
 // scale = max|a| / 448 per vector).
+// Widened elements [i0, i0 + N) of a key-axis vector in the stage.
+template <int N>
+__device__ __forceinline__ void ld_chunk(const uint8_t* base, int i0, bool bf16, float (&x)[N]) {
+    if constexpr (N % 4 == 0) {
+#pragma unroll
+        for (int t = 0; t < N; t += 4) {
+            const float4 v = ld_vec4(base, i0 + t, bf16);
+            x[t] = v.x; x[t + 1] = v.y; x[t + 2] = v.z; x[t + 3] = v.w;
+        }
+    } else {
+#pragma unroll
+        for (int t = 0; t < N; ++t) x[t] = ld_vec(base, i0 + t, bf16);
+    }
+}
+
+// One slot of the pure-write window for this lane's chunk of rows: decode a,
+// propagate a' = alpha * fma(-beta (k.a), k, a), and z = a'.q (k.q for the
+// slot that takes the new write).  Dots: each chunk in increasing row order,
+// the 8 chunks combined by the XOR butterfly d = 1, 2, 4.
+template <int CH>
+__device__ __forceinline__ float pw_slot(const uint8_t* stage, int off_wa, int off_was, int slot, int dk,
+                                         int i0, const float (&kk)[CH], const float (&qq)[CH], float alpha,
+                                         float beta, bool merging, float (&a)[CH]) {
+    const float as = reinterpret_cast<const float*>(stage + off_was)[slot];
+    const uint16_t* ab = reinterpret_cast<const uint16_t*>(stage + off_wa + slot * dk + i0);
+#pragma unroll
+    for (int t = 0; t < CH; t += 2) {
+        float lo, hi;
+        e4m3x2_to_f32(ab[t / 2], lo, hi);
+        a[t] = __fmul_rn(lo, as);
+        a[t + 1] = __fmul_rn(hi, as);
+    }
+    float ka = 0.f;
+#pragma unroll
+    for (int t = 0; t < CH; ++t) ka = __fmaf_rn(kk[t], a[t], ka);
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) ka = __fadd_rn(ka, __shfl_xor_sync(0xffffffffu, ka, d));
+    const float gg = __fmul_rn(beta, ka);
+    float z = 0.f;
+#pragma unroll
+    for (int t = 0; t < CH; ++t) {
+        a[t] = __fmul_rn(alpha, __fmaf_rn(-gg, kk[t], a[t]));
+        z = __fmaf_rn(merging ? kk[t] : a[t], qq[t], z);
+    }
+#pragma unroll
+    for (int d = 1; d < 8; d <<= 1) z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, d));
+    return z;
+}
+
+// Pure-write window ("Low-Bit GDN Recurrent-State Quantization: ... Pure-Write
+// Sliding Windows", abstract), per warp: every slot's a vector goes through
+// the step's transition a <- alpha (a - beta k (k.a)); the slot `ps` leaving
+// the window leaves its propagated a in the pair array `pm` (rows as
+// duplicated pairs) for the merge into the history; z_w = a_w . q (slot ps:
+// k . q, its new write) goes to `zs`.  Lane (slot group, chunk) handles rows
+// [chunk * DK/8, (chunk+1) * DK/8) of slots slot group, +4, +8, ...  The writer
+// warp also encodes the new a vectors (FP8 E4M3, one scale = max|a| / 448).
 template <int DK, int PST>
 __device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* stage, int off_wa,
                                          int off_was, int off_va, int off_vb, int hu, int ps,
@@ -183,40 +240,18 @@ __device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* s
     constexpr int CH = DK / 8;
     const bool bf16 = p.in_bf16 != 0;
     const int sl = lane >> 3, chunk = lane & 7, i0 = chunk * CH;
-    for (int pass = 0; pass * 4 < p.W; ++pass) {
-        const int slot = pass * 4 + sl;
+    float kk[CH], qq[CH];
+    ld_chunk<CH>(stage + off_vb, i0, bf16, kk);
+    ld_chunk<CH>(stage + off_va, i0, bf16, qq);
+    auto finish = [&](int slot, float z, float (&a)[CH]) {
         const bool merging = (slot == ps);
-        const float as = reinterpret_cast<const float*>(stage + off_was)[slot];
-        const uint16_t* ab = reinterpret_cast<const uint16_t*>(stage + off_wa + slot * DK + i0);
-        float a[CH], kk[CH];
-        float ka = 0.f;
+        if (merging) {
 #pragma unroll
-        for (int t = 0; t < CH; t += 2) {
-            float lo, hi;
-            e4m3x2_to_f32(ab[t / 2], lo, hi);
-            a[t] = __fmul_rn(lo, as);
-            a[t + 1] = __fmul_rn(hi, as);
-            kk[t] = ld_vec(stage + off_vb, i0 + t, bf16);
-            kk[t + 1] = ld_vec(stage + off_vb, i0 + t + 1, bf16);
-        }
-#pragma unroll
-        for (int t = 0; t < CH; ++t) ka = __fmaf_rn(kk[t], a[t], ka);
-#pragma unroll
-        for (int d = 1; d < 8; d <<= 1) ka = __fadd_rn(ka, __shfl_xor_sync(0xffffffffu, ka, d));
-        const float gg = __fmul_rn(beta, ka);
-        float z = 0.f;
-#pragma unroll
-        for (int t = 0; t < CH; ++t) {
-            a[t] = __fmul_rn(alpha, __fmaf_rn(-gg, kk[t], a[t]));  // propagated a'
-            const float q = ld_vec(stage + off_va, i0 + t, bf16);
-            z = __fmaf_rn(merging ? kk[t] : a[t], q, z);
-            if (merging) {
+            for (int t = 0; t < CH; ++t) {
                 const int i = i0 + t;
                 pm[(i & (kR - 1)) * PST + i / kR] = pk(a[t], a[t]);
             }
         }
-#pragma unroll
-        for (int d = 1; d < 8; d <<= 1) z = __fadd_rn(z, __shfl_xor_sync(0xffffffffu, z, d));
         if (chunk == 0) zs[slot] = z;
         if (writer) {
             // the stored a: propagated for the slots that stay, k for the new write
@@ -237,6 +272,22 @@ __device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* s
             }
             if (chunk == 0) p.win_as_out[(long long)hu * p.W + slot] = __fdiv_rn(m, 448.f);
         }
+    };
+    int pass = 0;
+    // two slots per lane at a time where possible (independent dependency chains)
+    for (; (pass + 2) * 4 <= p.W; pass += 2) {
+        const int s0 = pass * 4 + sl, s1 = s0 + 4;
+        float a0[CH], a1[CH];
+        const float z0 = pw_slot<CH>(stage, off_wa, off_was, s0, DK, i0, kk, qq, alpha, beta, s0 == ps, a0);
+        const float z1 = pw_slot<CH>(stage, off_wa, off_was, s1, DK, i0, kk, qq, alpha, beta, s1 == ps, a1);
+        finish(s0, z0, a0);
+        finish(s1, z1, a1);
+    }
+    for (; pass * 4 < p.W; ++pass) {
+        const int s0 = pass * 4 + sl;
+        float a0[CH];
+        const float z0 = pw_slot<CH>(stage, off_wa, off_was, s0, DK, i0, kk, qq, alpha, beta, s0 == ps, a0);
+        finish(s0, z0, a0);
     }
 }
 
@@ -551,25 +602,18 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
         const long long nblk = p.dv / kBlockCols;
         uint8_t* bdst = p.win_b_out + ((long long)hu * nblk + blk) * p.W * 16;
         if (lane < p.W) {
-            uint4 row;
-            if (lane != ps) {
-                row = *reinterpret_cast<const uint4*>(stage + C::OFF_WB + (w * p.W + lane) * 16);
-            } else {
-                uint32_t wd[4];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    float x[4];
-#pragma unroll
-                    for (int e = 0; e < 4; ++e)
-                        x[e] = __fmul_rn(__fmul_rn(beta, ld_vec(stage + C::OFF_VF, j0 + 4 * q4 + e, bf16)), invb);
-                    wd[q4] = e4m3x2_from_f32(x[1], x[0]) | (e4m3x2_from_f32(x[3], x[2]) << 16);
-                }
-                row = make_uint4(wd[0], wd[1], wd[2], wd[3]);
-            }
-            *reinterpret_cast<uint4*>(bdst + lane * 16) = row;
+            // the slots that stay: copied
+            if (lane != ps)
+                *reinterpret_cast<uint4*>(bdst + lane * 16) =
+                    *reinterpret_cast<const uint4*>(stage + C::OFF_WB + (w * p.W + lane) * 16);
             if (un.cb == 0 && w == 0)
                 p.win_bs_out[(long long)hu * p.W + lane] =
                     (lane == ps) ? __fdiv_rn(mb, 448.f) : reinterpret_cast<const float*>(stage + C::OFF_WBS)[lane];
+        } else if (lane >= 16) {
+            // the new write: one column per lane
+            const int jj = lane - 16;
+            const float x = __fmul_rn(__fmul_rn(beta, ld_vec(stage + C::OFF_VF, j0 + jj, bf16)), invb);
+            bdst[ps * 16 + jj] = static_cast<uint8_t>(e4m3x2_from_f32(0.f, x));
         }
     }
 

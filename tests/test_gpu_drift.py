@@ -26,6 +26,8 @@ def _oracle_series(w, steps, every, variants):
     rnd = {"sr": oracle.SR, "rtn": oracle.RTN, "bdr": oracle.BDR, "sr_bdr": oracle.SR_BDR}
     ref = oracle.zero_state(w.B, w.H, w.dk, w.dv, fp32=True)
     qs = {lab: oracle.zero_state(w.B, w.H, w.dk, w.dv, fp32=False) for lab, _, _, _ in variants}
+    wins = {lab: oracle.zero_window(w.B, w.H, int(src[1:]), w.dk, w.dv)
+            for lab, _, _, src in variants if src.startswith("w")}
     out = {lab: [] for lab, _, _, _ in variants}
     f32 = np.full(w.H, 32, np.int8)
     for t in range(steps):
@@ -34,11 +36,16 @@ def _oracle_series(w, steps, every, variants):
         m = np.abs(ref["f"]).max(axis=2)
         for lab, bits, r, src in variants:
             hb = np.full(w.H, bits, np.int8)
-            qs[lab], o = oracle.gdn_step(qs[lab], inp, hb, rounding=rnd[r], seed=w.sr_seed, step=t,
-                                         copy_absmax=m if src == "copy" else None)
+            if lab in wins:
+                qs[lab], wins[lab], o = oracle.gdn_pw_step(qs[lab], wins[lab], inp, hb, rounding=rnd[r],
+                                                           seed=w.sr_seed, step=t)
+            else:
+                qs[lab], o = oracle.gdn_step(qs[lab], inp, hb, rounding=rnd[r], seed=w.sr_seed, step=t,
+                                             copy_absmax=m if src == "copy" else None)
             if (t + 1) % every == 0:
                 F = oracle.dequantize(ref, f32).astype(np.float64)
-                D = oracle.dequantize(qs[lab], hb).astype(np.float64)
+                D = (oracle.window_full_state(qs[lab], wins[lab], hb) if lab in wins
+                     else oracle.dequantize(qs[lab], hb).astype(np.float64))
                 num = ((D - F) ** 2).sum(axis=(2, 3))
                 den = (F ** 2).sum(axis=(2, 3))
                 o64, r64 = o.astype(np.float64), o_ref.astype(np.float64)
