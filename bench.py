@@ -201,6 +201,23 @@ def oracle_rate(w: W.Workload, head_bits, budget_s: float, heads_per_call: int =
     return n_done / t_used, n_done, t
 
 
+def _oracle_rate_job(job):
+    w, bits, budget_s = job
+    rate, n, _ = oracle_rate(w, bits, budget_s)
+    return n, n / rate
+
+
+def oracle_rate_all_cores(w: W.Workload, head_bits, budget_s: float):
+    """The same oracle sample run by one spawned process per host core at once
+    (each core its own heads): head updates of all processes / the longest
+    process time.  Returns (rate, processes)."""
+    import multiprocessing as mp
+    n = max(1, os.cpu_count() or 1)
+    with mp.get_context("spawn").Pool(n) as pool:
+        res = pool.map(_oracle_rate_job, [(w, head_bits, budget_s)] * n)
+    return sum(r[0] for r in res) / max(r[1] for r in res), n
+
+
 def _oracle_step(oracle, w: W.Workload, st, inp, bits, rounding, t, R, heads):
     kw = dict(rounding=rounding, seed=w.sr_seed, step=t, R=R, heads=heads)
     if w.family == "gdn":
@@ -488,6 +505,11 @@ def run_ours(args, w: W.Workload):
         line["cpu_baseline"] = {"value": rate, "unit": "head-updates/s", "cores": 1, "kind": "oracle",
                                 "sample": "%d head updates (%d decode steps of the first requests) "
                                           "in ~%.0f s, single-threaded C oracle" % (n, steps, args.cpu_seconds)}
+        rate_all, procs = oracle_rate_all_cores(w, bits, args.cpu_seconds)
+        line["cpu_baseline_all_cores"] = {
+            "value": rate_all, "unit": "head-updates/s", "cores": procs, "kind": "oracle",
+            "sample": "the same sample in %d concurrent processes (one per host core), ~%.0f s each"
+                      % (procs, args.cpu_seconds)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     for gr in list(graph_cache.values()) + warm_graphs:
