@@ -27,7 +27,9 @@ RSQ_DECLARE(decode_info_gla_copy)
 RSQ_DECLARE(decode_info_gla_copy_bdr)
 RSQ_DECLARE(decode_info_kda_copy)
 RSQ_DECLARE(decode_info_kda_copy_bdr)
-RSQ_DECLARE(decode_info_gdn_pw)
+RSQ_DECLARE(decode_info_gdn_pw4)
+RSQ_DECLARE(decode_info_gdn_pw8)
+RSQ_DECLARE(decode_info_gdn_pw16)
 #undef RSQ_DECLARE
 
 int decode_kernel_info(int family, int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
@@ -40,8 +42,10 @@ int decode_kernel_info(int family, int dk, int ub, bool f32state, int rnd, int* 
         {decode_info_kda, decode_info_kda_bdr, decode_info_kda_copy, decode_info_kda_copy_bdr}};
     if (rnd < 0 || rnd > 7) return -1;
     const int group = f32state ? 0 : (rnd >> 1);
-    if (family == kFamGdnPw)  // pure-write window: plain rules only
-        return group == 0 ? decode_info_gdn_pw(dk, ub, f32state, rnd, threads, smem, func) : -1;
+    if (is_pw_family(family)) {  // pure-write window: plain rules only
+        static const InfoFn pw[3] = {decode_info_gdn_pw4, decode_info_gdn_pw8, decode_info_gdn_pw16};
+        return group == 0 ? pw[family - kFamGdnPw](dk, ub, f32state, rnd, threads, smem, func) : -1;
+    }
     if (family < 0 || family > 3) return -1;
     return table[family][group](dk, ub, f32state, rnd, threads, smem, func);
 }

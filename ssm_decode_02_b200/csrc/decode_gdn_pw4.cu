@@ -1,0 +1,11 @@
+// decode_gdn_pw4.cu -- Gated DeltaNet with a 4-slot pure-write window:
+// instantiations of the fused decode kernel with nearest and stochastic
+// rounding (and the full-precision history).
+#include "decode_kernel.cuh"
+
+namespace rsq {
+int decode_info_gdn_pw4(int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
+                        const void** func) {
+    return decode_info_family<kFamGdnPw + 0, 0, kRndSr>(dk, ub, f32state, rnd, threads, smem, func);
+}
+}  // namespace rsq

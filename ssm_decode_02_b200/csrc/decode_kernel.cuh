@@ -35,7 +35,7 @@ struct DecodeCfg {
     static constexpr int NT = 32 * UB;         // one warp per 16-column block
     static constexpr int UCOLS = 16 * UB;      // columns per unit
     // pipeline stages (KDA's extra pair array leaves room for three)
-    static constexpr int NS = F32STATE ? 2 : ((FAM == RSQ_KDA || FAM == kFamGdnPw) ? 3 : 4);
+    static constexpr int NS = F32STATE ? 2 : ((FAM == RSQ_KDA || is_pw_family(FAM)) ? 3 : 4);
     static constexpr int CODE_BYTES = F32STATE ? DK * UCOLS * 4 : DK * UCOLS;  // largest tile (8-bit)
     static constexpr int OFF_SCALES = CODE_BYTES;
     static constexpr int OFF_VA = OFF_SCALES + UCOLS * 4;  // GDN q / Mamba-2 C   (<= DK floats)
@@ -45,7 +45,8 @@ struct DecodeCfg {
     static constexpr bool DIAG = (FAM == RSQ_GLA || FAM == RSQ_KDA);
     // pure-write window: the whole v (<= 256 floats), the slots' a codes and
     // scales, this unit's b codes (W x 16 per block) and the b scales
-    static constexpr bool PW = (FAM == kFamGdnPw);
+    static constexpr bool PW = is_pw_family(FAM);
+    static constexpr int WIN = pw_window(FAM);  // window slots
     static constexpr int OFF_VF = OFF_VD;
     static constexpr int OFF_WA = OFF_VF + 256 * 4;
     static constexpr int OFF_WAS = OFF_WA + kMaxWindow * DK;
@@ -58,10 +59,10 @@ struct DecodeCfg {
     static constexpr int PST = L::RPT + 2;
     // pair arrays: q, k (+ the decay per key channel for GLA, + decay and
     // decay * k for KDA)
-    static constexpr int NPAIR = FAM == RSQ_KDA ? 4 : ((DIAG || FAM == kFamGdnPw) ? 3 : 2);
+    static constexpr int NPAIR = FAM == RSQ_KDA ? 4 : ((DIAG || is_pw_family(FAM)) ? 3 : 2);
     // (+ the window's z_w = a_w . q for the pure-write window)
     static constexpr int OFF_PZ = NPAIR * kR * PST * 8;
-    static constexpr int P_WARP = OFF_PZ + (FAM == kFamGdnPw ? kMaxWindow * 4 : 0);
+    static constexpr int P_WARP = OFF_PZ + (is_pw_family(FAM) ? kMaxWindow * 4 : 0);
     static constexpr int OFF_P = NS * STAGE;
     static constexpr int OFF_CNT = OFF_P + UB * P_WARP;  // NS release counters
     static constexpr int OFF_BAR = OFF_CNT + 16;
@@ -103,7 +104,7 @@ __device__ __forceinline__ void issue_unit(const DecodeParams& p, const UnitIt& 
     const int hu = un.hu(p);
     const uint32_t code_bytes = static_cast<uint32_t>(DK * UCOLS * bits / 8);
     const uint32_t esz = p.in_bf16 ? 2u : 4u;
-    const uint32_t W = static_cast<uint32_t>(p.W);
+    const uint32_t W = static_cast<uint32_t>(C::WIN);
     const uint32_t total = code_bytes + (F32STATE ? 0u : UCOLS * 4u) + 2u * DK * esz + UCOLS * esz +
                            (C::DIAG ? DK * 4u : 0u) +
                            (C::PW ? p.dv * esz + W * DK + 2u * W * 4u + UB * W * 16u : 0u);
@@ -232,7 +233,7 @@ __device__ __forceinline__ float pw_slot(const uint8_t* stage, int off_wa, int o
 // k . q, its new write) goes to `zs`.  Lane (slot group, chunk) handles rows
 // [chunk * DK/8, (chunk+1) * DK/8) of slots slot group, +4, +8, ...  The writer
 // warp also encodes the new a vectors (FP8 E4M3, one scale = max|a| / 448).
-template <int DK, int PST>
+template <int DK, int PST, int WIN>
 __device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* stage, int off_wa,
                                          int off_was, int off_va, int off_vb, int hu, int ps,
                                          float alpha, float beta, bool writer, uint64_t* pm,
@@ -264,18 +265,19 @@ __device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* s
 #pragma unroll
             for (int d = 1; d < 8; d <<= 1) m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, d));
             const float inv = (m > 0.f && isfinite(m)) ? __fdiv_rn(448.f, m) : 0.f;
-            uint8_t* dst = p.win_a_out + ((long long)hu * p.W + slot) * DK + i0;
+            uint8_t* dst = p.win_a_out + ((long long)hu * WIN + slot) * DK + i0;
 #pragma unroll
             for (int t = 0; t < CH; t += 2) {
                 const uint32_t two = e4m3x2_from_f32(__fmul_rn(a[t + 1], inv), __fmul_rn(a[t], inv));
                 *reinterpret_cast<uint16_t*>(dst + t) = static_cast<uint16_t>(two);
             }
-            if (chunk == 0) p.win_as_out[(long long)hu * p.W + slot] = __fdiv_rn(m, 448.f);
+            if (chunk == 0) p.win_as_out[(long long)hu * WIN + slot] = __fdiv_rn(m, 448.f);
         }
     };
     int pass = 0;
     // two slots per lane at a time where possible (independent dependency chains)
-    for (; (pass + 2) * 4 <= p.W; pass += 2) {
+#pragma unroll
+    for (; (pass + 2) * 4 <= WIN; pass += 2) {
         const int s0 = pass * 4 + sl, s1 = s0 + 4;
         float a0[CH], a1[CH];
         const float z0 = pw_slot<CH>(stage, off_wa, off_was, s0, DK, i0, kk, qq, alpha, beta, s0 == ps, a0);
@@ -283,7 +285,8 @@ __device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* s
         finish(s0, z0, a0);
         finish(s1, z1, a1);
     }
-    for (; pass * 4 < p.W; ++pass) {
+#pragma unroll
+    for (; pass * 4 < WIN; ++pass) {
         const int s0 = pass * 4 + sl;
         float a0[CH];
         const float z0 = pw_slot<CH>(stage, off_wa, off_was, s0, DK, i0, kk, qq, alpha, beta, s0 == ps, a0);
@@ -328,9 +331,9 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
     }
     __syncwarp();
     float* zs = reinterpret_cast<float*>(smem + C::OFF_P + w * C::P_WARP + C::OFF_PZ);  // window z_w
-    const int ps = C::PW ? static_cast<int>(p.step % static_cast<uint32_t>(p.W)) : 0;  // slot leaving
+    const int ps = C::PW ? static_cast<int>(p.step % static_cast<uint32_t>(C::WIN)) : 0;  // slot leaving
     if constexpr (C::PW) {
-        pw_slots<DK, C::PST>(p, stage, C::OFF_WA, C::OFF_WAS, C::OFF_VA, C::OFF_VB, hu, ps, gt.g0, gt.g1,
+        pw_slots<DK, C::PST, C::WIN>(p, stage, C::OFF_WA, C::OFF_WAS, C::OFF_VA, C::OFF_VB, hu, ps, gt.g0, gt.g1,
                              un.cb == 0 && w == 0, pc, zs, lane);
         __syncwarp();
     }
@@ -406,7 +409,7 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
         if constexpr (C::PW) {
             // the slot leaving the window merges into the history: S += a'_ps b_ps^T
             const float bsc = reinterpret_cast<const float*>(stage + C::OFF_WBS)[ps];
-            const uint32_t b4 = *reinterpret_cast<const uint32_t*>(stage + C::OFF_WB + (w * p.W + ps) * 16 + 4 * cw);
+            const uint32_t b4 = *reinterpret_cast<const uint32_t*>(stage + C::OFF_WB + (w * C::WIN + ps) * 16 + 4 * cw);
             float b0, b1, b2, b3;
             e4m3x2_to_f32(b4 & 0xFFFFu, b0, b1);
             e4m3x2_to_f32(b4 >> 16, b2, b3);
@@ -512,9 +515,10 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
     if constexpr (C::PW) {
         // the window's part of the readout: o_j += b_w,j z_w in slot order
         const float vcol = ld_vec(stage + C::OFF_VC, 16 * w + 4 * cw + c, bf16);
-        const uint8_t* bcol = stage + C::OFF_WB + w * p.W * 16 + 4 * cw + c;
+        const uint8_t* bcol = stage + C::OFF_WB + w * C::WIN * 16 + 4 * cw + c;
         const float* bscale = reinterpret_cast<const float*>(stage + C::OFF_WBS);
-        for (int ws = 0; ws < p.W; ++ws) {
+#pragma unroll
+        for (int ws = 0; ws < C::WIN; ++ws) {
             float bw, unused;
             e4m3x2_to_f32(bcol[ws * 16], bw, unused);
             bw = (ws == ps) ? __fmul_rn(gt.g1, vcol) : __fmul_rn(bw, bscale[ws]);
@@ -600,14 +604,14 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
         for (int d = 16; d >= 1; d >>= 1) mb = max_nan(mb, __shfl_xor_sync(0xffffffffu, mb, d));
         const float invb = (mb > 0.f && isfinite(mb)) ? __fdiv_rn(448.f, mb) : 0.f;
         const long long nblk = p.dv / kBlockCols;
-        uint8_t* bdst = p.win_b_out + ((long long)hu * nblk + blk) * p.W * 16;
-        if (lane < p.W) {
+        uint8_t* bdst = p.win_b_out + ((long long)hu * nblk + blk) * C::WIN * 16;
+        if (lane < C::WIN) {
             // the slots that stay: copied
             if (lane != ps)
                 *reinterpret_cast<uint4*>(bdst + lane * 16) =
-                    *reinterpret_cast<const uint4*>(stage + C::OFF_WB + (w * p.W + lane) * 16);
+                    *reinterpret_cast<const uint4*>(stage + C::OFF_WB + (w * C::WIN + lane) * 16);
             if (un.cb == 0 && w == 0)
-                p.win_bs_out[(long long)hu * p.W + lane] =
+                p.win_bs_out[(long long)hu * C::WIN + lane] =
                     (lane == ps) ? __fdiv_rn(mb, 448.f) : reinterpret_cast<const float*>(stage + C::OFF_WBS)[lane];
         } else if (lane >= 16) {
             // the new write: one column per lane
@@ -642,7 +646,7 @@ constexpr int decode_min_blocks() {
     using C = DecodeCfg<FAM, DK, UB, F32STATE>;
     // BDR: about 168 registers per thread (65536 / (168 * 128) = 3 CTAs of 128 threads)
     // (the pure-write window's slot pass needs as many)
-    return ((RND & kRndBdr) != 0 || FAM == kFamGdnPw) ? 384 / C::NT : C::MINB;
+    return ((RND & kRndBdr) != 0 || is_pw_family(FAM)) ? 384 / C::NT : C::MINB;
 }
 
 template <int FAM, int DK, int UB, bool F32STATE, int RND>

@@ -43,7 +43,10 @@ rsq_status cuda_fail(int err, const char* what) {
 
 constexpr int kCopyScaleBit = 4;  // kernel rule bit of the copy scale (beside the rsq_rounding bits)
 // Kernel family of a configuration (Gated DeltaNet with a window has its own kernels).
-int kernel_family(const rsq_config& c) { return (c.family == RSQ_GDN && c.window > 0) ? rsq::kFamGdnPw : c.family; }
+int kernel_family(const rsq_config& c) {
+    if (c.family != RSQ_GDN || c.window <= 0) return c.family;
+    return rsq::kFamGdnPw + (c.window == 4 ? 0 : (c.window == 8 ? 1 : 2));
+}
 bool family_ok(int f) { return f == RSQ_GDN || f == RSQ_MAMBA2 || f == RSQ_GLA || f == RSQ_KDA; }
 bool rounding_ok(int r) { return r == RSQ_RTN || r == RSQ_SR || r == RSQ_BDR || r == RSQ_SR_BDR; }
 bool dk_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }

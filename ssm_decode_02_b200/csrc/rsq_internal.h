@@ -8,10 +8,12 @@
 
 namespace rsq {
 
-// Internal family value of Gated DeltaNet with a pure-write window (the public
-// family is RSQ_GDN with rsq_config.window > 0).
-constexpr int kFamGdnPw = 4;
+// Internal family values of Gated DeltaNet with a pure-write window of 4, 8
+// or 16 slots (the public family is RSQ_GDN with rsq_config.window > 0).
+constexpr int kFamGdnPw = 4;  // + log2(W / 4)
 constexpr int kMaxWindow = 16;
+constexpr bool is_pw_family(int fam) { return fam >= kFamGdnPw && fam < kFamGdnPw + 3; }
+constexpr int pw_window(int fam) { return is_pw_family(fam) ? 4 << (fam - kFamGdnPw) : 0; }
 
 constexpr unsigned kFlagNonFinite = 1u;  // a column's absmax was inf or NaN
 constexpr unsigned kFlagTimeout = 2u;    // a bounded barrier wait ran out
