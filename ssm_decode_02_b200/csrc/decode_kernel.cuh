@@ -10,14 +10,22 @@
 //   1. decodes the codes to exact floats (packed pairs),
 //   2. (Gated DeltaNet) forms u = S^T k as s_j * sum_i c_ij k_i,
 //   3. updates the state in registers (full precision, packed f32x2),
-//   4. reads out o = S^T q (GDN) or y = S^T C + D x (Mamba-2) from that state,
-//   5. takes each column's absmax as its new scale (the dynamic "noisy" scale),
-//   6. requantizes (round-to-nearest or Philox stochastic rounding) and stores.
+//   4. reads out o = S^T q (GDN, GLA, KDA) or y = S^T C + D x (Mamba-2) from
+//      that state,
+//   5. takes each column's absmax as its new scale (the dynamic "noisy" scale;
+//      or the column maxima of an unquantized copy: the copy scale),
+//   6. requantizes (round-to-nearest or Philox stochastic rounding, optionally
+//      with Bounded Directional Rounding) and stores.
+// Template parameters: the family (GDN, Mamba-2, GLA, KDA, or GDN with a 4-,
+// 8- or 16-slot pure-write window), dk, the blocks per unit, a full-precision
+// state, and the rule bits (stochastic, BDR, copy scale).
 // Method: LoReS ("Quantizing Recurrent Language Models Is Easier Than You
 // Think", sections "LoReS: State Quantization", "(1/4) Scale grouping", "(3/4)
-// Rounding"); recurrences as named in "Preserving Updates in Low-Bit Recurrent
-// State Quantization" (abstract).  No tensor cores: per head this is two
-// matrix-vector products over a state read once from HBM.
+// Rounding", "(4/4) Rotations"); recurrences and BDR as named in "Preserving
+// Updates in Low-Bit Recurrent State Quantization" (abstract); the pure-write
+// window of "Low-Bit GDN Recurrent-State Quantization: Global Gradient-aware
+// Allocation and Pure-Write Sliding Windows" (abstract).  No tensor cores: per
+// head this is two matrix-vector products over a state read once from HBM.
 #pragma once
 
 #include <cuda_runtime.h>

@@ -45,26 +45,6 @@ __device__ __forceinline__ float4 unpk4(uint64_t a, uint64_t b) {
     return r;
 }
 
-// Butterfly over the 8 row groups (lanes 4, 8, 16 apart) in the order d = 1, 2, 4.
-__device__ __forceinline__ void warp_sum4(float4& v) {
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        v.x = __fadd_rn(v.x, __shfl_xor_sync(0xffffffffu, v.x, off));
-        v.y = __fadd_rn(v.y, __shfl_xor_sync(0xffffffffu, v.y, off));
-        v.z = __fadd_rn(v.z, __shfl_xor_sync(0xffffffffu, v.z, off));
-        v.w = __fadd_rn(v.w, __shfl_xor_sync(0xffffffffu, v.w, off));
-    }
-}
-__device__ __forceinline__ void warp_max4(float4& m) {
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        m.x = max_nan(m.x, __shfl_xor_sync(0xffffffffu, m.x, off));
-        m.y = max_nan(m.y, __shfl_xor_sync(0xffffffffu, m.y, off));
-        m.z = max_nan(m.z, __shfl_xor_sync(0xffffffffu, m.z, off));
-        m.w = max_nan(m.w, __shfl_xor_sync(0xffffffffu, m.w, off));
-    }
-}
-
 // Reduce-scatter over the 8 row groups of a column group.  Afterwards lane
 // (cw, g) holds the total of column 4cw + col_of(g), col_of(g) = 2*(g&1) +
 // ((g>>1)&1); lanes g and g^4 hold the same column.  Every addition pairs the
@@ -102,10 +82,6 @@ __device__ __forceinline__ float4 gather_cols(float mine, int cw, int base) {
     r.z = __shfl_sync(0xffffffffu, mine, base + cw + 4);
     r.w = __shfl_sync(0xffffffffu, mine, base + cw + 12);
     return r;
-}
-
-__device__ __forceinline__ float pick4(const float4& v, int j) {
-    return j == 0 ? v.x : (j == 1 ? v.y : (j == 2 ? v.z : v.w));
 }
 
 // Column finalisation after the reduce-scatter (m = absmax of this lane's
