@@ -77,6 +77,11 @@ def lib():
                                            P, P, P, P, P, P, ctypes.c_float, ctypes.c_float, P, P, P,
                                            P, P, P, P, P]
         L.orc_gdn_pw_head_step.restype = ctypes.c_int
+        L.orc_gdn_ka_head_step.argtypes = [ctypes.POINTER(_Head), P, P, P, P, P, ctypes.c_float,
+                                           ctypes.c_float, P, P, P]
+        L.orc_gdn_ka_head_step.restype = ctypes.c_int
+        L.orc_quantize_ka_head.argtypes = [ctypes.POINTER(_Head), P, P, P]
+        L.orc_quantize_ka_head.restype = ctypes.c_int
         L.orc_allocate_bits.argtypes = [P, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                         ctypes.c_int, P]
         _lib = L
@@ -297,6 +302,56 @@ def kda_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, ste
              mode: int = CANONICAL, R: int = 8, heads=None, copy_absmax=None):
     """One KDA decode step (delta rule with a decay vector alpha [B][H][dk] and gate beta [B][H])."""
     return _diag_step(1, state, inp, head_bits, rounding, seed, step, mode, R, heads, copy_absmax)
+
+
+def zero_state_ka(B: int, H: int, dk: int, dv: int) -> dict:
+    """S_0 = 0 with key-axis scales: codes [B][H][dk][dv], scales [B][H][dk]."""
+    return {"codes": np.zeros((B, H, dk, dv), np.int8), "scales": np.zeros((B, H, dk), np.float32)}
+
+
+def gdn_ka_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, step: int,
+                mode: int = CANONICAL, R: int = 8, heads=None):
+    """One Gated DeltaNet decode step with key-axis scales (one per row i)."""
+    B, H, dk, dv = state["codes"].shape
+    q, k, v = widen(inp["q"]), widen(inp["k"]), widen(inp["v"])
+    alpha, beta = _c(inp["alpha"], np.float32), _c(inp["beta"], np.float32)
+    new = {"codes": state["codes"].copy(), "scales": state["scales"].copy()}
+    o = np.zeros((B, H, dv), np.float32)
+    L = lib()
+    for b, h in _heads(B, H, heads):
+        hd = _head(dk, dv, int(head_bits[h]), rounding, mode, R, seed, b, h, step)
+        c_in, s_in = _c(state["codes"][b, h], np.int8), _c(state["scales"][b, h], np.float32)
+        c_out = np.zeros((dk, dv), np.int8)
+        s_out = np.zeros(dk, np.float32)
+        o_h = np.zeros(dv, np.float32)
+        qh, kh, vh = _c(q[b, h], np.float32), _c(k[b, h], np.float32), _c(v[b, h], np.float32)
+        assert L.orc_gdn_ka_head_step(ctypes.byref(hd), _p(c_in), _p(s_in), _p(qh), _p(kh), _p(vh),
+                                      float(alpha[b, h]), float(beta[b, h]), _p(c_out), _p(s_out),
+                                      _p(o_h)) == 0
+        new["codes"][b, h], new["scales"][b, h], o[b, h] = c_out, s_out, o_h
+    return new, o
+
+
+def quantize_ka(S: np.ndarray, head_bits, *, rounding: int, seed: int, step: int,
+                mode: int = CANONICAL) -> dict:
+    """Quantize a full-precision state [B][H][dk][dv] with key-axis scales."""
+    B, H, dk, dv = S.shape
+    st = zero_state_ka(B, H, dk, dv)
+    L = lib()
+    for b in range(B):
+        for h in range(H):
+            hd = _head(dk, dv, int(head_bits[h]), rounding, mode, 1, seed, b, h, step)
+            c_out = np.zeros((dk, dv), np.int8)
+            s_out = np.zeros(dk, np.float32)
+            assert L.orc_quantize_ka_head(ctypes.byref(hd), _p(_c(S[b, h], np.float32)), _p(c_out),
+                                          _p(s_out)) == 0
+            st["codes"][b, h], st["scales"][b, h] = c_out, s_out
+    return st
+
+
+def dequantize_ka(st: dict) -> np.ndarray:
+    """Key-axis state -> float32 [B][H][dk][dv]: c_ij * s_i (binary32 products)."""
+    return (st["codes"].astype(np.float32) * st["scales"][..., :, None]).astype(np.float32)
 
 
 def e4m3_encode(x: float) -> int:

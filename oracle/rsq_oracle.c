@@ -494,6 +494,89 @@ int orc_diag_head_step(const orc_head* hd, int delta, const int8_t* c_in, const 
 }
 
 /* ------------------------------------------------------------------------- */
+/* Key-axis scale groups ([LoReS] (1/4) Scale grouping: the alternative to the */
+/* value-axis groups; one scale per key row i, s_i = max_j |S_ij| / r).       */
+/* ------------------------------------------------------------------------- */
+/* Quantize row i of S (dk x dv) with its own maximum; same rounding rules as
+ * a column.  Non-finite rows keep their scale and get codes 0.             */
+static void orc_quantize_row(const float* S, int dk, int dv, int i, int bits, int rounding,
+                             int mode, uint64_t seed, uint32_t b, uint32_t h, uint32_t step,
+                             int8_t* codes, float* scale_out)
+{
+    const float rf = (float)orc_rmax(bits);
+    float m = 0.0f;
+    for (int j = 0; j < dv; ++j) {
+        const float a = fabsf(S[(int64_t)i * dv + j]);
+        if (isnan(a) || isnan(m)) m = NAN;
+        else if (a > m) m = a;
+    }
+    *scale_out = m / rf;
+    const int usable = (m > 0.0f) && isfinite(m);
+    for (int j = 0; j < dv; ++j) {
+        int c = 0;
+        if (usable) {
+            const uint32_t u = ORC_SR_BASE(rounding) ? orc_sr_uniform16(seed, b, h, step, dk, i, j) : 0u;
+            c = orc_quantize_scalar(S[(int64_t)i * dv + j], m, bits, rounding, mode, u);
+        }
+        codes[(int64_t)i * dv + j] = (int8_t)c;
+    }
+}
+
+/* Gated DeltaNet decode step with key-axis scales s_in[dk] (everything else as
+ * orc_gdn_head_step).  Canonical c-form with a per-row scale:
+ *   u_j = sum_i c_ij (s_i k_i),  w_j = beta * fma(-alpha, u_j, v_j),
+ *   S_ij = fma(c_ij, alpha s_i, k_i w_j),  o_j = sum_i S_ij q_i,
+ * then each row is requantized with its own maximum.                       */
+int orc_gdn_ka_head_step(const orc_head* hd, const int8_t* c_in, const float* s_in,
+                         const float* q, const float* k, const float* v, float alpha, float beta,
+                         int8_t* c_out, float* s_out, float* o)
+{
+    const int dk = hd->dk, dv = hd->dv;
+    const int R = (hd->mode == ORC_PLAIN) ? 1 : hd->R;
+    const size_t n = (size_t)dk * (size_t)dv;
+    float* S = (float*)malloc(sizeof(float) * n);
+    float* cf = (float*)malloc(sizeof(float) * n);
+    float* ks = (float*)malloc(sizeof(float) * (size_t)dk);
+    if (!S || !cf || !ks) { free(S); free(cf); free(ks); return 1; }
+    if (hd->mode == ORC_PLAIN) {
+        for (int i = 0; i < dk; ++i)
+            for (int j = 0; j < dv; ++j)
+                cf[(int64_t)i * dv + j] = (float)c_in[(int64_t)i * dv + j] * s_in[i];  /* S^ */
+        for (int j = 0; j < dv; ++j) {
+            const float u = orc_dot_rows(cf + j, dv, k, dk, 1);
+            const float w = beta * fmaf(-alpha, u, v[j]);
+            for (int i = 0; i < dk; ++i)
+                S[(int64_t)i * dv + j] = fmaf(alpha, cf[(int64_t)i * dv + j], k[i] * w);
+        }
+    } else {
+        for (size_t t = 0; t < n; ++t) cf[t] = (float)c_in[t];
+        for (int i = 0; i < dk; ++i) ks[i] = s_in[i] * k[i];
+        for (int j = 0; j < dv; ++j) {
+            const float u = orc_dot_rows(cf + j, dv, ks, dk, R);
+            const float w = beta * fmaf(-alpha, u, v[j]);
+            for (int i = 0; i < dk; ++i)
+                S[(int64_t)i * dv + j] = fmaf(cf[(int64_t)i * dv + j], alpha * s_in[i], k[i] * w);
+        }
+    }
+    for (int j = 0; j < dv; ++j) o[j] = orc_dot_rows(S + j, dv, q, dk, R);
+    for (int i = 0; i < dk; ++i)
+        orc_quantize_row(S, dk, dv, i, hd->bits, hd->rounding & 1, hd->mode, hd->seed, hd->b, hd->h,
+                         hd->step, c_out, &s_out[i]);
+    free(S); free(cf); free(ks);
+    return 0;
+}
+
+/* Quantize a full-precision head with key-axis scales. */
+int orc_quantize_ka_head(const orc_head* hd, const float* S, int8_t* c_out, float* s_out)
+{
+    if (hd->bits != 4 && hd->bits != 8) return 1;
+    for (int i = 0; i < hd->dk; ++i)
+        orc_quantize_row(S, hd->dk, hd->dv, i, hd->bits, hd->rounding & 1, hd->mode, hd->seed, hd->b,
+                         hd->h, hd->step, c_out, &s_out[i]);
+    return 0;
+}
+
+/* ------------------------------------------------------------------------- */
 /* FP8 E4M3 [OCP8]: round to nearest even, saturating to +-448.              */
 /* ------------------------------------------------------------------------- */
 uint8_t orc_e4m3_encode(float x)

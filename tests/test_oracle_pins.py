@@ -795,3 +795,76 @@ def test_pure_write_window_fp8_error_is_bounded():
     full = oracle.window_full_state(st, win, hb)
     for h in range(w.H):
         assert _rel(full[0, h], _gdn_closed_form(ins, T, 0, h)) <= 0.08
+
+
+# ---------------------------------------------------------------------------
+# Key-axis scale groups (LoReS (1/4) Scale grouping: the alternative grouping,
+# one scale per key row)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("bits", [8, 4])
+def test_key_axis_quantizer_is_the_value_axis_quantizer_transposed(bits):
+    """Rows of S grouped by key are the columns of S^T: nearest rounding of S with
+    key-axis scales equals the (pinned) value-axis quantizer applied to S^T."""
+    rng = np.random.default_rng(bits + 1)
+    S = rng.standard_normal((2, 3, 32, 48)).astype(np.float32)
+    hb = np.full(3, bits, np.int8)
+    ka = oracle.quantize_ka(S, hb, rounding=oracle.RTN, seed=0, step=0)
+    va = oracle.quantize(np.ascontiguousarray(S.transpose(0, 1, 3, 2)), hb, rounding=oracle.RTN, seed=0,
+                         step=0)
+    assert np.array_equal(ka["codes"], va["codes"].transpose(0, 1, 3, 2))
+    assert np.array_equal(ka["scales"], va["scales"])
+
+
+@pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
+def test_key_axis_first_step_rank_one_codes(mode):
+    """From S_0 = 0, S_1 = beta k v^T: every row's codes are round(r * v_j *
+    sign(k_i) / max|v|) and its scale beta |k_i| max|v| / r."""
+    w = TINY
+    inp = W.gdn_inputs(w, 0)
+    hb = np.full(w.H, 8, np.int8)
+    st1, o = oracle.gdn_ka_step(oracle.zero_state_ka(w.B, w.H, w.dk, w.dv), inp, hb, rounding=oracle.RTN,
+                                seed=0, step=0, mode=mode)
+    for h in range(w.H):
+        k = inp["k"][0, h].astype(np.float64)
+        v = inp["v"][0, h].astype(np.float64)
+        beta = float(inp["beta"][0, h])
+        expect = 127 * np.outer(np.sign(k), v) / np.abs(v).max()
+        assert np.all(np.abs(st1["codes"][0, h] - expect) <= 0.5 + 1e-4)
+        assert np.allclose(st1["scales"][0, h], beta * np.abs(k) * np.abs(v).max() / 127, rtol=1e-5)
+        assert np.allclose(o[0, h], beta * float(k @ inp["q"][0, h]) * v, rtol=1e-5, atol=1e-6)
+
+
+def test_key_axis_readout_error_variance():
+    """With key-axis groups the readout error of column j mixes the row scales:
+    E[e_j^2] = sum_i q_i^2 s_i^2 / 12 under uniform rounding error (within 10%) --
+    the quantity the value-axis proposition of (1/4) compares against."""
+    rng = np.random.default_rng(43)
+    ratios = []
+    for rep in range(40):
+        S = rng.standard_normal((1, 1, 64, 64)).astype(np.float32)
+        st = oracle.quantize_ka(S, np.array([8], np.int8), rounding=oracle.RTN, seed=0, step=0)
+        E = (oracle.dequantize_ka(st) - S)[0, 0].astype(np.float64)
+        q = rng.standard_normal((64, 64))
+        q /= np.linalg.norm(q, axis=0, keepdims=True)
+        e = E.T @ q                                          # e[j, n] = sum_i E_ij q_in
+        s = st["scales"][0, 0].astype(np.float64)
+        pred = (q ** 2 * (s ** 2)[:, None]).sum(axis=0) / 12  # per query n
+        ratios.append(np.mean(e ** 2, axis=0) / pred)
+    assert abs(np.mean(ratios) - 1.0) <= 0.10
+
+
+def test_key_axis_step_plain_and_canonical_agree():
+    """The literal and the canonical evaluation order of the key-axis step differ
+    only by rounding: codes within one step, readouts within 1e-5 relative."""
+    w = dataclasses.replace(TINY, B=2, H=2)
+    hb = np.full(w.H, 8, np.int8)
+    rng = np.random.default_rng(9)
+    st = oracle.quantize_ka((rng.standard_normal((2, 2, 16, 16)) * 0.3).astype(np.float32), hb,
+                            rounding=oracle.RTN, seed=0, step=0)
+    for t in range(8):
+        inp = W.gdn_inputs(w, t)
+        a, oa = oracle.gdn_ka_step(st, inp, hb, rounding=oracle.SR, seed=3, step=t, mode=oracle.CANONICAL)
+        b, ob = oracle.gdn_ka_step(st, inp, hb, rounding=oracle.SR, seed=3, step=t, mode=oracle.PLAIN)
+        assert np.abs(a["codes"].astype(int) - b["codes"].astype(int)).max() <= 1
+        assert _rel(oa, ob) <= 1e-5
+        st = a
