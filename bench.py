@@ -313,7 +313,8 @@ def run_ours(args, w: W.Workload):
     ctx = rsq.Context(fam, w.B, w.H, w.dk, w.dv, head_bits=bits,
                       rounding=ROUNDING[w.rounding],
                       in_dtype=rsq.RSQ_BF16 if w.in_dtype == "bf16" else rsq.RSQ_F32,
-                      seed=w.sr_seed + 7919 * rank, ngroups=w.ngroups, window=args.window)
+                      seed=w.sr_seed + 7919 * rank, ngroups=w.ngroups, window=args.window,
+                      key_axis=int(args.key_axis))
     state_bytes = ctx.code_bytes + ctx.scale_bytes
     layers = max(2, -(-3 * l2 // state_bytes))
     if args.layers:
@@ -504,7 +505,7 @@ def run_ours(args, w: W.Workload):
         "data": "synthetic",
         "config": {"workload": w.name, "global_batch": w.B * world, "heads": w.H, "dk": w.dk,
                    "dv": w.dv, "state": w.state, "rounding": w.rounding, "inputs": w.in_dtype,
-                   "window": args.window,
+                   "window": args.window, "scale_groups": "key-axis" if args.key_axis else "value-axis",
                    "parallelism": "dp%d" % world, "layers_rotated": layers,
                    "l2": "inputs larger than L2: %d layer states + %d input sets = %.0f MB per "
                          "rotation (L2 %.0f MB)" % (layers, n_sets,
@@ -553,14 +554,17 @@ def run_ours(args, w: W.Workload):
 # ---------------------------------------------------------------------------
 # (label, bits, rounding, variant): "noisy" = the quantized state's own column
 # maxima as scales, "copy" = the column maxima of the FP32 trajectory, "wN" = a
-# pure-write window of N FP8 slots beside the low-bit history (GDN)
+# pure-write window of N FP8 slots beside the low-bit history (GDN),
+# "keyaxis" = one scale per key row instead of per value column (GDN)
 DRIFT_VARIANTS = (("int4_sr", 4, "sr", "noisy"), ("int4_rtn", 4, "rtn", "noisy"),
                   ("int4_bdr", 4, "bdr", "noisy"), ("int4_sr_bdr", 4, "sr_bdr", "noisy"),
                   ("int4_sr_copy", 4, "sr", "copy"), ("int4_rtn_copy", 4, "rtn", "copy"),
                   ("int4_sr_w8", 4, "sr", "w8"), ("int4_rtn_w8", 4, "rtn", "w8"),
                   ("int8_sr", 8, "sr", "noisy"), ("int8_rtn", 8, "rtn", "noisy"),
                   ("int8_bdr", 8, "bdr", "noisy"), ("int8_sr_copy", 8, "sr", "copy"),
-                  ("int8_sr_w8", 8, "sr", "w8"))
+                  ("int8_sr_w8", 8, "sr", "w8"),
+                  ("int4_sr_keyaxis", 4, "sr", "keyaxis"), ("int4_rtn_keyaxis", 4, "rtn", "keyaxis"),
+                  ("int8_sr_keyaxis", 8, "sr", "keyaxis"))
 ROUNDING = {"rtn": 0, "sr": 1, "bdr": 2, "sr_bdr": 3}   # rsq_rounding values
 
 
@@ -587,10 +591,11 @@ def drift_series(w: W.Workload, steps: int, every: int, B: int | None = None, va
     fam = FAMILY[w.family]
     in_dtype = rsq.RSQ_BF16 if w.in_dtype == "bf16" else rsq.RSQ_F32
 
-    def make(bits, rounding, window=0):
+    def make(bits, rounding, window=0, key_axis=0):
         ctx = rsq.Context(fam, B, w.H, w.dk, w.dv, head_bits=np.full(w.H, bits, np.int8),
                           rounding=ROUNDING[rounding],
-                          in_dtype=in_dtype, seed=w.sr_seed, ngroups=w.ngroups, window=window)
+                          in_dtype=in_dtype, seed=w.sr_seed, ngroups=w.ngroups, window=window,
+                          key_axis=key_axis)
         st = ctx.alloc_state(device)
         ctx.quantize(torch.zeros((B, w.H, w.dk, w.dv), dtype=torch.float32, device=device), st)
         out = torch.empty((B, w.H, w.dv), dtype=torch.float32, device=device)
@@ -600,7 +605,7 @@ def drift_series(w: W.Workload, steps: int, every: int, B: int | None = None, va
         return int(src[1:]) if src.startswith("w") else 0
 
     ref = make(32, "rtn")
-    runs = {label: make(bits, rnd, window_of(src)) for label, bits, rnd, src in variants}
+    runs = {label: make(bits, rnd, window_of(src), int(src == "keyaxis")) for label, bits, rnd, src in variants}
     source = {label: src for label, _, _, src in variants}
     wins = {label: [runs[label][0].alloc_window(device), runs[label][0].alloc_window(device)]
             for label, _, _, src in variants if window_of(src)}
@@ -624,8 +629,9 @@ def drift_series(w: W.Workload, steps: int, every: int, B: int | None = None, va
         if (t + 1) % every == 0:
             o_ref = ref[2].double()
             for label, (ctx, st, out) in runs.items():
-                if label in wins:
-                    num, den = _window_drift_sums(rsq, ctx, st, wins[label][(t + 1) % 2], ref, B, w, device)
+                if label in wins or source[label] == "keyaxis":
+                    num, den = _full_drift_sums(ctx, st, wins[label][(t + 1) % 2] if label in wins else None,
+                                                ref, B, w, device)
                 else:
                     rsq.rsq_state_drift(ctx.ctx, st, ref[0].ctx, ref[1], sums)
                     s = sums.cpu().numpy()
@@ -642,19 +648,22 @@ def drift_series(w: W.Workload, steps: int, every: int, B: int | None = None, va
     return series
 
 
-def _window_drift_sums(rsq, ctx, st, win, ref, B, w, device):
-    """Per-head sums of (full state - FP32 state)^2 and FP32 state^2 for a state
-    with a pure-write window: full state = dequantized history + sum_w a_w b_w^T."""
+def _full_drift_sums(ctx, st, win, ref, B, w, device):
+    """Per-head sums of (state - FP32 state)^2 and FP32 state^2 through the
+    library's dequantization (any scale grouping); with a pure-write window the
+    state is the dequantized history + sum_w a_w b_w^T."""
     import torch
     Hq = torch.empty((B, w.H, w.dk, w.dv), dtype=torch.float32, device=device)
     F = torch.empty_like(Hq)
     ctx.dequantize(st, Hq)
     ref[0].dequantize(ref[1], F)
-    Wn = ctx.window
-    dec = lambda codes: codes.view(torch.float8_e4m3fn).to(torch.float32)
-    a = dec(win.a) * win.a_scale[..., None]                                   # [B][H][W][dk]
-    b = dec(win.b).permute(0, 1, 3, 2, 4).reshape(B, w.H, Wn, w.dv) * win.b_scale[..., None]
-    full = Hq.double() + torch.einsum("bhwi,bhwj->bhij", a.double(), b.double())
+    full = Hq.double()
+    if win is not None:
+        Wn = ctx.window
+        dec = lambda codes: codes.view(torch.float8_e4m3fn).to(torch.float32)
+        a = dec(win.a) * win.a_scale[..., None]                                   # [B][H][W][dk]
+        b = dec(win.b).permute(0, 1, 3, 2, 4).reshape(B, w.H, Wn, w.dv) * win.b_scale[..., None]
+        full = full + torch.einsum("bhwi,bhwj->bhij", a.double(), b.double())
     F = F.double()
     num = ((full - F) ** 2).sum(dim=(2, 3)).cpu().numpy()
     den = (F ** 2).sum(dim=(2, 3)).cpu().numpy()
@@ -754,6 +763,8 @@ def main():
                     help="override the workload's requantization rule")
     ap.add_argument("--window", type=int, default=0,
                     help="pure-write window slots (Gated DeltaNet): 0, 4, 8 or 16")
+    ap.add_argument("--key-axis", action="store_true",
+                    help="one scale per key row instead of per value column (Gated DeltaNet)")
     ap.add_argument("--drift", action="store_true",
                     help="run the long-horizon state drift study instead of the throughput bench")
     ap.add_argument("--drift-steps", type=int, default=0, help="horizon (default: the workload's)")

@@ -124,6 +124,10 @@ typedef struct {
     uint64_t seed;   /* stochastic-rounding key */
     int window;      /* pure-write window slots W for Gated DeltaNet ([PW]): 0 (none), 4, 8
                         or 16; needs RSQ_RTN or RSQ_SR and rsq_decode_step_window */
+    int key_axis;    /* 0: one scale per value column (the method's grouping); 1: one scale
+                        per key row, s_i = max_j |S_ij| / r ([LoReS] (1/4), the grouping
+                        ablation).  Key-axis: Gated DeltaNet, 4/8-bit heads, RSQ_RTN or
+                        RSQ_SR; scales are [B][H][dk]; one CTA per head. */
 } rsq_config;
 
 typedef struct rsq_ctx rsq_ctx;

@@ -306,7 +306,8 @@ def kda_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, ste
 
 def zero_state_ka(B: int, H: int, dk: int, dv: int) -> dict:
     """S_0 = 0 with key-axis scales: codes [B][H][dk][dv], scales [B][H][dk]."""
-    return {"codes": np.zeros((B, H, dk, dv), np.int8), "scales": np.zeros((B, H, dk), np.float32)}
+    return {"codes": np.zeros((B, H, dk, dv), np.int8), "scales": np.zeros((B, H, dk), np.float32),
+            "f": None}
 
 
 def gdn_ka_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, step: int,
@@ -315,7 +316,7 @@ def gdn_ka_step(state: dict, inp: dict, head_bits, *, rounding: int, seed: int, 
     B, H, dk, dv = state["codes"].shape
     q, k, v = widen(inp["q"]), widen(inp["k"]), widen(inp["v"])
     alpha, beta = _c(inp["alpha"], np.float32), _c(inp["beta"], np.float32)
-    new = {"codes": state["codes"].copy(), "scales": state["scales"].copy()}
+    new = {"codes": state["codes"].copy(), "scales": state["scales"].copy(), "f": None}
     o = np.zeros((B, H, dv), np.float32)
     L = lib()
     for b, h in _heads(B, H, heads):

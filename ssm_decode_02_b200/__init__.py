@@ -36,7 +36,8 @@ class rsq_config(ctypes.Structure):
     _fields_ = [("family", ctypes.c_int), ("batch", ctypes.c_int), ("heads", ctypes.c_int),
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("ngroups", ctypes.c_int),
                 ("head_bits", ctypes.POINTER(ctypes.c_int8)), ("rounding", ctypes.c_int),
-                ("in_dtype", ctypes.c_int), ("seed", ctypes.c_uint64), ("window", ctypes.c_int)]
+                ("in_dtype", ctypes.c_int), ("seed", ctypes.c_uint64), ("window", ctypes.c_int),
+                ("key_axis", ctypes.c_int)]
 
 
 class rsq_state(ctypes.Structure):
@@ -150,21 +151,23 @@ def _stream(stream) -> int | None:
 # ---------------------------------------------------------------------------
 def rsq_create(family: int, batch: int, heads: int, dk: int, dv: int, *, head_bits=None,
                rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0,
-               ngroups: int = 1, window: int = 0) -> int:
+               ngroups: int = 1, window: int = 0, key_axis: int = 0) -> int:
     cfg, bits_arr = _config(family, batch, heads, dk, dv, head_bits, rounding, in_dtype, seed, ngroups,
-                            window)
+                            window, key_axis)
     out = ctypes.c_void_p()
     _check(lib.rsq_create(ctypes.byref(cfg), ctypes.byref(out)))
     return int(out.value)
 
 
-def _config(family, batch, heads, dk, dv, head_bits, rounding, in_dtype, seed, ngroups, window=0):
+def _config(family, batch, heads, dk, dv, head_bits, rounding, in_dtype, seed, ngroups, window=0,
+            key_axis=0):
     bits_arr = None
     if head_bits is not None:
         bits_arr = (ctypes.c_int8 * heads)(*[int(b) for b in head_bits])
     cfg = rsq_config(int(family), int(batch), int(heads), int(dk), int(dv), int(ngroups),
                      ctypes.cast(bits_arr, ctypes.POINTER(ctypes.c_int8)) if bits_arr else None,
-                     int(rounding), int(in_dtype), int(seed) & (2 ** 64 - 1), int(window))
+                     int(rounding), int(in_dtype), int(seed) & (2 ** 64 - 1), int(window),
+                     int(key_axis))
     return cfg, bits_arr
 
 
@@ -323,13 +326,14 @@ class Context:
 
     def __init__(self, family: int, batch: int, heads: int, dk: int, dv: int, *, head_bits=None,
                  rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0, ngroups: int = 1,
-                 window: int = 0):
+                 window: int = 0, key_axis: int = 0):
         self.family, self.batch, self.heads, self.dk, self.dv = family, batch, heads, dk, dv
         self.head_bits = None if head_bits is None else np.asarray(head_bits, np.int8)
         self.rounding, self.in_dtype, self.seed, self.ngroups = rounding, in_dtype, seed, ngroups
-        self.window = window
+        self.window, self.key_axis = window, key_axis
         self.ctx = rsq_create(family, batch, heads, dk, dv, head_bits=head_bits, rounding=rounding,
-                              in_dtype=in_dtype, seed=seed, ngroups=ngroups, window=window)
+                              in_dtype=in_dtype, seed=seed, ngroups=ngroups, window=window,
+                              key_axis=key_axis)
         self.code_bytes, self.scale_bytes = rsq_state_bytes(self.ctx)
 
     def close(self):
@@ -346,7 +350,8 @@ class Context:
     def alloc_state(self, device="cuda") -> State:
         import torch
         codes = torch.empty((self.batch, self.code_bytes // self.batch), dtype=torch.uint8, device=device)
-        scales = torch.empty((self.batch, self.heads, self.dv), dtype=torch.float32, device=device)
+        scales = torch.empty((self.batch, self.heads, self.dk if self.key_axis else self.dv),
+                             dtype=torch.float32, device=device)
         return State(codes, scales)
 
     def decode_step(self, state_in: State, state_out: State, inputs, out, step: int, stream=None):

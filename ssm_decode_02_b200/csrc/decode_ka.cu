@@ -1,0 +1,356 @@
+// decode_ka.cu -- Gated DeltaNet decode step with key-axis scale groups.
+//
+// The grouping ablation of LoReS ("Quantizing Recurrent Language Models Is
+// Easier Than You Think", section "(1/4) Scale grouping"): one scale per key
+// row, s_i = max_j |S_ij| / r, instead of one per value column.  A row's
+// maximum runs over all d_v columns of the head, so one CTA owns one head:
+// warp w holds the 16-column block w (the same lane tile as the value-axis
+// kernel), the row maxima of the warps meet in shared memory, and two CTA
+// barriers separate the phases.  There are no early exits, so every thread
+// reaches both barriers.
+//
+// Per head, in the canonical order the oracle follows:
+//   u_j = sum_i c_ij (s_i k_i)  (8 partials + XOR butterfly),
+//   w_j = beta * fma(-alpha, u_j, v_j),   S_ij = fma(c_ij, alpha s_i, k_i w_j),
+//   o_j = sum_i S_ij q_i,   m_i = max_j |S_ij|,   s_i = m_i / r,
+//   inv_i = r / m_i rounded toward zero,   codes as in the value-axis kernel.
+#include <cuda_runtime.h>
+
+#include "rsq_internal.h"
+#include "rsq_tile.cuh"
+
+namespace rsq {
+namespace {
+
+template <int DK>
+struct KaCfg {
+    static constexpr int RPT = DK / kR;
+    static constexpr int PST = RPT + 2;          // padded row-group stride of the pair arrays
+    static constexpr int PAIRS = kR * PST;        // uint64 per pair array
+};
+
+__device__ __forceinline__ float ka_vec(const void* base, long long e, bool bf16) {
+    if (bf16) return bf16_bits_to_f32(static_cast<const uint16_t*>(base)[e]);
+    return static_cast<const float*>(base)[e];
+}
+
+// Requantize this lane's rows with one multiplier per row (pairs (inv_i, inv_i)
+// at invp[k] for row g + 8k) and store them; RTN or Philox SR as in the
+// value-axis requantizer.
+template <int BITS, bool SR, int RPT>
+__device__ __forceinline__ void ka_requantize_store(const uint64_t (&S2)[RPT][2], const uint64_t* invp,
+                                                    uint8_t* dst, int g, int cw, uint32_t gcol,
+                                                    uint32_t h, uint32_t b, uint32_t step,
+                                                    const PhiloxKeys& rk) {
+    uint8_t* const row0 = dst + (BITS == 8 ? g * 16 + 4 * cw : g * 8 + 2 * cw);
+    auto store_row = [&](int k, uint32_t word) {
+        if constexpr (BITS == 8)
+            *reinterpret_cast<uint32_t*>(row0 + k * (kR * 16)) = word;
+        else
+            *reinterpret_cast<uint16_t*>(row0 + k * (kR * 8)) = static_cast<uint16_t>(word);
+    };
+    constexpr float kOff = (BITS == 8) ? 128.0f : 8.0f;
+    if constexpr (!SR) {
+        const uint64_t moff = pk(kMagic + kOff, kMagic + kOff);
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            float t0, t1, t2, t3;
+            upk(fma2(S2[k][0], invp[k], moff), t0, t1);
+            upk(fma2(S2[k][1], invp[k], moff), t2, t3);
+            store_row(k, pack_row<BITS>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
+                                        __float_as_uint(t3), false));
+        }
+    } else {
+        constexpr uint32_t vb = (BITS == 8) ? kSrBits8 : kSrBits4;
+        const uint64_t mm = pk(kMagic, kMagic);
+#pragma unroll
+        for (int k = 0; k < RPT / 2; ++k) {
+            const uint32_t i = static_cast<uint32_t>(g + kR * k);  // partner row i + dk/2
+            const U4 rnd = philox4x32_10(U4{i | (gcol << 16), h, b, step}, rk.k0, rk.k1);
+            const uint32_t u[2][2] = {{rnd.x, rnd.y}, {rnd.z, rnd.w}};
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                const int kk = k + half * (RPT / 2);
+                const uint32_t w0 = u[half][0], w1 = u[half][1];
+                const uint64_t V01 = pk(__uint_as_float(vb | (w0 & 0xFFFFu)), __uint_as_float(umulhi_add(w0, 0x10000u, vb)));
+                const uint64_t V23 = pk(__uint_as_float(vb | (w1 & 0xFFFFu)), __uint_as_float(umulhi_add(w1, 0x10000u, vb)));
+                uint64_t t01 = fma2(S2[kk][0], invp[kk], V01);
+                uint64_t t23 = fma2(S2[kk][1], invp[kk], V23);
+                if constexpr (BITS == 8) {
+                    t01 = add2_rm(t01, mm);
+                    t23 = add2_rm(t23, mm);
+                }
+                float t0, t1, t2, t3;
+                upk(t01, t0, t1);
+                upk(t23, t2, t3);
+                store_row(kk, pack_row<BITS>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
+                                             __float_as_uint(t3), BITS == 4));
+            }
+        }
+    }
+}
+
+template <int DK, int BITS, bool SR>
+__device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, int b, int h, int hu) {
+    using K = KaCfg<DK>;
+    constexpr int RPT = K::RPT;
+    constexpr int BLOCK_BYTES = DK * kBlockCols * BITS / 8;
+    constexpr float r = float((1 << (BITS - 1)) - 1);
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nt = blockDim.x, nw = nt >> 5;
+    const int g = lane >> 2, cw = lane & 3;
+    const bool bf16 = p.in_bf16 != 0;
+    uint64_t* pq = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* pkk = pq + K::PAIRS;   // k
+    uint64_t* pks = pkk + K::PAIRS;  // s_i k_i
+    uint64_t* pas = pks + K::PAIRS;  // alpha s_i
+    uint64_t* pin = pas + K::PAIRS;  // inv_i (after the row maxima)
+    float* rowmax = reinterpret_cast<float*>(pin + K::PAIRS);  // [nw][DK]
+    const float alpha = __ldg(p.g0 + hu), beta = __ldg(p.g1 + hu);
+
+    // ---- key-axis vectors and row scales as duplicated pairs (shared by all warps)
+    for (int i = tid; i < DK; i += nt) {
+        const float q = ka_vec(p.vA, (long long)hu * DK + i, bf16);
+        const float k = ka_vec(p.vB, (long long)hu * DK + i, bf16);
+        const float s = __ldg(p.scales_in + (long long)hu * DK + i);
+        const int pos = (i & (kR - 1)) * K::PST + i / kR;
+        const float ks = __fmul_rn(s, k), as = __fmul_rn(alpha, s);
+        pq[pos] = pk(q, q);
+        pkk[pos] = pk(k, k);
+        pks[pos] = pk(ks, ks);
+        pas[pos] = pk(as, as);
+    }
+    __syncthreads();
+
+    // ---- this warp's block: decode, update, read out -------------------------
+    const int j0 = w * kBlockCols;
+    const long long rowoff = (long long)b * p.row_bytes + p.head_off[h] + (long long)w * BLOCK_BYTES;
+    uint64_t S2[RPT][2];
+    load_codes<BITS, RPT>(p.codes_in + rowoff, g, cw, S2);
+    const uint64_t* kq = pq + g * K::PST;
+    const uint64_t* kk = pkk + g * K::PST;
+    const uint64_t* kks = pks + g * K::PST;
+    const uint64_t* kas = pas + g * K::PST;
+    uint64_t a01 = pk(0.f, 0.f), a23 = pk(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < RPT; k += 2) {
+        const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(kks + k);
+        a01 = fma2(S2[k][0], x.x, a01);
+        a23 = fma2(S2[k][1], x.x, a23);
+        a01 = fma2(S2[k + 1][0], x.y, a01);
+        a23 = fma2(S2[k + 1][1], x.y, a23);
+    }
+    const float4 u4 = gather_cols(reduce_scatter4(unpk4(a01, a23), g, AddOp()), cw, 0);
+    const float uv[4] = {u4.x, u4.y, u4.z, u4.w};
+    float wj[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float v = ka_vec(p.vC, (long long)hu * p.dv + j0 + 4 * cw + j, bf16);
+        wj[j] = __fmul_rn(beta, __fmaf_rn(-alpha, uv[j], v));
+    }
+    const uint64_t W01 = pk(wj[0], wj[1]), W23 = pk(wj[2], wj[3]);
+#pragma unroll
+    for (int k = 0; k < RPT; k += 2) {
+        const ulonglong2 ka = *reinterpret_cast<const ulonglong2*>(kas + k);
+        const ulonglong2 kv = *reinterpret_cast<const ulonglong2*>(kk + k);
+        S2[k][0] = fma2(S2[k][0], ka.x, mul2(kv.x, W01));
+        S2[k][1] = fma2(S2[k][1], ka.x, mul2(kv.x, W23));
+        S2[k + 1][0] = fma2(S2[k + 1][0], ka.y, mul2(kv.y, W01));
+        S2[k + 1][1] = fma2(S2[k + 1][1], ka.y, mul2(kv.y, W23));
+    }
+    uint64_t o01 = pk(0.f, 0.f), o23 = pk(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k < RPT; k += 2) {
+        const ulonglong2 x = *reinterpret_cast<const ulonglong2*>(kq + k);
+        o01 = fma2(S2[k][0], x.x, o01);
+        o23 = fma2(S2[k][1], x.x, o23);
+        o01 = fma2(S2[k + 1][0], x.y, o01);
+        o23 = fma2(S2[k + 1][1], x.y, o23);
+    }
+    const float o = reduce_scatter4(unpk4(o01, o23), g, AddOp());
+    if (g < 4) p.out[(long long)hu * p.dv + j0 + 4 * cw + col_of(g)] = o;
+
+    // ---- row maxima: this warp's 16 columns, then across the warps -----------
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+        const float4 x = unpk4(S2[k][0], S2[k][1]);
+        float m = max3_nan(fabsf(x.x), fabsf(x.y), max_nan(fabsf(x.z), fabsf(x.w)));
+        m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        if (cw == 0) rowmax[w * DK + g + kR * k] = m;
+    }
+    __syncthreads();
+    for (int i = tid; i < DK; i += nt) {
+        float m = 0.f;
+        for (int ww = 0; ww < nw; ++ww) m = max_nan(m, rowmax[ww * DK + i]);
+        const float s = __fdiv_rn(m, r);
+        float inv = 0.f;
+        if (!isfinite(m)) {
+            inv = -0.0f;  // marks a non-finite row
+        } else if (m > 0.f) {
+            const float q = __fdiv_rn(r, m);
+            inv = (__fmaf_rn(q, m, -r) > 0.f) ? __uint_as_float(__float_as_uint(q) - 1u) : q;
+        }
+        p.scales_out[(long long)hu * DK + i] = s;
+        pin[(i & (kR - 1)) * K::PST + i / kR] = pk(inv, inv);
+    }
+    __syncthreads();
+
+    // ---- requantize with the row multipliers ----------------------------------
+    const uint64_t* ki = pin + g * K::PST;
+    uint64_t invp[RPT];
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) invp[k] = ki[k];
+    uint8_t* dst = p.codes_out + rowoff;
+    const uint32_t gcol = static_cast<uint32_t>(j0 / 4 + cw);
+    ka_requantize_store<BITS, SR, RPT>(S2, invp, dst, g, cw, gcol, h, b, p.step, p.rk);
+    // rare: non-finite rows (multiplier -0.0) are stored as the zero code
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) bad |= is_neg_zero(__uint_as_float(static_cast<uint32_t>(invp[k])));
+    if (bad) {
+        if (cw == 0 && g == 0) atomicOr(p.flag, kFlagNonFinite);
+#pragma unroll
+        for (int k = 0; k < RPT; ++k)
+            if (is_neg_zero(__uint_as_float(static_cast<uint32_t>(invp[k])))) {
+                S2[k][0] = pk(0.f, 0.f);
+                S2[k][1] = pk(0.f, 0.f);
+            }
+        ka_requantize_store<BITS, SR, RPT>(S2, invp, dst, g, cw, gcol, h, b, p.step, p.rk);
+    }
+}
+
+template <int DK, bool SR>
+__global__ void __launch_bounds__(512) rsq_decode_ka_kernel(const __grid_constant__ DecodeParams p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int hu = blockIdx.x;
+    const int b = hu / p.H, h = hu - b * p.H;
+    if (p.head_bits[h] == 8)
+        ka_head<DK, 8, SR>(p, smem, b, h, hu);
+    else
+        ka_head<DK, 4, SR>(p, smem, b, h, hu);
+}
+
+// Quantize a full-precision head (natural [dk][dv] layout) with key-axis
+// scales: warp w owns block w, row maxima meet in shared memory.
+template <int DK, int BITS, bool SR>
+__device__ __forceinline__ void ka_quantize_head(const QuantParams& p, uint8_t* smem, int b, int h, int hu) {
+    using K = KaCfg<DK>;
+    constexpr int RPT = K::RPT;
+    constexpr int BLOCK_BYTES = DK * kBlockCols * BITS / 8;
+    constexpr float r = float((1 << (BITS - 1)) - 1);
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nt = blockDim.x, nw = nt >> 5;
+    const int g = lane >> 2, cw = lane & 3;
+    uint64_t* pin = reinterpret_cast<uint64_t*>(smem);
+    float* rowmax = reinterpret_cast<float*>(pin + K::PAIRS);
+    const int j0 = w * kBlockCols;
+    const float* src = p.S + (long long)hu * DK * p.dv + j0 + 4 * cw;
+    uint64_t S2[RPT][2];
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+        const ulonglong2 t = __ldg(reinterpret_cast<const ulonglong2*>(src + (long long)(g + kR * k) * p.dv));
+        S2[k][0] = t.x;
+        S2[k][1] = t.y;
+        const float4 x = unpk4(t.x, t.y);
+        float m = max3_nan(fabsf(x.x), fabsf(x.y), max_nan(fabsf(x.z), fabsf(x.w)));
+        m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
+        m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
+        if (cw == 0) rowmax[w * DK + g + kR * k] = m;
+    }
+    __syncthreads();
+    for (int i = tid; i < DK; i += nt) {
+        float m = 0.f;
+        for (int ww = 0; ww < nw; ++ww) m = max_nan(m, rowmax[ww * DK + i]);
+        float inv = 0.f;
+        if (!isfinite(m)) {
+            inv = -0.0f;
+        } else if (m > 0.f) {
+            const float q = __fdiv_rn(r, m);
+            inv = (__fmaf_rn(q, m, -r) > 0.f) ? __uint_as_float(__float_as_uint(q) - 1u) : q;
+        }
+        p.scales[(long long)hu * DK + i] = __fdiv_rn(m, r);
+        pin[(i & (kR - 1)) * K::PST + i / kR] = pk(inv, inv);
+    }
+    __syncthreads();
+    uint64_t invp[RPT];
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+        invp[k] = pin[g * K::PST + k];
+        if (is_neg_zero(__uint_as_float(static_cast<uint32_t>(invp[k])))) {
+            bad = true;
+            S2[k][0] = pk(0.f, 0.f);
+            S2[k][1] = pk(0.f, 0.f);
+        }
+    }
+    if (bad && cw == 0 && g == 0) atomicOr(p.flag, kFlagNonFinite);
+    uint8_t* dst = p.codes + (long long)b * p.row_bytes + p.head_off[h] + (long long)w * BLOCK_BYTES;
+    ka_requantize_store<BITS, SR, RPT>(S2, invp, dst, g, cw, static_cast<uint32_t>(j0 / 4 + cw), h, b, p.step,
+                                       p.rk);
+}
+
+template <int DK>
+__global__ void __launch_bounds__(512) rsq_quantize_ka_kernel(const __grid_constant__ QuantParams p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int hu = blockIdx.x;
+    const int b = hu / p.H, h = hu - b * p.H;
+    const bool bits8 = p.head_bits[h] == 8;
+    if (p.sr) {
+        if (bits8) ka_quantize_head<DK, 8, true>(p, smem, b, h, hu);
+        else ka_quantize_head<DK, 4, true>(p, smem, b, h, hu);
+    } else {
+        if (bits8) ka_quantize_head<DK, 8, false>(p, smem, b, h, hu);
+        else ka_quantize_head<DK, 4, false>(p, smem, b, h, hu);
+    }
+}
+
+template <int DK>
+int launch_quantize_ka_dk(const QuantParams& p, void* stream) {
+    const int nw = p.dv / kBlockCols;
+    const size_t smem = KaCfg<DK>::PAIRS * sizeof(uint64_t) + static_cast<size_t>(nw) * DK * sizeof(float);
+    rsq_quantize_ka_kernel<DK><<<p.B * p.H, 32 * nw, smem, static_cast<cudaStream_t>(stream)>>>(p);
+    return static_cast<int>(cudaGetLastError());
+}
+
+template <int DK>
+size_t ka_smem(int nw) {
+    return 5 * KaCfg<DK>::PAIRS * sizeof(uint64_t) + static_cast<size_t>(nw) * DK * sizeof(float);
+}
+
+template <int DK>
+int launch_ka_dk(const DecodeParams& p, bool sr, void* stream) {
+    const int nw = p.dv / kBlockCols;
+    const size_t smem = ka_smem<DK>(nw);
+    const void* f = sr ? reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, true>)
+                       : reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, false>);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(p.B * p.H);
+    cfg.blockDim = dim3(32 * nw);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    void* args[] = {const_cast<DecodeParams*>(&p)};
+    return static_cast<int>(cudaLaunchKernelExC(&cfg, f, args));
+}
+
+}  // namespace
+
+int launch_quantize_ka(int dk, const QuantParams& p, void* stream) {
+    switch (dk) {
+        case 16: return launch_quantize_ka_dk<16>(p, stream);
+        case 32: return launch_quantize_ka_dk<32>(p, stream);
+        case 64: return launch_quantize_ka_dk<64>(p, stream);
+        case 128: return launch_quantize_ka_dk<128>(p, stream);
+        default: return static_cast<int>(cudaErrorInvalidValue);
+    }
+}
+
+int launch_decode_ka(int dk, const DecodeParams& p, bool sr, void* stream) {
+    switch (dk) {
+        case 16: return launch_ka_dk<16>(p, sr, stream);
+        case 32: return launch_ka_dk<32>(p, sr, stream);
+        case 64: return launch_ka_dk<64>(p, sr, stream);
+        case 128: return launch_ka_dk<128>(p, sr, stream);
+        default: return static_cast<int>(cudaErrorInvalidValue);
+    }
+}
+
+}  // namespace rsq

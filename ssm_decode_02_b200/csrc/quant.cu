@@ -109,12 +109,23 @@ __device__ __forceinline__ void dequantize_block(const DequantParams& p, const B
         }
     } else {
         load_codes<BITS, RPT>(src, g, cw, S2);
-        const float4 s = *reinterpret_cast<const float4*>(p.scales + (long long)bi.hu * p.dv + j0 + 4 * cw);
-        const uint64_t s01 = pk(s.x, s.y), s23 = pk(s.z, s.w);
+        if (p.key_axis) {
+            // one scale per key row
 #pragma unroll
-        for (int k = 0; k < RPT; ++k) {
-            S2[k][0] = mul2(S2[k][0], s01);
-            S2[k][1] = mul2(S2[k][1], s23);
+            for (int k = 0; k < RPT; ++k) {
+                const float si = p.scales[(long long)bi.hu * DK + g + kR * k];
+                const uint64_t ss = pk(si, si);
+                S2[k][0] = mul2(S2[k][0], ss);
+                S2[k][1] = mul2(S2[k][1], ss);
+            }
+        } else {
+            const float4 s = *reinterpret_cast<const float4*>(p.scales + (long long)bi.hu * p.dv + j0 + 4 * cw);
+            const uint64_t s01 = pk(s.x, s.y), s23 = pk(s.z, s.w);
+#pragma unroll
+            for (int k = 0; k < RPT; ++k) {
+                S2[k][0] = mul2(S2[k][0], s01);
+                S2[k][1] = mul2(S2[k][1], s23);
+            }
         }
     }
     if (p.absmax != nullptr) {

@@ -133,6 +133,9 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
         return fail(RSQ_E_UNSUPPORTED, "create: the pure-write window is defined for Gated DeltaNet");
     if (c.window && c.rounding != RSQ_RTN && c.rounding != RSQ_SR)
         return fail(RSQ_E_UNSUPPORTED, "create: the pure-write window takes nearest or stochastic rounding");
+    if (c.key_axis != 0 && c.key_axis != 1) return fail(RSQ_E_INVAL, "create: key_axis must be 0 or 1");
+    if (c.key_axis && (c.family != RSQ_GDN || c.window || (c.rounding != RSQ_RTN && c.rounding != RSQ_SR)))
+        return fail(RSQ_E_UNSUPPORTED, "create: key-axis scales: Gated DeltaNet, no window, nearest or stochastic rounding");
 
     rsq_ctx* ctx = new (std::nothrow) rsq_ctx();
     if (!ctx) return fail(RSQ_E_NOMEM, "create: host allocation failed");
@@ -151,6 +154,10 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
     if (n32 != 0 && n32 != c.heads) {
         delete ctx;
         return fail(RSQ_E_UNSUPPORTED, "create: 32-bit heads cannot be mixed with 4/8-bit heads");
+    }
+    if (n32 && c.key_axis) {
+        delete ctx;
+        return fail(RSQ_E_UNSUPPORTED, "create: key-axis scales need 4/8-bit heads");
     }
     ctx->f32state = (n32 == c.heads);
     long long off = 0;
@@ -214,7 +221,8 @@ void rsq_destroy(rsq_ctx* ctx) {
 rsq_status rsq_state_bytes(const rsq_ctx* ctx, size_t* code_bytes, size_t* scale_bytes) {
     if (!ctx || !code_bytes || !scale_bytes) return fail(RSQ_E_INVAL, "state_bytes: null argument");
     *code_bytes = static_cast<size_t>(ctx->row_bytes) * ctx->cfg.batch;
-    *scale_bytes = static_cast<size_t>(ctx->cfg.batch) * ctx->cfg.heads * ctx->cfg.dv * sizeof(float);
+    *scale_bytes = static_cast<size_t>(ctx->cfg.batch) * ctx->cfg.heads *
+                   (ctx->cfg.key_axis ? ctx->cfg.dk : ctx->cfg.dv) * sizeof(float);
     return RSQ_OK;
 }
 
@@ -288,6 +296,7 @@ rsq_status rsq_column_absmax(const rsq_ctx* ctx, const rsq_state* state, float* 
     p.codes = static_cast<const uint8_t*>(state->codes);
     p.scales = state->scales;
     p.absmax = absmax;
+    p.key_axis = c.key_axis;
     fill_heads(ctx, p);
     const int err = rsq::launch_dequantize(c.dk, p, stream);
     if (err) return cuda_fail(err, "column_absmax launch");
@@ -369,6 +378,12 @@ rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const
     const int ghu = ctx->grid / ctx->ncb;
     p.gh = ghu % c.heads;
     p.gb = ghu / c.heads;
+    if (c.key_axis) {
+        if (copy_absmax) return fail(RSQ_E_UNSUPPORTED, "decode_step_copy_scale: not with key-axis scales");
+        const int e = rsq::launch_decode_ka(c.dk, p, (c.rounding & RSQ_SR) != 0, stream);
+        if (e) return cuda_fail(e, "decode_step launch");
+        return RSQ_OK;
+    }
     const int err = rsq::launch_decode(kernel_family(c), c.dk, ctx->ub, ctx->f32state,
                                        c.rounding | (copy_absmax ? kCopyScaleBit : 0), p,
                                        stream);
@@ -399,7 +414,7 @@ rsq_status rsq_quantize(const rsq_ctx* ctx, const float* S, const rsq_state* sta
     p.key1 = static_cast<uint32_t>(c.seed >> 32);
     p.rk = rsq::philox_round_keys(p.key0, p.key1);
     fill_heads(ctx, p);
-    const int err = rsq::launch_quantize(c.dk, p, stream);
+    const int err = c.key_axis ? rsq::launch_quantize_ka(c.dk, p, stream) : rsq::launch_quantize(c.dk, p, stream);
     if (err) return cuda_fail(err, "quantize launch");
     return RSQ_OK;
 }
@@ -417,6 +432,7 @@ rsq_status rsq_dequantize(const rsq_ctx* ctx, const rsq_state* state_in, float* 
     p.codes = static_cast<const uint8_t*>(state_in->codes);
     p.scales = state_in->scales;
     p.S = S_out;
+    p.key_axis = c.key_axis;
     fill_heads(ctx, p);
     const int err = rsq::launch_dequantize(c.dk, p, stream);
     if (err) return cuda_fail(err, "dequantize launch");
@@ -428,6 +444,8 @@ rsq_status rsq_state_drift(const rsq_ctx* q_ctx, const rsq_state* q_state, const
     if (!q_ctx || !f_ctx || !sums) return fail(RSQ_E_INVAL, "state_drift: null argument");
     if (q_ctx->f32state || !f_ctx->f32state)
         return fail(RSQ_E_INVAL, "state_drift: need a quantized and a full-precision context");
+    if (q_ctx->cfg.key_axis)
+        return fail(RSQ_E_UNSUPPORTED, "state_drift: key-axis scales (use rsq_dequantize)");
     const rsq_config& a = q_ctx->cfg;
     const rsq_config& b = f_ctx->cfg;
     if (a.batch != b.batch || a.heads != b.heads || a.dk != b.dk || a.dv != b.dv)
@@ -530,8 +548,8 @@ extern "C" rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_s
         return fail(RSQ_E_INVAL, "decode_step_noalloc: bad in_dtype %d", c.in_dtype);
     if (c.family == RSQ_MAMBA2 && (c.ngroups < 1 || c.heads % c.ngroups != 0))
         return fail(RSQ_E_INVAL, "decode_step_noalloc: ngroups must divide heads");
-    if (c.window != 0)
-        return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: no pure-write window in this entry point");
+    if (c.window != 0 || c.key_axis != 0)
+        return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: no pure-write window or key-axis scales here");
     if (kNoallocWordsNeeded > kNoallocScratchWords)
         return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: needs %d scratch words, the static array holds %d",
                     kNoallocWordsNeeded, kNoallocScratchWords);

@@ -97,6 +97,7 @@ struct DequantParams {
     const float* scales;
     float* S;                      // natural [B][H][dk][dv] (dequantize), or null
     float* absmax;                 // [B][H][dv] column maxima of |S| (column_absmax), or null
+    int key_axis;                  // scales are per key row ([B][H][dk]) instead of per column
     uint32_t head_off[RSQ_MAX_HEADS];
     uint8_t head_bits[RSQ_MAX_HEADS];
 };
@@ -120,6 +121,9 @@ int decode_kernel_info(int family, int dk, int ub, bool f32state, int rnd, int* 
                        const void** func);
 int launch_quantize(int dk, const QuantParams& p, void* stream);
 int launch_dequantize(int dk, const DequantParams& p, void* stream);
+// key-axis scale groups (one CTA per head)
+int launch_decode_ka(int dk, const DecodeParams& p, bool sr, void* stream);
+int launch_quantize_ka(int dk, const QuantParams& p, void* stream);
 int launch_drift(const DriftParams& p, void* stream);
 
 }  // namespace rsq

@@ -64,6 +64,10 @@ def _create(**kw):
     (dict(window=3), rsq.RSQ_E_INVAL),
     (dict(window=8, family=rsq.RSQ_MAMBA2), rsq.RSQ_E_UNSUPPORTED),
     (dict(window=8, rounding=rsq.RSQ_BDR), rsq.RSQ_E_UNSUPPORTED),
+    (dict(key_axis=2), rsq.RSQ_E_INVAL),
+    (dict(key_axis=1, family=rsq.RSQ_KDA), rsq.RSQ_E_UNSUPPORTED),
+    (dict(key_axis=1, window=4), rsq.RSQ_E_UNSUPPORTED),
+    (dict(key_axis=1, head_bits=[32, 32, 32, 32]), rsq.RSQ_E_UNSUPPORTED),
 ])
 def test_create_rejects_bad_configs_on_host(kw, status):
     with pytest.raises(rsq.RsqError) as e:

@@ -25,7 +25,8 @@ import bench  # noqa: E402
 def _oracle_series(w, steps, every, variants):
     rnd = {"sr": oracle.SR, "rtn": oracle.RTN, "bdr": oracle.BDR, "sr_bdr": oracle.SR_BDR}
     ref = oracle.zero_state(w.B, w.H, w.dk, w.dv, fp32=True)
-    qs = {lab: oracle.zero_state(w.B, w.H, w.dk, w.dv, fp32=False) for lab, _, _, _ in variants}
+    qs = {lab: (oracle.zero_state_ka(w.B, w.H, w.dk, w.dv) if src == "keyaxis"
+                else oracle.zero_state(w.B, w.H, w.dk, w.dv, fp32=False)) for lab, _, _, src in variants}
     wins = {lab: oracle.zero_window(w.B, w.H, int(src[1:]), w.dk, w.dv)
             for lab, _, _, src in variants if src.startswith("w")}
     out = {lab: [] for lab, _, _, _ in variants}
@@ -39,13 +40,19 @@ def _oracle_series(w, steps, every, variants):
             if lab in wins:
                 qs[lab], wins[lab], o = oracle.gdn_pw_step(qs[lab], wins[lab], inp, hb, rounding=rnd[r],
                                                            seed=w.sr_seed, step=t)
+            elif src == "keyaxis":
+                qs[lab], o = oracle.gdn_ka_step(qs[lab], inp, hb, rounding=rnd[r], seed=w.sr_seed, step=t)
             else:
                 qs[lab], o = oracle.gdn_step(qs[lab], inp, hb, rounding=rnd[r], seed=w.sr_seed, step=t,
                                              copy_absmax=m if src == "copy" else None)
             if (t + 1) % every == 0:
                 F = oracle.dequantize(ref, f32).astype(np.float64)
-                D = (oracle.window_full_state(qs[lab], wins[lab], hb) if lab in wins
-                     else oracle.dequantize(qs[lab], hb).astype(np.float64))
+                if lab in wins:
+                    D = oracle.window_full_state(qs[lab], wins[lab], hb)
+                elif src == "keyaxis":
+                    D = oracle.dequantize_ka(qs[lab]).astype(np.float64)
+                else:
+                    D = oracle.dequantize(qs[lab], hb).astype(np.float64)
                 num = ((D - F) ** 2).sum(axis=(2, 3))
                 den = (F ** 2).sum(axis=(2, 3))
                 o64, r64 = o.astype(np.float64), o_ref.astype(np.float64)

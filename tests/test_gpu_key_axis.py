@@ -1,0 +1,101 @@
+"""GPU parity of key-axis scale groups (LoReS "(1/4) Scale grouping": one scale
+per key row, the grouping ablation) against the CPU oracle.
+
+The key-axis decode kernel (one CTA per head) and its quantize / dequantize
+paths must match the oracle bit for bit on free-running trajectories.
+"""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ssm_decode_02_b200 as rsq
+import workloads as W
+from gpu_harness import assert_out_equal, dev, host, sample_heads
+
+pytestmark = pytest.mark.gpu
+
+
+class KaRun:
+    def __init__(self, w, bits, rounding):
+        self.w, self.bits, self.rounding = w, np.asarray(bits, np.int8), rounding
+        self.B, self.H, self.dk, self.dv = w.B, w.H, w.dk, w.dv
+        self.in_dtype = rsq.RSQ_BF16 if w.in_dtype == "bf16" else rsq.RSQ_F32
+        self.ctx = rsq.Context(rsq.RSQ_GDN, self.B, self.H, self.dk, self.dv, head_bits=self.bits,
+                               rounding=rounding, in_dtype=self.in_dtype, seed=w.sr_seed, key_axis=1)
+
+    def upload(self, st):
+        return rsq.State(dev(oracle.pack_state(st, self.bits)), dev(st["scales"]))
+
+    def download(self, s, heads=None):
+        dummy = np.zeros((self.B, self.H, self.dv), np.float32)
+        st = oracle.unpack_state(host(s.codes), dummy, self.bits, self.B, self.H, self.dk, self.dv,
+                                 heads=heads)
+        return {"codes": st["codes"], "scales": host(s.scales)}
+
+    def inputs(self, t):
+        return W.gdn_inputs(self.w, t)
+
+
+def _assert_ka_equal(g, o, heads, what):
+    for b, h in heads:
+        assert np.array_equal(g["codes"][b, h], o["codes"][b, h]), "%s codes (%d,%d)" % (what, b, h)
+        assert np.array_equal(g["scales"][b, h].view(np.uint32), o["scales"][b, h].view(np.uint32)), \
+            "%s scales (%d,%d)" % (what, b, h)
+
+
+def _trajectory(run: KaRun, steps, heads=None, seed=5):
+    rng = np.random.default_rng(seed)
+    S = (rng.standard_normal((run.B, run.H, run.dk, run.dv)) * 0.2).astype(np.float32)
+    st = oracle.quantize_ka(S, run.bits, rounding=run.rounding, seed=run.w.sr_seed, step=0)
+    g = run.upload(st)
+    sel = heads if heads is not None else [(b, h) for b in range(run.B) for h in range(run.H)]
+    for t in range(steps):
+        inp = run.inputs(t)
+        keep = {k: dev(v) for k, v in inp.items()}
+        ins = rsq.gdn_inputs(keep["q"], keep["k"], keep["v"], keep["alpha"], keep["beta"])
+        out = torch.empty((run.B, run.H, run.dv), dtype=torch.float32, device="cuda")
+        run.ctx.decode_step(g, g, ins, out, t)
+        torch.cuda.synchronize()
+        st, o = oracle.gdn_ka_step(st, inp, run.bits, rounding=run.rounding, seed=run.w.sr_seed, step=t,
+                                   heads=heads)
+        _assert_ka_equal(run.download(g, heads=heads), st, sel, "step %d" % t)
+        assert_out_equal(host(out), o, heads=heads, what="step %d" % t)
+
+
+@pytest.mark.parametrize("dk,dv", [(128, 128), (16, 16), (32, 64), (64, 256), (128, 32)])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR])
+def test_key_axis_decode_bit_exact(dk, dv, rounding):
+    w = dataclasses.replace(W.WORKLOADS[1], B=3, H=4, dk=dk, dv=dv)
+    _trajectory(KaRun(w, [8, 4, 4, 8], rounding), 4, seed=dk + dv)
+
+
+def test_key_axis_f32_inputs():
+    w = dataclasses.replace(W.WORKLOADS[0], B=2, H=3)
+    _trajectory(KaRun(w, [8, 8, 4], rsq.RSQ_SR), 6)
+
+
+def test_key_axis_full_size_sampled_heads():
+    w = W.WORKLOADS[1]
+    run = KaRun(w, np.full(w.H, 8, np.int8), rsq.RSQ_SR)
+    _trajectory(run, 2, heads=sample_heads(w.B, w.H, 32, seed=7))
+
+
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR])
+def test_key_axis_quantize_dequantize_and_maxima(rounding):
+    w = dataclasses.replace(W.WORKLOADS[1], B=2, H=3, dk=64, dv=128)
+    run = KaRun(w, [8, 4, 8], rounding)
+    rng = np.random.default_rng(3)
+    S = rng.standard_normal((2, 3, 64, 128)).astype(np.float32)
+    g = run.ctx.alloc_state()
+    run.ctx.quantize(dev(S), g, step=4)
+    want = oracle.quantize_ka(S, run.bits, rounding=rounding, seed=w.sr_seed, step=4)
+    _assert_ka_equal(run.download(g), want, [(b, h) for b in range(2) for h in range(3)], "quantize")
+    D = torch.empty((2, 3, 64, 128), dtype=torch.float32, device="cuda")
+    run.ctx.dequantize(g, D)
+    assert np.array_equal(host(D), oracle.dequantize_ka(want))
+    m = torch.empty((2, 3, 128), dtype=torch.float32, device="cuda")
+    run.ctx.column_absmax(g, m)
+    assert np.array_equal(host(m), np.abs(oracle.dequantize_ka(want)).max(axis=2))
