@@ -125,16 +125,31 @@ def _check(status: int) -> int:
 
 
 def _ptr(t) -> int | None:
-    """Device (or host) address of a tensor / buffer; ints pass through; None stays None."""
+    """Host address of a numpy array (host arguments); ints pass through; None stays None."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
-    if hasattr(t, "data_ptr"):
-        return int(t.data_ptr())
     if isinstance(t, np.ndarray):
         return int(t.ctypes.data)
+    if hasattr(t, "data_ptr"):
+        return int(t.data_ptr())
     raise TypeError("cannot take the address of %r" % type(t))
+
+
+def _dptr(t) -> int | None:
+    """Device address of a CUDA tensor argument; a CPU or non-contiguous tensor is
+    refused here instead of reaching the kernel.  Ints (raw device addresses) pass
+    through; None stays None."""
+    if t is None or isinstance(t, int):
+        return t
+    if not hasattr(t, "data_ptr"):
+        raise TypeError("expected a CUDA tensor, got %r" % type(t))
+    if not getattr(t, "is_cuda", False):
+        raise ValueError("expected a CUDA tensor, got one on %s" % getattr(t, "device", "the host"))
+    if not t.is_contiguous():
+        raise ValueError("expected a contiguous CUDA tensor")
+    return int(t.data_ptr())
 
 
 def _stream(stream) -> int | None:
@@ -180,7 +195,7 @@ def rsq_decode_step_noalloc(family: int, batch: int, heads: int, dk: int, dv: in
     cfg, keep = _config(family, batch, heads, dk, dv, head_bits, rounding, in_dtype, seed, ngroups)
     si, so = _state(state_in), _state(state_out)
     _check(lib.rsq_decode_step_noalloc(ctypes.byref(cfg), ctypes.byref(si), ctypes.byref(so),
-                                       ctypes.byref(inputs), _ptr(out), int(step) & 0xFFFFFFFF,
+                                       ctypes.byref(inputs), _dptr(out), int(step) & 0xFFFFFFFF,
                                        _stream(stream)))
     del keep
 
@@ -202,7 +217,7 @@ def rsq_head_offset(ctx: int, h: int) -> int:
 
 
 def _state(st) -> rsq_state:
-    return rsq_state(_ptr(st.codes), _ptr(st.scales))
+    return rsq_state(_dptr(st.codes), _dptr(st.scales))
 
 
 def rsq_decode_step(ctx: int, state_in, state_out, inputs, out, step: int, stream=None) -> None:
@@ -210,7 +225,7 @@ def rsq_decode_step(ctx: int, state_in, state_out, inputs, out, step: int, strea
     mamba2_inputs, diag_inputs)."""
     si, so = _state(state_in), _state(state_out)
     _check(lib.rsq_decode_step(ctx, ctypes.byref(si), ctypes.byref(so), ctypes.byref(inputs),
-                               _ptr(out), int(step) & 0xFFFFFFFF, _stream(stream)))
+                               _dptr(out), int(step) & 0xFFFFFFFF, _stream(stream)))
 
 
 def rsq_decode_step_copy_scale(ctx: int, state_in, state_out, inputs, copy_absmax, out, step: int,
@@ -219,14 +234,14 @@ def rsq_decode_step_copy_scale(ctx: int, state_in, state_out, inputs, copy_absma
     unquantized copy of the state) instead of the state's own columns."""
     si, so = _state(state_in), _state(state_out)
     _check(lib.rsq_decode_step_copy_scale(ctx, ctypes.byref(si), ctypes.byref(so), ctypes.byref(inputs),
-                                          _ptr(copy_absmax), _ptr(out), int(step) & 0xFFFFFFFF,
+                                          _dptr(copy_absmax), _dptr(out), int(step) & 0xFFFFFFFF,
                                           _stream(stream)))
 
 
 def rsq_column_absmax(ctx: int, state, absmax, stream=None) -> None:
     """Column maxima of |S^| of a stored state into absmax ([B][H][dv] float32, device)."""
     si = _state(state)
-    _check(lib.rsq_column_absmax(ctx, ctypes.byref(si), _ptr(absmax), _stream(stream)))
+    _check(lib.rsq_column_absmax(ctx, ctypes.byref(si), _dptr(absmax), _stream(stream)))
 
 
 def rsq_window_bytes(ctx: int) -> tuple[int, int, int]:
@@ -236,7 +251,7 @@ def rsq_window_bytes(ctx: int) -> tuple[int, int, int]:
 
 
 def _window(win) -> rsq_window:
-    return rsq_window(_ptr(win.a), _ptr(win.a_scale), _ptr(win.b), _ptr(win.b_scale))
+    return rsq_window(_dptr(win.a), _dptr(win.a_scale), _dptr(win.b), _dptr(win.b_scale))
 
 
 def rsq_decode_step_window(ctx: int, state_in, state_out, win_in, win_out, inputs, out, step: int,
@@ -244,23 +259,23 @@ def rsq_decode_step_window(ctx: int, state_in, state_out, win_in, win_out, input
     si, so = _state(state_in), _state(state_out)
     wi, wo = _window(win_in), _window(win_out)
     _check(lib.rsq_decode_step_window(ctx, ctypes.byref(si), ctypes.byref(so), ctypes.byref(wi),
-                                      ctypes.byref(wo), ctypes.byref(inputs), _ptr(out),
+                                      ctypes.byref(wo), ctypes.byref(inputs), _dptr(out),
                                       int(step) & 0xFFFFFFFF, _stream(stream)))
 
 
 def rsq_quantize(ctx: int, S, state_out, step: int, stream=None) -> None:
     so = _state(state_out)
-    _check(lib.rsq_quantize(ctx, _ptr(S), ctypes.byref(so), int(step) & 0xFFFFFFFF, _stream(stream)))
+    _check(lib.rsq_quantize(ctx, _dptr(S), ctypes.byref(so), int(step) & 0xFFFFFFFF, _stream(stream)))
 
 
 def rsq_dequantize(ctx: int, state_in, S_out, stream=None) -> None:
     si = _state(state_in)
-    _check(lib.rsq_dequantize(ctx, ctypes.byref(si), _ptr(S_out), _stream(stream)))
+    _check(lib.rsq_dequantize(ctx, ctypes.byref(si), _dptr(S_out), _stream(stream)))
 
 
 def rsq_state_drift(q_ctx: int, q_state, f_ctx: int, f_state, sums, stream=None) -> None:
     a, b = _state(q_state), _state(f_state)
-    _check(lib.rsq_state_drift(q_ctx, ctypes.byref(a), f_ctx, ctypes.byref(b), _ptr(sums),
+    _check(lib.rsq_state_drift(q_ctx, ctypes.byref(a), f_ctx, ctypes.byref(b), _dptr(sums),
                                _stream(stream)))
 
 
@@ -309,16 +324,16 @@ class Window:
 
 
 def gdn_inputs(q, k, v, alpha, beta) -> rsq_gdn_inputs:
-    return rsq_gdn_inputs(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta))
+    return rsq_gdn_inputs(_dptr(q), _dptr(k), _dptr(v), _dptr(alpha), _dptr(beta))
 
 
 def diag_inputs(q, k, v, alpha, beta=None) -> rsq_diag_inputs:
     """GLA / KDA inputs: alpha is the decay per key channel ([B][H][dk] float32)."""
-    return rsq_diag_inputs(_ptr(q), _ptr(k), _ptr(v), _ptr(alpha), _ptr(beta))
+    return rsq_diag_inputs(_dptr(q), _dptr(k), _dptr(v), _dptr(alpha), _dptr(beta))
 
 
 def mamba2_inputs(x, Bm, Cm, dt, A, D, decay=None) -> rsq_mamba2_inputs:
-    return rsq_mamba2_inputs(_ptr(x), _ptr(Bm), _ptr(Cm), _ptr(dt), _ptr(A), _ptr(D), _ptr(decay))
+    return rsq_mamba2_inputs(_dptr(x), _dptr(Bm), _dptr(Cm), _dptr(dt), _dptr(A), _dptr(D), _dptr(decay))
 
 
 class Context:

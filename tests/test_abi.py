@@ -107,3 +107,16 @@ def test_allocate_bits_validation():
         rsq.rsq_allocate_bits(np.ones(4), 5)
     with pytest.raises(rsq.RsqError):
         rsq.rsq_allocate_bits(np.ones(4), 1, high_bits=16)
+
+
+def test_binding_refuses_host_tensors_for_device_arguments():
+    """A CPU or non-contiguous tensor passed where the ABI expects device memory
+    is refused by the binding before any call reaches the library."""
+    import torch
+    with pytest.raises(ValueError):
+        rsq.gdn_inputs(torch.zeros(4), 0, 0, 0, 0)
+    with pytest.raises(ValueError):
+        rsq._state(rsq.State(torch.zeros(8, dtype=torch.uint8), 0))
+    with pytest.raises(TypeError):
+        rsq.gdn_inputs(object(), 0, 0, 0, 0)
+    assert rsq.gdn_inputs(0, 0, 0, 0, 0).q is None
