@@ -60,8 +60,14 @@ struct DecodeCfg {
     static constexpr int OFF_WAS = OFF_WA + kMaxWindow * DK;
     static constexpr int OFF_WB = OFF_WAS + kMaxWindow * 4;
     static constexpr int OFF_WBS = OFF_WB + UB * kMaxWindow * 16;
+    // the slot pass's results, shared by the unit's warps: z_w and the leaving
+    // slot's propagated a as duplicated pairs (row-group layout of the pairs)
+    static constexpr int OFF_WZ = OFF_WBS + kMaxWindow * 4;
+    static constexpr int OFF_WM = OFF_WZ + kMaxWindow * 4;
     static constexpr int END_BASE = DIAG ? OFF_VD + DK * 4 : OFF_VD;
-    static constexpr int STAGE = ((PW ? OFF_WBS + kMaxWindow * 4 : END_BASE) + 127) / 128 * 128;
+    static constexpr int STAGE = ((PW ? OFF_WM + kR * (DK / kR + 2) * 8 : END_BASE) + 127) / 128 * 128;
+    // warps that run the slot passes (passes of 4 slots spread over the unit's warps)
+    static constexpr int NPROD = PW ? (WIN / 4 < UB ? WIN / 4 : UB) : 0;
     // per warp: the two key-axis vectors as duplicated pairs (x, x), one row of
     // PST pairs per row group (padded so the row groups hit different banks)
     static constexpr int PST = L::RPT + 2;
@@ -74,7 +80,8 @@ struct DecodeCfg {
     static constexpr int OFF_P = NS * STAGE;
     static constexpr int OFF_CNT = OFF_P + UB * P_WARP;  // NS release counters
     static constexpr int OFF_BAR = OFF_CNT + 16;
-    static constexpr int SMEM = OFF_BAR + NS * 8;
+    static constexpr int OFF_SBAR = OFF_BAR + NS * 8;  // window: "slot results ready" per stage
+    static constexpr int SMEM = OFF_SBAR + (PW ? NS * 8 : 0);
     // resident CTAs per SM the register budget is sized for: shared memory holds
     // four 128-thread CTAs per SM (4 x ~50 KB), so 128 registers per thread
     static constexpr int MINB = F32STATE ? 1 : (NT < 128 ? 8 : 4);
@@ -175,7 +182,8 @@ __device__ __forceinline__ Gates load_gates(const DecodeParams& p, const UnitIt&
 }
 
 // Pure-write window ("Low-Bit GDN Recurrent-State Quantization: ... Pure-Write
-// Sliding Windows", abstract), per warp: every slot's a vector goes through
+// Sliding Windows", abstract), for the slot passes given to this warp: each
+// slot's a vector goes through
 // the step's transition a <- alpha (a - beta k (k.a)); the slot `ps` leaving
 // the window leaves its propagated a in the pair array `pm` (rows as
 // duplicated pairs) for the merge into the history; z_w = a_w . q (slot ps:
@@ -234,18 +242,20 @@ __device__ __forceinline__ float pw_slot(const uint8_t* stage, int off_wa, int o
 }
 
 // Pure-write window ("Low-Bit GDN Recurrent-State Quantization: ... Pure-Write
-// Sliding Windows", abstract), per warp: every slot's a vector goes through
+// Sliding Windows", abstract), for the slot passes given to this warp: each
+// slot's a vector goes through
 // the step's transition a <- alpha (a - beta k (k.a)); the slot `ps` leaving
 // the window leaves its propagated a in the pair array `pm` (rows as
 // duplicated pairs) for the merge into the history; z_w = a_w . q (slot ps:
 // k . q, its new write) goes to `zs`.  Lane (slot group, chunk) handles rows
-// [chunk * DK/8, (chunk+1) * DK/8) of slots slot group, +4, +8, ...  The writer
-// warp also encodes the new a vectors (FP8 E4M3, one scale = max|a| / 448).
+// [chunk * DK/8, (chunk+1) * DK/8) of the slots (slot group) + 4 * pass.  In a
+// writer unit the warp also encodes its slots' new a vectors (FP8 E4M3, one
+// scale = max|a| / 448).
 template <int DK, int PST, int WIN>
 __device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* stage, int off_wa,
                                          int off_was, int off_va, int off_vb, int hu, int ps,
-                                         float alpha, float beta, bool writer, uint64_t* pm,
-                                         float* zs, int lane) {
+                                         float alpha, float beta, int pass0, int pstep, bool writer,
+                                         uint64_t* pm, float* zs, int lane) {
     constexpr int CH = DK / 8;
     const bool bf16 = p.in_bf16 != 0;
     const int sl = lane >> 3, chunk = lane & 7, i0 = chunk * CH;
@@ -282,19 +292,19 @@ __device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* s
             if (chunk == 0) p.win_as_out[(long long)hu * WIN + slot] = __fdiv_rn(m, 448.f);
         }
     };
-    int pass = 0;
-    // two slots per lane at a time where possible (independent dependency chains)
-#pragma unroll
-    for (; (pass + 2) * 4 <= WIN; pass += 2) {
-        const int s0 = pass * 4 + sl, s1 = s0 + 4;
+    // passes pass0, pass0 + pstep, ... of 4 slots each; two slots per lane at a
+    // time where possible (independent dependency chains)
+    constexpr int NPASS = WIN / 4;
+    int pass = pass0;
+    for (; pass + pstep < NPASS; pass += 2 * pstep) {
+        const int s0 = pass * 4 + sl, s1 = (pass + pstep) * 4 + sl;
         float a0[CH], a1[CH];
         const float z0 = pw_slot<CH>(stage, off_wa, off_was, s0, DK, i0, kk, qq, alpha, beta, s0 == ps, a0);
         const float z1 = pw_slot<CH>(stage, off_wa, off_was, s1, DK, i0, kk, qq, alpha, beta, s1 == ps, a1);
         finish(s0, z0, a0);
         finish(s1, z1, a1);
     }
-#pragma unroll
-    for (; pass * 4 < WIN; ++pass) {
+    for (; pass < NPASS; pass += pstep) {
         const int s0 = pass * 4 + sl;
         float a0[CH];
         const float z0 = pw_slot<CH>(stage, off_wa, off_was, s0, DK, i0, kk, qq, alpha, beta, s0 == ps, a0);
@@ -304,8 +314,8 @@ __device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* s
 
 // One 16-column block of one unit, processed by warp w.
 template <int FAM, int DK, int UB, bool F32STATE, int RND, int BITS>
-__device__ __forceinline__ void process_block(const DecodeParams& p, const UnitIt& un, uint8_t* stage,
-                                              uint8_t* smem, int stage_idx, uint32_t bar,
+__device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitIt& un, uint8_t* stage,
+                                              uint8_t* smem, int stage_idx, uint32_t bar, uint32_t parity,
                                               const Gates& gt, int w, int lane, int g, int cw) {
     using L = Layout<DK>;
     using C = DecodeCfg<FAM, DK, UB, F32STATE>;
@@ -338,12 +348,21 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
         }
     }
     __syncwarp();
-    float* zs = reinterpret_cast<float*>(smem + C::OFF_P + w * C::P_WARP + C::OFF_PZ);  // window z_w
+    // window: z_w and the leaving slot's propagated a, computed by the unit's
+    // first NPROD warps into the stage and published through a stage barrier
+    float* zs = reinterpret_cast<float*>(stage + C::OFF_WZ);
     const int ps = C::PW ? static_cast<int>(p.step % static_cast<uint32_t>(C::WIN)) : 0;  // slot leaving
     if constexpr (C::PW) {
-        pw_slots<DK, C::PST, C::WIN>(p, stage, C::OFF_WA, C::OFF_WAS, C::OFF_VA, C::OFF_VB, hu, ps, gt.g0, gt.g1,
-                             un.cb == 0 && w == 0, pc, zs, lane);
-        __syncwarp();
+        const uint32_t sbar = smem_u32(smem + C::OFF_SBAR) + 8 * stage_idx;
+        if (w < C::NPROD) {
+            pw_slots<DK, C::PST, C::WIN>(p, stage, C::OFF_WA, C::OFF_WAS, C::OFF_VA, C::OFF_VB, hu, ps, gt.g0,
+                                         gt.g1, w, C::NPROD, un.cb == 0,
+                                         reinterpret_cast<uint64_t*>(stage + C::OFF_WM), zs, lane);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(sbar);
+        }
+        const bool ok = mbar_wait(sbar, parity, kWaitIters);
+        if (!__all_sync(0xffffffffu, ok)) return false;
     }
     const uint64_t* qa = pa + g * C::PST;  // q (GDN, GLA, KDA) / C (Mamba-2) of rows g + 8k
     const uint64_t* kb = pb + g * C::PST;  // k / B
@@ -423,7 +442,7 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
             e4m3x2_to_f32(b4 >> 16, b2, b3);
             const uint64_t B01 = pk(__fmul_rn(b0, bsc), __fmul_rn(b1, bsc));
             const uint64_t B23 = pk(__fmul_rn(b2, bsc), __fmul_rn(b3, bsc));
-            const uint64_t* mg = pc + g * C::PST;
+            const uint64_t* mg = reinterpret_cast<const uint64_t*>(stage + C::OFF_WM) + g * C::PST;
 #pragma unroll
             for (int k = 0; k < RPT; k += 2) {
                 const ulonglong2 aa = *reinterpret_cast<const ulonglong2*>(mg + k);
@@ -644,6 +663,7 @@ __device__ __forceinline__ void process_block(const DecodeParams& p, const UnitI
             }
         }
     }
+    return true;
 }
 
 // Resident CTAs per SM the register budget is sized for: Bounded Directional
@@ -671,6 +691,7 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_
         uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + C::OFF_CNT);
         for (int s = 0; s < C::NS; ++s) {
             mbar_init(bar0 + 8 * s, 1);
+            if constexpr (C::PW) mbar_init(smem_u32(smem + C::OFF_SBAR) + 8 * s, C::NPROD);
             cnt[s] = 0u;
         }
         fence_mbar_init();
@@ -701,13 +722,18 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_
             return;  // this warp stops; the others see their own waits expire
         }
         uint8_t* st = smem + stage * C::STAGE;
+        bool done;
         if constexpr (F32STATE) {
-            process_block<FAM, DK, UB, true, 0, 32>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
+            done = process_block<FAM, DK, UB, true, 0, 32>(p, cur, st, smem, stage, bar, parity, gt, w, lane, g, cw);
         } else {
             if (p.head_bits[cur.h] == 8)
-                process_block<FAM, DK, UB, false, RND, 8>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
+                done = process_block<FAM, DK, UB, false, RND, 8>(p, cur, st, smem, stage, bar, parity, gt, w, lane, g, cw);
             else
-                process_block<FAM, DK, UB, false, RND, 4>(p, cur, st, smem, stage, bar, gt, w, lane, g, cw);
+                done = process_block<FAM, DK, UB, false, RND, 4>(p, cur, st, smem, stage, bar, parity, gt, w, lane, g, cw);
+        }
+        if (!done) {  // a bounded wait inside the block ran out (window slot results)
+            if (lane == 0) atomicOr(p.flag, kFlagTimeout);
+            return;
         }
         cur = nxt;
         gt = ng;
