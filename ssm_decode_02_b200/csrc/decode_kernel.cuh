@@ -73,10 +73,8 @@ struct DecodeCfg {
     static constexpr int PST = L::RPT + 2;
     // pair arrays: q, k (+ the decay per key channel for GLA, + decay and
     // decay * k for KDA)
-    static constexpr int NPAIR = FAM == RSQ_KDA ? 4 : ((DIAG || is_pw_family(FAM)) ? 3 : 2);
-    // (+ the window's z_w = a_w . q for the pure-write window)
-    static constexpr int OFF_PZ = NPAIR * kR * PST * 8;
-    static constexpr int P_WARP = OFF_PZ + (is_pw_family(FAM) ? kMaxWindow * 4 : 0);
+    static constexpr int NPAIR = FAM == RSQ_KDA ? 4 : (DIAG ? 3 : 2);
+    static constexpr int P_WARP = NPAIR * kR * PST * 8;
     static constexpr int OFF_P = NS * STAGE;
     static constexpr int OFF_CNT = OFF_P + UB * P_WARP;  // NS release counters
     static constexpr int OFF_BAR = OFF_CNT + 16;
