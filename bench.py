@@ -291,6 +291,7 @@ def run_reference(args, w: W.Workload):
 def run_ours(args, w: W.Workload):
     import torch
     import torch.distributed as dist
+    from torch.cuda import nvtx  # ranges rsq.warmup / rsq.timed / rsq.l2_hot / rsq.e2e for ncu --nvtx
 
     import ssm_decode_02_b200 as rsq
 
@@ -396,7 +397,7 @@ def run_ours(args, w: W.Workload):
     clocks.start()
     time.sleep(0.3)
     # graphs replay on the current stream: make it the timed stream
-    with torch.cuda.stream(stream):
+    with torch.cuda.stream(stream), nvtx.range("rsq.warmup"):
         for gr in warm_graphs:
             gr.replay()
     stream.synchronize()
@@ -405,7 +406,7 @@ def run_ours(args, w: W.Workload):
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    with torch.cuda.stream(stream):
+    with torch.cuda.stream(stream), nvtx.range("rsq.timed"):
         ev0.record(stream)
         for t0, n in timed_plan:
             graph_cache[n].replay()
@@ -430,9 +431,10 @@ def run_ours(args, w: W.Workload):
                 step_on(0, structs[0], args.warmup + t, t)
         hot.replay()
         h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        h0.record(stream)
-        hot.replay()
-        h1.record(stream)
+        with nvtx.range("rsq.l2_hot"):
+            h0.record(stream)
+            hot.replay()
+            h1.record(stream)
     h1.synchronize()
     hot_ms = h0.elapsed_time(h1) / n_hot
     del hot
@@ -466,6 +468,7 @@ def run_ours(args, w: W.Workload):
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
+    nvtx.range_push("rsq.e2e")
     e0.record(s_in)
     for t in range(n_e2e):
         i = t % 2
@@ -486,6 +489,7 @@ def run_ours(args, w: W.Workload):
     s_in.wait_stream(stream)
     s_in.wait_stream(s_out)
     e1.record(s_in)
+    nvtx.range_pop()
     e1.synchronize()
     e2e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist if world > 1 else None, dev)
 

@@ -38,7 +38,8 @@ _lib = None
 def lib():
     global _lib
     if _lib is None:
-        path = _build.build()
+        # RSQ_ORACLE_LIB selects another build of the same source (the sanitizer build)
+        path = os.environ.get("RSQ_ORACLE_LIB") or _build.build()
         L = ctypes.CDLL(path)
         P = ctypes.c_void_p
         L.orc_philox4x32_10.argtypes = [P, P, P]

@@ -26,5 +26,22 @@ def build(force: bool = False) -> str:
     return LIB
 
 
+SAN_LIB = os.path.join(HERE, "librsq_oracle_san.so")
+
+
+def build_sanitized() -> str:
+    """The same library under AddressSanitizer and UndefinedBehaviorSanitizer
+    (for the sanitizer test; load it with RSQ_ORACLE_LIB and libasan preloaded)."""
+    if os.path.exists(SAN_LIB) and os.path.getmtime(SAN_LIB) >= os.path.getmtime(SRC):
+        return SAN_LIB
+    tmp = SAN_LIB + ".tmp.%d" % os.getpid()
+    cmd = ["gcc", "-O1", "-g", "-std=c11", "-fPIC", "-shared", "-ffp-contract=off", "-fno-fast-math",
+           "-fsanitize=address,undefined", "-fno-sanitize-recover=all", "-fno-omit-frame-pointer",
+           SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, SAN_LIB)
+    return SAN_LIB
+
+
 if __name__ == "__main__":
     print(build(force="--force" in sys.argv))
