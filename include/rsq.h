@@ -109,6 +109,17 @@ typedef enum { RSQ_GDN = 0, RSQ_MAMBA2 = 1, RSQ_GLA = 2, RSQ_KDA = 3 } rsq_famil
 typedef enum { RSQ_RTN = 0, RSQ_SR = 1, RSQ_BDR = 2, RSQ_SR_BDR = 3 } rsq_rounding;
 typedef enum { RSQ_F32 = 0, RSQ_BF16 = 1 } rsq_dtype;
 
+/* Device allocator hook for the context's own allocation (its 4-byte flag
+ * word).  alloc returns device memory of at least `bytes` bytes, 16-byte
+ * aligned, on the current device, or NULL when it cannot (rsq_create then
+ * returns RSQ_E_NOMEM and allocates nothing else); release gives it back and
+ * is called once, by rsq_destroy or by a failing rsq_create.  `user` is
+ * rsq_config.alloc_user, passed through.  Both NULL: cudaMalloc / cudaFree.
+ * The hook lets a caller place the word in its own pool, and lets a test
+ * make the allocation fail. */
+typedef void* (*rsq_alloc_fn)(size_t bytes, void* user);
+typedef void (*rsq_release_fn)(void* ptr, void* user);
+
 /* Layer configuration, read once by rsq_create. */
 typedef struct {
     int family;      /* rsq_family */
@@ -128,6 +139,9 @@ typedef struct {
                         per key row, s_i = max_j |S_ij| / r ([LoReS] (1/4), the grouping
                         ablation).  Key-axis: Gated DeltaNet, 4/8-bit heads, RSQ_RTN or
                         RSQ_SR; scales are [B][H][dk]; one CTA per head. */
+    rsq_alloc_fn alloc;      /* allocator hook (above); NULL with release NULL: cudaMalloc */
+    rsq_release_fn release;  /* its release; set both or neither (else RSQ_E_INVAL) */
+    void* alloc_user;        /* passed to both */
 } rsq_config;
 
 typedef struct rsq_ctx rsq_ctx;
@@ -179,8 +193,9 @@ typedef struct {
 
 /* Create a context for one layer configuration.  Validates the configuration
  * (RSQ_E_INVAL / RSQ_E_UNSUPPORTED, nothing allocated), then allocates a
- * 4-byte device flag word on the current device (RSQ_E_NOMEM / RSQ_E_CUDA on
- * failure).  *out receives the context; release it with rsq_destroy. */
+ * 4-byte device flag word on the current device, through cfg->alloc when set
+ * (RSQ_E_NOMEM / RSQ_E_CUDA on failure).  *out receives the context; release
+ * it with rsq_destroy. */
 rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out);
 
 /* Release a context (NULL is a no-op).  Not stream-ordered: call it only after
@@ -328,10 +343,11 @@ int rsq_reduction_partials(int dk);
  *
  * Same computation, arguments and results as rsq_decode_step, but without a
  * context: the configuration is passed directly and nothing is allocated.
- * rsq_create allocates a 4-byte device flag word with cudaMalloc; callers that
- * may not allocate device memory -- code running inside CUDA stream capture
- * (allocation calls are not capturable) or a runtime whose device memory is
- * owned entirely by its own pool allocator -- use this entry point instead.
+ * rsq_create allocates a 4-byte device flag word (cudaMalloc, or the
+ * config's allocator hook); callers that may not allocate device memory at
+ * all -- code running inside CUDA stream capture (allocation calls are not
+ * capturable) -- use this entry point instead.  cfg->alloc, release and
+ * alloc_user are ignored here.
  *
  * Its scratch (the decode kernel's flag word) lives in a statically allocated
  * device array of 64 words (256 bytes) that every GPU loading the library

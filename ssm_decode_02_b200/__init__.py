@@ -32,12 +32,17 @@ class RsqError(RuntimeError):
         self.status = status
 
 
+rsq_alloc_fn = ctypes.CFUNCTYPE(ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p)
+rsq_release_fn = ctypes.CFUNCTYPE(None, ctypes.c_void_p, ctypes.c_void_p)
+
+
 class rsq_config(ctypes.Structure):
     _fields_ = [("family", ctypes.c_int), ("batch", ctypes.c_int), ("heads", ctypes.c_int),
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("ngroups", ctypes.c_int),
                 ("head_bits", ctypes.POINTER(ctypes.c_int8)), ("rounding", ctypes.c_int),
                 ("in_dtype", ctypes.c_int), ("seed", ctypes.c_uint64), ("window", ctypes.c_int),
-                ("key_axis", ctypes.c_int)]
+                ("key_axis", ctypes.c_int), ("alloc", rsq_alloc_fn), ("release", rsq_release_fn),
+                ("alloc_user", ctypes.c_void_p)]
 
 
 class rsq_state(ctypes.Structure):
@@ -166,9 +171,15 @@ def _stream(stream) -> int | None:
 # ---------------------------------------------------------------------------
 def rsq_create(family: int, batch: int, heads: int, dk: int, dv: int, *, head_bits=None,
                rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0,
-               ngroups: int = 1, window: int = 0, key_axis: int = 0) -> int:
+               ngroups: int = 1, window: int = 0, key_axis: int = 0, alloc=None, release=None) -> int:
+    """``alloc`` / ``release``: rsq_alloc_fn / rsq_release_fn objects (the
+    allocator hook; the caller keeps them alive as long as the context)."""
     cfg, bits_arr = _config(family, batch, heads, dk, dv, head_bits, rounding, in_dtype, seed, ngroups,
                             window, key_axis)
+    if alloc is not None:
+        cfg.alloc = alloc
+    if release is not None:
+        cfg.release = release
     out = ctypes.c_void_p()
     _check(lib.rsq_create(ctypes.byref(cfg), ctypes.byref(out)))
     return int(out.value)
@@ -341,14 +352,20 @@ class Context:
 
     def __init__(self, family: int, batch: int, heads: int, dk: int, dv: int, *, head_bits=None,
                  rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0, ngroups: int = 1,
-                 window: int = 0, key_axis: int = 0):
+                 window: int = 0, key_axis: int = 0, allocator=None):
+        """``allocator``: optional (alloc(nbytes) -> device address or None,
+        release(address)) pair for the context's own device word."""
         self.family, self.batch, self.heads, self.dk, self.dv = family, batch, heads, dk, dv
         self.head_bits = None if head_bits is None else np.asarray(head_bits, np.int8)
         self.rounding, self.in_dtype, self.seed, self.ngroups = rounding, in_dtype, seed, ngroups
         self.window, self.key_axis = window, key_axis
+        self._hooks = (None, None)
+        if allocator is not None:
+            a, r = allocator
+            self._hooks = (rsq_alloc_fn(lambda n, _u: a(int(n))), rsq_release_fn(lambda p, _u: r(int(p))))
         self.ctx = rsq_create(family, batch, heads, dk, dv, head_bits=head_bits, rounding=rounding,
                               in_dtype=in_dtype, seed=seed, ngroups=ngroups, window=window,
-                              key_axis=key_axis)
+                              key_axis=key_axis, alloc=self._hooks[0], release=self._hooks[1])
         self.code_bytes, self.scale_bytes = rsq_state_bytes(self.ctx)
 
     def close(self):

@@ -27,6 +27,16 @@ struct rsq_ctx {
 
 namespace {
 
+// The context's flag word goes back to whoever allocated it.
+void release_flag(rsq_ctx* ctx) {
+    if (!ctx->flag) return;
+    if (ctx->cfg.release)
+        ctx->cfg.release(ctx->flag, ctx->cfg.alloc_user);
+    else
+        cudaFree(ctx->flag);
+    ctx->flag = nullptr;
+}
+
 thread_local char g_err[512] = "";
 
 rsq_status fail(rsq_status s, const char* fmt, ...) {
@@ -134,6 +144,8 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
     if (c.window && c.rounding != RSQ_RTN && c.rounding != RSQ_SR)
         return fail(RSQ_E_UNSUPPORTED, "create: the pure-write window takes nearest or stochastic rounding");
     if (c.key_axis != 0 && c.key_axis != 1) return fail(RSQ_E_INVAL, "create: key_axis must be 0 or 1");
+    if ((c.alloc == nullptr) != (c.release == nullptr))
+        return fail(RSQ_E_INVAL, "create: set both alloc and release, or neither");
     if (c.key_axis && (c.family != RSQ_GDN || c.window || (c.rounding != RSQ_RTN && c.rounding != RSQ_SR)))
         return fail(RSQ_E_UNSUPPORTED, "create: key-axis scales: Gated DeltaNet, no window, nearest or stochastic rounding");
 
@@ -199,10 +211,21 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
                                     &f2) == 0)
             err = cudaFuncSetAttribute(f2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2));
     }
-    if (!err) err = cudaMalloc(&ctx->flag, sizeof(unsigned));
+    if (!err) {
+        if (c.alloc) {
+            ctx->flag = static_cast<unsigned*>(c.alloc(sizeof(unsigned), c.alloc_user));
+            if (!ctx->flag || (reinterpret_cast<uintptr_t>(ctx->flag) & 15u)) {
+                if (ctx->flag) c.release(ctx->flag, c.alloc_user);
+                delete ctx;
+                return fail(RSQ_E_NOMEM, "create: the allocator hook returned no 16-byte aligned memory");
+            }
+        } else {
+            err = cudaMalloc(&ctx->flag, sizeof(unsigned));
+        }
+    }
     if (!err) err = cudaMemset(ctx->flag, 0, sizeof(unsigned));
     if (err) {
-        if (ctx->flag) cudaFree(ctx->flag);
+        release_flag(ctx);
         delete ctx;
         if (err == cudaErrorMemoryAllocation) return fail(RSQ_E_NOMEM, "create: flag allocation failed");
         return cuda_fail(err, "create");
@@ -214,7 +237,7 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
 
 void rsq_destroy(rsq_ctx* ctx) {
     if (!ctx) return;
-    if (ctx->flag) cudaFree(ctx->flag);
+    release_flag(ctx);
     delete ctx;
 }
 
@@ -492,8 +515,8 @@ rsq_status rsq_check_flags(const rsq_ctx* ctx, int* seen, void* stream) {
 // ---------------------------------------------------------------------------
 // Decode step without any allocation.
 //
-// rsq_create allocates the context's 4-byte device flag word with cudaMalloc.
-// This entry point instead keeps that word in a small statically allocated
+// rsq_create allocates the context's 4-byte device flag word with cudaMalloc
+// (or the configuration's allocator hook).  This entry point instead keeps that word in a small statically allocated
 // device array, so a caller that may not allocate device memory can still run
 // a decode step: code inside stream capture, where allocation calls are not
 // allowed, or a runtime whose memory is owned entirely by its own pool

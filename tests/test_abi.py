@@ -68,6 +68,8 @@ def _create(**kw):
     (dict(key_axis=1, family=rsq.RSQ_KDA), rsq.RSQ_E_UNSUPPORTED),
     (dict(key_axis=1, window=4), rsq.RSQ_E_UNSUPPORTED),
     (dict(key_axis=1, head_bits=[32, 32, 32, 32]), rsq.RSQ_E_UNSUPPORTED),
+    (dict(alloc=rsq.rsq_alloc_fn(lambda n, u: None)), rsq.RSQ_E_INVAL),      # hook without release
+    (dict(release=rsq.rsq_release_fn(lambda p, u: None)), rsq.RSQ_E_INVAL),  # release without hook
 ])
 def test_create_rejects_bad_configs_on_host(kw, status):
     with pytest.raises(rsq.RsqError) as e:
@@ -120,3 +122,33 @@ def test_binding_refuses_host_tensors_for_device_arguments():
     with pytest.raises(TypeError):
         rsq.gdn_inputs(object(), 0, 0, 0, 0)
     assert rsq.gdn_inputs(0, 0, 0, 0, 0).q is None
+
+
+def test_binding_structs_match_the_c_header_layout(tmp_path):
+    """Every ctypes struct of the binding has the size and field offsets that a C
+    compiler gives the declarations in include/rsq.h."""
+    import ctypes
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("gcc not available")
+    structs = {"rsq_config": rsq.rsq_config, "rsq_state": rsq.rsq_state, "rsq_gdn_inputs": rsq.rsq_gdn_inputs,
+               "rsq_mamba2_inputs": rsq.rsq_mamba2_inputs, "rsq_diag_inputs": rsq.rsq_diag_inputs,
+               "rsq_window": rsq.rsq_window}
+    lines = ["#include <stdio.h>", "#include <stddef.h>", '#include "rsq.h"', "int main(void) {"]
+    for name, cls in structs.items():
+        lines.append('printf("%s %%zu\\n", sizeof(%s));' % (name, name))
+        for f in cls._fields_:
+            lines.append('printf("%s.%s %%zu\\n", offsetof(%s, %s));' % (name, f[0], name, f[0]))
+    lines += ["return 0;", "}"]
+    src = tmp_path / "layout.c"
+    src.write_text("\n".join(lines))
+    exe = tmp_path / "layout"
+    inc = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include")
+    subprocess.run(["gcc", "-std=c11", "-I", inc, str(src), "-o", str(exe)], check=True)
+    got = dict(l.split() for l in subprocess.run([str(exe)], capture_output=True, text=True,
+                                                 check=True).stdout.splitlines())
+    for name, cls in structs.items():
+        assert int(got[name]) == ctypes.sizeof(cls), name
+        for f in cls._fields_:
+            assert int(got["%s.%s" % (name, f[0])]) == getattr(cls, f[0]).offset, (name, f[0])
