@@ -177,6 +177,21 @@ static float orc_inv_rz(float r, float m)
  *               even) of the exact product S*inv;  SR: t = S*inv + (o + u/2^16)
  *               rounded once to binary32, c = floor(t) - o, with the offset
  *               o = 128 (8-bit) or 136 (4-bit) so that t stays in [1, 256).  */
+/* S / s of the plain order, made safe to convert to an integer.  When the
+ * scale s = m / r underflows to zero (m below r * 2^-150, deep in the
+ * subnormal range) S / s is +-inf, which the clamp to [-r, r] turns into +-r,
+ * or 0 / 0 for an element that is zero, whose code is 0.  Values beyond
+ * +-(r + 1) clamp to +-r either way, so they are cut there first.         */
+static float orc_plain_ratio(float S, float s, int r)
+{
+    const float x = S / s;
+    const float lim = (float)(r + 1);
+    if (isnan(x)) return 0.0f;
+    if (x > lim) return lim;
+    if (x < -lim) return -lim;
+    return x;
+}
+
 int orc_quantize_scalar(float S, float m, int bits, int rounding, int mode, uint32_t u)
 {
     const int r = orc_rmax(bits);
@@ -184,7 +199,7 @@ int orc_quantize_scalar(float S, float m, int bits, int rounding, int mode, uint
     int c;
     if (mode == ORC_PLAIN) {
         const float s = m / rf;
-        const float x = S / s;
+        const float x = orc_plain_ratio(S, s, r);
         if (!ORC_SR_BASE(rounding))
             c = (int)rintf(x);
         else
@@ -221,7 +236,8 @@ int orc_bdr_adjust(int c, float S, float prev, float m, int bits, int mode)
     const int up = (S > prev) && (now < prev);
     const int down = (S < prev) && (now > prev);
     if (!up && !down) return c;
-    const double x = (mode == ORC_PLAIN) ? (double)(S / s_new) : (double)S * (double)orc_inv_rz(rf, m);
+    const double x = (mode == ORC_PLAIN) ? (double)orc_plain_ratio(S, s_new, orc_rmax(bits))
+                                         : (double)S * (double)orc_inv_rz(rf, m);
     int d = up ? (int)ceil(x) : (int)floor(x);
     const int r = orc_rmax(bits);
     if (d > r) d = r;

@@ -170,6 +170,39 @@ def test_rtn_brute_force_nearest_code(bits):
             assert errs[c + r] <= best + s * r * 2.0 ** -22
 
 
+@pytest.mark.parametrize("bits", [8, 4])
+def test_subnormal_column_maxima(bits):
+    """Columns whose maximum m is so small that r/m overflows binary32.
+    Canonical order: the multiplier r/m rounded toward zero saturates at FLT_MAX,
+    so codes are the nearest integers of the exact products S * FLT_MAX (closed
+    form, float64).  Plain order: once s = m/r underflows to zero, every nonzero
+    element gets the code sign(S) r and a zero element 0; the stored scale is 0
+    either way, so both orders dequantize such a column to zeros."""
+    r = oracle.rmax(bits)
+    fmax = np.float64(np.finfo(np.float32).max)
+    hb = np.array([bits], np.int8)
+    for m in (np.float32(1e-38), np.float32(3e-39), np.float32(1e-40)):
+        assert np.float64(r) / np.float64(m) > fmax      # r/m overflows
+        col = np.array([m, -m, m / 2, -m / 3, 0, m / 7, -m, m / 5], np.float32)
+        S = np.zeros((1, 1, 8, 2), np.float32)
+        S[0, 0, :, 0] = col
+        st = oracle.quantize(S, hb, rounding=oracle.RTN, seed=0, step=0, mode=oracle.CANONICAL)
+        want = np.rint(col.astype(np.float64) * fmax).astype(np.int64)
+        assert np.array_equal(st["codes"][0, 0, :, 0], want)
+        assert st["scales"][0, 0, 0] == np.float32(m) / np.float32(r)
+        assert st["scales"][0, 0, 1] == 0 and not st["codes"][0, 0, :, 1].any()   # all-zero column
+    m = np.float32(2 * np.finfo(np.float32).smallest_subnormal)
+    assert np.float32(m) / np.float32(r) == 0                                        # s underflows
+    col = np.array([m, -m, 0, np.float32(m / 4), -np.float32(m / 2), 0, m, -m], np.float32)
+    S = np.zeros((1, 1, 8, 1), np.float32)
+    S[0, 0, :, 0] = col
+    for rnd in (oracle.RTN, oracle.SR):
+        st = oracle.quantize(S, hb, rounding=rnd, seed=3, step=1, mode=oracle.PLAIN)
+        assert np.array_equal(st["codes"][0, 0, :, 0], (np.sign(col) * r).astype(np.int64))
+        assert st["scales"][0, 0, 0] == 0
+        assert not oracle.dequantize(st, hb).any()
+
+
 # ---------------------------------------------------------------------------
 # (c) stochastic rounding is (conditionally) unbiased
 # ---------------------------------------------------------------------------

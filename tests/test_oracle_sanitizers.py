@@ -50,6 +50,19 @@ q = oracle.quantize(S, hb, rounding=oracle.SR, seed=1, step=0, copy_absmax=np.ab
 oracle.dequantize(q, hb)
 oracle.unpack_state(oracle.pack_state(q, hb), q["scales"], hb, 1, 2, 16, 16)
 oracle.quantize_ka(S, hb, rounding=oracle.RTN, seed=0, step=0)
+# columns whose maxima span the float range, down to scales that underflow to zero
+E = np.zeros((1, 1, 16, 16), np.float32)
+for j, m in enumerate([0.0, 1e-45, 1e-43, 1e-41, 3e-39, 1e-37, 1e-30, 1.0, 1e30, 3.4e38]):
+    E[0, 0, :, j] = np.linspace(-m, m, 16, dtype=np.float64).astype(np.float32)
+E[0, 0, 5, 10] = np.float32(3.4028235e38)
+for mode in (oracle.PLAIN, oracle.CANONICAL):
+    for rnd in (oracle.RTN, oracle.SR):
+        for b in (8, 4):
+            oracle.quantize(E, np.array([b], np.int8), rounding=rnd, seed=1, step=0, mode=mode)
+    oracle.quantize_ka(E, np.array([4], np.int8), rounding=oracle.SR, seed=1, step=0, mode=mode)
+    tinyst = oracle.quantize(E, np.array([8], np.int8), rounding=oracle.RTN, seed=1, step=0)
+    oracle.gdn_step(tinyst, W.gdn_inputs(dataclasses.replace(tiny, B=1, H=1), 0), np.array([8], np.int8),
+                    rounding=oracle.SR_BDR, seed=1, step=0, mode=mode)
 [oracle.e4m3_decode(c) for c in range(256)]
 [oracle.e4m3_encode(x) for x in (0.0, 1e-9, 0.3, 448.0, 1e6, -3.0)]
 oracle.allocate_bits(np.arange(8, dtype=np.float64), 2)
