@@ -10,6 +10,7 @@ model do, so every step reads its state from HBM.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
   python bench.py --drift [--workload W] [--drift-steps T] [--drift-every E]
+  python bench.py --sweep [--steps K] [--jsonl results.jsonl]
 
 N > 1 is launched by torchrun (one process per GPU); every rank runs its own
 requests (weak scaling, no collective on the data path); the time is the max
@@ -17,7 +18,9 @@ over ranks.  --impl reference times the CPU oracle on the host cores instead.
 --drift runs the long-horizon study instead (default: Gated DeltaNet B=1024,
 H=16, d=128, 4096 steps): the relative state drift of INT4/INT8 trajectories
 with stochastic and nearest rounding against the FP32 trajectory, every 256
-steps, as one JSON line.
+steps, as one JSON line.  --sweep measures every row of the throughput table
+(each workload and rounding, key-axis and window variant) in one process, one
+line each; --jsonl appends every line to a file as well.
 """
 from __future__ import annotations
 
@@ -135,6 +138,48 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
                 "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def emit(line: dict, args) -> None:
+    """Print the result line; with --jsonl also append it to that file."""
+    text = json.dumps(line)
+    print(text, flush=True)
+    if getattr(args, "jsonl", None):
+        with open(args.jsonl, "a") as f:
+            f.write(text + "\n")
+
+
+# The rows of the throughput table: (workload, rounding or None, window, key-axis)
+SWEEP = (
+    ("gdn_b64_h16_d128_int8_sr", None, 0, False), ("gdn_b64_h16_d128_int8_sr", "rtn", 0, False),
+    ("gdn_b64_h16_d128_int8_sr", "bdr", 0, False), ("gdn_b64_h16_d128_int8_sr", "sr_bdr", 0, False),
+    ("gdn_b256_h32_d128_mixed_sr", None, 0, False), ("mamba2_b128_h80_p64_n128_int8_sr", None, 0, False),
+    ("gdn_b1024_h16_d128_int4_sr_long", None, 0, False), ("gla_b64_h16_d128_int8_sr", None, 0, False),
+    ("kda_b64_h16_d128_int8_sr", None, 0, False), ("gdn_b1024_h16_d128_int4_sr_long", "sr_bdr", 0, False),
+    ("gdn_b64_h16_d128_int8_sr", None, 0, True), ("gdn_b64_h16_d128_int8_sr", "rtn", 0, True),
+    ("gdn_b1024_h16_d128_int4_sr_long", None, 0, True), ("gdn_b64_h16_d128_int8_sr", None, 4, False),
+    ("gdn_b64_h16_d128_int8_sr", None, 8, False), ("gdn_b64_h16_d128_int8_sr", None, 16, False),
+    ("gdn_b1024_h16_d128_int4_sr_long", None, 8, False),
+)
+
+
+def run_sweep(args) -> int:
+    """Every row of SWEEP on one GPU, one JSON line each (and --jsonl records)."""
+    import copy
+    import dataclasses
+    if int(os.environ.get("WORLD_SIZE", "1")) > 1:
+        print("--sweep runs on one GPU", file=sys.stderr)
+        return 2
+    for name, rounding, window, key_axis in SWEEP:
+        a = copy.copy(args)
+        a.window, a.key_axis, a.no_cpu_baseline = window, key_axis, True
+        w = W.BY_NAME[name]
+        if rounding:
+            w = dataclasses.replace(w, rounding=rounding)
+        rc = run_ours(a, w)
+        if rc:
+            return rc
+    return 0
 
 
 def max_over_ranks(x: float, dist=None, device=None) -> float:
@@ -281,7 +326,7 @@ def run_reference(args, w: W.Workload):
         "e2e": {"value": value, "unit": "head-updates/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
-    print(json.dumps(line), flush=True)
+    emit(line, args)
     return 0
 
 
@@ -542,7 +587,7 @@ def run_ours(args, w: W.Workload):
             "sample": "the same sample in %d concurrent processes (one per host core), ~%.0f s each"
                       % (procs, args.cpu_seconds)}
     if rank == 0:
-        print(json.dumps(line), flush=True)
+        emit(line, args)
     for gr in list(graph_cache.values()) + warm_graphs:
         del gr
     graph_cache.clear()
@@ -689,7 +734,7 @@ def run_drift(args, w: W.Workload, pool) -> int:
         "series": series, "input_workers": getattr(pool, "_processes", 0),
         "wall_s": time.perf_counter() - t0,
     }
-    print(json.dumps(line), flush=True)
+    emit(line, args)
     return 0
 
 
@@ -773,8 +818,13 @@ def main():
                     help="run the long-horizon state drift study instead of the throughput bench")
     ap.add_argument("--drift-steps", type=int, default=0, help="horizon (default: the workload's)")
     ap.add_argument("--drift-every", type=int, default=256)
+    ap.add_argument("--jsonl", default=None, help="also append each result line to this file")
+    ap.add_argument("--sweep", action="store_true",
+                    help="measure every row of the throughput table (one GPU), one line each")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
+    if args.sweep:
+        return run_sweep(args)
     if args.drift:
         w = W.BY_NAME[args.workload if args.workload != DEFAULT_WORKLOAD else DRIFT_WORKLOAD]
         # the input generator pool starts before the first CUDA call

@@ -85,3 +85,28 @@ def test_reference_arm_under_torchrun_prints_one_line():
     assert len(lines) == 1
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["value"] > 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_emit_appends_jsonl_records(tmp_path):
+    """--jsonl: each result line is printed and appended to the file."""
+    import argparse
+    sys.path.insert(0, ROOT)
+    import bench
+    path = tmp_path / "r.jsonl"
+    args = argparse.Namespace(jsonl=str(path))
+    bench.emit({"metric": "head-updates/s", "value": 1.0}, args)
+    bench.emit({"metric": "head-updates/s", "value": 2.0}, args)
+    recs = [json.loads(l) for l in path.read_text().splitlines()]
+    assert [r["value"] for r in recs] == [1.0, 2.0]
+    bench.emit({"value": 3.0}, argparse.Namespace(jsonl=None))   # no file: print only
+    assert len(path.read_text().splitlines()) == 2
+
+
+def test_sweep_rows_name_known_workloads():
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    for name, rounding, window, key_axis in bench.SWEEP:
+        assert name in W.BY_NAME
+        assert rounding is None or rounding in bench.ROUNDING
+        assert window in (0, 4, 8, 16) and not (window and key_axis)
