@@ -63,8 +63,8 @@
  *
  * Arithmetic (binary32 throughout; fixed evaluation order, see rsq_decode_step)
  * ------------------------------------------------------------------------
- *  Sums over the key axis i use R = rsq_reduction_partials(dk) = 8 partial
- *  sums: partial p accumulates rows i = p, p+R, p+2R, ... in increasing i with
+ *  Sums over the key axis i use R = rsq_reduction_partials(dk) partial sums
+ *  (8 up to dk = 128, 16 for dk = 256): partial p accumulates rows i = p, p+R, p+2R, ... in increasing i with
  *  one fused multiply-add per term; then for d = 1, 2, ..., R/2 every partial p
  *  becomes P[p] + P[p^d]; the sum is P[0].
  */
@@ -125,7 +125,8 @@ typedef struct {
     int family;      /* rsq_family */
     int batch;       /* B >= 1 independent requests */
     int heads;       /* H, 1..RSQ_MAX_HEADS */
-    int dk;          /* rows: GDN key dim d_k / Mamba-2 state dim N; one of 16, 32, 64, 128 */
+    int dk;          /* rows: GDN key dim d_k / Mamba-2 state dim N; one of 16, 32, 64, 128,
+                        256 (256: no pure-write window, no key-axis scales) */
     int dv;          /* columns: GDN value dim d_v / Mamba-2 head dim P; one of 16,32,64,128,256 */
     int ngroups;     /* Mamba-2 B/C groups (divides heads); ignored for GDN */
     const int8_t* head_bits; /* host [heads]: each 4 or 8, or every entry 32 (full-precision
@@ -336,7 +337,7 @@ rsq_status rsq_allocate_bits(const double* score, int heads, int n_high, int hig
                              int low_bits, int8_t* bits_out);
 
 /* Number of partial sums R of the key-axis reduction order for a given dk
- * (host-only; 8 for every supported dk). */
+ * (host-only): 8 for dk <= 128, 16 for dk = 256. */
 int rsq_reduction_partials(int dk);
 
 /* Decode step that allocates nothing (no counterpart in the method's pages).

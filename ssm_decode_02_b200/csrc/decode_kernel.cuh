@@ -39,8 +39,14 @@ constexpr uint32_t kWaitIters = 1u << 22;  // bounded mbarrier waits (error flag
 
 template <int FAM, int DK, int UB, bool F32STATE>
 struct DecodeCfg {
-    using L = Layout<DK>;
-    static constexpr int NT = 32 * UB;         // one warp per 16-column block
+    // warps per 16-column block: one holds all rows up to d_k = 128; at d_k = 256
+    // two warps share the block, warp half hh holding the rows i with
+    // (i mod 16) div 8 = hh (the register footprint of d_k = 128)
+    static constexpr int SPLIT = DK > 128 ? 2 : 1;
+    using L = Layout<DK / SPLIT>;
+    static constexpr int RS = kR * SPLIT;      // row stride of a lane's rows
+    static constexpr int NW = UB * SPLIT;      // warps per CTA
+    static constexpr int NT = 32 * NW;
     static constexpr int UCOLS = 16 * UB;      // columns per unit
     // pipeline stages (KDA's extra pair array leaves room for three)
     static constexpr int NS = F32STATE ? 2 : ((FAM == RSQ_KDA || is_pw_family(FAM)) ? 3 : 4);
@@ -76,13 +82,19 @@ struct DecodeCfg {
     static constexpr int NPAIR = FAM == RSQ_KDA ? 4 : (DIAG ? 3 : 2);
     static constexpr int P_WARP = NPAIR * kR * PST * 8;
     static constexpr int OFF_P = NS * STAGE;
-    static constexpr int OFF_CNT = OFF_P + UB * P_WARP;  // NS release counters
+    static constexpr int OFF_CNT = OFF_P + NW * P_WARP;  // NS release counters
     static constexpr int OFF_BAR = OFF_CNT + 16;
     static constexpr int OFF_SBAR = OFF_BAR + NS * 8;  // window: "slot results ready" per stage
-    static constexpr int SMEM = OFF_SBAR + (PW ? NS * 8 : 0);
+    // d_k = 256: the two warps of a block exchange column totals (k^T S, the
+    // readout, the absmax) in three slots of 2 x 16 floats, behind one mbarrier
+    // per block (two arrivals per phase)
+    static constexpr int OFF_XCH = OFF_SBAR + (PW ? NS * 8 : 0);
+    static constexpr int OFF_XBAR = OFF_XCH + (SPLIT > 1 ? UB * 3 * 32 * 4 : 0);
+    static constexpr int SMEM = OFF_XBAR + (SPLIT > 1 ? UB * 8 : 0);
     // resident CTAs per SM the register budget is sized for: shared memory holds
     // four 128-thread CTAs per SM (4 x ~50 KB), so 128 registers per thread
-    static constexpr int MINB = F32STATE ? 1 : (NT < 128 ? 8 : 4);
+    static constexpr int MINB = F32STATE ? 1 : (NT < 128 ? 8 : 512 / NT);
+    static_assert(!PW || SPLIT == 1, "the pure-write window is built for d_k <= 128");
 };
 
 // Grid-stride walk over units without divisions: (b, h, cb) advance by the
@@ -310,19 +322,48 @@ __device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* s
     }
 }
 
-// One 16-column block of one unit, processed by warp w.
+// Two warps sharing a block (d_k = 256): combine this lane's column total v
+// (after the in-warp reduce-scatter) with the other warp's total of the same
+// column, through exchange slot `xs` (2 x 16 floats) and the block's mbarrier.
+// Both warps compute op(v_0, v_1) with operands in the same order as the
+// butterfly's last stage d = 8 (partials p and p ^ 8).  False if the bounded
+// wait ran out.
+template <class Op>
+__device__ __forceinline__ bool pair_combine(float& v, float* xs, uint32_t xbar, uint32_t& xphase, int hh,
+                                             int col16, int lane, int g, Op op) {
+    if (g < 4) xs[hh * 16 + col16] = v;  // lanes g and g ^ 4 hold the same column
+    __syncwarp();
+    if (lane == 0) mbar_arrive(xbar);
+    const bool ok = mbar_wait(xbar, xphase & 1u, kWaitIters);
+    ++xphase;
+    if (!__all_sync(0xffffffffu, ok)) return false;
+    const float other = xs[(hh ^ 1) * 16 + col16];
+    v = hh == 0 ? op(v, other) : op(other, v);
+    return true;
+}
+
+// One 16-column block of one unit, processed by warp w (with d_k = 256, by
+// warps w and w + UB, each with half of the rows).
 template <int FAM, int DK, int UB, bool F32STATE, int RND, int BITS>
 __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitIt& un, uint8_t* stage,
                                               uint8_t* smem, int stage_idx, uint32_t bar, uint32_t parity,
-                                              const Gates& gt, int w, int lane, int g, int cw) {
-    using L = Layout<DK>;
+                                              uint32_t& xphase, const Gates& gt, int w, int lane, int g,
+                                              int cw) {
     using C = DecodeCfg<FAM, DK, UB, F32STATE>;
+    using L = typename C::L;
     constexpr int RPT = L::RPT;
+    constexpr int RS = C::RS;
     constexpr int BLOCK_BYTES = DK * kBlockCols * BITS / 8;
     const bool bf16 = p.in_bf16 != 0;
     const int hu = un.hu(p);
-    const int blk = un.cb * UB + w;  // block index within the head
+    const int hh = (C::SPLIT > 1) ? w / UB : 0;  // which rows of the block (d_k = 256)
+    const int wb = (C::SPLIT > 1) ? w - hh * UB : w;  // block within the unit
+    const int gr = g + kR * hh;                  // this lane's first row
+    const int blk = un.cb * UB + wb;  // block index within the head
     const int j0 = blk * kBlockCols;  // its first column
+    const int col16 = 4 * cw + col_of(g);  // the column this lane finalises (within the block)
+    float* xs = reinterpret_cast<float*>(smem + C::OFF_XCH) + wb * 96;
+    const uint32_t xbar = smem_u32(smem + C::OFF_XBAR) + 8 * wb;
 
     // ---- this warp's copy of the key-axis vectors as duplicated pairs --------
     uint64_t* pa = reinterpret_cast<uint64_t*>(smem + C::OFF_P + w * C::P_WARP);
@@ -331,9 +372,10 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     uint64_t* pd = pc + kR * C::PST;  // KDA: alpha_i * k_i
 #pragma unroll
     for (int i = lane; i < DK; i += 32) {
+        if (C::SPLIT > 1 && ((i / kR) & 1) != hh) continue;  // the other warp's rows
         const float a = ld_vec(stage + C::OFF_VA, i, bf16);
         const float b = ld_vec(stage + C::OFF_VB, i, bf16);
-        const int pos = (i & (kR - 1)) * C::PST + i / kR;
+        const int pos = (i & (kR - 1)) * C::PST + i / RS;
         pa[pos] = pk(a, a);
         pb[pos] = pk(b, b);
         if constexpr (C::DIAG) {
@@ -368,27 +410,27 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     const uint64_t* gk = pd + g * C::PST;  // decay * k (KDA)
 
     // ---- state block -> registers (packed pairs) ------------------------------
-    const uint8_t* tile = stage + w * BLOCK_BYTES;
+    const uint8_t* tile = stage + wb * BLOCK_BYTES;
     uint64_t S2[RPT][2];
     if constexpr (BITS == 32) {
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
-            const ulonglong2 t = *reinterpret_cast<const ulonglong2*>(tile + ((g + kR * k) * 16 + 4 * cw) * 4);
+            const ulonglong2 t = *reinterpret_cast<const ulonglong2*>(tile + ((gr + RS * k) * 16 + 4 * cw) * 4);
             S2[k][0] = t.x;
             S2[k][1] = t.y;
         }
     } else {
-        load_codes<BITS, RPT>(tile, g, cw, S2);  // exact float codes c
+        load_codes<BITS, RPT, RS>(tile, gr, cw, S2);  // exact float codes c
     }
     // scales and v (GDN) / x (Mamba-2) of this lane's columns, read where needed
     // (keeping them live across the reductions costs registers)
     auto load_s4 = [&]() {
         if constexpr (BITS != 32)
-            return *reinterpret_cast<const float4*>(stage + C::OFF_SCALES + (16 * w + 4 * cw) * 4);
+            return *reinterpret_cast<const float4*>(stage + C::OFF_SCALES + (16 * wb + 4 * cw) * 4);
         else
             return make_float4(1.f, 1.f, 1.f, 1.f);
     };
-    auto load_vc = [&]() { return ld_vec4(stage + C::OFF_VC, 16 * w + 4 * cw, bf16); };
+    auto load_vc = [&]() { return ld_vec4(stage + C::OFF_VC, 16 * wb + 4 * cw, bf16); };
 
     // ---- state update ---------------------------------------------------------
     if constexpr (FAM == RSQ_GDN || C::PW) {
@@ -402,7 +444,10 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
             a01 = fma2(S2[k + 1][0], kk.y, a01);
             a23 = fma2(S2[k + 1][1], kk.y, a23);
         }
-        const float4 ck = gather_cols(reduce_scatter4(unpk4(a01, a23), g, AddOp()), cw, 0);
+        float cpart = reduce_scatter4(unpk4(a01, a23), g, AddOp());
+        if constexpr (C::SPLIT > 1)
+            if (!pair_combine(cpart, xs, xbar, xphase, hh, col16, lane, g, AddOp())) return false;
+        const float4 ck = gather_cols(cpart, cw, 0);
         // reload the k pairs below instead of keeping 16 of them live across the
         // reduction (register pressure)
         asm volatile("" ::: "memory");
@@ -467,7 +512,10 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
                 a01 = fma2(S2[k + 1][0], kk.y, a01);
                 a23 = fma2(S2[k + 1][1], kk.y, a23);
             }
-            const float4 ck = gather_cols(reduce_scatter4(unpk4(a01, a23), g, AddOp()), cw, 0);
+            float cpart = reduce_scatter4(unpk4(a01, a23), g, AddOp());
+            if constexpr (C::SPLIT > 1)
+                if (!pair_combine(cpart, xs, xbar, xphase, hh, col16, lane, g, AddOp())) return false;
+            const float4 ck = gather_cols(cpart, cw, 0);
             asm volatile("" ::: "memory");
             const float ckv[4] = {ck.x, ck.y, ck.z, ck.w};
             const float beta = gt.g1;
@@ -536,10 +584,12 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     }
     const int c = col_of(g);  // the column this lane finalises
     float o = reduce_scatter4(unpk4(o01, o23), g, AddOp());
-    if constexpr (FAM == RSQ_MAMBA2) o = __fmaf_rn(gt.D, ld_vec(stage + C::OFF_VC, 16 * w + 4 * cw + c, bf16), o);
+    if constexpr (C::SPLIT > 1)
+        if (!pair_combine(o, xs + 32, xbar, xphase, hh, col16, lane, g, AddOp())) return false;
+    if constexpr (FAM == RSQ_MAMBA2) o = __fmaf_rn(gt.D, ld_vec(stage + C::OFF_VC, 16 * wb + 4 * cw + c, bf16), o);
     if constexpr (C::PW) {
         // the window's part of the readout: o_j += b_w,j z_w in slot order
-        const float vcol = ld_vec(stage + C::OFF_VC, 16 * w + 4 * cw + c, bf16);
+        const float vcol = ld_vec(stage + C::OFF_VC, 16 * wb + 4 * cw + c, bf16);
         const uint8_t* bcol = stage + C::OFF_WB + w * C::WIN * 16 + 4 * cw + c;
         const float* bscale = reinterpret_cast<const float*>(stage + C::OFF_WBS);
 #pragma unroll
@@ -551,7 +601,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
         }
     }
     const long long col = (long long)hu * p.dv + j0 + 4 * cw + c;
-    if (g < 4) p.out[col] = o;
+    if (g < 4 && hh == 0) p.out[col] = o;
     float4 iv = make_float4(0.f, 0.f, 0.f, 0.f);
     float mine_scale = 0.f;  // the scale (lanes g < 4) or multiplier (g >= 4) of this lane's column
     if constexpr (BITS != 32) {
@@ -565,7 +615,9 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
             m2 = max3_nan(m2, fabsf(x.z), fabsf(y.z));
             m3 = max3_nan(m3, fabsf(x.w), fabsf(y.w));
         }
-        const float m = reduce_scatter4(make_float4(m0, m1, m2, m3), g, MaxOp());
+        float m = reduce_scatter4(make_float4(m0, m1, m2, m3), g, MaxOp());
+        if constexpr (C::SPLIT > 1)
+            if (!pair_combine(m, xs + 64, xbar, xphase, hh, col16, lane, g, MaxOp())) return false;
         if constexpr ((RND & kRndCopy) == 0) {
             mine_scale = scale_or_inv<BITS>(m, g);
         } else {
@@ -574,7 +626,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
             mine_scale = scale_or_inv<BITS>(__ldg(p.copy_absmax + col), g);
             if (g >= 4 && !isfinite(m)) mine_scale = -0.0f;
         }
-        if (g < 4) p.scales_out[col] = mine_scale;
+        if (g < 4 && hh == 0) p.scales_out[col] = mine_scale;
         iv = gather_cols(mine_scale, cw, 16);
     }
 
@@ -585,7 +637,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     if constexpr (BITS == 32) {
 #pragma unroll
         for (int k = 0; k < RPT; ++k)
-            *reinterpret_cast<ulonglong2*>(dst + ((g + kR * k) * 16 + 4 * cw) * 4) =
+            *reinterpret_cast<ulonglong2*>(dst + ((gr + RS * k) * 16 + 4 * cw) * 4) =
                 make_ulonglong2(S2[k][0], S2[k][1]);
     } else {
         BdrRef bdr{};
@@ -609,12 +661,13 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
                 S2[k][1] = pk(fminf(fmaxf(v.z, -mc.z), mc.z), fminf(fmaxf(v.w, -mc.w), mc.w));
             }
         }
-        requantize_store<BITS, RND, RPT>(S2, iv, dst, g, cw, gcol, un.h, un.b, p.step, p.rk, bdr);
+        requantize_store<BITS, RND, RPT, PhiloxKeys, RS>(S2, iv, dst, gr, cw, gcol, un.h, un.b, p.step, p.rk, bdr);
         // rare: a non-finite column (multiplier -0.0) is stored as the zero code
         if (is_neg_zero(iv.x) || is_neg_zero(iv.y) || is_neg_zero(iv.z) || is_neg_zero(iv.w)) {
             atomicOr(p.flag, kFlagNonFinite);
             clear_nonfinite_columns<RPT>(S2, iv);
-            requantize_store<BITS, RND, RPT>(S2, iv, dst, g, cw, gcol, un.h, un.b, p.step, p.rk, bdr);
+            requantize_store<BITS, RND, RPT, PhiloxKeys, RS>(S2, iv, dst, gr, cw, gcol, un.h, un.b, p.step, p.rk,
+                                                             bdr);
         }
     }
 
@@ -650,7 +703,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     __syncwarp();
     if (lane == 0) {
         uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + C::OFF_CNT) + stage_idx;
-        if (atomicAdd(cnt, 1u) == UB - 1) {
+        if (atomicAdd(cnt, 1u) == C::NW - 1) {
             *cnt = 0u;
             UnitIt refill = un;  // the unit NS ahead of this one
 #pragma unroll
@@ -692,6 +745,8 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_
             if constexpr (C::PW) mbar_init(smem_u32(smem + C::OFF_SBAR) + 8 * s, C::NPROD);
             cnt[s] = 0u;
         }
+        if constexpr (C::SPLIT > 1)
+            for (int b = 0; b < UB; ++b) mbar_init(smem_u32(smem + C::OFF_XBAR) + 8 * b, C::SPLIT);
         fence_mbar_init();
     }
     __syncthreads();
@@ -708,6 +763,7 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_
     if (cur.u < p.units) gt = load_gates<FAM>(p, cur);
     int stage = 0;
     uint32_t parity = 0;
+    uint32_t xphase = 0;  // phases of the block's exchange barrier (d_k = 256)
     while (cur.u < p.units) {
         UnitIt nxt = cur;
         nxt.advance(p);
@@ -722,12 +778,12 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_
         uint8_t* st = smem + stage * C::STAGE;
         bool done;
         if constexpr (F32STATE) {
-            done = process_block<FAM, DK, UB, true, 0, 32>(p, cur, st, smem, stage, bar, parity, gt, w, lane, g, cw);
+            done = process_block<FAM, DK, UB, true, 0, 32>(p, cur, st, smem, stage, bar, parity, xphase, gt, w, lane, g, cw);
         } else {
             if (p.head_bits[cur.h] == 8)
-                done = process_block<FAM, DK, UB, false, RND, 8>(p, cur, st, smem, stage, bar, parity, gt, w, lane, g, cw);
+                done = process_block<FAM, DK, UB, false, RND, 8>(p, cur, st, smem, stage, bar, parity, xphase, gt, w, lane, g, cw);
             else
-                done = process_block<FAM, DK, UB, false, RND, 4>(p, cur, st, smem, stage, bar, parity, gt, w, lane, g, cw);
+                done = process_block<FAM, DK, UB, false, RND, 4>(p, cur, st, smem, stage, bar, parity, xphase, gt, w, lane, g, cw);
         }
         if (!done) {  // a bounded wait inside the block ran out (window slot results)
             if (lane == 0) atomicOr(p.flag, kFlagTimeout);
@@ -775,6 +831,9 @@ int decode_info_family(int dk, int ub, bool f32state, int rnd, int* threads, siz
     RSQ_CASE(32, 1) RSQ_CASE(32, 2) RSQ_CASE(32, 4)
     RSQ_CASE(64, 1) RSQ_CASE(64, 2) RSQ_CASE(64, 4)
     RSQ_CASE(128, 1) RSQ_CASE(128, 2) RSQ_CASE(128, 4)
+    if constexpr (!is_pw_family(FAM)) {
+        RSQ_CASE(256, 1) RSQ_CASE(256, 2) RSQ_CASE(256, 4)
+    }
 #undef RSQ_CASE
     return -1;
 }

@@ -227,6 +227,7 @@ int launch_quantize(int dk, const QuantParams& p, void* stream) {
         case 32: rsq_quantize_kernel<32><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
         case 64: rsq_quantize_kernel<64><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
         case 128: rsq_quantize_kernel<128><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
+        case 256: rsq_quantize_kernel<256><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
         default: return static_cast<int>(cudaErrorInvalidValue);
     }
     return static_cast<int>(cudaGetLastError());
@@ -240,6 +241,7 @@ int launch_dequantize(int dk, const DequantParams& p, void* stream) {
         case 32: rsq_dequantize_kernel<32><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
         case 64: rsq_dequantize_kernel<64><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
         case 128: rsq_dequantize_kernel<128><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
+        case 256: rsq_dequantize_kernel<256><<<grid, 32 * kWarpsPerCta, 0, st>>>(p); break;
         default: return static_cast<int>(cudaErrorInvalidValue);
     }
     return static_cast<int>(cudaGetLastError());

@@ -59,7 +59,7 @@ int kernel_family(const rsq_config& c) {
 }
 bool family_ok(int f) { return f == RSQ_GDN || f == RSQ_MAMBA2 || f == RSQ_GLA || f == RSQ_KDA; }
 bool rounding_ok(int r) { return r == RSQ_RTN || r == RSQ_SR || r == RSQ_BDR || r == RSQ_SR_BDR; }
-bool dk_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128; }
+bool dk_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
 bool dv_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -103,8 +103,9 @@ const char* rsq_status_string(rsq_status s) {
 }
 
 int rsq_reduction_partials(int dk) {
-    (void)dk;
-    return rsq::kR;  // one partial per row group of a warp tile (rsq_tile.cuh)
+    // one partial per row group of a warp tile (rsq_tile.cuh); at dk = 256 two
+    // warps share a block, each with 8 row groups of its own
+    return dk > 128 ? 2 * rsq::kR : rsq::kR;
 }
 
 rsq_status rsq_allocate_bits(const double* score, int heads, int n_high, int high_bits,
@@ -132,7 +133,7 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
     if (c.batch < 1) return fail(RSQ_E_INVAL, "create: batch must be >= 1");
     if (c.heads < 1 || c.heads > RSQ_MAX_HEADS) return fail(RSQ_E_INVAL, "create: heads must be in [1, %d]", RSQ_MAX_HEADS);
     if (!dk_ok(c.dk) || !dv_ok(c.dv))
-        return fail(RSQ_E_UNSUPPORTED, "create: dk must be one of 16, 32, 64, 128 and dv one of 16, 32, 64, 128, 256 (got %d, %d)", c.dk, c.dv);
+        return fail(RSQ_E_UNSUPPORTED, "create: dk and dv must be one of 16, 32, 64, 128, 256 (got %d, %d)", c.dk, c.dv);
     if (!rounding_ok(c.rounding)) return fail(RSQ_E_INVAL, "create: bad rounding %d", c.rounding);
     if (c.in_dtype != RSQ_F32 && c.in_dtype != RSQ_BF16) return fail(RSQ_E_INVAL, "create: bad in_dtype %d", c.in_dtype);
     if (c.family == RSQ_MAMBA2 && (c.ngroups < 1 || c.heads % c.ngroups != 0))
@@ -148,6 +149,8 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
         return fail(RSQ_E_INVAL, "create: set both alloc and release, or neither");
     if (c.key_axis && (c.family != RSQ_GDN || c.window || (c.rounding != RSQ_RTN && c.rounding != RSQ_SR)))
         return fail(RSQ_E_UNSUPPORTED, "create: key-axis scales: Gated DeltaNet, no window, nearest or stochastic rounding");
+    if ((c.window || c.key_axis) && c.dk > 128)
+        return fail(RSQ_E_UNSUPPORTED, "create: the pure-write window and key-axis scales are built for dk <= 128");
 
     rsq_ctx* ctx = new (std::nothrow) rsq_ctx();
     if (!ctx) return fail(RSQ_E_NOMEM, "create: host allocation failed");

@@ -107,14 +107,15 @@ __device__ __forceinline__ bool is_neg_zero(float x) { return __float_as_uint(x)
 
 // Decode this lane's RPT rows of 4 codes of a stored block into exact float
 // codes, kept as packed pairs: S2[k][0] = columns 0,1 and S2[k][1] = columns
-// 2,3 of row g + 8k.
-template <int BITS, int RPT>
+// 2,3 of row g + RS k (g: the lane's first row; RS: the row stride, 8 when one
+// warp holds every row of the block, 16 when two warps share it).
+template <int BITS, int RPT, int RS = kR>
 __device__ __forceinline__ void load_codes(const uint8_t* blk, int g, int cw, uint64_t (&S2)[RPT][2]) {
     if constexpr (BITS == 8) {
         const uint64_t off = pk(-(kMagic + 128.0f), -(kMagic + 128.0f));
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
-            const uint32_t w = *reinterpret_cast<const uint32_t*>(blk + (g + kR * k) * 16 + 4 * cw);
+            const uint32_t w = *reinterpret_cast<const uint32_t*>(blk + (g + RS * k) * 16 + 4 * cw);
             const uint64_t f01 = pk(__uint_as_float(prmt(w, kMagicBits, 0x7650u)),
                                     __uint_as_float(prmt(w, kMagicBits, 0x7651u)));
             const uint64_t f23 = pk(__uint_as_float(prmt(w, kMagicBits, 0x7652u)),
@@ -126,7 +127,7 @@ __device__ __forceinline__ void load_codes(const uint8_t* blk, int g, int cw, ui
         const uint64_t off = pk(-(kMagic + 8.0f), -(kMagic + 8.0f));
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
-            const uint32_t h16 = *reinterpret_cast<const uint16_t*>(blk + (g + kR * k) * 8 + 2 * cw);
+            const uint32_t h16 = *reinterpret_cast<const uint16_t*>(blk + (g + RS * k) * 8 + 2 * cw);
             const uint32_t lo = h16 & 0x0F0Fu;         // columns 0 and 2
             const uint32_t hi = (h16 >> 4) & 0x0F0Fu;  // columns 1 and 3
             const uint64_t f01 = pk(__uint_as_float(prmt(lo, kMagicBits, 0x7650u)),
@@ -139,15 +140,15 @@ __device__ __forceinline__ void load_codes(const uint8_t* blk, int g, int cw, ui
     }
 }
 
-// Exact float codes of row g + 8k of a stored block (this lane's 4 columns).
-template <int BITS>
+// Exact float codes of row g + RS k of a stored block (this lane's 4 columns).
+template <int BITS, int RS = kR>
 __device__ __forceinline__ void load_code_row(const uint8_t* blk, int g, int cw, int k, uint64_t& c01,
                                               uint64_t& c23) {
     uint64_t S2[1][2];
     if constexpr (BITS == 8)
-        load_codes<8, 1>(blk + kR * k * 16, g, cw, S2);
+        load_codes<8, 1>(blk + RS * k * 16, g, cw, S2);
     else
-        load_codes<4, 1>(blk + kR * k * 8, g, cw, S2);
+        load_codes<4, 1>(blk + RS * k * 8, g, cw, S2);
     c01 = S2[0][0];
     c23 = S2[0][1];
 }
@@ -212,8 +213,10 @@ __device__ __forceinline__ float bdr_pick(float S, float prev, float now, float 
 //        Philox4x32-10 with counter {i mod dk/2 | (j/4) << 16, h, b, step}.
 //   +BDR: the base code is replaced by ceil / floor of the exact S*inv when it
 //        moves the element opposite to its update (see bdr_pick).
-// `gcol` is j/4 of this lane's first column.
-template <int BITS, int RND, int RPT, class PhiloxKeysT>
+// `gcol` is j/4 of this lane's first column; the lane's rows are g + RS k
+// (RS: as for load_codes; RS * RPT / 2 = dk / 2, so rows k and k + RPT/2 are
+// the pair i, i + dk/2 that one Philox call serves).
+template <int BITS, int RND, int RPT, class PhiloxKeysT, int RS = kR>
 __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], const float4& iv,
                                                  uint8_t* dst, int g, int cw, uint32_t gcol,
                                                  uint32_t h, uint32_t b, uint32_t step,
@@ -222,13 +225,13 @@ __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], c
     constexpr bool BDR = (RND & kRndBdr) != 0;
     constexpr float kOff = (BITS == 8) ? 128.0f : 8.0f;  // stored code = c + kOff
     const uint64_t inv01 = pk(iv.x, iv.y), inv23 = pk(iv.z, iv.w);
-    // this lane's first row; row k sits k * 8 rows further
+    // this lane's first row; row k sits k * RS rows further
     uint8_t* const row0 = dst + (BITS == 8 ? g * 16 + 4 * cw : g * 8 + 2 * cw);
     auto store_row = [&](int k, uint32_t word) {
         if constexpr (BITS == 8)
-            *reinterpret_cast<uint32_t*>(row0 + k * (kR * 16)) = word;
+            *reinterpret_cast<uint32_t*>(row0 + k * (RS * 16)) = word;
         else
-            *reinterpret_cast<uint16_t*>(row0 + k * (kR * 8)) = static_cast<uint16_t>(word);
+            *reinterpret_cast<uint16_t*>(row0 + k * (RS * 8)) = static_cast<uint16_t>(word);
     };
     const uint64_t moff = pk(kMagic + kOff, kMagic + kOff);
     // Row k with its base codes T = c + M + kOff (two packed pairs): apply the
@@ -237,7 +240,7 @@ __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], c
         if constexpr (BDR) {
             const uint64_t nmoff = pk(-(kMagic + kOff), -(kMagic + kOff));
             uint64_t c01, c23;
-            load_code_row<BITS>(bdr.old_block, g, cw, k, c01, c23);
+            load_code_row<BITS, RS>(bdr.old_block, g, cw, k, c01, c23);
             const float4 prev = unpk4(mul2(c01, bdr.s_old01), mul2(c23, bdr.s_old23));
             const float4 now = unpk4(mul2(add2(T01, nmoff), bdr.s_new01), mul2(add2(T23, nmoff), bdr.s_new23));
             const float4 tu = unpk4(fma2_rp(S2[k][0], inv01, moff), fma2_rp(S2[k][1], inv23, moff));
@@ -261,7 +264,7 @@ __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], c
         const uint64_t mm = pk(kMagic, kMagic);
 #pragma unroll
         for (int k = 0; k < RPT / 2; ++k) {
-            const uint32_t i = static_cast<uint32_t>(g + kR * k);  // i < dk/2; partner i + dk/2
+            const uint32_t i = static_cast<uint32_t>(g + RS * k);  // i < dk/2; partner i + dk/2
             const U4 rnd = philox4x32_10(U4{i | (gcol << 16), h, b, step}, rk.k0, rk.k1);
             const uint32_t u[2][2] = {{rnd.x, rnd.y}, {rnd.z, rnd.w}};
 #pragma unroll

@@ -53,7 +53,9 @@ def _create(**kw):
     (dict(heads=0), rsq.RSQ_E_INVAL),
     (dict(heads=rsq.RSQ_MAX_HEADS + 1), rsq.RSQ_E_INVAL),
     (dict(dk=100), rsq.RSQ_E_UNSUPPORTED),
-    (dict(dk=256), rsq.RSQ_E_UNSUPPORTED),
+    (dict(dk=512), rsq.RSQ_E_UNSUPPORTED),
+    (dict(dk=256, window=8), rsq.RSQ_E_UNSUPPORTED),
+    (dict(dk=256, key_axis=1), rsq.RSQ_E_UNSUPPORTED),
     (dict(dv=8), rsq.RSQ_E_UNSUPPORTED),
     (dict(rounding=4), rsq.RSQ_E_INVAL),
     (dict(rounding=-1), rsq.RSQ_E_INVAL),
@@ -88,7 +90,7 @@ def test_null_arguments_rejected():
 
 
 def test_reduction_partials():
-    assert [rsq.rsq_reduction_partials(d) for d in (16, 32, 64, 128)] == [8, 8, 8, 8]
+    assert [rsq.rsq_reduction_partials(d) for d in (16, 32, 64, 128, 256)] == [8, 8, 8, 8, 16]
 
 
 def test_allocate_bits_matches_oracle_brute_force():

@@ -59,6 +59,23 @@ def test_gdn_fp32_state_matches_closed_form(mode):
                 assert _rel(o[0, h].astype(np.float64), o_ref) <= 1e-5
 
 
+@pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
+def test_gdn_fp32_state_matches_closed_form_dk256(mode):
+    """The benchmark spec (a) at d_k = 256, with the 16-partial canonical order the
+    library uses there (rsq_reduction_partials(256) = 16)."""
+    w = dataclasses.replace(TINY, B=1, H=2, dk=256, dv=32)
+    ins = [W.gdn_inputs(w, t) for t in range(6)]
+    bits = np.full(w.H, 32, np.int8)
+    st = oracle.zero_state(w.B, w.H, w.dk, w.dv)
+    for t in range(6):
+        st, o = oracle.gdn_step(st, ins[t], bits, rounding=oracle.RTN, seed=0, step=t, mode=mode, R=16)
+        for h in range(w.H):
+            S_ref = _gdn_closed_form(ins, t + 1, 0, h)
+            assert _rel(st["f"][0, h].astype(np.float64), S_ref) <= 1e-5
+            o_ref = S_ref.T @ ins[t]["q"][0, h].astype(np.float64)
+            assert _rel(o[0, h].astype(np.float64), o_ref) <= 1e-5
+
+
 def _mamba_closed_form(ins, t_end, b, h, D):
     """S_t = sum_tau (prod_{s>tau} exp(dt_s A)) dt_tau B_tau x_tau^T;  y_t = S_t^T C_t + D x_t."""
     S = np.zeros((ins[0]["Bm"].shape[-1], ins[0]["x"].shape[-1]))
