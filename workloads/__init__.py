@@ -74,6 +74,12 @@ EXTRA_WORKLOADS = [
              input_seed=5, sr_seed=1005),
     Workload("kda_b64_h16_d128_int8_sr", "kda", 64, 16, 128, 128, 1024, "int8", "sr", "bf16",
              input_seed=6, sr_seed=1006),
+    # d_k = 256 (two warps per block): Gated DeltaNet with 256-wide heads, and
+    # Mamba-2 with a 256-wide SSM state (N = 256)
+    Workload("gdn_b64_h8_d256_int8_sr", "gdn", 64, 8, 256, 256, 1024, "int8", "sr", "bf16",
+             input_seed=7, sr_seed=1007),
+    Workload("mamba2_b128_h80_p64_n256_int8_sr", "mamba2", 128, 80, 256, 64, 512, "int8", "sr",
+             "bf16", input_seed=8, sr_seed=1008),
 ]
 BY_NAME = {w.name: w for w in WORKLOADS + EXTRA_WORKLOADS}
 
