@@ -10,6 +10,9 @@
 // accumulated in increasing i, then combined by the XOR butterfly over p with
 // d = 1, 2, 4 -- shuffles across lanes 4, 8, 16 apart.  A warp-wide shared load
 // of one row per lane group reads 8 consecutive rows: no bank conflicts.
+// The decode kernel at dk = 256 splits a block over two warps: each lane then
+// holds the rows g + 8hh + 16k (row stride RS = 16), giving R = 16 partials
+// p = i mod 16; the helpers below take the lane's first row and RS.
 #pragma once
 
 #include "rsq_device.cuh"

@@ -114,16 +114,21 @@ CASES = [
     ("gdn_b64_h16_d128_int8_sr", 2, 3, 64, 64, [32, 32, 32], rsq.RSQ_SR, 1),
     ("gla_b64_h16_d128_int8_sr", 2, 3, 32, 64, [8, 4, 8], rsq.RSQ_BDR, 1),
     ("kda_b64_h16_d128_int8_sr", 3, 2, 64, 32, [4, 8], rsq.RSQ_SR, 1),
+    ("gdn_b64_h8_d256_int8_sr", 3, 3, 256, 16, [8, 4, 8], rsq.RSQ_SR_BDR, 1),   # two warps per block
+    ("gdn_b64_h8_d256_int8_sr", 2, 2, 256, 64, [32, 32], rsq.RSQ_SR, 1),
+    ("kda_b64_h16_d128_int8_sr", 2, 3, 256, 32, [4, 8, 4], rsq.RSQ_SR, 1),
 ]
 
 
-@pytest.mark.parametrize("case", range(len(CASES) + 1))
+@pytest.mark.parametrize("case", range(len(CASES) + 2))
 def test_decode_step_stays_inside_its_buffers(case):
     if case < len(CASES):
         name, B, H, dk, dv, bits, rnd, ng = CASES[case]
         base = W.BY_NAME[name]
-    else:  # Mamba-2 with shared B/C groups and a ragged group count
+    elif case == len(CASES):  # Mamba-2 with shared B/C groups and a ragged group count
         base, B, H, dk, dv, bits, rnd, ng = W.WORKLOADS[3], 2, 6, 32, 64, [8, 4, 8, 4, 4, 8], rsq.RSQ_SR, 3
+    else:  # Mamba-2 with a 256-wide state
+        base, B, H, dk, dv, bits, rnd, ng = W.WORKLOADS[3], 2, 4, 256, 32, [8, 4, 4, 8], rsq.RSQ_RTN, 2
     w = dataclasses.replace(base, B=B, H=H, dk=dk, dv=dv, ngroups=ng)
     bits = np.array(bits, np.int8)
     run = Run(w, bits, rounding=rnd)

@@ -26,11 +26,14 @@ def _copy(s: rsq.State) -> rsq.State:
     return rsq.State(s.codes.clone(), s.scales.clone())
 
 
-@pytest.mark.parametrize("family", ["gdn", "mamba2"])
+@pytest.mark.parametrize("family", ["gdn", "mamba2", "gdn_dk256"])
 def test_noalloc_step_matches_context_step_twice(family):
     if family == "gdn":
         w = dataclasses.replace(W.WORKLOADS[1], B=6, H=8)
         bits = np.array([8, 4, 8, 4, 4, 8, 4, 4], np.int8)
+    elif family == "gdn_dk256":
+        w = dataclasses.replace(W.WORKLOADS[1], B=3, H=4, dk=256, dv=64)
+        bits = np.array([8, 4, 4, 8], np.int8)
     else:
         w = dataclasses.replace(W.WORKLOADS[3], B=3, H=8)
         bits = np.full(8, 8, np.int8)
