@@ -486,57 +486,37 @@ def run_ours(args, w: W.Workload):
     del hot
 
     # end-to-end through the public API with host buffers (pinned), per step:
-    # H2D of that step's inputs (one packed buffer), the decode step, D2H of its
-    # output.  Copies run on their own streams and overlap the neighbouring
-    # steps' kernels (double-buffered inputs and outputs), as a server would.
+    # the library's host-buffer pipeline (rsq_pipe) copies the step's packed
+    # inputs in, runs the decode step and copies its output back, with three
+    # steps in flight on its own copy-in / compute / copy-out streams, as a
+    # server would.  Timed with events on the pipe's streams.
     n_e2e = max(2, min(args.steps, 500))
-    packed = [_pack_inputs(W.inputs(w, rank_input_step(200000 + t, rank))) for t in range(4)]
-    h2d = packed[0][0].numel()
-    dev_buf = [torch.empty(h2d, dtype=torch.uint8, device=dev) for _ in range(2)]
-    dev_views = [_unpack_views(buf, packed[0][1]) for buf in dev_buf]
-    e2e_structs = [_inputs_struct(rsq, w, v) for v in dev_views]
-    out_dev = [torch.empty((w.B, w.H, w.dv), dtype=torch.float32, device=dev) for _ in range(2)]
-    out_host = [torch.empty((w.B, w.H, w.dv), dtype=torch.float32, pin_memory=True) for _ in range(2)]
-    d2h = out_host[0].numel() * 4
-    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
-    ev_copied = [torch.cuda.Event() for _ in range(2)]
-    ev_done = [torch.cuda.Event() for _ in range(2)]
-    ev_read = [torch.cuda.Event() for _ in range(2)]
+    pipe = rsq.Pipe(ctx)
+    host_in = [rsq.pack_host_inputs(ctx, W.inputs(w, rank_input_step(200000 + t, rank))) for t in range(4)]
+    h2d = host_in[0].numel()
+    host_out = [torch.empty((w.B, w.H, w.dv), dtype=torch.float32, pin_memory=True) for _ in range(4)]
+    d2h = host_out[0].numel() * 4
+    s_in = torch.cuda.ExternalStream(pipe.copy_in, device=dev)
+    s_out = torch.cuda.ExternalStream(pipe.copy_out, device=dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-
-    def e2e_step(t, i):
-        if wins is None:
-            ctx.decode_step(states[0], states[0], e2e_structs[i], out_dev[i], t, stream.cuda_stream)
-        else:
-            ctx.decode_step_window(states[0], states[0], wins[0][t % 2], wins[0][(t + 1) % 2],
-                                   e2e_structs[i], out_dev[i], t, stream.cuda_stream)
-
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     nvtx.range_push("rsq.e2e")
     e0.record(s_in)
     for t in range(n_e2e):
-        i = t % 2
-        with torch.cuda.stream(s_in):
-            if t >= 2:
-                s_in.wait_event(ev_done[i])          # step t-2 has consumed dev_buf[i]
-            dev_buf[i].copy_(packed[t % 4][0], non_blocking=True)
-            ev_copied[i].record(s_in)
-        stream.wait_event(ev_copied[i])
-        if t >= 2:
-            stream.wait_event(ev_read[i])            # out_dev[i] of step t-2 has been read back
-        e2e_step(args.warmup + args.steps + t, i)
-        ev_done[i].record(stream)
-        with torch.cuda.stream(s_out):
-            s_out.wait_event(ev_done[i])
-            out_host[i].copy_(out_dev[i], non_blocking=True)
-            ev_read[i].record(s_out)
-    s_in.wait_stream(stream)
-    s_in.wait_stream(s_out)
-    e1.record(s_in)
+        step_t = args.warmup + args.steps + t
+        if wins is None:
+            pipe.step(states[0], states[0], host_in[t % 4], host_out[t % 4], step_t)
+        else:
+            pipe.step(states[0], states[0], host_in[t % 4], host_out[t % 4], step_t,
+                      wins[0][t % 2], wins[0][(t + 1) % 2])
+    # the last output copy follows every earlier copy and kernel of the pipe
+    e1.record(s_out)
     nvtx.range_pop()
     e1.synchronize()
+    pipe.sync()
+    pipe.close()
     e2e_elapsed = max_over_ranks(e0.elapsed_time(e1) / 1e3, dist if world > 1 else None, dev)
 
     hu_step = w.B * w.H
@@ -762,33 +742,6 @@ def _to_pinned(a: np.ndarray):
     if a.dtype == np.uint16:
         a = a.view(np.int16)
     return torch.from_numpy(a.copy()).pin_memory()
-
-
-def _pack_inputs(host: dict):
-    """One pinned host buffer holding every input array of a step, each at a
-    16-byte aligned offset; returns (buffer, [(name, offset, shape, dtype)])."""
-    import torch
-    layout, off = [], 0
-    for k, v in host.items():
-        a = np.ascontiguousarray(v)
-        layout.append((k, off, a.shape, a.dtype))
-        off += (a.nbytes + 15) // 16 * 16
-    buf = np.zeros(off, np.uint8)
-    for (k, o, shape, dt), v in zip(layout, host.values()):
-        a = np.ascontiguousarray(v)
-        buf[o:o + a.nbytes] = a.view(np.uint8).ravel()
-    return torch.from_numpy(buf).pin_memory(), layout
-
-
-def _unpack_views(buf, layout) -> dict:
-    """Typed views into a packed device buffer (same layout as _pack_inputs)."""
-    import torch
-    tmap = {np.dtype(np.float32): torch.float32, np.dtype(np.uint16): torch.int16}
-    out = {}
-    for k, o, shape, dt in layout:
-        n = int(np.prod(shape)) * np.dtype(dt).itemsize
-        out[k] = buf[o:o + n].view(tmap[np.dtype(dt)]).view(shape)
-    return out
 
 
 def _inputs_struct(rsq, w: W.Workload, d: dict):

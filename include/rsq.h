@@ -363,6 +363,45 @@ rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_state* state
                                    const rsq_state* state_out, const void* inputs, float* out,
                                    uint32_t step, void* stream);
 
+/* End-to-end pipeline over host buffers (no counterpart in the method's pages:
+ * the serving-side plumbing of the decode step).
+ *
+ * rsq_host_input_layout: one step's inputs packed in one host buffer, the
+ *   arrays of the family's input struct in its field order, each starting at
+ *   a 16-byte aligned offset: GDN q, k, v, alpha, beta; GLA / KDA q, k, v,
+ *   alpha (float [B][H][dk]), beta (GLA: 0 bytes); Mamba-2 x, Bm, Cm, dt, A, D
+ *   (the decay is computed on the device).  Array shapes and types as in the
+ *   input structs above.  offsets[6], sizes[6]: host arrays filled with each
+ *   field's byte offset and byte count (unused entries 0); *total: the buffer
+ *   size.  Host-only.
+ * rsq_pipe_create: three non-blocking streams (input copy, compute, output
+ *   copy), events and device staging for 3 steps in flight, on the current
+ *   device (RSQ_E_NOMEM / RSQ_E_CUDA).  The pipe borrows ctx: destroy the pipe
+ *   first.
+ * rsq_pipe_step: one decode step.  Copies host_inputs (the packed layout;
+ *   page-locked memory for the copies to overlap) to the device, runs
+ *   rsq_decode_step (rsq_decode_step_window with win_in / win_out for a window
+ *   context, else both NULL) on the compute stream, and copies the output
+ *   [B][H][dv] to host_out.  Returns once the work is queued; when the pipe
+ *   already has 3 steps in flight it first waits for the oldest to finish, so
+ *   the host buffers of step n may be reused once step n + 3 has been issued
+ *   (or after rsq_pipe_sync).  The states are read and written on the compute
+ *   stream, in step order; a caller using them on another stream orders it
+ *   against rsq_pipe_streams' compute stream.  Errors as rsq_decode_step.
+ * rsq_pipe_sync: wait for every queued step.
+ * rsq_pipe_streams: the pipe's three streams (cudaStream_t), e.g. to time it
+ *   with events.  rsq_pipe_destroy waits for the pipe's work, then frees it
+ *   (NULL is a no-op). */
+typedef struct rsq_pipe rsq_pipe;
+rsq_status rsq_host_input_layout(const rsq_ctx* ctx, size_t* offsets, size_t* sizes, size_t* total);
+rsq_status rsq_pipe_create(const rsq_ctx* ctx, rsq_pipe** out);
+void rsq_pipe_destroy(rsq_pipe* pipe);
+rsq_status rsq_pipe_step(rsq_pipe* pipe, const rsq_state* state_in, const rsq_state* state_out,
+                         const rsq_window* win_in, const rsq_window* win_out, const void* host_inputs,
+                         float* host_out, uint32_t step);
+rsq_status rsq_pipe_sync(rsq_pipe* pipe);
+rsq_status rsq_pipe_streams(const rsq_pipe* pipe, void** copy_in, void** compute, void** copy_out);
+
 const char* rsq_status_string(rsq_status s);
 const char* rsq_last_error(void);
 const char* rsq_version(void);

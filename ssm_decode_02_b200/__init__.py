@@ -108,6 +108,14 @@ def _load():
         "rsq_decode_step_window": ([P, ctypes.POINTER(rsq_state), ctypes.POINTER(rsq_state),
                                     ctypes.POINTER(rsq_window), ctypes.POINTER(rsq_window), P, P,
                                     ctypes.c_uint32, P], C),
+        "rsq_host_input_layout": ([P, ctypes.POINTER(ctypes.c_size_t), ctypes.POINTER(ctypes.c_size_t),
+                                   ctypes.POINTER(ctypes.c_size_t)], C),
+        "rsq_pipe_create": ([P, ctypes.POINTER(P)], C),
+        "rsq_pipe_destroy": ([P], None),
+        "rsq_pipe_step": ([P, ctypes.POINTER(rsq_state), ctypes.POINTER(rsq_state), ctypes.POINTER(rsq_window),
+                           ctypes.POINTER(rsq_window), P, P, ctypes.c_uint32], C),
+        "rsq_pipe_sync": ([P], C),
+        "rsq_pipe_streams": ([P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P)], C),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -155,6 +163,21 @@ def _dptr(t) -> int | None:
     if not t.is_contiguous():
         raise ValueError("expected a contiguous CUDA tensor")
     return int(t.data_ptr())
+
+
+def _hptr(t) -> int:
+    """Host address of a host buffer argument (numpy array or CPU tensor); a CUDA
+    tensor is refused here."""
+    if getattr(t, "is_cuda", False):
+        raise ValueError("expected a host buffer, got a CUDA tensor")
+    if isinstance(t, np.ndarray) and not t.flags.c_contiguous:
+        raise ValueError("expected a contiguous host buffer")
+    if hasattr(t, "is_contiguous") and not t.is_contiguous():
+        raise ValueError("expected a contiguous host buffer")
+    p = _ptr(t)
+    if not p:
+        raise ValueError("null host buffer")
+    return p
 
 
 def _stream(stream) -> int | None:
@@ -272,6 +295,45 @@ def rsq_decode_step_window(ctx: int, state_in, state_out, win_in, win_out, input
     _check(lib.rsq_decode_step_window(ctx, ctypes.byref(si), ctypes.byref(so), ctypes.byref(wi),
                                       ctypes.byref(wo), ctypes.byref(inputs), _dptr(out),
                                       int(step) & 0xFFFFFFFF, _stream(stream)))
+
+
+def rsq_host_input_layout(ctx: int) -> tuple[list[int], list[int], int]:
+    """(offsets, sizes, total) of the packed host input buffer of one step."""
+    off = (ctypes.c_size_t * 6)()
+    size = (ctypes.c_size_t * 6)()
+    total = ctypes.c_size_t()
+    _check(lib.rsq_host_input_layout(ctx, off, size, ctypes.byref(total)))
+    return list(off), list(size), int(total.value)
+
+
+def rsq_pipe_create(ctx: int) -> int:
+    out = ctypes.c_void_p()
+    _check(lib.rsq_pipe_create(ctx, ctypes.byref(out)))
+    return int(out.value)
+
+
+def rsq_pipe_destroy(pipe: int) -> None:
+    lib.rsq_pipe_destroy(pipe)
+
+
+def rsq_pipe_step(pipe: int, state_in, state_out, host_inputs, host_out, step: int, win_in=None,
+                  win_out=None) -> None:
+    """host_inputs: the packed host buffer (pack_host_inputs); host_out: host float [B][H][dv]."""
+    si, so = _state(state_in), _state(state_out)
+    wi = ctypes.byref(_window(win_in)) if win_in is not None else None
+    wo = ctypes.byref(_window(win_out)) if win_out is not None else None
+    _check(lib.rsq_pipe_step(pipe, ctypes.byref(si), ctypes.byref(so), wi, wo, _hptr(host_inputs),
+                             _hptr(host_out), int(step) & 0xFFFFFFFF))
+
+
+def rsq_pipe_sync(pipe: int) -> None:
+    _check(lib.rsq_pipe_sync(pipe))
+
+
+def rsq_pipe_streams(pipe: int) -> tuple[int, int, int]:
+    a, b, c = ctypes.c_void_p(), ctypes.c_void_p(), ctypes.c_void_p()
+    _check(lib.rsq_pipe_streams(pipe, ctypes.byref(a), ctypes.byref(b), ctypes.byref(c)))
+    return int(a.value), int(b.value), int(c.value)
 
 
 def rsq_quantize(ctx: int, S, state_out, step: int, stream=None) -> None:
@@ -417,3 +479,51 @@ class Context:
 
     def check_flags(self, stream=None) -> int:
         return rsq_check_flags(self.ctx, stream)
+
+
+def pack_host_inputs(ctx: "Context", inputs: dict, out=None):
+    """Pack one step's host input arrays (numpy; bf16 as uint16 bits) into the
+    library's host layout (rsq_host_input_layout), in page-locked memory.
+    Marshalling only: each array is copied byte for byte to its offset."""
+    import torch
+    names = (("x", "Bm", "Cm", "dt", "A", "D") if ctx.family == RSQ_MAMBA2
+             else ("q", "k", "v", "alpha", "beta"))
+    off, size, total = rsq_host_input_layout(ctx.ctx)
+    if out is None:
+        out = torch.empty(total, dtype=torch.uint8, pin_memory=True)
+    buf = out.numpy()
+    for f, name in enumerate(names):
+        if size[f] == 0:
+            continue
+        a = np.ascontiguousarray(inputs[name]).reshape(-1).view(np.uint8)
+        if a.size != size[f]:
+            raise ValueError("input %s has %d bytes, the layout expects %d" % (name, a.size, size[f]))
+        buf[off[f]:off[f] + size[f]] = a
+    return out
+
+
+class Pipe:
+    """An end-to-end pipeline over host buffers for one Context (rsq_pipe)."""
+
+    def __init__(self, ctx: "Context"):
+        self.context = ctx  # the pipe borrows the context: keep it alive
+        self.pipe = rsq_pipe_create(ctx.ctx)
+        self.copy_in, self.compute, self.copy_out = rsq_pipe_streams(self.pipe)
+
+    def step(self, state_in: State, state_out: State, host_inputs, host_out, step: int, win_in=None,
+             win_out=None):
+        rsq_pipe_step(self.pipe, state_in, state_out, host_inputs, host_out, step, win_in, win_out)
+
+    def sync(self):
+        rsq_pipe_sync(self.pipe)
+
+    def close(self):
+        if getattr(self, "pipe", None):
+            rsq_pipe_destroy(self.pipe)
+            self.pipe = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

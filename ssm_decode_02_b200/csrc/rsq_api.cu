@@ -632,3 +632,173 @@ extern "C" rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_s
     ctx.flag = scratch;
     return rsq_decode_step(&ctx, state_in, state_out, inputs, out, step, stream);
 }
+
+// ---------------------------------------------------------------------------
+// Host-buffer pipeline (rsq_pipe): one call per step copies the step's packed
+// inputs host -> device, runs the decode step and copies the output back, on
+// three streams ordered by events, so step t's input copy, step t-1's kernel
+// and step t-2's output copy overlap.  Device staging is owned by the pipe.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr int kPipeDepth = 3;   // steps in flight (staging and output buffers)
+constexpr int kHostFields = 6;  // largest input struct (Mamba-2 without decay)
+
+size_t round16(size_t n) { return (n + 15) / 16 * 16; }
+
+// Byte sizes of the host input fields of a context, in its input struct's
+// field order (unused entries 0).
+void host_field_sizes(const rsq_config& c, size_t sizes[kHostFields]) {
+    const size_t esz = (c.in_dtype == RSQ_BF16) ? 2 : 4;
+    const size_t bh = static_cast<size_t>(c.batch) * c.heads;
+    for (int f = 0; f < kHostFields; ++f) sizes[f] = 0;
+    if (c.family == RSQ_MAMBA2) {
+        const size_t bg = static_cast<size_t>(c.batch) * c.ngroups;
+        sizes[0] = bh * c.dv * esz;  // x
+        sizes[1] = bg * c.dk * esz;  // B
+        sizes[2] = bg * c.dk * esz;  // C
+        sizes[3] = bh * 4;           // dt
+        sizes[4] = static_cast<size_t>(c.heads) * 4;  // A
+        sizes[5] = static_cast<size_t>(c.heads) * 4;  // D
+        return;
+    }
+    sizes[0] = bh * c.dk * esz;  // q
+    sizes[1] = bh * c.dk * esz;  // k
+    sizes[2] = bh * c.dv * esz;  // v
+    sizes[3] = (c.family == RSQ_GDN) ? bh * 4 : bh * c.dk * 4;  // alpha: gate / decay per key channel
+    sizes[4] = (c.family == RSQ_GLA) ? 0 : bh * 4;              // beta
+}
+
+}  // namespace
+
+struct rsq_pipe {
+    const rsq_ctx* ctx;
+    size_t off[kHostFields], size[kHostFields];
+    size_t in_bytes, out_bytes;
+    uint8_t* stage[kPipeDepth];
+    float* out_dev[kPipeDepth];
+    cudaStream_t s_in, s_cmp, s_out;
+    cudaEvent_t copied[kPipeDepth], done[kPipeDepth], read[kPipeDepth];
+    unsigned long long issued;
+};
+
+rsq_status rsq_host_input_layout(const rsq_ctx* ctx, size_t* offsets, size_t* sizes, size_t* total) {
+    if (!ctx || !offsets || !sizes || !total) return fail(RSQ_E_INVAL, "host_input_layout: null argument");
+    host_field_sizes(ctx->cfg, sizes);
+    size_t off = 0;
+    for (int f = 0; f < kHostFields; ++f) {
+        offsets[f] = off;
+        off += round16(sizes[f]);
+    }
+    *total = off;
+    return RSQ_OK;
+}
+
+void rsq_pipe_destroy(rsq_pipe* pipe) {
+    if (!pipe) return;
+    if (pipe->s_out) cudaStreamSynchronize(pipe->s_out);
+    if (pipe->s_cmp) cudaStreamSynchronize(pipe->s_cmp);
+    if (pipe->s_in) cudaStreamSynchronize(pipe->s_in);
+    for (int i = 0; i < kPipeDepth; ++i) {
+        if (pipe->stage[i]) cudaFree(pipe->stage[i]);
+        if (pipe->out_dev[i]) cudaFree(pipe->out_dev[i]);
+        if (pipe->copied[i]) cudaEventDestroy(pipe->copied[i]);
+        if (pipe->done[i]) cudaEventDestroy(pipe->done[i]);
+        if (pipe->read[i]) cudaEventDestroy(pipe->read[i]);
+    }
+    if (pipe->s_in) cudaStreamDestroy(pipe->s_in);
+    if (pipe->s_cmp) cudaStreamDestroy(pipe->s_cmp);
+    if (pipe->s_out) cudaStreamDestroy(pipe->s_out);
+    delete pipe;
+}
+
+rsq_status rsq_pipe_create(const rsq_ctx* ctx, rsq_pipe** out) {
+    if (!ctx || !out) return fail(RSQ_E_INVAL, "pipe_create: null argument");
+    *out = nullptr;
+    rsq_pipe* p = new (std::nothrow) rsq_pipe();
+    if (!p) return fail(RSQ_E_NOMEM, "pipe_create: host allocation failed");
+    p->ctx = ctx;
+    size_t total = 0;
+    rsq_host_input_layout(ctx, p->off, p->size, &total);
+    p->in_bytes = total;
+    p->out_bytes = static_cast<size_t>(ctx->cfg.batch) * ctx->cfg.heads * ctx->cfg.dv * sizeof(float);
+    int err = cudaStreamCreateWithFlags(&p->s_in, cudaStreamNonBlocking);
+    if (!err) err = cudaStreamCreateWithFlags(&p->s_cmp, cudaStreamNonBlocking);
+    if (!err) err = cudaStreamCreateWithFlags(&p->s_out, cudaStreamNonBlocking);
+    for (int i = 0; i < kPipeDepth && !err; ++i) {
+        err = cudaMalloc(&p->stage[i], p->in_bytes);
+        if (!err) err = cudaMalloc(&p->out_dev[i], p->out_bytes);
+        if (!err) err = cudaEventCreateWithFlags(&p->copied[i], cudaEventDisableTiming);
+        if (!err) err = cudaEventCreateWithFlags(&p->done[i], cudaEventDisableTiming);
+        if (!err) err = cudaEventCreateWithFlags(&p->read[i], cudaEventDisableTiming);
+    }
+    if (err) {
+        rsq_pipe_destroy(p);
+        if (err == cudaErrorMemoryAllocation) return fail(RSQ_E_NOMEM, "pipe_create: device allocation failed");
+        return cuda_fail(err, "pipe_create");
+    }
+    *out = p;
+    return RSQ_OK;
+}
+
+rsq_status rsq_pipe_step(rsq_pipe* pipe, const rsq_state* state_in, const rsq_state* state_out,
+                         const rsq_window* win_in, const rsq_window* win_out, const void* host_inputs,
+                         float* host_out, uint32_t step) {
+    if (!pipe || !host_inputs || !host_out) return fail(RSQ_E_INVAL, "pipe_step: null argument");
+    const int i = static_cast<int>(pipe->issued % kPipeDepth);
+    // the step that used slot i (kPipeDepth steps ago) has finished its output
+    // copy, hence also its kernel and its input copy: the slot's buffers and
+    // that step's host buffers are free again
+    int err = 0;
+    if (pipe->issued >= kPipeDepth) err = cudaEventSynchronize(pipe->read[i]);
+    if (!err) err = cudaMemcpyAsync(pipe->stage[i], host_inputs, pipe->in_bytes, cudaMemcpyHostToDevice, pipe->s_in);
+    if (!err) err = cudaEventRecord(pipe->copied[i], pipe->s_in);
+    if (!err) err = cudaStreamWaitEvent(pipe->s_cmp, pipe->copied[i], 0);
+    if (err) return cuda_fail(err, "pipe_step: input copy");
+    const uint8_t* b = pipe->stage[i];
+    const size_t* o = pipe->off;
+    const rsq_config& c = pipe->ctx->cfg;
+    rsq_gdn_inputs gi;
+    rsq_diag_inputs di;
+    rsq_mamba2_inputs mi;
+    const void* inputs;
+    if (c.family == RSQ_GDN) {
+        gi = {b + o[0], b + o[1], b + o[2], reinterpret_cast<const float*>(b + o[3]),
+              reinterpret_cast<const float*>(b + o[4])};
+        inputs = &gi;
+    } else if (c.family == RSQ_MAMBA2) {
+        mi = {b + o[0], b + o[1], b + o[2], reinterpret_cast<const float*>(b + o[3]),
+              reinterpret_cast<const float*>(b + o[4]), reinterpret_cast<const float*>(b + o[5]), nullptr};
+        inputs = &mi;
+    } else {
+        di = {b + o[0], b + o[1], b + o[2], reinterpret_cast<const float*>(b + o[3]),
+              c.family == RSQ_KDA ? reinterpret_cast<const float*>(b + o[4]) : nullptr};
+        inputs = &di;
+    }
+    rsq_status s = decode_step_impl(pipe->ctx, state_in, state_out, inputs, nullptr, win_in, win_out,
+                                    pipe->out_dev[i], step, pipe->s_cmp);
+    if (s) return s;
+    err = cudaEventRecord(pipe->done[i], pipe->s_cmp);
+    if (!err) err = cudaStreamWaitEvent(pipe->s_out, pipe->done[i], 0);
+    if (!err) err = cudaMemcpyAsync(host_out, pipe->out_dev[i], pipe->out_bytes, cudaMemcpyDeviceToHost, pipe->s_out);
+    if (!err) err = cudaEventRecord(pipe->read[i], pipe->s_out);
+    if (err) return cuda_fail(err, "pipe_step: output copy");
+    ++pipe->issued;
+    return RSQ_OK;
+}
+
+rsq_status rsq_pipe_sync(rsq_pipe* pipe) {
+    if (!pipe) return fail(RSQ_E_INVAL, "pipe_sync: null pipe");
+    int err = cudaStreamSynchronize(pipe->s_in);
+    if (!err) err = cudaStreamSynchronize(pipe->s_cmp);
+    if (!err) err = cudaStreamSynchronize(pipe->s_out);
+    return err ? cuda_fail(err, "pipe_sync") : RSQ_OK;
+}
+
+rsq_status rsq_pipe_streams(const rsq_pipe* pipe, void** copy_in, void** compute, void** copy_out) {
+    if (!pipe || !copy_in || !compute || !copy_out) return fail(RSQ_E_INVAL, "pipe_streams: null argument");
+    *copy_in = pipe->s_in;
+    *compute = pipe->s_cmp;
+    *copy_out = pipe->s_out;
+    return RSQ_OK;
+}
