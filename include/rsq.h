@@ -376,8 +376,9 @@ rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_state* state
  *   size.  Host-only.
  * rsq_pipe_create: three non-blocking streams (input copy, compute, output
  *   copy), events and device staging for 3 steps in flight, on the current
- *   device (RSQ_E_NOMEM / RSQ_E_CUDA).  The pipe borrows ctx: destroy the pipe
- *   first.
+ *   device, which must be the context's (else RSQ_E_INVAL; RSQ_E_NOMEM /
+ *   RSQ_E_CUDA on failure).  The pipe borrows ctx: destroy the pipe first.
+ *   rsq_pipe_step also returns RSQ_E_INVAL when called on another device.
  * rsq_pipe_step: one decode step.  Copies host_inputs (the packed layout;
  *   page-locked memory for the copies to overlap) to the device, runs
  *   rsq_decode_step (rsq_decode_step_window with win_in / win_out for a window

@@ -98,6 +98,18 @@ struct DecodeCfg {
     // four 128-thread CTAs per SM (4 x ~50 KB), so 128 registers per thread
     static constexpr int MINB = F32STATE ? 1 : (NT < 128 ? 8 : 512 / NT);
     static_assert(!PW || SPLIT == 1, "the pure-write window is built for d_k <= 128");
+    // the shared-memory layout, checked for every instance at compile time
+    static_assert(SMEM <= 227 * 1024, "shared memory beyond the per-CTA limit");
+    static_assert(STAGE % 128 == 0 && OFF_P >= NS * STAGE, "stages overlap the pair arrays");
+    static_assert(OFF_SCALES % 16 == 0 && OFF_VA % 16 == 0 && OFF_VB % 16 == 0 && OFF_VC % 16 == 0 &&
+                      OFF_VD % 16 == 0, "bulk-copy destinations must be 16-byte aligned");
+    static_assert(P_WARP % 16 == 0 && OFF_P % 16 == 0 && OFF_CNT - OFF_P >= NW * P_WARP,
+                  "one 16-byte aligned pair-array set per warp");
+    static_assert(OFF_BAR >= OFF_CNT + 4 * NS && OFF_BAR % 8 == 0 && OFF_SBAR % 8 == 0 && OFF_XBAR % 8 == 0,
+                  "mbarriers need their own 8-byte aligned words");
+    static_assert(L::RPT * RS == DK && RS * (L::RPT / 2) == DK / 2,
+                  "a lane's rows cover the block once, Philox row pairs are i and i + dk/2");
+    static_assert(PST > (DK - 1) / RS, "pair arrays hold a lane's rows");
 };
 
 // Grid-stride walk over units without divisions: (b, h, cb) advance by the

@@ -715,6 +715,9 @@ void rsq_pipe_destroy(rsq_pipe* pipe) {
 rsq_status rsq_pipe_create(const rsq_ctx* ctx, rsq_pipe** out) {
     if (!ctx || !out) return fail(RSQ_E_INVAL, "pipe_create: null argument");
     *out = nullptr;
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != ctx->device)
+        return fail(RSQ_E_INVAL, "pipe_create: the current device is not the context's device");
     rsq_pipe* p = new (std::nothrow) rsq_pipe();
     if (!p) return fail(RSQ_E_NOMEM, "pipe_create: host allocation failed");
     p->ctx = ctx;
@@ -745,6 +748,9 @@ rsq_status rsq_pipe_step(rsq_pipe* pipe, const rsq_state* state_in, const rsq_st
                          const rsq_window* win_in, const rsq_window* win_out, const void* host_inputs,
                          float* host_out, uint32_t step) {
     if (!pipe || !host_inputs || !host_out) return fail(RSQ_E_INVAL, "pipe_step: null argument");
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev != pipe->ctx->device)
+        return fail(RSQ_E_INVAL, "pipe_step: the current device is not the context's device");
     const int i = static_cast<int>(pipe->issued % kPipeDepth);
     // the step that used slot i (kPipeDepth steps ago) has finished its output
     // copy, hence also its kernel and its input copy: the slot's buffers and
