@@ -44,7 +44,8 @@ def _gdn_closed_form(ins, t_end, b, h):
 
 @pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
 def test_gdn_fp32_state_matches_closed_form(mode):
-    """The benchmark spec (a); recurrence of the gated delta rule (Gated DeltaNet)."""
+    """Quantization disabled: the closed-form unrolled sum of decayed outer
+    products; recurrence of the gated delta rule (Gated DeltaNet)."""
     w = TINY
     ins = [W.gdn_inputs(w, t) for t in range(w.steps)]
     bits = np.full(w.H, 32, np.int8)
@@ -61,7 +62,7 @@ def test_gdn_fp32_state_matches_closed_form(mode):
 
 @pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
 def test_gdn_fp32_state_matches_closed_form_dk256(mode):
-    """The benchmark spec (a) at d_k = 256, with the 16-partial canonical order the
+    """The closed-form unrolled sum at d_k = 256, with the 16-partial canonical order the
     library uses there (rsq_reduction_partials(256) = 16)."""
     w = dataclasses.replace(TINY, B=1, H=2, dk=256, dv=32)
     ins = [W.gdn_inputs(w, t) for t in range(6)]
@@ -90,7 +91,8 @@ def _mamba_closed_form(ins, t_end, b, h, D):
 
 @pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
 def test_mamba2_fp32_state_matches_closed_form(mode):
-    """The benchmark spec (a); Mamba-2 scalar-decay recurrence."""
+    """Quantization disabled: the closed-form unrolled sum of decayed outer
+    products; Mamba-2 scalar-decay recurrence."""
     w = TINY_M
     ins = [W.mamba2_inputs(w, t) for t in range(w.steps)]
     # exp(dt*A) passed explicitly (correctly rounded) so the closed form uses the same decays
@@ -153,7 +155,8 @@ def test_gdn_error_contraction_delta_rule():
 @pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
 def test_rtn_error_at_most_half_step(bits, mode):
-    """The benchmark spec (b); (1/4) Proposition: rounding errors within half a grid step."""
+    """Round-to-nearest error at most half a step; (1/4) Proposition: rounding
+    errors within half a grid step."""
     rng = np.random.default_rng(bits)
     S = (rng.standard_normal((3, 4, 32, 24)) * rng.uniform(0.01, 10, (3, 4, 1, 24))).astype(np.float32)
     st = oracle.quantize(S, np.full(4, bits, np.int8), rounding=oracle.RTN, seed=0, step=0, mode=mode)
@@ -244,7 +247,7 @@ def test_sr_exhaustive_probability(bits, mode):
 
 
 def test_sr_unbiased_over_draws():
-    """The benchmark spec (c): the mean of SR-dequantized values over many independent
+    """Stochastic rounding is unbiased: the mean of SR-dequantized values over many independent
     draws (steps) converges to the value (5 sigma)."""
     rng = np.random.default_rng(11)
     S = (rng.standard_normal((1, 2, 16, 16))).astype(np.float32)
@@ -268,7 +271,7 @@ def test_sr_unbiased_over_draws():
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("bits", [8, 4])
 def test_rtn_quantize_dequantize_idempotent(bits):
-    """The benchmark spec (d): Q(D(Q(S))) == Q(S) for round-to-nearest (codes bit-exact,
+    """quantize o dequantize is idempotent: Q(D(Q(S))) == Q(S) for round-to-nearest (codes bit-exact,
     scales within one ulp)."""
     rng = np.random.default_rng(21 + bits)
     S = (rng.standard_normal((2, 3, 32, 64)) * 3).astype(np.float32)
@@ -282,7 +285,7 @@ def test_rtn_quantize_dequantize_idempotent(bits):
 
 @pytest.mark.parametrize("bits", [8, 4])
 def test_sr_quantize_dequantize_nearly_idempotent(bits):
-    """The benchmark spec (d) for stochastic rounding: re-quantizing dequantized codes moves
+    """Idempotence for stochastic rounding: re-quantizing dequantized codes moves
     at most a 1e-5 fraction of the codes, each by at most one step."""
     rng = np.random.default_rng(31 + bits)
     S = (rng.standard_normal((4, 4, 64, 64)) * 2).astype(np.float32)
