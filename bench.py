@@ -406,7 +406,7 @@ def run_ours(args, w: W.Workload):
     # CUDA graphs of up to CH consecutive steps (launch-bound inner loop); CH is a
     # multiple of the layer count so the rotation continues across graph replays
     # (an even number of visits per layer, so the window ping-pong ends where it began)
-    CH = 2 * max(1, 1024 // layers) * layers
+    CH = 2 * max(1, (args.chunk or 1024) // layers) * layers
 
     def capture(t0, n):
         gr = torch.cuda.CUDAGraph()
@@ -777,6 +777,9 @@ def main():
     ap.add_argument("--drift-steps", type=int, default=0, help="horizon (default: the workload's)")
     ap.add_argument("--drift-every", type=int, default=256)
     ap.add_argument("--jsonl", default=None, help="also append each result line to this file")
+    ap.add_argument("--seed", type=int, default=None, help="override the workload's stochastic-rounding seed")
+    ap.add_argument("--chunk", type=int, default=0,
+                    help="steps per captured CUDA graph (rounded to an even number of visits per layer)")
     ap.add_argument("--sweep", action="store_true",
                     help="measure every row of the throughput table (one GPU), one line each")
     args = ap.parse_args()
@@ -790,9 +793,12 @@ def main():
         with mp.get_context("spawn").Pool(max(1, min(32, (os.cpu_count() or 2) - 1))) as pool:
             return run_drift(args, w, pool)
     w = W.BY_NAME[args.workload]
-    if args.rounding:
+    if args.rounding or args.seed is not None:
         import dataclasses
-        w = dataclasses.replace(w, rounding=args.rounding)
+        if args.rounding:
+            w = dataclasses.replace(w, rounding=args.rounding)
+        if args.seed is not None:
+            w = dataclasses.replace(w, sr_seed=args.seed)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)
