@@ -317,7 +317,8 @@ def run_reference(args, w: W.Workload):
     value = n_heads * args.steps / elapsed
     line = {
         "impl": "reference", "metric": "head-updates/s", "value": value, "unit": "head-updates/s",
-        "n_gpus": 0, "steps": args.steps, "warmup": args.warmup,
+        "n_gpus": args.gpus, "runs_on": "host CPU, rank 0 only (the oracle uses no GPU)",
+        "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1e3 * elapsed / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": w.name, "global_batch": w.B, "heads": w.H, "dk": w.dk, "dv": w.dv,
