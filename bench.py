@@ -160,7 +160,8 @@ SWEEP = (
     ("gdn_b1024_h16_d128_int4_sr_long", None, 0, True), ("gdn_b64_h16_d128_int8_sr", None, 4, False),
     ("gdn_b64_h16_d128_int8_sr", None, 8, False), ("gdn_b64_h16_d128_int8_sr", None, 16, False),
     ("gdn_b1024_h16_d128_int4_sr_long", None, 8, False),
-    ("gdn_b64_h8_d256_int8_sr", None, 0, False), ("mamba2_b128_h80_p64_n256_int8_sr", None, 0, False),
+    ("gdn_b64_h8_d256_int8_sr", None, 0, False), ("gdn_b64_h8_d256_int8_sr", "rtn", 0, False),
+    ("gdn_b64_h8_d256_int8_sr", "sr_bdr", 0, False), ("mamba2_b128_h80_p64_n256_int8_sr", None, 0, False),
 )
 
 

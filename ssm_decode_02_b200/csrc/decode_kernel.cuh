@@ -739,8 +739,10 @@ template <int FAM, int DK, int UB, bool F32STATE, int RND>
 constexpr int decode_min_blocks() {
     using C = DecodeCfg<FAM, DK, UB, F32STATE>;
     // BDR: about 168 registers per thread (65536 / (168 * 128) = 3 CTAs of 128 threads)
-    // (the pure-write window's slot pass needs as many)
-    return ((RND & kRndBdr) != 0 || is_pw_family(FAM)) ? 384 / C::NT : C::MINB;
+    // (the pure-write window's slot pass needs as many, and so does stochastic
+    // rounding at dk = 256 with its pair exchanges, run with two blocks per unit)
+    constexpr bool wide = (RND & kRndBdr) != 0 || is_pw_family(FAM) || (C::SPLIT > 1 && (RND & kRndSr) != 0);
+    return wide ? 384 / C::NT : C::MINB;
 }
 
 template <int FAM, int DK, int UB, bool F32STATE, int RND>

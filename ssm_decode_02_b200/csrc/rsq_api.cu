@@ -59,6 +59,11 @@ int kernel_family(const rsq_config& c) {
 }
 bool family_ok(int f) { return f == RSQ_GDN || f == RSQ_MAMBA2 || f == RSQ_GLA || f == RSQ_KDA; }
 bool rounding_ok(int r) { return r == RSQ_RTN || r == RSQ_SR || r == RSQ_BDR || r == RSQ_SR_BDR; }
+// 16-column blocks per work unit (at most): four, except stochastic rounding
+// at dk = 256, whose two-warp blocks run faster as 128-thread CTAs at three
+// per SM (168 registers, no spills) than as 256-thread CTAs at two.
+int unit_blocks(const rsq_config& c) { return (c.dk > 128 && (c.rounding & RSQ_SR)) ? 2 : 4; }
+
 bool dk_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
 bool dv_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
 
@@ -181,7 +186,7 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
         off += static_cast<long long>(c.dk) * c.dv * ctx->bits[h] / 8;
     }
     ctx->row_bytes = off;
-    ctx->ub = std::min(c.dv / rsq::kBlockCols, 4);
+    ctx->ub = std::min(c.dv / rsq::kBlockCols, unit_blocks(c));
     ctx->ncb = c.dv / (rsq::kBlockCols * ctx->ub);
     const long long units = static_cast<long long>(c.batch) * c.heads * ctx->ncb;
     if (units > (1LL << 30)) {
@@ -602,7 +607,7 @@ extern "C" rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_s
         off += static_cast<long long>(c.dk) * c.dv * ctx.bits[h] / 8;
     }
     ctx.row_bytes = off;
-    ctx.ub = std::min(c.dv / rsq::kBlockCols, 4);
+    ctx.ub = std::min(c.dv / rsq::kBlockCols, unit_blocks(c));
     ctx.ncb = c.dv / (rsq::kBlockCols * ctx.ub);
     const long long units = static_cast<long long>(c.batch) * c.heads * ctx.ncb;
     if (units > (1LL << 30)) return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: too many work units");
