@@ -50,7 +50,7 @@ def algorithmic_bytes_per_head(w: W.Workload, bits: int) -> int:
     written, the input vectors and gates, and the float output."""
     esz = 2 if w.in_dtype == "bf16" else 4
     codes = w.dk * w.dv * bits // 8
-    scales = 4 * w.dv
+    scales = 0 if bits == 32 else 4 * w.dv   # a full-precision state has no scales
     out = 4 * w.dv
     if w.family == "gdn":
         vecs = esz * (2 * w.dk + w.dv) + 8          # q, k, v, alpha, beta

@@ -110,3 +110,25 @@ def test_sweep_rows_name_known_workloads():
         assert name in W.BY_NAME
         assert rounding is None or rounding in bench.ROUNDING
         assert window in (0, 4, 8, 16) and not (window and key_axis)
+
+
+def test_algorithmic_bytes_match_the_hand_counts():
+    """The roofline numerator: bytes one head update must move (codes and scales
+    read and written, inputs, gates, fp32 output), counted by hand per format.
+    GDN d=128 bf16: codes 2*16384 (INT8) or 2*8192 (INT4), scales 2*512,
+    q/k/v 3*256 + alpha/beta 8, output 512."""
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads as W
+    gdn = W.BY_NAME["gdn_b64_h16_d128_int8_sr"]
+    assert bench.algorithmic_bytes_per_head(gdn, 8) == 32768 + 1024 + 776 + 512 == 35080
+    assert bench.algorithmic_bytes_per_head(gdn, 4) == 16384 + 1024 + 776 + 512 == 18696
+    # full-precision state: 4-byte values in both directions, no scales
+    assert bench.algorithmic_bytes_per_head(gdn, 32) == 2 * 65536 + 776 + 512 == 132360
+    mamba = W.BY_NAME["mamba2_b128_h80_p64_n128_int8_sr"]
+    # Mamba-2 N=128, P=64: codes 2*8192, scales 2*256, x 128 + dt 4, output 256
+    assert bench.algorithmic_bytes_per_head(mamba, 8) == 16384 + 512 + 132 + 256 == 17284
+    # per step: every head, plus B and C once per request (ngroups = 1) and A, D per head
+    assert bench.step_bytes(mamba, [8] * mamba.H) == (17284 * mamba.H + 2 * 128 * 2) * mamba.B + 8 * mamba.H
+    # the benchmark workload: 1024 head updates of 35080 bytes
+    assert bench.step_bytes(gdn, [8] * gdn.H) == 1024 * 35080 == 35921920
