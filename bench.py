@@ -45,12 +45,13 @@ DEFAULT_WORKLOAD = "gdn_b64_h16_d128_int8_sr"
 DRIFT_WORKLOAD = "gdn_b1024_h16_d128_int4_sr_long"
 
 
-def algorithmic_bytes_per_head(w: W.Workload, bits: int) -> int:
+def algorithmic_bytes_per_head(w: W.Workload, bits: int, key_axis: bool = False) -> int:
     """Bytes the method must move per head update: codes and scales read and
     written, the input vectors and gates, and the float output."""
     esz = 2 if w.in_dtype == "bf16" else 4
     codes = w.dk * w.dv * bits // 8
-    scales = 0 if bits == 32 else 4 * w.dv   # a full-precision state has no scales
+    # a full-precision state has no scales; key-axis groups keep one per row
+    scales = 0 if bits == 32 else 4 * (w.dk if key_axis else w.dv)
     out = 4 * w.dv
     if w.family == "gdn":
         vecs = esz * (2 * w.dk + w.dv) + 8          # q, k, v, alpha, beta
@@ -67,8 +68,8 @@ def window_bytes_per_head(w: W.Workload, window: int) -> int:
     return 2 * (window * (w.dk + w.dv) + 2 * 4 * window) if window else 0
 
 
-def step_bytes(w: W.Workload, head_bits, window: int = 0) -> int:
-    per = sum(algorithmic_bytes_per_head(w, int(b)) + window_bytes_per_head(w, window)
+def step_bytes(w: W.Workload, head_bits, window: int = 0, key_axis: bool = False) -> int:
+    per = sum(algorithmic_bytes_per_head(w, int(b), key_axis) + window_bytes_per_head(w, window)
               for b in head_bits) * w.B
     if w.family == "mamba2":
         esz = 2 if w.in_dtype == "bf16" else 4
@@ -528,7 +529,7 @@ def run_ours(args, w: W.Workload):
     value = world * hu_step * args.steps / elapsed
     e2e_value = world * hu_step * n_e2e / e2e_elapsed
     per_launch = elapsed / args.steps
-    alg = step_bytes(w, bits, args.window)
+    alg = step_bytes(w, bits, args.window, bool(args.key_axis))
     peak, peak_kind = measured_peak_gbs()
     achieved = alg / per_launch / 1e9
     kernel_tag = "rsq_decode_kernel<%s,dk=%d,blocks=%d,%s>" % (w.family, w.dk, min(4, w.dv // 16),

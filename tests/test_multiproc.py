@@ -132,3 +132,8 @@ def test_algorithmic_bytes_match_the_hand_counts():
     assert bench.step_bytes(mamba, [8] * mamba.H) == (17284 * mamba.H + 2 * 128 * 2) * mamba.B + 8 * mamba.H
     # the benchmark workload: 1024 head updates of 35080 bytes
     assert bench.step_bytes(gdn, [8] * gdn.H) == 1024 * 35080 == 35921920
+    # key-axis groups: one scale per key row (d_k of them)
+    import dataclasses
+    wide = dataclasses.replace(gdn, dk=64, dv=128)
+    assert (bench.algorithmic_bytes_per_head(wide, 8, key_axis=True)
+            == bench.algorithmic_bytes_per_head(wide, 8) - 2 * 4 * (128 - 64))
