@@ -19,11 +19,11 @@ from gpu_harness import Run, dev, host
 pytestmark = pytest.mark.gpu
 
 
-def _state_from(ctx, st, bits, key_axis=False):
+def _state_from(st, bits):
     return rsq.State(dev(oracle.pack_state(st, bits)), dev(np.ascontiguousarray(st["scales"], np.float32)))
 
 
-def _window(ctx, win, dv):
+def _window(win, dv):
     B, H, Wn, _ = win["b"].shape
     b = np.ascontiguousarray(win["b"].reshape(B, H, Wn, dv // 16, 16).transpose(0, 1, 3, 2, 4))
     return rsq.Window(dev(win["a"]), dev(win["as"]), dev(b), dev(win["bs"]))
@@ -61,13 +61,13 @@ def test_pipe_matches_device_entry_points(name):
         st["f"] = S
     else:
         st = oracle.quantize(S, bits, rounding=oracle.SR, seed=1, step=0)
-    a = [_state_from(ctx, st, bits), _state_from(ctx, st, bits)]
-    b = [_state_from(ctx, st, bits), _state_from(ctx, st, bits)]
+    a = [_state_from(st, bits), _state_from(st, bits)]
+    b = [_state_from(st, bits), _state_from(st, bits)]
     wa = wb = None
     if Wn:
         win = oracle.zero_window(w.B, w.H, Wn, w.dk, w.dv)
-        wa = [_window(ctx, win, w.dv), _window(ctx, win, w.dv)]
-        wb = [_window(ctx, win, w.dv), _window(ctx, win, w.dv)]
+        wa = [_window(win, w.dv), _window(win, w.dv)]
+        wb = [_window(win, w.dv), _window(win, w.dv)]
     torch.cuda.synchronize()        # uploads done before the pipe's own streams start
     pipe = rsq.Pipe(ctx)
     steps = 7                       # more than the 3 steps in flight: every slot reused
