@@ -12,6 +12,7 @@ import pytest
 
 import oracle
 import workloads as W
+import plain_order
 import workloads as W_mod
 
 TINY = W.WORKLOADS[0]                      # GDN B=1 H=2 d=16, fp32 inputs, 64 steps
@@ -488,28 +489,61 @@ def test_sr_uniforms_distinct_per_element():
 # ---------------------------------------------------------------------------
 # Reduction order, mixed precision allocation, storage format
 # ---------------------------------------------------------------------------
-def test_canonical_and_plain_agree_teacher_forced():
-    """Both evaluation orders compute the same mathematics: from the same input
-    state they give codes that differ in few places, by at most one step, and
-    outputs within 1e-5 relative."""
-    w = dataclasses.replace(W.WORKLOADS[1], B=2, H=4)
-    hb = np.full(w.H, 8, np.int8)
-    rng = np.random.default_rng(51)
-    S = rng.standard_normal((w.B, w.H, w.dk, w.dv)).astype(np.float32)
-    st = oracle.quantize(S, hb, rounding=oracle.SR, seed=1, step=0)
-    n_diff = n_tot = 0
-    for t in range(1, 4):
-        inp = W.gdn_inputs(w, t, B=w.B)
-        a, oa = oracle.gdn_step(st, inp, hb, rounding=oracle.SR, seed=5, step=t, mode=oracle.PLAIN)
-        b, ob = oracle.gdn_step(st, inp, hb, rounding=oracle.SR, seed=5, step=t, mode=oracle.CANONICAL)
-        d = np.abs(a["codes"].astype(int) - b["codes"].astype(int))
-        assert d.max() <= 1
-        n_diff += int((d != 0).sum())
-        n_tot += d.size
-        assert np.max(np.abs(oa - ob)) <= 1e-5 * np.max(np.abs(oa))
-        assert np.allclose(a["scales"], b["scales"], rtol=1e-5)
+@pytest.mark.parametrize("family", ["gdn", "mamba2"])
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("rounding", [oracle.RTN, oracle.SR])
+def test_canonical_and_plain_agree_teacher_forced(family, bits, rounding):
+    """Both evaluation orders compute the same mathematics ("(1/4) Scale
+    grouping": s = max|S| / r, codes round(S / s); "(3/4) Rounding"): from the
+    same input state at most 1e-5 of the codes differ, each by one step, apart
+    from exact ties of nearest rounding (an element exactly a half-integer
+    number of steps), which the two orders break differently; scales and
+    outputs agree to 1e-5 relative."""
+    base = W.WORKLOADS[1] if family == "gdn" else W.WORKLOADS[3]
+    w = dataclasses.replace(base, B=8, H=8)
+    hb = np.full(w.H, bits, np.int8)
+    rng = np.random.default_rng(51 + bits + 7 * rounding)
+    S = (rng.standard_normal((w.B, w.H, w.dk, w.dv)) * 0.1).astype(np.float32)
+    st = oracle.quantize(S, hb, rounding=rounding, seed=1, step=0)
+    step = oracle.gdn_step if family == "gdn" else oracle.mamba2_step
+    n_other = n_tie = n_tot = 0
+    for t in range(1, 5):
+        inp = W.inputs(w, t, B=w.B)
+        a, oa = step(st, inp, hb, rounding=rounding, seed=5, step=t, mode=oracle.PLAIN)
+        b, ob = step(st, inp, hb, rounding=rounding, seed=5, step=t, mode=oracle.CANONICAL)
+        S_lit = plain_order.literal_state(family, st, inp, hb)
+        o, ti, tot = plain_order.compare_codes(b["codes"], a["codes"], S_lit, hb,
+                                               nearest=rounding == oracle.RTN)
+        n_other, n_tie, n_tot = n_other + o, n_tie + ti, n_tot + tot
+        assert plain_order.max_rel(ob, oa) <= 1e-5
+        assert np.allclose(a["scales"], b["scales"], rtol=1e-5, atol=0)
         st = b
-    assert n_diff / n_tot <= 1e-3
+    assert n_other <= 1e-5 * n_tot, (n_other, n_tie, n_tot)
+    assert n_tie <= 1e-3 * n_tot, (n_other, n_tie, n_tot)
+
+
+def test_exact_tie_broken_toward_zero_by_the_canonical_order():
+    """An element exactly half its column's maximum (x = S / s = r / 2) is an
+    exact tie of nearest rounding: the literal order's float scale and
+    quotient decide it, the canonical order's multiplier r / m rounded toward
+    zero rounds it toward zero unless r / m is exact in binary32, when the
+    product is the tie itself and goes to even ("(1/4) Scale grouping";
+    nearest with ties to even)."""
+    for bits in (4, 8):
+        r = (1 << (bits - 1)) - 1
+        for m in (1.0, 0.5, 0.75, 3.0e-3, 1.7):
+            m = float(np.float32(m))
+            S = m / 2.0                                  # exact
+            exact = float(np.float32(r / m)) == r / m    # r / m representable
+            want_c = (r + 1) // 2 if exact else (r - 1) // 2   # even (4 / 64) or toward zero
+            assert oracle.quantize_scalar(S, m, bits, oracle.RTN, oracle.CANONICAL) == want_c
+            assert oracle.quantize_scalar(-S, m, bits, oracle.RTN, oracle.CANONICAL) == -want_c
+            # the literal order: x = S / fl(m / r), nearest, ties to even
+            s = np.float32(np.float32(m) / np.float32(r))
+            x = np.float32(np.float32(S) / s)
+            want = int(np.rint(np.float64(x)))
+            assert oracle.quantize_scalar(S, m, bits, oracle.RTN, oracle.PLAIN) == want
+            assert want in ((r - 1) // 2, (r + 1) // 2)
 
 
 def test_allocation_matches_sort():
