@@ -23,6 +23,8 @@ from . import build as _build
 PLAIN, CANONICAL = 0, 1
 RTN, SR = 0, 1
 BDR, SR_BDR = 2, 3      # nearest / stochastic base rounding + Bounded Directional Rounding
+U8 = 4                  # stochastic rounding with 8-bit uniforms (SR alone: 16-bit uniforms)
+SR8, SR8_BDR = SR | U8, SR_BDR | U8
 
 
 class _Head(ctypes.Structure):
@@ -46,6 +48,8 @@ def lib():
         L.orc_sr_uniform16.argtypes = [ctypes.c_uint64, ctypes.c_uint32, ctypes.c_uint32,
                                        ctypes.c_uint32, ctypes.c_int, ctypes.c_int, ctypes.c_int]
         L.orc_sr_uniform16.restype = ctypes.c_uint32
+        L.orc_sr_uniform8.argtypes = L.orc_sr_uniform16.argtypes
+        L.orc_sr_uniform8.restype = ctypes.c_uint32
         L.orc_bf16_to_f32.argtypes = [P, P, ctypes.c_int64]
         L.orc_gdn_head_step.argtypes = [ctypes.POINTER(_Head), P, P, P, P, P, P, ctypes.c_float,
                                         ctypes.c_float, P, P, P, P]
@@ -117,8 +121,13 @@ def sr_uniform16(seed: int, b: int, h: int, step: int, dk: int, i: int, j: int) 
     return int(lib().orc_sr_uniform16(seed, b, h, step, dk, i, j))
 
 
+def sr_uniform8(seed: int, b: int, h: int, step: int, dk: int, i: int, j: int) -> int:
+    return int(lib().orc_sr_uniform8(seed, b, h, step, dk, i, j))
+
+
 def quantize_scalar(S: float, m: float, bits: int, rounding: int, mode: int, u: int = 0) -> int:
-    """Code of one element S of a column with absolute maximum m (> 0), given its uniform u."""
+    """Code of one element S of a column with absolute maximum m (> 0), given its
+    uniform u (16 bits wide, or 8 bits when ``rounding`` has the U8 bit)."""
     return int(lib().orc_quantize_scalar(float(S), float(m), int(bits), int(rounding), int(mode),
                                          int(u)))
 

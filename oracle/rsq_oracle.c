@@ -61,12 +61,15 @@
 #define ORC_PLAIN 0
 #define ORC_CANONICAL 1
 /* Rounding: bit 0 selects the base rounding (0 nearest, 1 stochastic); bit 1
- * adds the directional correction of [BDR] on top of it.                    */
+ * adds the directional correction of [BDR] on top of it; bit 2 makes the
+ * stochastic rounding's uniforms 8 bits wide instead of 16.                 */
 #define ORC_RTN 0
 #define ORC_SR 1
 #define ORC_BDR 2
+#define ORC_U8 4
 #define ORC_SR_BASE(rnd) ((rnd) & 1)
 #define ORC_HAS_BDR(rnd) (((rnd) & 2) != 0)
+#define ORC_UBITS(rnd) (((rnd) & ORC_U8) ? 8 : 16)
 
 /* ------------------------------------------------------------------------- */
 /* Philox4x32-10 [PHILOX]: 10 rounds of two 32x32->64 multiplies; the key is
@@ -112,6 +115,34 @@ uint32_t orc_sr_uniform16(uint64_t seed, uint32_t b, uint32_t h, uint32_t step,
     int chunk = 4 * (i >= half ? 1 : 0) + (j % 4);
     uint32_t word = out[chunk / 2];
     return (chunk % 2 == 0) ? (word & 0xFFFFu) : (word >> 16);
+}
+
+/* The 8-bit uniform of element (i, j) of head (b, h) at decode step `step`
+ * (stochastic rounding with 8-bit uniforms).  One Philox block serves 16
+ * elements: rows i', i' + dk/4, i' + dk/2, i' + 3dk/4 (i' = i mod dk/4) of the
+ * four columns 4g..4g+3 (g = j/4).
+ *   counter = { i' | g << 16, h, b, step },  key = { seed_lo, seed_hi }
+ *   word i div (dk/4), byte j mod 4 (lowest byte first).                   */
+uint32_t orc_sr_uniform8(uint64_t seed, uint32_t b, uint32_t h, uint32_t step,
+                         int dk, int i, int j)
+{
+    int quarter = dk / 4;
+    uint32_t ip = (uint32_t)(i % quarter);
+    uint32_t g = (uint32_t)(j / 4);
+    uint32_t ctr[4] = {ip | (g << 16), h, b, step};
+    uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+    uint32_t out[4];
+    orc_philox4x32_10(ctr, key, out);
+    uint32_t word = out[i / quarter];
+    return (word >> (8 * (j % 4))) & 0xFFu;
+}
+
+/* The uniform stochastic rounding of element (i, j) consumes under rule `rnd`. */
+static uint32_t orc_sr_uniform(int rnd, uint64_t seed, uint32_t b, uint32_t h, uint32_t step,
+                               int dk, int i, int j)
+{
+    return (rnd & ORC_U8) ? orc_sr_uniform8(seed, b, h, step, dk, i, j)
+                          : orc_sr_uniform16(seed, b, h, step, dk, i, j);
 }
 
 /* bfloat16 -> binary32 widening (exact): the bf16 bits are the upper half. */
@@ -168,15 +199,21 @@ static float orc_inv_rz(float r, float m)
 }
 
 /* Quantize one element S of a column whose absolute maximum is m (> 0 and
- * finite) to a symmetric b-bit code.  `u` is the element's 16-bit uniform
- * (used by stochastic rounding only).
+ * finite) to a symmetric b-bit code.  `u` is the element's uniform (used by
+ * stochastic rounding only): 16 bits wide, or 8 bits under ORC_U8.
  *   plain:      x = S / s with s = m / r;  RTN: nearest (ties to even);
- *               SR: floor(x + u/2^16), i.e. up with probability frac(x)
- *               ([LoReS] (3/4): SR is conditionally unbiased); clamp to [-r, r].
+ *               SR, 16-bit u: floor(x + u/2^16), up with probability frac(x)
+ *               to within 2^-16 ([LoReS] (3/4): SR is conditionally unbiased);
+ *               SR, 8-bit u: floor(x + (u + 1/2)/2^8), up with probability
+ *               frac(x) rounded to a multiple of 2^-8 (within 2^-9), and a
+ *               value within 2^-9 of an integer stays on it;  clamp to [-r, r].
  *   canonical:  inv = r/m rounded toward zero;  RTN: nearest integer (ties to
- *               even) of the exact product S*inv;  SR: t = S*inv + (o + u/2^16)
- *               rounded once to binary32, c = floor(t) - o, with the offset
- *               o = 128 (8-bit) or 136 (4-bit) so that t stays in [1, 256).  */
+ *               even) of the exact product S*inv;  SR: t = S*inv + (o + u/U)
+ *               rounded once to binary32, c = floor(t) - o, with U = 2^16 and
+ *               the offset o = 128 (8-bit codes) or 136 (4-bit codes), so that
+ *               t stays in [1, 256), or U = 2^8 and o = 2^15 + 128 or 2^15 + 8,
+ *               so that t stays in [2^15, 2^16) where the rounding of t to a
+ *               multiple of 2^-8 adds the half of (u + 1/2).                 */
 /* S / s of the plain order, made safe to convert to an integer.  When the
  * scale s = m / r underflows to zero (m below r * 2^-150, deep in the
  * subnormal range) S / s is +-inf, which the clamp to [-r, r] turns into +-r,
@@ -196,12 +233,15 @@ int orc_quantize_scalar(float S, float m, int bits, int rounding, int mode, uint
 {
     const int r = orc_rmax(bits);
     const float rf = (float)r;
+    const int u8 = (rounding & ORC_U8) != 0;
     int c;
     if (mode == ORC_PLAIN) {
         const float s = m / rf;
         const float x = orc_plain_ratio(S, s, r);
         if (!ORC_SR_BASE(rounding))
             c = (int)rintf(x);
+        else if (u8)
+            c = (int)floor((double)x + ((double)u + 0.5) / 256.0);
         else
             c = (int)floor((double)x + (double)u / 65536.0);
         if (c > r) c = r;
@@ -211,8 +251,9 @@ int orc_quantize_scalar(float S, float m, int bits, int rounding, int mode, uint
         if (!ORC_SR_BASE(rounding)) {
             c = (int)rint((double)S * (double)inv);
         } else {
-            const float off = (bits == 8) ? 128.0f : 136.0f;
-            const float V = off + (float)u / 65536.0f; /* exact */
+            const float off = u8 ? ((bits == 8) ? 32896.0f : 32776.0f)
+                                 : ((bits == 8) ? 128.0f : 136.0f);
+            const float V = off + (float)u / (u8 ? 256.0f : 65536.0f); /* exact */
             const float t = fmaf(S, inv, V);
             c = (int)floorf(t) - (int)off;
         }
@@ -279,7 +320,7 @@ static void orc_quantize_column(const float* S, const float* prev, const float* 
         if (usable) {
             float x = S[(int64_t)i * dv + j];
             if (m_copy) x = fminf(fmaxf(x, -ms), ms); /* clip to the copy's range */
-            uint32_t u = ORC_SR_BASE(rounding) ? orc_sr_uniform16(seed, b, h, step, dk, i, j) : 0u;
+            uint32_t u = ORC_SR_BASE(rounding) ? orc_sr_uniform(rounding, seed, b, h, step, dk, i, j) : 0u;
             c = orc_quantize_scalar(x, ms, bits, rounding, mode, u);
             /* without a previous state (initial quantization) there is no
              * update direction and the base rounding stands */
@@ -531,7 +572,7 @@ static void orc_quantize_row(const float* S, int dk, int dv, int i, int bits, in
     for (int j = 0; j < dv; ++j) {
         int c = 0;
         if (usable) {
-            const uint32_t u = ORC_SR_BASE(rounding) ? orc_sr_uniform16(seed, b, h, step, dk, i, j) : 0u;
+            const uint32_t u = ORC_SR_BASE(rounding) ? orc_sr_uniform(rounding, seed, b, h, step, dk, i, j) : 0u;
             c = orc_quantize_scalar(S[(int64_t)i * dv + j], m, bits, rounding, mode, u);
         }
         codes[(int64_t)i * dv + j] = (int8_t)c;
@@ -576,8 +617,8 @@ int orc_gdn_ka_head_step(const orc_head* hd, const int8_t* c_in, const float* s_
     }
     for (int j = 0; j < dv; ++j) o[j] = orc_dot_rows(S + j, dv, q, dk, R);
     for (int i = 0; i < dk; ++i)
-        orc_quantize_row(S, dk, dv, i, hd->bits, hd->rounding & 1, hd->mode, hd->seed, hd->b, hd->h,
-                         hd->step, c_out, &s_out[i]);
+        orc_quantize_row(S, dk, dv, i, hd->bits, hd->rounding & ~ORC_BDR, hd->mode, hd->seed, hd->b,
+                         hd->h, hd->step, c_out, &s_out[i]);
     free(S); free(cf); free(ks);
     return 0;
 }
@@ -587,8 +628,8 @@ int orc_quantize_ka_head(const orc_head* hd, const float* S, int8_t* c_out, floa
 {
     if (hd->bits != 4 && hd->bits != 8) return 1;
     for (int i = 0; i < hd->dk; ++i)
-        orc_quantize_row(S, hd->dk, hd->dv, i, hd->bits, hd->rounding & 1, hd->mode, hd->seed, hd->b,
-                         hd->h, hd->step, c_out, &s_out[i]);
+        orc_quantize_row(S, hd->dk, hd->dv, i, hd->bits, hd->rounding & ~ORC_BDR, hd->mode, hd->seed,
+                         hd->b, hd->h, hd->step, c_out, &s_out[i]);
     return 0;
 }
 
@@ -737,7 +778,7 @@ int orc_gdn_pw_head_step(const orc_head* hd, int W, int fp32window, const int8_t
     } else {
         for (int j = 0; j < dv; ++j)
             orc_quantize_column(S, NULL, hd->m_copy ? hd->m_copy + j : NULL, dk, dv, j, hd->bits,
-                                hd->rounding & 1, hd->mode, hd->seed, hd->b, hd->h, hd->step,
+                                hd->rounding & ~ORC_BDR, hd->mode, hd->seed, hd->b, hd->h, hd->step,
                                 c_out, &s_out[j]);
     }
     for (int w = 0; w < W; ++w) {

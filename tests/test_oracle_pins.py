@@ -247,6 +247,63 @@ def test_sr_exhaustive_probability(bits, mode):
         assert abs(p_up - (x - lo)) <= 2.0 ** -16 + 1e-12, (x, p_up)
 
 
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
+def test_sr8_exhaustive_probability(bits, mode):
+    """(3/4) Rounding with 8-bit uniforms: enumerating all 256 uniforms, every
+    code is floor(x) or floor(x) + 1, P(round up) equals frac(x) to within
+    2^-9, and a value within 2^-9 of an integer is never moved off it."""
+    r = oracle.rmax(bits)
+    m = float(r)               # column max r -> scale 1 and multiplier 1: x = S exactly
+    rng = np.random.default_rng(17 + bits)
+    xs = list(rng.uniform(-r, r, 24).astype(np.float32)) + [np.float32(v) for v in (
+        0.0, 0.5, -0.5, 3.25, -2.75, r, -r, 1e-3, -1e-3, 2.0 - 2.0 ** -10, 1.0 + 2.0 ** -10,
+        0.5 + 2.0 ** -9, 0.25 - 2.0 ** -11)]
+    for x in xs:
+        x = float(x)
+        lo = np.floor(x)
+        codes = np.array([oracle.quantize_scalar(x, m, bits, oracle.SR8, mode, u) for u in range(256)])
+        assert set(np.unique(codes)) <= {int(lo), int(lo) + 1}
+        p_up = float(np.mean(codes == lo + 1))
+        assert abs(p_up - (x - lo)) <= 2.0 ** -9 + 1e-12, (x, p_up)
+        near = np.round(x)
+        if abs(x - near) < 2.0 ** -9:
+            assert np.all(codes == near), (x, np.unique(codes))
+
+
+def test_sr8_unbiased_over_draws():
+    """Stochastic rounding with 8-bit uniforms is unbiased to within 2^-9 of a
+    step: the mean of dequantized values over many draws converges to the value."""
+    rng = np.random.default_rng(13)
+    S = (rng.standard_normal((1, 2, 16, 16))).astype(np.float32)
+    bits = np.full(2, 4, np.int8)
+    n = 400
+    acc = np.zeros(S.shape)
+    for t in range(n):
+        st = oracle.quantize(S, bits, rounding=oracle.SR8, seed=4321, step=t, mode=oracle.CANONICAL)
+        acc += oracle.dequantize(st, bits).astype(np.float64)
+    mean = acc / n
+    s = st["scales"][:, :, None, :].astype(np.float64)
+    x = S.astype(np.float64) / s
+    phi = x - np.floor(x)
+    sigma = s * np.sqrt(np.maximum(phi * (1 - phi), 1.0 / n) / n)
+    assert np.all(np.abs(mean - S) <= 5 * sigma + s * 2.0 ** -9)
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+def test_sr8_quantize_dequantize_idempotent(bits):
+    """With 8-bit uniforms (values within 2^-9 of an integer stay on it),
+    quantize o dequantize is idempotent for stochastic rounding: the codes of
+    Q(D(Q(S))) equal those of Q(S) whatever the second draw."""
+    rng = np.random.default_rng(41 + bits)
+    S = (rng.standard_normal((4, 4, 64, 64)) * 2).astype(np.float32)
+    hb = np.full(4, bits, np.int8)
+    for mode in (oracle.PLAIN, oracle.CANONICAL):
+        q1 = oracle.quantize(S, hb, rounding=oracle.SR8, seed=9, step=1, mode=mode)
+        q2 = oracle.quantize(oracle.dequantize(q1, hb), hb, rounding=oracle.SR8, seed=9, step=2, mode=mode)
+        assert np.array_equal(q1["codes"], q2["codes"])
+
+
 def test_sr_unbiased_over_draws():
     """Stochastic rounding is unbiased: the mean of SR-dequantized values over many independent
     draws (steps) converges to the value (5 sigma)."""
@@ -363,7 +420,7 @@ def _gdn_traj(w, steps, bits_h, rounding, seed, mode):
     return ins, out
 
 
-@pytest.mark.parametrize("rounding", [oracle.RTN, oracle.SR])
+@pytest.mark.parametrize("rounding", [oracle.RTN, oracle.SR, oracle.SR8])
 def test_decaying_error_bound(rounding):
     """(2/4) Proposition (decaying error): ||E_t||_F <= sum_tau alpha^(t-tau) ||eps_tau||_F
     with alpha = max alpha_t, unit-norm keys and 0 < beta < 2."""
@@ -486,12 +543,42 @@ def test_sr_uniforms_distinct_per_element():
     assert chi2 < 60
 
 
+def test_sr8_uniforms_distinct_per_element():
+    """With 8-bit uniforms each element of a head draws its own byte of a
+    Philox block: counter {i mod dk/4 | (j/4) << 16, h, b, step}, word i div
+    dk/4, byte j mod 4.  Over one head the (block, byte) pairs are all
+    distinct, each uniform is that byte of the oracle's (Triton-pinned) Philox
+    output, and the uniforms are uniform."""
+    for dk in (16, 128):
+        dv = 32
+        seen = set()
+        vals = []
+        for i in range(dk):
+            for j in range(dv):
+                blk = (i % (dk // 4), j // 4)
+                slot = 4 * (i // (dk // 4)) + j % 4
+                assert (blk, slot) not in seen
+                seen.add((blk, slot))
+                u = oracle.sr_uniform8(77, 2, 6, 9, dk, i, j)
+                vals.append(u)
+        if dk == 128:
+            for i, j in ((0, 0), (37, 5), (127, 31), (64, 17)):
+                ctr = np.array([(i % 32) | ((j // 4) << 16), 6, 2, 9], np.uint32)
+                out = oracle.philox4x32_10(ctr, np.array([77, 0], np.uint32))[0]
+                assert oracle.sr_uniform8(77, 2, 6, 9, dk, i, j) == (int(out[i // 32]) >> (8 * (j % 4))) & 0xFF
+        vals = np.array(vals)
+        assert vals.min() >= 0 and vals.max() < 256
+        hist = np.bincount(vals >> 4, minlength=16)
+        chi2 = float(((hist - len(vals) / 16) ** 2 / (len(vals) / 16)).sum())
+        assert chi2 < 60
+
+
 # ---------------------------------------------------------------------------
 # Reduction order, mixed precision allocation, storage format
 # ---------------------------------------------------------------------------
 @pytest.mark.parametrize("family", ["gdn", "mamba2"])
 @pytest.mark.parametrize("bits", [8, 4])
-@pytest.mark.parametrize("rounding", [oracle.RTN, oracle.SR])
+@pytest.mark.parametrize("rounding", [oracle.RTN, oracle.SR, oracle.SR8])
 def test_canonical_and_plain_agree_teacher_forced(family, bits, rounding):
     """Both evaluation orders compute the same mathematics ("(1/4) Scale
     grouping": s = max|S| / r, codes round(S / s); "(3/4) Rounding"): from the
@@ -636,7 +723,7 @@ def _one_step_f64(st, inp, b, h):
     return a * Sh + np.outer(k, w), Sh
 
 
-@pytest.mark.parametrize("base", [oracle.RTN, oracle.SR])
+@pytest.mark.parametrize("base", [oracle.RTN, oracle.SR, oracle.SR8])
 @pytest.mark.parametrize("bits", [8, 4])
 @pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
 def test_bdr_properties_on_trajectories(base, bits, mode):
@@ -763,7 +850,7 @@ def test_gla_constant_decay_is_the_scalar_decay_step():
 # unquantized copy of the state; "When Dynamic Scaling Fails", key points: the
 # dynamic scale feeds back on the state it is derived from)
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("rounding", [oracle.RTN, oracle.SR])
+@pytest.mark.parametrize("rounding", [oracle.RTN, oracle.SR, oracle.SR8])
 @pytest.mark.parametrize("mode", [oracle.PLAIN, oracle.CANONICAL])
 def test_copy_scale_equal_to_own_maximum_is_the_noisy_quantizer(rounding, mode):
     rng = np.random.default_rng(3)
