@@ -606,7 +606,9 @@ DRIFT_VARIANTS = (("int4_sr", 4, "sr", "noisy"), ("int4_rtn", 4, "rtn", "noisy")
                   ("int8_sr_w8", 8, "sr", "w8"),
                   ("int4_sr_keyaxis", 4, "sr", "keyaxis"), ("int4_rtn_keyaxis", 4, "rtn", "keyaxis"),
                   ("int8_sr_keyaxis", 8, "sr", "keyaxis"))
-ROUNDING = {"rtn": 0, "sr": 1, "bdr": 2, "sr_bdr": 3}   # rsq_rounding values
+# rsq_rounding values; "sr" is stochastic rounding with 8-bit uniforms, "sr16"
+# the same with 16-bit uniforms
+ROUNDING = {"rtn": 0, "sr": 5, "bdr": 2, "sr_bdr": 7, "sr16": 1, "sr16_bdr": 3}
 
 
 def _drift_inputs(job):

@@ -96,17 +96,28 @@ typedef enum {
  * RSQ_KDA: S_t = (I - beta k k^T) diag(alpha) S_{t-1} + beta k v^T.  GLA and
  * KDA are the diagonal-decay mixers of [LoReS] Table 1. */
 typedef enum { RSQ_GDN = 0, RSQ_MAMBA2 = 1, RSQ_GLA = 2, RSQ_KDA = 3 } rsq_family;
-/* Requantization rule.  RSQ_RTN: nearest code (ties to even).  RSQ_SR:
- * stochastic rounding with a 16-bit Philox uniform per element ([LoReS] (3/4)).
- * RSQ_BDR / RSQ_SR_BDR: the same base rounding followed by Bounded Directional
- * Rounding ("Preserving Updates in Low-Bit Recurrent State Quantization",
- * abstract): when the rounded value c_t s_t lies strictly on the other side of
- * the previous value c_{t-1} s_{t-1} than the updated state S_t does (the
- * element moved against its update), the code becomes the integer next to
- * S_t / s_t on the update's side (ceil for an upward update, floor for a
- * downward one), so the error stays below one step.  No extra storage.
- * rsq_quantize has no previous state and applies the base rounding. */
-typedef enum { RSQ_RTN = 0, RSQ_SR = 1, RSQ_BDR = 2, RSQ_SR_BDR = 3 } rsq_rounding;
+/* Requantization rule.  RSQ_RTN: nearest code (ties to even).  RSQ_SR8:
+ * stochastic rounding with an 8-bit Philox uniform per element, up with
+ * probability frac(x) rounded to a multiple of 2^-8 ([LoReS] (3/4)); RSQ_SR:
+ * the same with a 16-bit uniform per element, up with probability frac(x) to
+ * within 2^-16 (twice the random bits, twice the Philox work per element).
+ * Bit 0 = stochastic, bit 1 = directional correction, bit 2 = 8-bit uniforms.
+ * RSQ_BDR / RSQ_SR_BDR / RSQ_SR8_BDR: the same base rounding followed by
+ * Bounded Directional Rounding ("Preserving Updates in Low-Bit Recurrent State
+ * Quantization", abstract): when the rounded value c_t s_t lies strictly on
+ * the other side of the previous value c_{t-1} s_{t-1} than the updated state
+ * S_t does (the element moved against its update), the code becomes the
+ * integer next to S_t / s_t on the update's side (ceil for an upward update,
+ * floor for a downward one), so the error stays below one step.  No extra
+ * storage.  rsq_quantize has no previous state and applies the base rounding. */
+typedef enum {
+    RSQ_RTN = 0,
+    RSQ_SR = 1,
+    RSQ_BDR = 2,
+    RSQ_SR_BDR = 3,
+    RSQ_SR8 = 5,
+    RSQ_SR8_BDR = 7
+} rsq_rounding;
 typedef enum { RSQ_F32 = 0, RSQ_BF16 = 1 } rsq_dtype;
 
 /* Device allocator hook for the context's own allocation (its 4-byte flag
@@ -135,11 +146,11 @@ typedef struct {
     int in_dtype;    /* rsq_dtype of the vector inputs (q, k, v / x, B, C) */
     uint64_t seed;   /* stochastic-rounding key */
     int window;      /* pure-write window slots W for Gated DeltaNet ([PW]): 0 (none), 4, 8
-                        or 16; needs RSQ_RTN or RSQ_SR and rsq_decode_step_window */
+                        or 16; needs RSQ_RTN, RSQ_SR or RSQ_SR8 and rsq_decode_step_window */
     int key_axis;    /* 0: one scale per value column (the method's grouping); 1: one scale
                         per key row, s_i = max_j |S_ij| / r ([LoReS] (1/4), the grouping
-                        ablation).  Key-axis: Gated DeltaNet, 4/8-bit heads, RSQ_RTN or
-                        RSQ_SR; scales are [B][H][dk]; one CTA per head. */
+                        ablation).  Key-axis: Gated DeltaNet, 4/8-bit heads, RSQ_RTN,
+                        RSQ_SR or RSQ_SR8; scales are [B][H][dk]; one CTA per head. */
     rsq_alloc_fn alloc;      /* allocator hook (above); NULL with release NULL: cudaMalloc */
     rsq_release_fn release;  /* its release; set both or neither (else RSQ_E_INVAL) */
     void* alloc_user;        /* passed to both */
@@ -225,11 +236,18 @@ rsq_status rsq_head_offset(const rsq_ctx* ctx, int h, size_t* offset);
  *     m_j = max_i |S_ij|;  s'_j = m_j / r;  inv_j = r / m_j rounded toward zero
  *     (inv_j = 0 when m_j = 0);
  *     RTN: c'_ij = nearest integer (ties to even) of the exact S_ij * inv_j
+ *     SR8: t = fma(S_ij, inv_j, 2^15 + o + u_ij/256) in binary32 (t lies in
+ *          [2^15, 2^16), where rounding to the ulp 2^-8 adds the half of
+ *          u + 1/2), c'_ij = floor(t) - 2^15 - o, o = 128 (8-bit) / 8 (4-bit);
+ *          u_ij is an 8-bit uniform from Philox4x32-10 (Salmon et al., SC'11)
+ *          with key = seed and counter { (i mod dk/4) | (j/4) << 16, h, b,
+ *          step }; element (i, j) takes byte j mod 4 (lowest first) of word
+ *          i div (dk/4).
  *     SR : t = fma(S_ij, inv_j, o + u_ij/65536) in binary32, c'_ij = floor(t) - o,
  *          o = 128 (8-bit) / 136 (4-bit); u_ij is a 16-bit uniform from
- *          Philox4x32-10 (Salmon et al., SC'11) with key = seed and counter
- *          { (i mod dk/2) | (j/4) << 16, h, b, step }; element (i, j) takes
- *          16-bit chunk 4*[i >= dk/2] + (j mod 4) (word chunk/2, low half first).
+ *          Philox4x32-10 with counter { (i mod dk/2) | (j/4) << 16, h, b, step };
+ *          element (i, j) takes 16-bit chunk 4*[i >= dk/2] + (j mod 4) (word
+ *          chunk/2, low half first).
  *  32-bit heads skip the quantizer and store S_t; their update is
  *     GDN: u_j = sum_i S_ij k_i, S_ij = fma(alpha, S_ij, k_i*w_j);
  *     Mamba-2: S_ij = fma(a, S_ij, B_i*(dt*x_j)).

@@ -21,6 +21,7 @@ LIB_PATH = os.path.join(_HERE, "librsq.so")
 
 RSQ_GDN, RSQ_MAMBA2, RSQ_GLA, RSQ_KDA = 0, 1, 2, 3
 RSQ_RTN, RSQ_SR, RSQ_BDR, RSQ_SR_BDR = 0, 1, 2, 3
+RSQ_SR8, RSQ_SR8_BDR = 5, 7   # stochastic rounding with 8-bit uniforms (RSQ_SR: 16-bit)
 RSQ_F32, RSQ_BF16 = 0, 1
 RSQ_OK, RSQ_E_INVAL, RSQ_E_UNSUPPORTED, RSQ_E_CUDA, RSQ_E_NOMEM, RSQ_E_NONFINITE = range(6)
 RSQ_MAX_HEADS = 512
@@ -193,7 +194,7 @@ def _stream(stream) -> int | None:
 # C functions under their own names (argument marshalling only)
 # ---------------------------------------------------------------------------
 def rsq_create(family: int, batch: int, heads: int, dk: int, dv: int, *, head_bits=None,
-               rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0,
+               rounding: int = RSQ_SR8, in_dtype: int = RSQ_BF16, seed: int = 0,
                ngroups: int = 1, window: int = 0, key_axis: int = 0, alloc=None, release=None) -> int:
     """``alloc`` / ``release``: rsq_alloc_fn / rsq_release_fn objects (the
     allocator hook; the caller keeps them alive as long as the context)."""
@@ -222,7 +223,7 @@ def _config(family, batch, heads, dk, dv, head_bits, rounding, in_dtype, seed, n
 
 def rsq_decode_step_noalloc(family: int, batch: int, heads: int, dk: int, dv: int, state_in,
                             state_out, inputs, out, step: int, *, head_bits=None,
-                            rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0,
+                            rounding: int = RSQ_SR8, in_dtype: int = RSQ_BF16, seed: int = 0,
                             ngroups: int = 1, stream=None) -> None:
     """Decode step without a context and without any device allocation (the
     kernel's flag word lives in a static device array; see include/rsq.h)."""
@@ -413,7 +414,7 @@ class Context:
     """Owns one rsq_ctx (one layer configuration)."""
 
     def __init__(self, family: int, batch: int, heads: int, dk: int, dv: int, *, head_bits=None,
-                 rounding: int = RSQ_SR, in_dtype: int = RSQ_BF16, seed: int = 0, ngroups: int = 1,
+                 rounding: int = RSQ_SR8, in_dtype: int = RSQ_BF16, seed: int = 0, ngroups: int = 1,
                  window: int = 0, key_axis: int = 0, allocator=None):
         """``allocator``: optional (alloc(nbytes) -> device address or None,
         release(address)) pair for the context's own device word."""

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include "rsq_internal.h"
+#include "rsq_tile.cuh"
 
 namespace rsq {
 
@@ -40,8 +41,8 @@ int decode_kernel_info(int family, int dk, int ub, bool f32state, int rnd, int* 
         {decode_info_mamba2, decode_info_mamba2_bdr, decode_info_mamba2_copy, decode_info_mamba2_copy_bdr},
         {decode_info_gla, decode_info_gla_bdr, decode_info_gla_copy, decode_info_gla_copy_bdr},
         {decode_info_kda, decode_info_kda_bdr, decode_info_kda_copy, decode_info_kda_copy_bdr}};
-    if (rnd < 0 || rnd > 7) return -1;
-    const int group = f32state ? 0 : (rnd >> 1);
+    if (rnd < 0 || rnd > 15) return -1;
+    const int group = f32state ? 0 : (((rnd & kRndBdr) ? 1 : 0) + ((rnd & kRndCopy) ? 2 : 0));
     if (is_pw_family(family)) {  // pure-write window: plain rules only
         static const InfoFn pw[3] = {decode_info_gdn_pw4, decode_info_gdn_pw8, decode_info_gdn_pw16};
         return group == 0 ? pw[family - kFamGdnPw](dk, ub, f32state, rnd, threads, smem, func) : -1;

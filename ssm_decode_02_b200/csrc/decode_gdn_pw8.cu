@@ -6,6 +6,6 @@
 namespace rsq {
 int decode_info_gdn_pw8(int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
                         const void** func) {
-    return decode_info_family<kFamGdnPw + 1, 0, kRndSr>(dk, ub, f32state, rnd, threads, smem, func);
+    return decode_info_family<kFamGdnPw + 1, 0, kRndSr, kRndSr | kRndU8>(dk, ub, f32state, rnd, threads, smem, func);
 }
 }  // namespace rsq

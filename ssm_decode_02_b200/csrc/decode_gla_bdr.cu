@@ -5,7 +5,7 @@
 namespace rsq {
 int decode_info_gla_bdr(int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
                         const void** func) {
-    return decode_info_family<RSQ_GLA, kRndBdr, kRndBdr | kRndSr>(dk, ub, f32state, rnd, threads,
+    return decode_info_family<RSQ_GLA, kRndBdr, kRndBdr | kRndSr, kRndBdr | kRndSr | kRndU8>(dk, ub, f32state, rnd, threads,
                                                                  smem, func);
 }
 }  // namespace rsq

@@ -35,13 +35,16 @@ __device__ __forceinline__ float ka_vec(const void* base, long long e, bool bf16
 }
 
 // Requantize this lane's rows with one multiplier per row (pairs (inv_i, inv_i)
-// at invp[k] for row g + 8k) and store them; RTN or Philox SR as in the
-// value-axis requantizer.
-template <int BITS, bool SR, int RPT>
+// at invp[k] for row g + 8k) and store them; nearest or Philox stochastic
+// rounding (16- or 8-bit uniforms: rule bits RND) as in the value-axis
+// requantizer.
+template <int BITS, int RND, int RPT>
 __device__ __forceinline__ void ka_requantize_store(const uint64_t (&S2)[RPT][2], const uint64_t* invp,
                                                     uint8_t* dst, int g, int cw, uint32_t gcol,
                                                     uint32_t h, uint32_t b, uint32_t step,
                                                     const PhiloxKeys& rk) {
+    constexpr bool SR = (RND & kRndSr) != 0;
+    constexpr bool U8 = SR && (RND & kRndU8) != 0;
     uint8_t* const row0 = dst + (BITS == 8 ? g * 16 + 4 * cw : g * 8 + 2 * cw);
     auto store_row = [&](int k, uint32_t word) {
         if constexpr (BITS == 8)
@@ -57,9 +60,20 @@ __device__ __forceinline__ void ka_requantize_store(const uint64_t (&S2)[RPT][2]
             float t0, t1, t2, t3;
             upk(fma2(S2[k][0], invp[k], moff), t0, t1);
             upk(fma2(S2[k][1], invp[k], moff), t2, t3);
-            store_row(k, pack_row<BITS>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
-                                        __float_as_uint(t3), false));
+            store_row(k, pack_row<BITS, 0>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
+                                           __float_as_uint(t3)));
         }
+    } else if constexpr (U8) {
+        constexpr uint32_t vb = (BITS == 8) ? kSr8Bits8 : kSr8Bits4;
+        sr8_words<RPT, kR>(g, gcol, h, b, step, rk, [&](int kk, uint32_t word) {
+            uint64_t V01, V23;
+            sr8_offsets(word, vb, V01, V23);
+            float t0, t1, t2, t3;
+            upk(fma2(S2[kk][0], invp[kk], V01), t0, t1);
+            upk(fma2(S2[kk][1], invp[kk], V23), t2, t3);
+            store_row(kk, pack_row<BITS, 1>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
+                                            __float_as_uint(t3)));
+        });
     } else {
         constexpr uint32_t vb = (BITS == 8) ? kSrBits8 : kSrBits4;
         const uint64_t mm = pk(kMagic, kMagic);
@@ -83,14 +97,18 @@ __device__ __forceinline__ void ka_requantize_store(const uint64_t (&S2)[RPT][2]
                 float t0, t1, t2, t3;
                 upk(t01, t0, t1);
                 upk(t23, t2, t3);
-                store_row(kk, pack_row<BITS>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
-                                             __float_as_uint(t3), BITS == 4));
+                if constexpr (BITS == 8)
+                    store_row(kk, pack_row<8, 0>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
+                                                 __float_as_uint(t3)));
+                else
+                    store_row(kk, pack_row<4, 2>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
+                                                 __float_as_uint(t3)));
             }
         }
     }
 }
 
-template <int DK, int BITS, bool SR>
+template <int DK, int BITS, int RND>
 __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, int b, int h, int hu) {
     using K = KaCfg<DK>;
     constexpr int RPT = K::RPT;
@@ -202,7 +220,7 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, in
     for (int k = 0; k < RPT; ++k) invp[k] = ki[k];
     uint8_t* dst = p.codes_out + rowoff;
     const uint32_t gcol = static_cast<uint32_t>(j0 / 4 + cw);
-    ka_requantize_store<BITS, SR, RPT>(S2, invp, dst, g, cw, gcol, h, b, p.step, p.rk);
+    ka_requantize_store<BITS, RND, RPT>(S2, invp, dst, g, cw, gcol, h, b, p.step, p.rk);
     // rare: non-finite rows (multiplier -0.0) are stored as the zero code
     bool bad = false;
 #pragma unroll
@@ -215,24 +233,24 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, in
                 S2[k][0] = pk(0.f, 0.f);
                 S2[k][1] = pk(0.f, 0.f);
             }
-        ka_requantize_store<BITS, SR, RPT>(S2, invp, dst, g, cw, gcol, h, b, p.step, p.rk);
+        ka_requantize_store<BITS, RND, RPT>(S2, invp, dst, g, cw, gcol, h, b, p.step, p.rk);
     }
 }
 
-template <int DK, bool SR>
+template <int DK, int RND>
 __global__ void __launch_bounds__(512) rsq_decode_ka_kernel(const __grid_constant__ DecodeParams p) {
     extern __shared__ __align__(16) uint8_t smem[];
     const int hu = blockIdx.x;
     const int b = hu / p.H, h = hu - b * p.H;
     if (p.head_bits[h] == 8)
-        ka_head<DK, 8, SR>(p, smem, b, h, hu);
+        ka_head<DK, 8, RND>(p, smem, b, h, hu);
     else
-        ka_head<DK, 4, SR>(p, smem, b, h, hu);
+        ka_head<DK, 4, RND>(p, smem, b, h, hu);
 }
 
 // Quantize a full-precision head (natural [dk][dv] layout) with key-axis
 // scales: warp w owns block w, row maxima meet in shared memory.
-template <int DK, int BITS, bool SR>
+template <int DK, int BITS, int RND>
 __device__ __forceinline__ void ka_quantize_head(const QuantParams& p, uint8_t* smem, int b, int h, int hu) {
     using K = KaCfg<DK>;
     constexpr int RPT = K::RPT;
@@ -284,7 +302,7 @@ __device__ __forceinline__ void ka_quantize_head(const QuantParams& p, uint8_t* 
     }
     if (bad && cw == 0 && g == 0) atomicOr(p.flag, kFlagNonFinite);
     uint8_t* dst = p.codes + (long long)b * p.row_bytes + p.head_off[h] + (long long)w * BLOCK_BYTES;
-    ka_requantize_store<BITS, SR, RPT>(S2, invp, dst, g, cw, static_cast<uint32_t>(j0 / 4 + cw), h, b, p.step,
+    ka_requantize_store<BITS, RND, RPT>(S2, invp, dst, g, cw, static_cast<uint32_t>(j0 / 4 + cw), h, b, p.step,
                                        p.rk);
 }
 
@@ -294,12 +312,16 @@ __global__ void __launch_bounds__(512) rsq_quantize_ka_kernel(const __grid_const
     const int hu = blockIdx.x;
     const int b = hu / p.H, h = hu - b * p.H;
     const bool bits8 = p.head_bits[h] == 8;
-    if (p.sr) {
-        if (bits8) ka_quantize_head<DK, 8, true>(p, smem, b, h, hu);
-        else ka_quantize_head<DK, 4, true>(p, smem, b, h, hu);
+    constexpr int kSr8 = kRndSr | kRndU8;
+    if (p.rnd == kSr8) {
+        if (bits8) ka_quantize_head<DK, 8, kSr8>(p, smem, b, h, hu);
+        else ka_quantize_head<DK, 4, kSr8>(p, smem, b, h, hu);
+    } else if (p.rnd == kRndSr) {
+        if (bits8) ka_quantize_head<DK, 8, kRndSr>(p, smem, b, h, hu);
+        else ka_quantize_head<DK, 4, kRndSr>(p, smem, b, h, hu);
     } else {
-        if (bits8) ka_quantize_head<DK, 8, false>(p, smem, b, h, hu);
-        else ka_quantize_head<DK, 4, false>(p, smem, b, h, hu);
+        if (bits8) ka_quantize_head<DK, 8, 0>(p, smem, b, h, hu);
+        else ka_quantize_head<DK, 4, 0>(p, smem, b, h, hu);
     }
 }
 
@@ -317,11 +339,13 @@ size_t ka_smem(int nw) {
 }
 
 template <int DK>
-int launch_ka_dk(const DecodeParams& p, bool sr, void* stream) {
+int launch_ka_dk(const DecodeParams& p, void* stream) {
     const int nw = p.dv / kBlockCols;
     const size_t smem = ka_smem<DK>(nw);
-    const void* f = sr ? reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, true>)
-                       : reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, false>);
+    constexpr int kSr8 = kRndSr | kRndU8;
+    const void* f = p.rnd == kSr8    ? reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, kSr8>)
+                    : p.rnd == kRndSr ? reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, kRndSr>)
+                                      : reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, 0>);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.B * p.H);
     cfg.blockDim = dim3(32 * nw);
@@ -343,12 +367,12 @@ int launch_quantize_ka(int dk, const QuantParams& p, void* stream) {
     }
 }
 
-int launch_decode_ka(int dk, const DecodeParams& p, bool sr, void* stream) {
+int launch_decode_ka(int dk, const DecodeParams& p, void* stream) {
     switch (dk) {
-        case 16: return launch_ka_dk<16>(p, sr, stream);
-        case 32: return launch_ka_dk<32>(p, sr, stream);
-        case 64: return launch_ka_dk<64>(p, sr, stream);
-        case 128: return launch_ka_dk<128>(p, sr, stream);
+        case 16: return launch_ka_dk<16>(p, stream);
+        case 32: return launch_ka_dk<32>(p, stream);
+        case 64: return launch_ka_dk<64>(p, stream);
+        case 128: return launch_ka_dk<128>(p, stream);
         default: return static_cast<int>(cudaErrorInvalidValue);
     }
 }

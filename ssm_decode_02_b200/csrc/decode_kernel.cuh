@@ -826,24 +826,30 @@ int decode_info_one(int* threads, size_t* smem, const void** func) {
 }
 
 // All (dk, blocks per unit) instantiations of one family for the rounding
-// rules in RNDS (a full-precision state ignores the rounding: it is built with
-// the first rule only).  The rules are split over translation units so the
-// instantiations compile in parallel.
-template <int FAM, int RND0, int RND1>
+// rules RND0, RNDS... (a full-precision state ignores the rounding: it is built
+// with the first rule only, when that rule is plain nearest rounding).  The
+// rules are split over translation units so the instantiations compile in
+// parallel.
+template <int FAM, int DK, int UB, int RND0, int... RNDS>
+int decode_info_rules(bool f32state, int rnd, int* threads, size_t* smem, const void** func) {
+    if (f32state) {
+        if constexpr (RND0 == 0)
+            return decode_info_one<FAM, DK, UB, true, 0>(threads, smem, func);
+        else
+            return -1;
+    }
+    int found = -1;
+    if (rnd == RND0) found = decode_info_one<FAM, DK, UB, false, RND0>(threads, smem, func);
+    ((found != 0 && rnd == RNDS ? (found = decode_info_one<FAM, DK, UB, false, RNDS>(threads, smem, func)) : 0),
+     ...);
+    return found;
+}
+
+template <int FAM, int... RNDS>
 int decode_info_family(int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
                        const void** func) {
-#define RSQ_CASE(DK_, UB_)                                                                      \
-    if (dk == DK_ && ub == UB_) {                                                                \
-        if (f32state) {                                                                          \
-            if constexpr (RND0 == 0)                                                             \
-                return decode_info_one<FAM, DK_, UB_, true, 0>(threads, smem, func);             \
-            else                                                                                 \
-                return -1;                                                                       \
-        }                                                                                        \
-        if (rnd == RND0) return decode_info_one<FAM, DK_, UB_, false, RND0>(threads, smem, func); \
-        if (rnd == RND1) return decode_info_one<FAM, DK_, UB_, false, RND1>(threads, smem, func); \
-        return -1;                                                                               \
-    }
+#define RSQ_CASE(DK_, UB_)                                                                 \
+    if (dk == DK_ && ub == UB_) return decode_info_rules<FAM, DK_, UB_, RNDS...>(f32state, rnd, threads, smem, func);
     RSQ_CASE(16, 1) RSQ_CASE(16, 2) RSQ_CASE(16, 4)
     RSQ_CASE(32, 1) RSQ_CASE(32, 2) RSQ_CASE(32, 4)
     RSQ_CASE(64, 1) RSQ_CASE(64, 2) RSQ_CASE(64, 4)

@@ -1,10 +1,10 @@
 // decode_mamba2.cu -- Mamba-2 instantiations of the fused decode kernel with
-// nearest and stochastic rounding (and the full-precision state).
+// nearest and stochastic rounding, 16- and 8-bit uniforms (and the full-precision state).
 #include "decode_kernel.cuh"
 
 namespace rsq {
 int decode_info_mamba2(int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
                     const void** func) {
-    return decode_info_family<RSQ_MAMBA2, 0, kRndSr>(dk, ub, f32state, rnd, threads, smem, func);
+    return decode_info_family<RSQ_MAMBA2, 0, kRndSr, kRndSr | kRndU8>(dk, ub, f32state, rnd, threads, smem, func);
 }
 }  // namespace rsq

@@ -70,7 +70,9 @@ __device__ __forceinline__ void quantize_block(const QuantParams& p, const Block
         const uint32_t gcol = static_cast<uint32_t>(j0 / 4 + cw);
         // no previous state: the base rounding of the context's rule
         const BdrRef none{};
-        if (p.sr)
+        if (p.rnd == (kRndSr | kRndU8))
+            requantize_store<BITS, kRndSr | kRndU8, RPT>(S2, iv, dst, g, cw, gcol, bi.h, bi.b, p.step, p.rk, none);
+        else if (p.rnd == kRndSr)
             requantize_store<BITS, kRndSr, RPT>(S2, iv, dst, g, cw, gcol, bi.h, bi.b, p.step, p.rk, none);
         else
             requantize_store<BITS, 0, RPT>(S2, iv, dst, g, cw, gcol, bi.h, bi.b, p.step, p.rk, none);

@@ -51,14 +51,20 @@ rsq_status cuda_fail(int err, const char* what) {
     return fail(RSQ_E_CUDA, "%s: %s", what, cudaGetErrorString(static_cast<cudaError_t>(err)));
 }
 
-constexpr int kCopyScaleBit = 4;  // kernel rule bit of the copy scale (beside the rsq_rounding bits)
+constexpr int kCopyScaleBit = rsq::kRndCopy;  // kernel rule bit of the copy scale (beside the rsq_rounding bits)
 // Kernel family of a configuration (Gated DeltaNet with a window has its own kernels).
 int kernel_family(const rsq_config& c) {
     if (c.family != RSQ_GDN || c.window <= 0) return c.family;
     return rsq::kFamGdnPw + (c.window == 4 ? 0 : (c.window == 8 ? 1 : 2));
 }
 bool family_ok(int f) { return f == RSQ_GDN || f == RSQ_MAMBA2 || f == RSQ_GLA || f == RSQ_KDA; }
-bool rounding_ok(int r) { return r == RSQ_RTN || r == RSQ_SR || r == RSQ_BDR || r == RSQ_SR_BDR; }
+bool rounding_ok(int r) {
+    return r == RSQ_RTN || r == RSQ_SR || r == RSQ_BDR || r == RSQ_SR_BDR || r == RSQ_SR8 || r == RSQ_SR8_BDR;
+}
+// nearest or stochastic rounding without the directional correction
+bool plain_rounding(int r) { return r == RSQ_RTN || r == RSQ_SR || r == RSQ_SR8; }
+// base-rounding bits of the kernels (stochastic, 8-bit uniforms)
+int base_rule(int r) { return r & (rsq::kRndSr | rsq::kRndU8); }
 // 16-column blocks per work unit (at most): four, except stochastic rounding
 // at dk = 256, whose two-warp blocks run faster as 128-thread CTAs at three
 // per SM (168 registers, no spills) than as 256-thread CTAs at two.
@@ -147,12 +153,12 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
         return fail(RSQ_E_INVAL, "create: window must be 0, 4, 8 or 16 (got %d)", c.window);
     if (c.window && c.family != RSQ_GDN)
         return fail(RSQ_E_UNSUPPORTED, "create: the pure-write window is defined for Gated DeltaNet");
-    if (c.window && c.rounding != RSQ_RTN && c.rounding != RSQ_SR)
+    if (c.window && !plain_rounding(c.rounding))
         return fail(RSQ_E_UNSUPPORTED, "create: the pure-write window takes nearest or stochastic rounding");
     if (c.key_axis != 0 && c.key_axis != 1) return fail(RSQ_E_INVAL, "create: key_axis must be 0 or 1");
     if ((c.alloc == nullptr) != (c.release == nullptr))
         return fail(RSQ_E_INVAL, "create: set both alloc and release, or neither");
-    if (c.key_axis && (c.family != RSQ_GDN || c.window || (c.rounding != RSQ_RTN && c.rounding != RSQ_SR)))
+    if (c.key_axis && (c.family != RSQ_GDN || c.window || !plain_rounding(c.rounding)))
         return fail(RSQ_E_UNSUPPORTED, "create: key-axis scales: Gated DeltaNet, no window, nearest or stochastic rounding");
     if ((c.window || c.key_axis) && c.dk > 128)
         return fail(RSQ_E_UNSUPPORTED, "create: the pure-write window and key-axis scales are built for dk <= 128");
@@ -352,7 +358,7 @@ rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const
     std::memset(&p, 0, sizeof(p));
     p.B = c.batch; p.H = c.heads; p.dk = c.dk; p.dv = c.dv; p.ncb = ctx->ncb; p.units = ctx->units;
     p.in_bf16 = (c.in_dtype == RSQ_BF16);
-    p.sr = (c.rounding & RSQ_SR) != 0;
+    p.rnd = base_rule(c.rounding);
     p.row_bytes = ctx->row_bytes;
     p.codes_in = static_cast<const uint8_t*>(state_in->codes);
     p.codes_out = static_cast<uint8_t*>(state_out->codes);
@@ -411,7 +417,7 @@ rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const
     p.gb = ghu / c.heads;
     if (c.key_axis) {
         if (copy_absmax) return fail(RSQ_E_UNSUPPORTED, "decode_step_copy_scale: not with key-axis scales");
-        const int e = rsq::launch_decode_ka(c.dk, p, (c.rounding & RSQ_SR) != 0, stream);
+        const int e = rsq::launch_decode_ka(c.dk, p, stream);
         if (e) return cuda_fail(e, "decode_step launch");
         return RSQ_OK;
     }
@@ -434,7 +440,7 @@ rsq_status rsq_quantize(const rsq_ctx* ctx, const float* S, const rsq_state* sta
     rsq::QuantParams p;
     std::memset(&p, 0, sizeof(p));
     p.B = c.batch; p.H = c.heads; p.dk = c.dk; p.dv = c.dv; p.ncb = ctx->ncb; p.units = ctx->units;
-    p.sr = (c.rounding & RSQ_SR) != 0;
+    p.rnd = base_rule(c.rounding);
     p.row_bytes = ctx->row_bytes;
     p.S = S;
     p.codes = static_cast<uint8_t*>(state_out->codes);

@@ -42,7 +42,8 @@ struct DecodeParams {
     int gcb, gh, gb;               // G decomposed as (batch, head, column block) steps
     int ngroups, heads_per_group;
     int in_bf16;                   // vector inputs are bf16 (else float)
-    int sr;                        // stochastic rounding (else round-to-nearest)
+    int rnd;                       // base rounding: 0 nearest, kRndSr (16-bit uniforms),
+                                   // kRndSr | kRndU8 (8-bit uniforms)
     long long row_bytes;           // code bytes per batch row
     const uint8_t* codes_in;
     uint8_t* codes_out;
@@ -78,7 +79,7 @@ struct DecodeParams {
 
 struct QuantParams {
     int B, H, dk, dv, ncb, units;
-    int sr;
+    int rnd;                       // base rounding bits, as DecodeParams::rnd
     long long row_bytes;
     const float* S;                // natural [B][H][dk][dv]
     uint8_t* codes;
@@ -122,7 +123,7 @@ int decode_kernel_info(int family, int dk, int ub, bool f32state, int rnd, int* 
 int launch_quantize(int dk, const QuantParams& p, void* stream);
 int launch_dequantize(int dk, const DequantParams& p, void* stream);
 // key-axis scale groups (one CTA per head)
-int launch_decode_ka(int dk, const DecodeParams& p, bool sr, void* stream);
+int launch_decode_ka(int dk, const DecodeParams& p, void* stream);
 int launch_quantize_ka(int dk, const QuantParams& p, void* stream);
 int launch_drift(const DriftParams& p, void* stream);
 

@@ -21,15 +21,23 @@ namespace rsq {
 
 constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23: ulp 1, integers land in the low mantissa bits
 constexpr uint32_t kMagicBits = 0x4B400000u;
-constexpr uint32_t kSrBits8 = 0x43000000u;  // 128.0f: SR offset of 8-bit codes
-constexpr uint32_t kSrBits4 = 0x43080000u;  // 136.0f: SR offset of 4-bit codes
+constexpr uint32_t kSrBits8 = 0x43000000u;  // 128.0f: SR offset of 8-bit codes (16-bit uniforms)
+constexpr uint32_t kSrBits4 = 0x43080000u;  // 136.0f: SR offset of 4-bit codes (16-bit uniforms)
+// 8-bit uniforms: t = S*inv + 2^15 + o + u/2^8 lies in [2^15, 2^16), where the
+// ulp is 2^-8: u fills the low byte of the offset and floor(t) - 2^15 = c + o
+// lands in byte 1 of t.  o = 128 (8-bit codes) or 8 (4-bit codes).
+constexpr uint32_t kSr8Bits8 = 0x47008000u;  // 32896.0f
+constexpr uint32_t kSr8Bits4 = 0x47000800u;  // 32776.0f
 
 // Requantization rule of a kernel instance: bit 0 = stochastic base rounding
 // (else nearest), bit 1 = Bounded Directional Rounding on top of it, bit 2 =
-// scales from the column maxima of an unquantized copy (copy scale).
+// 8-bit uniforms for the stochastic rounding (else 16-bit), bit 3 = scales
+// from the column maxima of an unquantized copy (copy scale).  Bits 0-2 are
+// the public rsq_rounding value.
 constexpr int kRndSr = 1;
 constexpr int kRndBdr = 2;
-constexpr int kRndCopy = 4;
+constexpr int kRndU8 = 4;
+constexpr int kRndCopy = 8;
 
 constexpr int kBlockCols = 16;  // columns per stored block (one warp)
 constexpr int kR = 8;           // partial sums over the key axis (row groups)
@@ -156,25 +164,65 @@ __device__ __forceinline__ void load_code_row(const uint8_t* blk, int g, int cw,
     c23 = S2[0][1];
 }
 
-// Pack the 4 codes of one row held in the low byte (RTN) or byte 2 (4-bit SR)
-// of four floats into the stored representation.
-template <int BITS>
-__device__ __forceinline__ uint32_t pack_row(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3,
-                                             bool byte2) {
-    if constexpr (BITS == 8) {
+// Pack the 4 codes of one row held in byte B of four floats (byte 0: nearest
+// rounding and 8-bit codes with 16-bit uniforms; byte 1: 8-bit uniforms;
+// byte 2: 4-bit codes with 16-bit uniforms) into the stored representation.
+template <int BITS, int B>
+__device__ __forceinline__ uint32_t pack_row(uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3) {
+    if constexpr (BITS == 8 && B == 0) {
         // Byte 0 of each float holds c + 128 and byte 1 is zero, so t1*256 + t0
         // (mod 2^32) carries (byte0(t1), byte0(t0)) in its low 16 bits without any
         // carry between them; one byte permute joins the two halves.
         const uint32_t a = t1 * 256u + t0;
         const uint32_t b = t3 * 256u + t2;
         return prmt(a, b, 0x5410u);
+    } else if constexpr (BITS == 8) {
+        constexpr uint32_t sel = (4u + B) << 4 | B;  // bytes B of the two operands
+        return prmt(prmt(t0, t1, sel), prmt(t2, t3, sel), 0x5410u);
     } else {
-        // the code nibble c + 8 sits in byte 0 (RTN) or byte 2 (SR)
-        const uint32_t sel = byte2 ? 0x0062u : 0x0040u;
+        // the code nibble c + 8 sits in byte B
+        constexpr uint32_t sel = (4u + B) << 4 | B;
         const uint32_t a = prmt(t0, t2, sel);  // columns 0, 2
         const uint32_t b = prmt(t1, t3, sel);  // columns 1, 3
         return a + (b << 4);                   // low 16 bits are the two stored bytes
     }
+}
+
+// Stochastic rounding with 8-bit uniforms: the Philox4x32-10 words of this
+// lane's rows.  One block with counter {i mod dk/4 | (j/4) << 16, h, b, step}
+// serves rows i, i + dk/4, i + dk/2, i + 3dk/4 of four columns: word
+// i div (dk/4), byte j mod 4.  The lane's rows are g + RS k (k < RPT), so the
+// block of counter row g + RS k (k < RPT/4) gives rows k + q RPT/4 word q;
+// with two rows per lane (dk = 16) both rows share counter row g mod 4.
+// row_fn(k, word) is called once per row.
+template <int RPT, int RS, class PhiloxKeysT, class F>
+__device__ __forceinline__ void sr8_words(int g, uint32_t gcol, uint32_t h, uint32_t b, uint32_t step,
+                                          const PhiloxKeysT& rk, F&& row_fn) {
+    if constexpr (RPT >= 4) {
+        constexpr int Q = RPT / 4;
+#pragma unroll
+        for (int k = 0; k < Q; ++k) {
+            const uint32_t i = static_cast<uint32_t>(g + RS * k);
+            const U4 rnd = philox4x32_10(U4{i | (gcol << 16), h, b, step}, rk.k0, rk.k1);
+            row_fn(k, rnd.x);
+            row_fn(k + Q, rnd.y);
+            row_fn(k + 2 * Q, rnd.z);
+            row_fn(k + 3 * Q, rnd.w);
+        }
+    } else {
+        static_assert(RPT == 2 && RS == 8, "two rows per lane only at dk = 16");
+        const U4 rnd = philox4x32_10(U4{static_cast<uint32_t>(g & 3) | (gcol << 16), h, b, step}, rk.k0, rk.k1);
+        const bool upper = g >= 4;  // rows g, g + 8 are words g/4 and g/4 + 2
+        row_fn(0, upper ? rnd.y : rnd.x);
+        row_fn(1, upper ? rnd.w : rnd.z);
+    }
+}
+
+// The offsets 2^15 + o + u/2^8 of one row's four columns, u = byte jj of the
+// row's Philox word (column 4cw + jj), as two packed pairs.
+__device__ __forceinline__ void sr8_offsets(uint32_t word, uint32_t vb, uint64_t& V01, uint64_t& V23) {
+    V01 = pk(__uint_as_float(prmt(word, vb, 0x7650u)), __uint_as_float(prmt(word, vb, 0x7651u)));
+    V23 = pk(__uint_as_float(prmt(word, vb, 0x7652u)), __uint_as_float(prmt(word, vb, 0x7653u)));
 }
 
 // Non-finite columns (multiplier -0.0) must come out as the zero code; their
@@ -214,11 +262,13 @@ __device__ __forceinline__ float bdr_pick(float S, float prev, float now, float 
 //   RTN: nearest integer of the exact S*inv (fma with a magic offset).
 //   SR : t = fma(S, inv, o + u/2^16), c = floor(t) - o, u a 16-bit uniform from
 //        Philox4x32-10 with counter {i mod dk/2 | (j/4) << 16, h, b, step}.
+//   SR, 8-bit uniforms: t = fma(S, inv, 2^15 + o + u/2^8) in [2^15, 2^16),
+//        c = floor(t) - 2^15 - o (byte 1 of t), u from sr8_words.
 //   +BDR: the base code is replaced by ceil / floor of the exact S*inv when it
 //        moves the element opposite to its update (see bdr_pick).
 // `gcol` is j/4 of this lane's first column; the lane's rows are g + RS k
 // (RS: as for load_codes; RS * RPT / 2 = dk / 2, so rows k and k + RPT/2 are
-// the pair i, i + dk/2 that one Philox call serves).
+// the pair i, i + dk/2 that one 16-bit-uniform Philox call serves).
 template <int BITS, int RND, int RPT, class PhiloxKeysT, int RS = kR>
 __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], const float4& iv,
                                                  uint8_t* dst, int g, int cw, uint32_t gcol,
@@ -226,6 +276,7 @@ __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], c
                                                  const PhiloxKeysT& rk, const BdrRef& bdr) {
     constexpr bool SR = (RND & kRndSr) != 0;
     constexpr bool BDR = (RND & kRndBdr) != 0;
+    constexpr bool U8 = SR && (RND & kRndU8) != 0;
     constexpr float kOff = (BITS == 8) ? 128.0f : 8.0f;  // stored code = c + kOff
     const uint64_t inv01 = pk(iv.x, iv.y), inv23 = pk(iv.z, iv.w);
     // this lane's first row; row k sits k * RS rows further
@@ -256,12 +307,31 @@ __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], c
         float t0, t1, t2, t3;
         upk(T01, t0, t1);
         upk(T23, t2, t3);
-        store_row(k, pack_row<BITS>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
-                                    __float_as_uint(t3), false));
+        store_row(k, pack_row<BITS, 0>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
+                                       __float_as_uint(t3)));
     };
     if constexpr (!SR) {
 #pragma unroll
         for (int k = 0; k < RPT; ++k) finish_row(k, fma2(S2[k][0], inv01, moff), fma2(S2[k][1], inv23, moff));
+    } else if constexpr (U8) {
+        constexpr uint32_t vb = (BITS == 8) ? kSr8Bits8 : kSr8Bits4;
+        sr8_words<RPT, RS>(g, gcol, h, b, step, rk, [&](int kk, uint32_t word) {
+            uint64_t V01, V23;
+            sr8_offsets(word, vb, V01, V23);
+            const uint64_t t01 = fma2(S2[kk][0], inv01, V01);
+            const uint64_t t23 = fma2(S2[kk][1], inv23, V23);
+            if constexpr (BDR) {
+                // floor(t) - 2^15 + M: the magic domain of the directional rounding
+                const uint64_t to_magic = pk(kMagic - 32768.0f, kMagic - 32768.0f);
+                finish_row(kk, add2_rm(t01, to_magic), add2_rm(t23, to_magic));
+            } else {
+                float t0, t1, t2, t3;
+                upk(t01, t0, t1);
+                upk(t23, t2, t3);
+                store_row(kk, pack_row<BITS, 1>(__float_as_uint(t0), __float_as_uint(t1), __float_as_uint(t2),
+                                                __float_as_uint(t3)));
+            }
+        });
     } else {
         constexpr uint32_t vb = (BITS == 8) ? kSrBits8 : kSrBits4;
         const uint64_t mm = pk(kMagic, kMagic);
@@ -297,8 +367,8 @@ __device__ __forceinline__ void requantize_store(const uint64_t (&S2)[RPT][2], c
                     float t0, t1, t2, t3;
                     upk(t01, t0, t1);
                     upk(t23, t2, t3);
-                    store_row(kk, pack_row<BITS>(__float_as_uint(t0), __float_as_uint(t1),
-                                                 __float_as_uint(t2), __float_as_uint(t3), true));
+                    store_row(kk, pack_row<BITS, 2>(__float_as_uint(t0), __float_as_uint(t1),
+                                                    __float_as_uint(t2), __float_as_uint(t3)));
                 }
             }
         }

@@ -38,7 +38,9 @@ class Run:
         self.dk, self.dv = w.dk, w.dv
         self.head_bits = np.asarray(head_bits, np.int8)
         assert self.head_bits.shape == (self.H,)
-        self.rounding = {"rtn": rsq.RSQ_RTN, "sr": rsq.RSQ_SR}[w.rounding] if rounding is None else rounding
+        # the workloads' stochastic rounding is the 8-bit-uniform rule; "sr16" the 16-bit one
+        self.rounding = ({"rtn": rsq.RSQ_RTN, "sr": rsq.RSQ_SR8, "sr16": rsq.RSQ_SR}[w.rounding]
+                         if rounding is None else rounding)
         self.seed = w.sr_seed if seed is None else seed
         self.in_dtype = {"f32": rsq.RSQ_F32, "bf16": rsq.RSQ_BF16}[w.in_dtype] if in_dtype is None else in_dtype
         self.family = {"gdn": rsq.RSQ_GDN, "mamba2": rsq.RSQ_MAMBA2, "gla": rsq.RSQ_GLA,

@@ -58,6 +58,7 @@ def _create(**kw):
     (dict(dk=256, key_axis=1), rsq.RSQ_E_UNSUPPORTED),
     (dict(dv=8), rsq.RSQ_E_UNSUPPORTED),
     (dict(rounding=4), rsq.RSQ_E_INVAL),
+    (dict(rounding=6), rsq.RSQ_E_INVAL),
     (dict(rounding=-1), rsq.RSQ_E_INVAL),
     (dict(in_dtype=9), rsq.RSQ_E_INVAL),
     (dict(head_bits=[8, 4, 2, 8]), rsq.RSQ_E_INVAL),

@@ -29,7 +29,7 @@ def _start(run: Run, seed: int) -> dict:
     return oracle.quantize(S, run.head_bits, rounding=run.rounding, seed=run.seed, step=0)
 
 
-@pytest.mark.parametrize("rounding", [rsq.RSQ_BDR, rsq.RSQ_SR_BDR])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_BDR, rsq.RSQ_SR_BDR, rsq.RSQ_SR8_BDR])
 @pytest.mark.parametrize("family,dk,dv", [("gdn", 128, 128), ("gdn", 32, 16), ("gdn", 64, 256),
                                           ("mamba2", 128, 64), ("mamba2", 16, 32)])
 def test_bdr_bit_exact(rounding, family, dk, dv):
@@ -48,7 +48,7 @@ def test_bdr_full_size_sampled_heads():
     _trajectory(run, 3, heads=heads)
 
 
-@pytest.mark.parametrize("base,bdr", [(rsq.RSQ_RTN, rsq.RSQ_BDR), (rsq.RSQ_SR, rsq.RSQ_SR_BDR)])
+@pytest.mark.parametrize("base,bdr", [(rsq.RSQ_RTN, rsq.RSQ_BDR), (rsq.RSQ_SR, rsq.RSQ_SR_BDR), (rsq.RSQ_SR8, rsq.RSQ_SR8_BDR)])
 def test_bdr_changes_codes_only_by_one_step(base, bdr):
     """One step from the same state: the rule keeps the scales, moves codes by at
     most one step, and does move some (reversals are common at 4 bits)."""

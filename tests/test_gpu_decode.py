@@ -175,7 +175,7 @@ def test_shapes_mamba2_groups(dk, dv):
     _trajectory(run, 3)
 
 
-@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_SR8])
 @pytest.mark.parametrize("in_dtype", [rsq.RSQ_F32, rsq.RSQ_BF16])
 def test_rounding_and_input_dtypes(rounding, in_dtype):
     w = dataclasses.replace(WL[1], B=3, H=4)
@@ -255,7 +255,7 @@ def test_nonfinite_column_flagged_and_zeroed():
 
 
 def test_quantize_dequantize_kernels_bit_exact():
-    for rounding in (rsq.RSQ_RTN, rsq.RSQ_SR):
+    for rounding in (rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_SR8):
         w = dataclasses.replace(WL[1], B=3, H=4, dk=64, dv=128)
         run = Run(w, np.array([8, 4, 8, 4], np.int8), rounding=rounding)
         rng = np.random.default_rng(rounding)

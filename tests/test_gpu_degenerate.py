@@ -44,7 +44,7 @@ def _extreme_state(B, H, dk, dv, seed, maxima=MAXIMA, fmax=True):
     return S
 
 
-@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_SR8])
 def test_quantize_dequantize_extreme_magnitudes(rounding):
     w = dataclasses.replace(W.WORKLOADS[1], B=2, H=4, dk=32, dv=32)
     bits = np.array([8, 4, 4, 8], np.int8)
@@ -75,7 +75,7 @@ def _run_steps(run: Run, st: dict, inputs_at, steps: int, decay_at=None):
     return st
 
 
-@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_SR_BDR])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_SR8, rsq.RSQ_SR8_BDR])
 def test_decode_from_extreme_state(rounding):
     w = dataclasses.replace(W.WORKLOADS[1], B=2, H=4, dk=32, dv=32, in_dtype="f32")
     bits = np.array([8, 4, 8, 4], np.int8)
@@ -95,7 +95,7 @@ def test_decode_from_extreme_state(rounding):
     _run_steps(run, st, inputs_at, 3)
 
 
-@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_BDR])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR8, rsq.RSQ_BDR])
 def test_gdn_gate_and_vector_extremes(rounding):
     H = 8
     w = dataclasses.replace(W.WORKLOADS[1], B=2, H=H, dk=32, dv=64, in_dtype="f32")

@@ -29,7 +29,7 @@ def test_reduction_partials_at_256():
 
 
 @pytest.mark.parametrize("dv", [16, 32, 64, 256])
-@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_SR8])
 def test_gdn_dk256_bit_exact(dv, rounding):
     w = dataclasses.replace(GDN, B=3, H=4, dk=256, dv=dv)
     run = Run(w, np.array([8, 4, 4, 8], np.int8), rounding=rounding)
@@ -122,7 +122,7 @@ def test_dk256_copy_scale_bit_exact():
         assert_out_equal(host(out_q), o, what="step %d" % t)
 
 
-@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_SR8])
 def test_dk256_quantize_dequantize_drift(rounding):
     w = dataclasses.replace(GDN, B=2, H=3, dk=256, dv=64)
     bits = np.array([8, 4, 8], np.int8)

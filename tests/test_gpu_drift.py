@@ -23,7 +23,7 @@ import bench  # noqa: E402
 
 
 def _oracle_series(w, steps, every, variants):
-    rnd = {"sr": oracle.SR, "rtn": oracle.RTN, "bdr": oracle.BDR, "sr_bdr": oracle.SR_BDR}
+    rnd = {"sr": oracle.SR8, "rtn": oracle.RTN, "bdr": oracle.BDR, "sr_bdr": oracle.SR8_BDR, "sr16": oracle.SR}
     ref = oracle.zero_state(w.B, w.H, w.dk, w.dv, fp32=True)
     qs = {lab: (oracle.zero_state_ka(w.B, w.H, w.dk, w.dv) if src == "keyaxis"
                 else oracle.zero_state(w.B, w.H, w.dk, w.dv, fp32=False)) for lab, _, _, src in variants}

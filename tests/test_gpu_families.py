@@ -27,12 +27,12 @@ KDA = W.BY_NAME["kda_b64_h16_d128_int8_sr"]
 def _start(run: Run, seed: int) -> dict:
     rng = np.random.default_rng(seed)
     S = (rng.standard_normal((run.B, run.H, run.dk, run.dv)) * 0.2).astype(np.float32)
-    return oracle.quantize(S, run.head_bits, rounding=run.rounding & 1, seed=run.seed, step=0)
+    return oracle.quantize(S, run.head_bits, rounding=run.rounding & ~oracle.BDR, seed=run.seed, step=0)
 
 
 @pytest.mark.parametrize("base", [GLA, KDA], ids=["gla", "kda"])
 @pytest.mark.parametrize("dk,dv", [(128, 128), (16, 16), (32, 64), (64, 256)])
-@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_SR8])
 def test_diag_bit_exact(base, dk, dv, rounding):
     w = dataclasses.replace(base, B=3, H=4, dk=dk, dv=dv)
     run = Run(w, np.array([8, 4, 4, 8], np.int8), rounding=rounding)

@@ -66,7 +66,7 @@ def _trajectory(run: KaRun, steps, heads=None, seed=5):
 
 
 @pytest.mark.parametrize("dk,dv", [(128, 128), (16, 16), (32, 64), (64, 256), (128, 32)])
-@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_SR8])
 def test_key_axis_decode_bit_exact(dk, dv, rounding):
     w = dataclasses.replace(W.WORKLOADS[1], B=3, H=4, dk=dk, dv=dv)
     _trajectory(KaRun(w, [8, 4, 4, 8], rounding), 4, seed=dk + dv)
@@ -83,7 +83,7 @@ def test_key_axis_full_size_sampled_heads():
     _trajectory(run, 2, heads=sample_heads(w.B, w.H, 32, seed=7))
 
 
-@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_SR8])
 def test_key_axis_quantize_dequantize_and_maxima(rounding):
     w = dataclasses.replace(W.WORKLOADS[1], B=2, H=3, dk=64, dv=128)
     run = KaRun(w, [8, 4, 8], rounding)

@@ -70,7 +70,7 @@ def _run(w, bits, Wn, rounding, steps, heads=None):
 
 
 @pytest.mark.parametrize("Wn", [4, 8, 16])
-@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_RTN, rsq.RSQ_SR, rsq.RSQ_SR8])
 def test_window_bit_exact(Wn, rounding):
     w = dataclasses.replace(W.WORKLOADS[1], B=3, H=4)
     _run(w, np.array([4, 8, 4, 4], np.int8), Wn, rounding, 2 * Wn + 3)
