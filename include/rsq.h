@@ -30,8 +30,9 @@
  *    marked "host" are ordinary host memory.
  *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *    stream).  Every call that takes a stream is asynchronous on that stream
- *    and never synchronizes, except rsq_check_flags.  Calls may be captured
- *    into CUDA graphs.
+ *    and never synchronizes, except rsq_check_flags.  rsq_decode_step,
+ *    rsq_decode_step_window, rsq_quantize and rsq_dequantize may be captured
+ *    into CUDA graphs (the benchmark replays them from graphs).
  *  - Host-side validation happens before any CUDA call; a failing check
  *    returns RSQ_E_INVAL or RSQ_E_UNSUPPORTED and touches no memory.  A
  *    failed launch returns RSQ_E_CUDA.  rsq_last_error() then holds a
@@ -347,6 +348,20 @@ rsq_status rsq_decode_step_window(const rsq_ctx* ctx, const rsq_state* state_in,
  * column.  Returns RSQ_E_NONFINITE when *seen = 1. */
 rsq_status rsq_check_flags(const rsq_ctx* ctx, int* seen, void* stream);
 
+/* Failure-detection hook for tests (no counterpart in the method's pages).
+ * Sets the limit of this context's decode kernels' bounded barrier waits to
+ * `wait_iters` polls (0: the default, 2^22) and, with withhold = 1, makes
+ * the second warp of every two-warp
+ * block (dk = 256) skip its arrivals on the block's exchange barrier, so that
+ * both warps' waits on it run out.  A kernel whose wait runs out sets the
+ * context's timeout flag, waits (bounded) for the copies it still has in
+ * flight towards its shared memory, and ends; that step's outputs are
+ * incomplete and rsq_check_flags returns RSQ_E_CUDA.  withhold = 0 and
+ * wait_iters = 0 restore normal operation.  For tests of the failure path:
+ * call it while no step of the context is in flight, from one thread.
+ * RSQ_E_INVAL for a null context or withhold not 0 or 1. */
+rsq_status rsq_debug_waits(rsq_ctx* ctx, uint32_t wait_iters, int withhold);
+
 /* Decay-based mixed precision ([LoReS] (2/4)): host-only.  score: host
  * double [heads] (a decay statistic, e.g. the mean gate alpha; larger = slower
  * decay).  The n_high heads with the largest score get high_bits, the others
@@ -363,20 +378,24 @@ int rsq_reduction_partials(int dk);
  * Same computation, arguments and results as rsq_decode_step, but without a
  * context: the configuration is passed directly and nothing is allocated.
  * rsq_create allocates a 4-byte device flag word (cudaMalloc, or the
- * config's allocator hook); callers that may not allocate device memory at
- * all -- code running inside CUDA stream capture (allocation calls are not
- * capturable) -- use this entry point instead.  cfg->alloc, release and
- * alloc_user are ignored here.
+ * config's allocator hook).  Some callers cannot allocate device memory once
+ * they are running: serving runtimes that reserve nearly all GPU memory for
+ * their own pools at start-up (a later cudaMalloc could fail or fragment what
+ * the pool manages) and embedded hosts with a fixed memory budget.  They use
+ * this entry point instead.  cfg->alloc, release and alloc_user are ignored.
  *
  * Its scratch (the decode kernel's flag word) lives in a statically allocated
  * device array of 64 words (256 bytes) that every GPU loading the library
  * holds until the process exits; a call needing more scratch than that is
  * rejected with RSQ_E_UNSUPPORTED.  All calls share the array: the flag word is
- * cleared at the start of every call, the flags it collects are not reported
- * (use a context and rsq_check_flags for that), and calls that overlap on the
- * GPU race on it.  The first call on a device looks up the array's device
- * address (and sets kernel attributes) for that device; make that first call
- * before any stream capture.  Errors as rsq_create plus rsq_decode_step. */
+ * cleared on the stream at the start of every call, the flags it collects are
+ * not reported (use a context and rsq_check_flags for that), and calls that
+ * overlap on the GPU race on it.  The first call on a device looks up the
+ * array's device address for that device, and the first call with a given
+ * kernel sets its shared-memory attribute and queries its occupancy; make
+ * those first calls before any stream capture.  The remembered address
+ * belongs to the device's current context: after cudaDeviceReset it is
+ * stale.  Errors as rsq_create plus rsq_decode_step. */
 rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_state* state_in,
                                    const rsq_state* state_out, const void* inputs, float* out,
                                    uint32_t step, void* stream);

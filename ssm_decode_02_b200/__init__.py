@@ -75,7 +75,7 @@ _EXPORTS = ["rsq_create", "rsq_destroy", "rsq_state_bytes", "rsq_head_offset", "
             "rsq_quantize", "rsq_dequantize", "rsq_state_drift", "rsq_check_flags",
             "rsq_allocate_bits", "rsq_reduction_partials", "rsq_status_string", "rsq_last_error",
             "rsq_version", "rsq_decode_step_noalloc", "rsq_decode_step_copy_scale",
-            "rsq_column_absmax", "rsq_window_bytes", "rsq_decode_step_window"]
+            "rsq_column_absmax", "rsq_window_bytes", "rsq_decode_step_window", "rsq_debug_waits"]
 
 
 def _load():
@@ -117,6 +117,7 @@ def _load():
                            ctypes.POINTER(rsq_window), P, P, ctypes.c_uint32], C),
         "rsq_pipe_sync": ([P], C),
         "rsq_pipe_streams": ([P, ctypes.POINTER(P), ctypes.POINTER(P), ctypes.POINTER(P)], C),
+        "rsq_debug_waits": ([P, ctypes.c_uint32, C], C),
     }
     for name, (args, res) in sig.items():
         f = getattr(L, name)
@@ -360,6 +361,12 @@ def rsq_check_flags(ctx: int, stream=None) -> int:
     if st not in (RSQ_OK, RSQ_E_NONFINITE):
         _check(st)
     return int(seen.value)
+
+
+def rsq_debug_waits(ctx: int, wait_iters: int, withhold: int) -> None:
+    """Failure-detection tests: limit the kernels' bounded waits and withhold an
+    exchange-barrier arrival (see rsq.h)."""
+    _check(lib.rsq_debug_waits(ctx, int(wait_iters), int(withhold)))
 
 
 def rsq_allocate_bits(score, n_high: int, high_bits: int = 8, low_bits: int = 4) -> np.ndarray:

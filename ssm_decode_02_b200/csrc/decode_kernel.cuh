@@ -38,8 +38,6 @@
 
 namespace rsq {
 
-constexpr uint32_t kWaitIters = 1u << 22;  // bounded mbarrier waits (error flag on expiry)
-
 template <int FAM, int DK, int UB, bool F32STATE>
 struct DecodeCfg {
     // warps per 16-column block: one holds all rows up to d_k = 128; at d_k = 256
@@ -344,12 +342,14 @@ __device__ __forceinline__ void pw_slots(const DecodeParams& p, const uint8_t* s
 // butterfly's last stage d = 8 (partials p and p ^ 8).  False if the bounded
 // wait ran out.
 template <class Op>
-__device__ __forceinline__ bool pair_combine(float& v, float* xs, uint32_t xbar, uint32_t& xphase, int hh,
-                                             int col16, int lane, int g, Op op) {
+__device__ __forceinline__ bool pair_combine(const DecodeParams& p, float& v, float* xs, uint32_t xbar,
+                                             uint32_t& xphase, int hh, int col16, int lane, int g, Op op) {
     if (g < 4) xs[hh * 16 + col16] = v;  // lanes g and g ^ 4 hold the same column
     __syncwarp();
-    if (lane == 0) mbar_arrive(xbar);
-    const bool ok = mbar_wait(xbar, xphase & 1u, kWaitIters);
+    // (failure-detection tests: the second warp withholds its arrival, so the
+    // phase never completes and both warps' bounded waits run out)
+    if (lane == 0 && !(p.withhold && hh == 1)) mbar_arrive(xbar);
+    const bool ok = mbar_wait(xbar, xphase & 1u, p.wait_iters);
     ++xphase;
     if (!__all_sync(0xffffffffu, ok)) return false;
     const float other = xs[(hh ^ 1) * 16 + col16];
@@ -377,6 +377,12 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     const int blk = un.cb * UB + wb;  // block index within the head
     const int j0 = blk * kBlockCols;  // its first column
     const int col16 = 4 * cw + col_of(g);  // the column this lane finalises (within the block)
+    // Addresses are a per-unit base (the same in every thread of the CTA) plus a
+    // per-thread offset that does not change from unit to unit.
+    const long long unit_code = (long long)un.b * p.row_bytes + p.head_off[un.h] +
+                                (long long)(un.cb * UB) * BLOCK_BYTES;
+    const long long unit_col = (long long)hu * p.dv + un.cb * C::UCOLS;
+    const int lane_col = kBlockCols * wb + 4 * cw;  // this lane's first column within the unit
     float* xs = reinterpret_cast<float*>(smem + C::OFF_XCH) + wb * 96;
     const uint32_t xbar = smem_u32(smem + C::OFF_XBAR) + 8 * wb;
 
@@ -416,7 +422,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
             __syncwarp();
             if (lane == 0) mbar_arrive(sbar);
         }
-        const bool ok = mbar_wait(sbar, parity, kWaitIters);
+        const bool ok = mbar_wait(sbar, parity, p.wait_iters);
         if (!__all_sync(0xffffffffu, ok)) return false;
     }
     const uint64_t* qa = pa + g * C::PST;  // q (GDN, GLA, KDA) / C (Mamba-2) of rows g + 8k
@@ -461,7 +467,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
         }
         float cpart = reduce_scatter4(unpk4(a01, a23), g, AddOp());
         if constexpr (C::SPLIT > 1)
-            if (!pair_combine(cpart, xs, xbar, xphase, hh, col16, lane, g, AddOp())) return false;
+            if (!pair_combine(p, cpart, xs, xbar, xphase, hh, col16, lane, g, AddOp())) return false;
         const float4 ck = gather_cols(cpart, cw, 0);
         // reload the k pairs below instead of keeping 16 of them live across the
         // reduction (register pressure)
@@ -529,7 +535,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
             }
             float cpart = reduce_scatter4(unpk4(a01, a23), g, AddOp());
             if constexpr (C::SPLIT > 1)
-                if (!pair_combine(cpart, xs, xbar, xphase, hh, col16, lane, g, AddOp())) return false;
+                if (!pair_combine(p, cpart, xs, xbar, xphase, hh, col16, lane, g, AddOp())) return false;
             const float4 ck = gather_cols(cpart, cw, 0);
             asm volatile("" ::: "memory");
             const float ckv[4] = {ck.x, ck.y, ck.z, ck.w};
@@ -600,7 +606,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     const int c = col_of(g);  // the column this lane finalises
     float o = reduce_scatter4(unpk4(o01, o23), g, AddOp());
     if constexpr (C::SPLIT > 1)
-        if (!pair_combine(o, xs + 32, xbar, xphase, hh, col16, lane, g, AddOp())) return false;
+        if (!pair_combine(p, o, xs + 32, xbar, xphase, hh, col16, lane, g, AddOp())) return false;
     if constexpr (FAM == RSQ_MAMBA2) o = __fmaf_rn(gt.D, ld_vec(stage + C::OFF_VC, 16 * wb + 4 * cw + c, bf16), o);
     if constexpr (C::PW) {
         // the window's part of the readout: o_j += b_w,j z_w in slot order
@@ -615,7 +621,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
             o = __fmaf_rn(bw, zs[ws], o);
         }
     }
-    const long long col = (long long)hu * p.dv + j0 + 4 * cw + c;
+    const long long col = unit_col + (lane_col + c);
     if (g < 4 && hh == 0) p.out[col] = o;
     float4 iv = make_float4(0.f, 0.f, 0.f, 0.f);
     float mine_scale = 0.f;  // the scale (lanes g < 4) or multiplier (g >= 4) of this lane's column
@@ -632,7 +638,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
         }
         float m = reduce_scatter4(make_float4(m0, m1, m2, m3), g, MaxOp());
         if constexpr (C::SPLIT > 1)
-            if (!pair_combine(m, xs + 64, xbar, xphase, hh, col16, lane, g, MaxOp())) return false;
+            if (!pair_combine(p, m, xs + 64, xbar, xphase, hh, col16, lane, g, MaxOp())) return false;
         if constexpr ((RND & kRndCopy) == 0) {
             mine_scale = scale_or_inv<BITS>(m, g);
         } else {
@@ -646,9 +652,8 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     }
 
     // ---- store ------------------------------------------------------------------
-    uint8_t* dst = p.codes_out + (long long)un.b * p.row_bytes + p.head_off[un.h] +
-                   (long long)blk * BLOCK_BYTES;
-    const uint32_t gcol = static_cast<uint32_t>(j0 / 4 + cw);
+    uint8_t* dst = p.codes_out + unit_code + wb * BLOCK_BYTES;
+    const uint32_t gcol = static_cast<uint32_t>(un.cb * (C::UCOLS / 4)) + static_cast<uint32_t>(lane_col / 4);
     if constexpr (BITS == 32) {
 #pragma unroll
         for (int k = 0; k < RPT; ++k)
@@ -668,7 +673,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
         if constexpr ((RND & kRndCopy) != 0) {
             // a copy scale can lie below the state's own maximum: the state is
             // clipped to the copy's range first, so every code stays within +-r
-            const float4 mc = __ldg(reinterpret_cast<const float4*>(p.copy_absmax + (long long)hu * p.dv + j0 + 4 * cw));
+            const float4 mc = __ldg(reinterpret_cast<const float4*>(p.copy_absmax + unit_col + lane_col));
 #pragma unroll
             for (int k = 0; k < RPT; ++k) {
                 const float4 v = unpk4(S2[k][0], S2[k][1]);
@@ -715,10 +720,13 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     }
 
     // ---- release the stage; the last warp refills it with the unit NS ahead ----
+    // (the warp's reads of the stage are ordered before its release by the
+    // __syncwarp and the release half of the counter update; the last warp's
+    // acquire half orders every warp's reads before its refill)
     __syncwarp();
     if (lane == 0) {
         uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + C::OFF_CNT) + stage_idx;
-        if (atomicAdd(cnt, 1u) == C::NW - 1) {
+        if (atom_add_acq_rel_cta(cnt, 1u) == C::NW - 1) {
             *cnt = 0u;
             UnitIt refill = un;  // the unit NS ahead of this one
 #pragma unroll
@@ -781,15 +789,31 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_
     int stage = 0;
     uint32_t parity = 0;
     uint32_t xphase = 0;  // phases of the block's exchange barrier (d_k = 256)
+    // A warp that stops early (a bounded wait ran out) first waits, again
+    // bounded, for the stage copies that may still be in flight towards this
+    // CTA's shared memory: at every stage whose next unit exists, the phase
+    // this warp would wait for next (a copy not yet issued, which a slower
+    // warp may still issue, is waited for by that warp when it stops).  The
+    // last warp of the CTA to stop has then seen every copy the CTA issued land
+    // (or given up on it after the limit).
+    auto stop = [&](const UnitIt& at, int stage_now, uint32_t parity_now) {
+        if (lane == 0) atomicOr(p.flag, kFlagTimeout);
+        for (int s = 0; s < C::NS; ++s) {
+            const int ahead = (s - stage_now + C::NS) % C::NS;  // units between this one and stage s's next
+            if (static_cast<long long>(at.u) + static_cast<long long>(ahead) * p.grid >= p.units) continue;
+            mbar_wait(bar0 + 8 * s, s >= stage_now ? parity_now : (parity_now ^ 1u), kDrainIters);
+        }
+        __syncwarp();
+    };
     while (cur.u < p.units) {
         UnitIt nxt = cur;
         nxt.advance(p);
         Gates ng = gt;
         if (nxt.u < p.units) ng = load_gates<FAM>(p, nxt);
         const uint32_t bar = bar0 + 8 * stage;
-        const bool ok = mbar_wait(bar, parity, kWaitIters);
+        const bool ok = mbar_wait(bar, parity, p.wait_iters);
         if (__any_sync(0xffffffffu, !ok)) {
-            if (lane == 0) atomicOr(p.flag, kFlagTimeout);
+            stop(cur, stage, parity);
             return;  // this warp stops; the others see their own waits expire
         }
         uint8_t* st = smem + stage * C::STAGE;
@@ -802,8 +826,8 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_
             else
                 done = process_block<FAM, DK, UB, false, RND, 4>(p, cur, st, smem, stage, bar, parity, xphase, gt, w, lane, g, cw);
         }
-        if (!done) {  // a bounded wait inside the block ran out (window slot results)
-            if (lane == 0) atomicOr(p.flag, kFlagTimeout);
+        if (!done) {  // a bounded wait inside the block ran out (window slot results, pair exchange)
+            stop(cur, stage, parity);
             return;
         }
         cur = nxt;

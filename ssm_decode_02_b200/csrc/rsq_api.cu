@@ -23,6 +23,8 @@ struct rsq_ctx {
     int grid;        // persistent decode grid
     int device;
     unsigned* flag;  // device word: rsq::kFlag* bits
+    uint32_t wait_iters;  // limit of the kernels' bounded barrier waits (0: the default)
+    int withhold;         // failure-detection tests: withhold an exchange-barrier arrival
 };
 
 namespace {
@@ -96,6 +98,14 @@ rsq_status check_state(const rsq_ctx* c, const rsq_state* s, const char* name) {
 }  // namespace
 
 extern "C" {
+
+rsq_status rsq_debug_waits(rsq_ctx* ctx, uint32_t wait_iters, int withhold) {
+    if (!ctx) return fail(RSQ_E_INVAL, "debug_waits: null context");
+    if (withhold != 0 && withhold != 1) return fail(RSQ_E_INVAL, "debug_waits: withhold must be 0 or 1");
+    ctx->wait_iters = wait_iters;
+    ctx->withhold = withhold;
+    return RSQ_OK;
+}
 
 const char* rsq_last_error(void) { return g_err; }
 
@@ -382,6 +392,8 @@ rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const
     p.key0 = static_cast<uint32_t>(c.seed);
     p.key1 = static_cast<uint32_t>(c.seed >> 32);
     p.rk = rsq::philox_round_keys(p.key0, p.key1);
+    p.wait_iters = ctx->wait_iters ? ctx->wait_iters : rsq::kWaitIters;
+    p.withhold = ctx->withhold;
     if (c.family == RSQ_GDN) {
         const rsq_gdn_inputs* in = static_cast<const rsq_gdn_inputs*>(inputs);
         if (!in->q || !in->k || !in->v || !in->alpha || !in->beta)
@@ -530,17 +542,20 @@ rsq_status rsq_check_flags(const rsq_ctx* ctx, int* seen, void* stream) {
 // Decode step without any allocation.
 //
 // rsq_create allocates the context's 4-byte device flag word with cudaMalloc
-// (or the configuration's allocator hook).  This entry point instead keeps that word in a small statically allocated
-// device array, so a caller that may not allocate device memory can still run
-// a decode step: code inside stream capture, where allocation calls are not
-// allowed, or a runtime whose memory is owned entirely by its own pool
-// allocator.
+// (or the configuration's allocator hook).  Some callers cannot allocate
+// device memory after start-up: serving runtimes that reserve nearly all of
+// the GPU's memory for their own pools when they start (a later cudaMalloc
+// could fail, or fragment what the pool manages) and embedded hosts that run
+// under a fixed memory budget.  This entry point keeps the flag word in a
+// small statically allocated device array instead, so those callers can still
+// run a decode step.
 // ---------------------------------------------------------------------------
 namespace {
 
 constexpr int kNoallocScratchWords = 64;   // 256 bytes on every device that loads the library
 constexpr int kNoallocWordsNeeded = 1;     // the decode kernel's flag word
 constexpr int kNoallocMaxDevices = 64;
+constexpr int kNoallocMaxKernels = 16;     // launch geometries remembered per device
 
 // In host code this name is only a stand-in for the device array; its device
 // address comes from cudaGetSymbolAddress (per device) below.
@@ -548,6 +563,16 @@ static __device__ __align__(256) unsigned g_noalloc_scratch[kNoallocScratchWords
 
 std::mutex g_noalloc_mu;
 unsigned* g_noalloc_ptr[kNoallocMaxDevices] = {};
+
+// Per device: the kernels already prepared (dynamic shared memory attribute
+// set) and their resident CTAs per SM, so later calls make no attribute or
+// occupancy query.
+struct NoallocGeometry {
+    const void* func;
+    int per_sm;
+};
+NoallocGeometry g_noalloc_geom[kNoallocMaxDevices][kNoallocMaxKernels] = {};
+int g_noalloc_sms[kNoallocMaxDevices] = {};
 
 // Device address of the scratch array for the current device (resolved once
 // per device, with that device current).
@@ -562,6 +587,32 @@ rsq_status noalloc_scratch(int device, unsigned** out) {
         g_noalloc_ptr[device] = static_cast<unsigned*>(ptr);
     }
     *out = g_noalloc_ptr[device];
+    return RSQ_OK;
+}
+
+// SM count and resident CTAs per SM of `func` on `device` (current), set up
+// and queried on the first call for that kernel, remembered afterwards.
+rsq_status noalloc_geometry(int device, const void* func, int threads, size_t smem, int* sms, int* per_sm) {
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    int err = 0;
+    if (!g_noalloc_sms[device]) err = cudaDeviceGetAttribute(&g_noalloc_sms[device], cudaDevAttrMultiProcessorCount, device);
+    if (err) return cuda_fail(err, "decode_step_noalloc: SM count");
+    *sms = g_noalloc_sms[device];
+    NoallocGeometry* slot = nullptr;
+    for (auto& e : g_noalloc_geom[device]) {
+        if (e.func == func) {
+            *per_sm = e.per_sm;
+            return RSQ_OK;
+        }
+        if (!e.func && !slot) slot = &e;
+    }
+    int n = 0;
+    err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (!err) err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, func, threads, smem);
+    if (!err && n < 1) err = cudaErrorInvalidConfiguration;
+    if (err) return cuda_fail(err, "decode_step_noalloc: launch geometry");
+    if (slot) *slot = NoallocGeometry{func, n};  // a full table only means the query repeats
+    *per_sm = n;
     return RSQ_OK;
 }
 
@@ -626,17 +677,15 @@ extern "C" rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_s
                                 &func) != 0)
         return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: no kernel for dk=%d dv=%d", c.dk, c.dv);
     int err = cudaGetDevice(&ctx.device);
-    int sms = 0, per_sm = 0;
-    if (!err) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, ctx.device);
-    if (!err) err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (!err) err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, func, threads, smem);
-    if (!err && per_sm < 1) err = cudaErrorInvalidConfiguration;
-    if (err) return cuda_fail(err, "decode_step_noalloc: launch geometry");
-    ctx.grid = static_cast<int>(std::min<long long>(units, static_cast<long long>(sms) * per_sm));
-
+    if (err) return cuda_fail(err, "decode_step_noalloc: cudaGetDevice");
     unsigned* scratch = nullptr;
     rsq_status s = noalloc_scratch(ctx.device, &scratch);
     if (s) return s;
+    int sms = 0, per_sm = 0;
+    s = noalloc_geometry(ctx.device, func, threads, smem, &sms, &per_sm);
+    if (s) return s;
+    ctx.grid = static_cast<int>(std::min<long long>(units, static_cast<long long>(sms) * per_sm));
+
     // the flag word starts each call at zero (every call shares the array)
     err = cudaMemsetAsync(scratch, 0, kNoallocWordsNeeded * sizeof(unsigned), static_cast<cudaStream_t>(stream));
     if (err) return cuda_fail(err, "decode_step_noalloc: clear scratch");

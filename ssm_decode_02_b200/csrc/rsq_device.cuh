@@ -57,6 +57,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_
     return false;
 }
 
+// Shared-memory add with acquire-release semantics at CTA scope: the caller's
+// earlier accesses (and, through a preceding __syncwarp, its warp's) happen
+// before those of any thread that later reads the value it wrote.
+__device__ __forceinline__ uint32_t atom_add_acq_rel_cta(uint32_t* p, uint32_t v) {
+    uint32_t old;
+    asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v)
+                 : "memory");
+    return old;
+}
+
 // Global -> shared bulk copy of `bytes` (multiple of 16, both addresses 16-byte
 // aligned) completing as a transaction on `bar`.  No multicast.
 __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t bytes,
@@ -133,6 +143,14 @@ __device__ __forceinline__ void e4m3x2_to_f32(uint32_t two, float& lo, float& hi
 __device__ __forceinline__ uint32_t umulhi_add(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t d;
     asm("mad.hi.u32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(c));
+    return d;
+}
+
+// (a & MASK) | bits in one logic operation (the mask an immediate, `bits` a register)
+template <uint32_t MASK>
+__device__ __forceinline__ uint32_t and_or(uint32_t a, uint32_t bits) {
+    uint32_t d;
+    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(d) : "r"(a), "n"(MASK), "r"(bits));
     return d;
 }
 

@@ -17,6 +17,8 @@ constexpr int pw_window(int fam) { return is_pw_family(fam) ? 4 << (fam - kFamGd
 
 constexpr unsigned kFlagNonFinite = 1u;  // a column's absmax was inf or NaN
 constexpr unsigned kFlagTimeout = 2u;    // a bounded barrier wait ran out
+constexpr uint32_t kWaitIters = 1u << 22;  // default limit of a bounded barrier wait (polls)
+constexpr uint32_t kDrainIters = 1u << 16; // wait for in-flight stage copies before a CTA leaves early
 
 // The ten round keys of Philox4x32-10 for one (key0, key1): round r uses
 // key0 + r * 0x9E3779B9 and key1 + r * 0xBB67AE85 (mod 2^32).  Computed once on
@@ -73,6 +75,11 @@ struct DecodeParams {
     unsigned* flag;
     uint32_t step, key0, key1;
     PhiloxKeys rk;                 // Philox round keys of (key0, key1)
+    // bounded waits: polls before a barrier wait gives up (sets kFlagTimeout);
+    // withhold = 1 (failure-detection tests only): the second warp of a
+    // two-warp block never arrives on the block's exchange barrier
+    uint32_t wait_iters;
+    int withhold;
     uint32_t head_off[RSQ_MAX_HEADS];  // byte offset of each head in a batch row
     uint8_t head_bits[RSQ_MAX_HEADS];
 };

@@ -135,18 +135,20 @@ __device__ __forceinline__ void load_codes(const uint8_t* blk, int g, int cw, ui
             S2[k][1] = add2(f23, off);
         }
     } else {
-        const uint64_t off = pk(-(kMagic + 8.0f), -(kMagic + 8.0f));
+        // Nibble t of the row's 16 bits (column t, bits 4t..4t+3) is OR-ed in place
+        // into the float 2^E_t with E_t = 23 - 4t, whose ulp is 2^(4t) there: the
+        // float is exactly 2^E_t + (c + 8), one logic operation per code.
+        const uint64_t off01 = pk(-(8388608.0f + 8.0f), -(524288.0f + 8.0f));  // 2^23, 2^19
+        const uint64_t off23 = pk(-(32768.0f + 8.0f), -(2048.0f + 8.0f));      // 2^15, 2^11
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
             const uint32_t h16 = *reinterpret_cast<const uint16_t*>(blk + (g + RS * k) * 8 + 2 * cw);
-            const uint32_t lo = h16 & 0x0F0Fu;         // columns 0 and 2
-            const uint32_t hi = (h16 >> 4) & 0x0F0Fu;  // columns 1 and 3
-            const uint64_t f01 = pk(__uint_as_float(prmt(lo, kMagicBits, 0x7650u)),
-                                    __uint_as_float(prmt(hi, kMagicBits, 0x7650u)));
-            const uint64_t f23 = pk(__uint_as_float(prmt(lo, kMagicBits, 0x7651u)),
-                                    __uint_as_float(prmt(hi, kMagicBits, 0x7651u)));
-            S2[k][0] = add2(f01, off);
-            S2[k][1] = add2(f23, off);
+            const uint64_t f01 = pk(__uint_as_float(and_or<0x000Fu>(h16, 0x4B000000u)),
+                                    __uint_as_float(and_or<0x00F0u>(h16, 0x49000000u)));
+            const uint64_t f23 = pk(__uint_as_float(and_or<0x0F00u>(h16, 0x47000000u)),
+                                    __uint_as_float(and_or<0xF000u>(h16, 0x45000000u)));
+            S2[k][0] = add2(f01, off01);
+            S2[k][1] = add2(f23, off23);
         }
     }
 }

@@ -1,9 +1,9 @@
 """The decode step that allocates nothing, against the context-based entry point.
 
-rsq_decode_step_noalloc exists for callers that may not allocate device memory
-(code inside CUDA stream capture, runtimes whose device memory belongs to their
-own pool allocator): instead of the context's cudaMalloc'd flag word it uses a
-static device array.  Here it must produce exactly what rsq_decode_step
+rsq_decode_step_noalloc exists for callers that cannot allocate device memory
+once they run (serving runtimes that reserve nearly all GPU memory for their
+own pools at start-up, embedded hosts with a fixed memory budget): instead of
+the context's cudaMalloc'd flag word it uses a static device array.  Here it must produce exactly what rsq_decode_step
 produces, on two consecutive decode steps, through the C ABI.  This file is
 collected last on purpose, so a run that stops at the first failure has already
 run every other test.
