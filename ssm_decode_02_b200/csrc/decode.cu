@@ -9,8 +9,8 @@ namespace rsq {
 
 // One pair of lookup functions per family (plain rules / directional rules),
 // each defined in its own translation unit.
-using InfoFn = int (*)(int, int, bool, int, int*, size_t*, const void**);
-#define RSQ_DECLARE(NAME) int NAME(int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem, \
+using InfoFn = int (*)(int, int, int, bool, int, int*, size_t*, const void**);
+#define RSQ_DECLARE(NAME) int NAME(int dk, int ub, int bpw, bool f32state, int rnd, int* threads, size_t* smem, \
                                    const void** func);
 RSQ_DECLARE(decode_info_gdn)
 RSQ_DECLARE(decode_info_gdn_bdr)
@@ -33,7 +33,7 @@ RSQ_DECLARE(decode_info_gdn_pw8)
 RSQ_DECLARE(decode_info_gdn_pw16)
 #undef RSQ_DECLARE
 
-int decode_kernel_info(int family, int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
+int decode_kernel_info(int family, int dk, int ub, int bpw, bool f32state, int rnd, int* threads, size_t* smem,
                        const void** func) {
     // [family][rule group]: plain, BDR, copy scale, copy scale + BDR
     static const InfoFn table[4][4] = {
@@ -45,18 +45,18 @@ int decode_kernel_info(int family, int dk, int ub, bool f32state, int rnd, int* 
     const int group = f32state ? 0 : (((rnd & kRndBdr) ? 1 : 0) + ((rnd & kRndCopy) ? 2 : 0));
     if (is_pw_family(family)) {  // pure-write window: plain rules only
         static const InfoFn pw[3] = {decode_info_gdn_pw4, decode_info_gdn_pw8, decode_info_gdn_pw16};
-        return group == 0 ? pw[family - kFamGdnPw](dk, ub, f32state, rnd, threads, smem, func) : -1;
+        return group == 0 ? pw[family - kFamGdnPw](dk, ub, bpw, f32state, rnd, threads, smem, func) : -1;
     }
     if (family < 0 || family > 3) return -1;
-    return table[family][group](dk, ub, f32state, rnd, threads, smem, func);
+    return table[family][group](dk, ub, bpw, f32state, rnd, threads, smem, func);
 }
 
-int launch_decode(int family, int dk, int ub, bool f32state, int rnd, const DecodeParams& p,
+int launch_decode(int family, int dk, int ub, int bpw, bool f32state, int rnd, const DecodeParams& p,
                   void* stream) {
     int threads;
     size_t smem;
     const void* func;
-    if (decode_kernel_info(family, dk, ub, f32state, rnd, &threads, &smem, &func) != 0)
+    if (decode_kernel_info(family, dk, ub, bpw, f32state, rnd, &threads, &smem, &func) != 0)
         return static_cast<int>(cudaErrorInvalidValue);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(p.grid);

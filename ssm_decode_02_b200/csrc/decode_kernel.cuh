@@ -38,7 +38,7 @@
 
 namespace rsq {
 
-template <int FAM, int DK, int UB, bool F32STATE>
+template <int FAM, int DK, int UB, bool F32STATE, int BPW_ = 1>
 struct DecodeCfg {
     // warps per 16-column block: one holds all rows up to d_k = 128; at d_k = 256
     // two warps share the block, warp half hh holding the rows i with
@@ -46,11 +46,16 @@ struct DecodeCfg {
     static constexpr int SPLIT = DK > 128 ? 2 : 1;
     using L = Layout<DK / SPLIT>;
     static constexpr int RS = kR * SPLIT;      // row stride of a lane's rows
-    static constexpr int NW = UB * SPLIT;      // warps per CTA
+    // blocks each warp takes per unit: one, or two (BPW = 2, units of four
+    // one-warp blocks): a warp's per-unit work -- its pair arrays, the stage
+    // wait and release -- then serves two blocks
+    static constexpr int BPW = BPW_;
+    static constexpr int NW = UB * SPLIT / BPW;  // warps per CTA
     static constexpr int NT = 32 * NW;
     static constexpr int UCOLS = 16 * UB;      // columns per unit
-    // pipeline stages (KDA's extra pair array leaves room for three)
-    static constexpr int NS = F32STATE ? 2 : ((FAM == RSQ_KDA || is_pw_family(FAM)) ? 3 : 4);
+    // pipeline stages (KDA's extra pair array leaves room for three; two-block
+    // warps keep two so that eight 64-thread CTAs fit an SM)
+    static constexpr int NS = F32STATE ? 2 : (BPW == 2 ? 2 : ((FAM == RSQ_KDA || is_pw_family(FAM)) ? 3 : 4));
     static constexpr int CODE_BYTES = F32STATE ? DK * UCOLS * 4 : DK * UCOLS;  // largest tile (8-bit)
     static constexpr int OFF_SCALES = CODE_BYTES;
     static constexpr int OFF_VA = OFF_SCALES + UCOLS * 4;  // GDN q / Mamba-2 C   (<= DK floats)
@@ -96,6 +101,8 @@ struct DecodeCfg {
     // four 128-thread CTAs per SM (4 x ~50 KB), so 128 registers per thread
     static constexpr int MINB = F32STATE ? 1 : (NT < 128 ? 8 : 512 / NT);
     static_assert(!PW || SPLIT == 1, "the pure-write window is built for d_k <= 128");
+    static_assert(BPW == 1 || (BPW == 2 && SPLIT == 1 && UB == 4 && !F32STATE && !PW),
+                  "two blocks per warp only for units of four one-warp blocks");
     // the shared-memory layout, checked for every instance at compile time
     static_assert(SMEM <= 227 * 1024, "shared memory beyond the per-CTA limit");
     static_assert(STAGE % 128 == 0 && OFF_P >= NS * STAGE, "stages overlap the pair arrays");
@@ -133,10 +140,10 @@ struct UnitIt {
 };
 
 // Issue the bulk copies of one unit into a stage (one thread).
-template <int FAM, int DK, int UB, bool F32STATE>
+template <int FAM, int DK, int UB, bool F32STATE, int BPW>
 __device__ __forceinline__ void issue_unit(const DecodeParams& p, const UnitIt& un, uint8_t* stage,
                                            uint32_t bar) {
-    using C = DecodeCfg<FAM, DK, UB, F32STATE>;
+    using C = DecodeCfg<FAM, DK, UB, F32STATE, BPW>;
     constexpr int UCOLS = C::UCOLS;
     const int bits = F32STATE ? 32 : p.head_bits[un.h];
     const int hu = un.hu(p);
@@ -359,12 +366,12 @@ __device__ __forceinline__ bool pair_combine(const DecodeParams& p, float& v, fl
 
 // One 16-column block of one unit, processed by warp w (with d_k = 256, by
 // warps w and w + UB, each with half of the rows).
-template <int FAM, int DK, int UB, bool F32STATE, int RND, int BITS>
+template <int FAM, int DK, int UB, bool F32STATE, int RND, int BITS, int BPW>
 __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitIt& un, uint8_t* stage,
                                               uint8_t* smem, int stage_idx, uint32_t bar, uint32_t parity,
                                               uint32_t& xphase, const Gates& gt, int w, int lane, int g,
-                                              int cw) {
-    using C = DecodeCfg<FAM, DK, UB, F32STATE>;
+                                              int cw, int wblk) {
+    using C = DecodeCfg<FAM, DK, UB, F32STATE, BPW>;
     using L = typename C::L;
     constexpr int RPT = L::RPT;
     constexpr int RS = C::RS;
@@ -372,7 +379,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     const bool bf16 = p.in_bf16 != 0;
     const int hu = un.hu(p);
     const int hh = (C::SPLIT > 1) ? w / UB : 0;  // which rows of the block (d_k = 256)
-    const int wb = (C::SPLIT > 1) ? w - hh * UB : w;  // block within the unit
+    const int wb = (C::SPLIT > 1) ? w - hh * UB : w + wblk * C::NW;  // block within the unit (warp's wblk-th)
     const int gr = g + kR * hh;                  // this lane's first row
     const int blk = un.cb * UB + wb;  // block index within the head
     const int j0 = blk * kBlockCols;  // its first column
@@ -393,6 +400,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     uint64_t* pd = pc + kR * C::PST;  // KDA: alpha_i * k_i
 #pragma unroll
     for (int i = lane; i < DK; i += 32) {
+        if (wblk != 0) break;  // built once per unit, for the warp's first block
         if (C::SPLIT > 1 && ((i / kR) & 1) != hh) continue;  // the other warp's rows
         const float a = ld_vec(stage + C::OFF_VA, i, bf16);
         const float b = ld_vec(stage + C::OFF_VB, i, bf16);
@@ -724,7 +732,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
     // __syncwarp and the release half of the counter update; the last warp's
     // acquire half orders every warp's reads before its refill)
     __syncwarp();
-    if (lane == 0) {
+    if (wblk == C::BPW - 1 && lane == 0) {  // after the warp's last block of the unit
         uint32_t* cnt = reinterpret_cast<uint32_t*>(smem + C::OFF_CNT) + stage_idx;
         if (atom_add_acq_rel_cta(cnt, 1u) == C::NW - 1) {
             *cnt = 0u;
@@ -733,7 +741,7 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
             for (int s = 0; s < C::NS; ++s) refill.advance(p);
             if (refill.u < p.units) {
                 asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-                issue_unit<FAM, DK, UB, F32STATE>(p, refill, stage, bar);
+                issue_unit<FAM, DK, UB, F32STATE, BPW>(p, refill, stage, bar);
             }
         }
     }
@@ -743,9 +751,9 @@ __device__ __forceinline__ bool process_block(const DecodeParams& p, const UnitI
 // Resident CTAs per SM the register budget is sized for: Bounded Directional
 // Rounding re-decodes the previous codes while requantizing and needs more
 // registers than the plain rules.
-template <int FAM, int DK, int UB, bool F32STATE, int RND>
+template <int FAM, int DK, int UB, bool F32STATE, int RND, int BPW>
 constexpr int decode_min_blocks() {
-    using C = DecodeCfg<FAM, DK, UB, F32STATE>;
+    using C = DecodeCfg<FAM, DK, UB, F32STATE, BPW>;
     // BDR: about 168 registers per thread (65536 / (168 * 128) = 3 CTAs of 128 threads)
     // (the pure-write window's slot pass needs as many, and so does stochastic
     // rounding at dk = 256 with its pair exchanges, run with two blocks per unit)
@@ -753,10 +761,11 @@ constexpr int decode_min_blocks() {
     return wide ? 384 / C::NT : C::MINB;
 }
 
-template <int FAM, int DK, int UB, bool F32STATE, int RND>
-__global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_min_blocks<FAM, DK, UB, F32STATE, RND>()))
+template <int FAM, int DK, int UB, bool F32STATE, int RND, int BPW>
+__global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE, BPW>::NT,
+                                  (decode_min_blocks<FAM, DK, UB, F32STATE, RND, BPW>()))
     rsq_decode_kernel(const __grid_constant__ DecodeParams p) {
-    using C = DecodeCfg<FAM, DK, UB, F32STATE>;
+    using C = DecodeCfg<FAM, DK, UB, F32STATE, BPW>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int tid = threadIdx.x;
     const int lane = tid & 31, w = tid >> 5;
@@ -780,7 +789,7 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_
     if (tid == 0) {
         UnitIt it = cur;
         for (int s = 0; s < C::NS; ++s) {
-            if (it.u < p.units) issue_unit<FAM, DK, UB, F32STATE>(p, it, smem + s * C::STAGE, bar0 + 8 * s);
+            if (it.u < p.units) issue_unit<FAM, DK, UB, F32STATE, BPW>(p, it, smem + s * C::STAGE, bar0 + 8 * s);
             it.advance(p);
         }
     }
@@ -817,14 +826,20 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_
             return;  // this warp stops; the others see their own waits expire
         }
         uint8_t* st = smem + stage * C::STAGE;
-        bool done;
-        if constexpr (F32STATE) {
-            done = process_block<FAM, DK, UB, true, 0, 32>(p, cur, st, smem, stage, bar, parity, xphase, gt, w, lane, g, cw);
-        } else {
-            if (p.head_bits[cur.h] == 8)
-                done = process_block<FAM, DK, UB, false, RND, 8>(p, cur, st, smem, stage, bar, parity, xphase, gt, w, lane, g, cw);
-            else
-                done = process_block<FAM, DK, UB, false, RND, 4>(p, cur, st, smem, stage, bar, parity, xphase, gt, w, lane, g, cw);
+        bool done = true;
+#pragma unroll 1
+        for (int wblk = 0; wblk < C::BPW && done; ++wblk) {
+            if constexpr (F32STATE) {
+                done = process_block<FAM, DK, UB, true, 0, 32, BPW>(p, cur, st, smem, stage, bar, parity, xphase, gt,
+                                                                    w, lane, g, cw, wblk);
+            } else {
+                if (p.head_bits[cur.h] == 8)
+                    done = process_block<FAM, DK, UB, false, RND, 8, BPW>(p, cur, st, smem, stage, bar, parity, xphase,
+                                                                          gt, w, lane, g, cw, wblk);
+                else
+                    done = process_block<FAM, DK, UB, false, RND, 4, BPW>(p, cur, st, smem, stage, bar, parity, xphase,
+                                                                          gt, w, lane, g, cw, wblk);
+            }
         }
         if (!done) {  // a bounded wait inside the block ran out (window slot results, pair exchange)
             stop(cur, stage, parity);
@@ -840,40 +855,50 @@ __global__ void __launch_bounds__(DecodeCfg<FAM, DK, UB, F32STATE>::NT, (decode_
 }
 
 // Kernel attributes for one instantiation.
-template <int FAM, int DK, int UB, bool F32, int RND>
+template <int FAM, int DK, int UB, bool F32, int RND, int BPW = 1>
 int decode_info_one(int* threads, size_t* smem, const void** func) {
-    using C = DecodeCfg<FAM, DK, UB, F32>;
+    using C = DecodeCfg<FAM, DK, UB, F32, BPW>;
     *threads = C::NT;
     *smem = C::SMEM;
-    *func = reinterpret_cast<const void*>(&rsq_decode_kernel<FAM, DK, UB, F32, RND>);
+    *func = reinterpret_cast<const void*>(&rsq_decode_kernel<FAM, DK, UB, F32, RND, BPW>);
     return 0;
 }
 
-// All (dk, blocks per unit) instantiations of one family for the rounding
-// rules RND0, RNDS... (a full-precision state ignores the rounding: it is built
-// with the first rule only, when that rule is plain nearest rounding).  The
-// rules are split over translation units so the instantiations compile in
-// parallel.
-template <int FAM, int DK, int UB, int RND0, int... RNDS>
+// All (dk, blocks per unit, blocks per warp) instantiations of one family for
+// the rounding rules RND0, RNDS... (a full-precision state ignores the
+// rounding: it is built with the first rule only, when that rule is plain
+// nearest rounding).  The rules are split over translation units so the
+// instantiations compile in parallel.
+template <int FAM, int DK, int UB, int BPW, int RND0, int... RNDS>
 int decode_info_rules(bool f32state, int rnd, int* threads, size_t* smem, const void** func) {
     if (f32state) {
-        if constexpr (RND0 == 0)
+        if constexpr (RND0 == 0 && BPW == 1)
             return decode_info_one<FAM, DK, UB, true, 0>(threads, smem, func);
         else
             return -1;
     }
     int found = -1;
-    if (rnd == RND0) found = decode_info_one<FAM, DK, UB, false, RND0>(threads, smem, func);
-    ((found != 0 && rnd == RNDS ? (found = decode_info_one<FAM, DK, UB, false, RNDS>(threads, smem, func)) : 0),
+    if (rnd == RND0) found = decode_info_one<FAM, DK, UB, false, RND0, BPW>(threads, smem, func);
+    ((found != 0 && rnd == RNDS ? (found = decode_info_one<FAM, DK, UB, false, RNDS, BPW>(threads, smem, func)) : 0),
      ...);
     return found;
 }
 
+// Two blocks per warp are built for d_k = 128 units of four blocks (not for the
+// pure-write window).
 template <int FAM, int... RNDS>
-int decode_info_family(int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
+int decode_info_family(int dk, int ub, int bpw, bool f32state, int rnd, int* threads, size_t* smem,
                        const void** func) {
+    if (bpw == 2) {
+        if constexpr (!is_pw_family(FAM)) {
+            if (dk == 128 && ub == 4 && !f32state)
+                return decode_info_rules<FAM, 128, 4, 2, RNDS...>(f32state, rnd, threads, smem, func);
+        }
+        return -1;
+    }
+    if (bpw != 1) return -1;
 #define RSQ_CASE(DK_, UB_)                                                                 \
-    if (dk == DK_ && ub == UB_) return decode_info_rules<FAM, DK_, UB_, RNDS...>(f32state, rnd, threads, smem, func);
+    if (dk == DK_ && ub == UB_) return decode_info_rules<FAM, DK_, UB_, 1, RNDS...>(f32state, rnd, threads, smem, func);
     RSQ_CASE(16, 1) RSQ_CASE(16, 2) RSQ_CASE(16, 4)
     RSQ_CASE(32, 1) RSQ_CASE(32, 2) RSQ_CASE(32, 4)
     RSQ_CASE(64, 1) RSQ_CASE(64, 2) RSQ_CASE(64, 4)

@@ -4,9 +4,9 @@
 #include "decode_kernel.cuh"
 
 namespace rsq {
-int decode_info_mamba2_copy(int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
+int decode_info_mamba2_copy(int dk, int ub, int bpw, bool f32state, int rnd, int* threads, size_t* smem,
                          const void** func) {
-    return decode_info_family<RSQ_MAMBA2, kRndCopy, kRndCopy | kRndSr, kRndCopy | kRndSr | kRndU8>(dk, ub, f32state, rnd, threads,
+    return decode_info_family<RSQ_MAMBA2, kRndCopy, kRndCopy | kRndSr, kRndCopy | kRndSr | kRndU8>(dk, ub, bpw, f32state, rnd, threads,
                                                                    smem, func);
 }
 }  // namespace rsq

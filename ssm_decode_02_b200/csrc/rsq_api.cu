@@ -20,6 +20,7 @@ struct rsq_ctx {
     long long row_bytes;
     bool f32state;
     int ub, ncb, units;   // 16-column blocks per unit, units per head, units per step
+    int bpw;              // blocks each warp of the decode kernel takes per unit (1 or 2)
     int grid;        // persistent decode grid
     int device;
     unsigned* flag;  // device word: rsq::kFlag* bits
@@ -76,6 +77,44 @@ bool dk_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256
 bool dv_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Resident CTAs per SM of a decode kernel instance, after allowing its dynamic
+// shared memory.  Nonzero cudaError_t on failure.
+int instance_occupancy(const rsq_config& c, int ub, int bpw, bool f32state, int* per_sm, const void** func_out) {
+    int threads = 0;
+    size_t smem = 0;
+    const void* func = nullptr;
+    if (rsq::decode_kernel_info(kernel_family(c), c.dk, ub, bpw, f32state, c.rounding, &threads, &smem, &func) != 0)
+        return -1;
+    int err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (!err) err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(per_sm, func, threads, smem);
+    if (!err && *per_sm < 1) err = cudaErrorInvalidConfiguration;
+    if (func_out) *func_out = func;
+    return err;
+}
+
+// Decode kernel geometry of a configuration: one block per warp, or two (64-
+// thread CTAs, d_k = 128 units of four blocks) when the step has at least four
+// units per resident CTA of that geometry -- there a warp's per-unit work
+// serving two blocks pays off, while small steps keep more CTAs busy with one.
+rsq_status choose_geometry(const rsq_config& c, int ub, bool f32state, long long units, int sms, int* bpw,
+                           int* per_sm) {
+    int err = instance_occupancy(c, ub, 1, f32state, per_sm, nullptr);
+    if (err == -1) return fail(RSQ_E_UNSUPPORTED, "create: no kernel for dk=%d dv=%d", c.dk, c.dv);
+    if (err) return cuda_fail(err, "create: launch geometry");
+    *bpw = 1;
+    if (!f32state && c.dk == 128 && ub == 4 && c.window == 0 && c.key_axis == 0) {
+        int per_sm2 = 0;
+        err = instance_occupancy(c, ub, 2, false, &per_sm2, nullptr);
+        if (err == -1) return RSQ_OK;  // no two-block instance for this rule
+        if (err) return cuda_fail(err, "create: launch geometry");
+        if (units >= 4LL * sms * per_sm2) {
+            *bpw = 2;
+            *per_sm = per_sm2;
+        }
+    }
+    return RSQ_OK;
+}
 
 template <class P>
 void fill_heads(const rsq_ctx* c, P& p) {
@@ -212,27 +251,25 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
     ctx->units = static_cast<int>(units);
 
     // launch geometry: persistent grid of every resident CTA
-    int threads = 0;
-    size_t smem = 0;
-    const void* func = nullptr;
-    if (rsq::decode_kernel_info(kernel_family(c), c.dk, ctx->ub, ctx->f32state, c.rounding, &threads,
-                                &smem, &func) != 0) {
-        delete ctx;
-        return fail(RSQ_E_UNSUPPORTED, "create: no kernel for dk=%d dv=%d", c.dk, c.dv);
-    }
     int err = cudaGetDevice(&ctx->device);
     int sms = 0, per_sm = 0;
     if (!err) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, ctx->device);
-    if (!err) err = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (!err) err = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, func, threads, smem);
-    if (!err && per_sm < 1) err = cudaErrorInvalidConfiguration;
-    if (!err && !ctx->f32state) {
+    if (err) {
+        delete ctx;
+        return cuda_fail(err, "create");
+    }
+    const rsq_status gs = choose_geometry(c, ctx->ub, ctx->f32state, units, sms, &ctx->bpw, &per_sm);
+    if (gs) {
+        delete ctx;
+        return gs;
+    }
+    if (!ctx->f32state) {
         // the copy-scale instance of the same rule (rsq_decode_step_copy_scale)
         int t2 = 0;
         size_t sm2 = 0;
         const void* f2 = nullptr;
-        if (rsq::decode_kernel_info(kernel_family(c), c.dk, ctx->ub, false, c.rounding | kCopyScaleBit, &t2, &sm2,
-                                    &f2) == 0)
+        if (rsq::decode_kernel_info(kernel_family(c), c.dk, ctx->ub, ctx->bpw, false, c.rounding | kCopyScaleBit, &t2,
+                                    &sm2, &f2) == 0)
             err = cudaFuncSetAttribute(f2, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(sm2));
     }
     if (!err) {
@@ -433,7 +470,7 @@ rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const
         if (e) return cuda_fail(e, "decode_step launch");
         return RSQ_OK;
     }
-    const int err = rsq::launch_decode(kernel_family(c), c.dk, ctx->ub, ctx->f32state,
+    const int err = rsq::launch_decode(kernel_family(c), c.dk, ctx->ub, ctx->bpw, ctx->f32state,
                                        c.rounding | (copy_absmax ? kCopyScaleBit : 0), p,
                                        stream);
     if (err) return cuda_fail(err, "decode_step launch");
@@ -673,7 +710,8 @@ extern "C" rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_s
     int threads = 0;
     size_t smem = 0;
     const void* func = nullptr;
-    if (rsq::decode_kernel_info(kernel_family(c), c.dk, ctx.ub, ctx.f32state, c.rounding, &threads, &smem,
+    ctx.bpw = 1;  // one block per warp (results do not depend on the geometry)
+    if (rsq::decode_kernel_info(kernel_family(c), c.dk, ctx.ub, ctx.bpw, ctx.f32state, c.rounding, &threads, &smem,
                                 &func) != 0)
         return fail(RSQ_E_UNSUPPORTED, "decode_step_noalloc: no kernel for dk=%d dv=%d", c.dk, c.dv);
     int err = cudaGetDevice(&ctx.device);

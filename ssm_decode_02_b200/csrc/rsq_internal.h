@@ -122,10 +122,11 @@ struct DriftParams {
 };
 
 // Launchers (defined in the .cu files).  Return a cudaError_t value.
-// ub = 16-column blocks per decode work unit (1, 2 or 4)
-int launch_decode(int family, int dk, int ub, bool f32state, int rnd, const DecodeParams& p,
+// ub = 16-column blocks per decode work unit (1, 2 or 4); bpw = blocks each
+// warp takes per unit (1, or 2 for d_k = 128 units of four blocks)
+int launch_decode(int family, int dk, int ub, int bpw, bool f32state, int rnd, const DecodeParams& p,
                   void* stream);
-int decode_kernel_info(int family, int dk, int ub, bool f32state, int rnd, int* threads, size_t* smem,
+int decode_kernel_info(int family, int dk, int ub, int bpw, bool f32state, int rnd, int* threads, size_t* smem,
                        const void** func);
 int launch_quantize(int dk, const QuantParams& p, void* stream);
 int launch_dequantize(int dk, const DequantParams& p, void* stream);

@@ -316,3 +316,18 @@ def test_misaligned_pointer_rejected_without_launch():
     with pytest.raises(rsq.RsqError) as e:
         run.ctx.decode_step(bad, s, ins, out, 0)
     assert e.value.status == rsq.RSQ_E_INVAL
+
+
+@pytest.mark.parametrize("family,rounding", [("gdn", rsq.RSQ_RTN), ("gdn", rsq.RSQ_SR), ("gdn", rsq.RSQ_SR8_BDR),
+                                             ("mamba2", rsq.RSQ_SR8), ("gla", rsq.RSQ_SR8), ("kda", rsq.RSQ_RTN)])
+def test_large_batch_geometry_sampled(family, rounding):
+    """Enough units per resident CTA that the library gives each warp two
+    blocks per unit (d_k = 128): sampled heads bit-exact against the oracle for
+    every family and several rules."""
+    base = {"gdn": WL[1], "mamba2": WL[3], "gla": W.BY_NAME["gla_b64_h16_d128_int8_sr"],
+            "kda": W.BY_NAME["kda_b64_h16_d128_int8_sr"]}[family]
+    w = dataclasses.replace(base, B=320, H=16)
+    bits = np.array([8, 4] * 8, np.int8)
+    run = Run(w, bits, rounding=rounding)
+    heads = sample_heads(run.B, run.H, 40, seed=17)
+    _trajectory(run, 2, heads=heads)
