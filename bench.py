@@ -163,6 +163,9 @@ SWEEP = (
     ("gdn_b1024_h16_d128_int4_sr_long", None, 8, False),
     ("gdn_b64_h8_d256_int8_sr", None, 0, False), ("gdn_b64_h8_d256_int8_sr", "rtn", 0, False),
     ("gdn_b64_h8_d256_int8_sr", "sr_bdr", 0, False), ("mamba2_b128_h80_p64_n256_int8_sr", None, 0, False),
+    ("gdn_b64_h16_d128_int8_sr", "sr16", 0, False), ("gdn_b1024_h16_d128_int4_sr_long", "sr16", 0, False),
+    ("gdn_b1024_h16_d128_int4_sr_long", "rtn", 0, False), ("gdn_b256_h32_d128_mixed_sr", "rtn", 0, False),
+    ("mamba2_b128_h80_p64_n128_int8_sr", "rtn", 0, False),
 )
 
 
@@ -211,15 +214,15 @@ def measured_peak_gbs():
         return 6650.0, "fallback"
 
 
-def profiled_traffic(kernel_tag: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on the
-    current kernel sources; else None."""
+def profiled_traffic(workload: str, kernel_tag: str):
+    """DRAM bytes per launch of `kernel_tag` on `workload` from a committed ncu
+    summary, if it was taken on the current kernel sources; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     try:
         with open(path) as f:
             d = json.load(f)
-        e = d.get(kernel_tag)
-        if e and e.get("source_hash") == source_hash():
+        e = d.get(workload)
+        if e and e.get("kernel") == kernel_tag and e.get("source_hash") == source_hash():
             return float(e["dram_bytes_per_launch"])
     except (OSError, ValueError, KeyError):
         pass
@@ -555,7 +558,8 @@ def run_ours(args, w: W.Workload):
         "hbm_gbs": achieved,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
-                     "traffic": profiled_traffic(kernel_tag),
+                     "traffic": (profiled_traffic(w.name, kernel_tag)
+                                 if not args.window and not args.key_axis else None),
                      "algorithmic_bytes_per_launch": alg, "kernel": kernel_tag},
         "frac_of_8tbs_datasheet": achieved / 8000.0,
         "e2e": {"value": e2e_value, "unit": "head-updates/s", "h2d_bytes_per_step": h2d,

@@ -3,11 +3,15 @@
 // The grouping ablation of LoReS ("Quantizing Recurrent Language Models Is
 // Easier Than You Think", section "(1/4) Scale grouping"): one scale per key
 // row, s_i = max_j |S_ij| / r, instead of one per value column.  A row's
-// maximum runs over all d_v columns of the head, so one CTA owns one head:
-// warp w holds the 16-column block w (the same lane tile as the value-axis
-// kernel), the row maxima of the warps meet in shared memory, and two CTA
-// barriers separate the phases.  There are no early exits, so every thread
-// reaches both barriers.
+// maximum runs over all d_v columns of the head, so a CTA works on one head at
+// a time: warp w holds the 16-column block w (the same lane tile as the
+// value-axis kernel), the row maxima of the warps meet in shared memory, and
+// CTA barriers separate the phases.  CTAs are persistent and walk the heads
+// with a grid stride; each head (its codes, row scales, q, k and v) arrives in
+// a two-stage shared-memory ring by bulk asynchronous copies, so the next
+// head's copy overlaps this head's arithmetic.  Every thread takes the same
+// path through the barriers: the one early exit (a stage wait that ran out) is
+// decided for the whole CTA at once.
 //
 // Per head, in the canonical order the oracle follows:
 //   u_j = sum_i c_ij (s_i k_i)  (8 partials + XOR butterfly),
@@ -27,6 +31,21 @@ struct KaCfg {
     static constexpr int RPT = DK / kR;
     static constexpr int PST = RPT + 2;          // padded row-group stride of the pair arrays
     static constexpr int PAIRS = kR * PST;        // uint64 per pair array
+};
+
+// One head in a stage: codes (sized for 8-bit heads), the row scales, q and k
+// (d_k each) and v (d_v), the vectors as delivered (bf16 or f32); every part
+// at a 16-byte aligned offset.
+constexpr int kKaStages = 2;
+struct KaStage {
+    int off_s, off_q, off_k, off_v, bytes;
+    __host__ __device__ KaStage(int dk, int dv) {
+        off_s = dk * dv;
+        off_q = off_s + dk * 4;
+        off_k = off_q + dk * 4;
+        off_v = off_k + dk * 4;
+        bytes = (off_v + dv * 4 + 127) / 128 * 128;
+    }
 };
 
 __device__ __forceinline__ float ka_vec(const void* base, long long e, bool bf16) {
@@ -108,8 +127,28 @@ __device__ __forceinline__ void ka_requantize_store(const uint64_t (&S2)[RPT][2]
     }
 }
 
+// Issue the bulk copies of head hu into a stage (one thread).
+template <int DK>
+__device__ __forceinline__ void ka_issue(const DecodeParams& p, int hu, uint8_t* st, uint32_t bar,
+                                         const KaStage& L) {
+    const int b = hu / p.H, h = hu - b * p.H;
+    const uint32_t cb = static_cast<uint32_t>(DK * p.dv * p.head_bits[h] / 8);
+    const uint32_t esz = p.in_bf16 ? 2u : 4u;
+    const uint32_t vk = DK * esz, vv = static_cast<uint32_t>(p.dv) * esz;
+    const uint32_t s = smem_u32(st);
+    mbar_arrive_expect_tx(bar, cb + DK * 4u + 2u * vk + vv);
+    bulk_g2s(s, p.codes_in + (long long)b * p.row_bytes + p.head_off[h], cb, bar);
+    bulk_g2s(s + L.off_s, p.scales_in + (long long)hu * DK, DK * 4u, bar);
+    bulk_g2s(s + L.off_q, static_cast<const char*>(p.vA) + (long long)hu * vk, vk, bar);
+    bulk_g2s(s + L.off_k, static_cast<const char*>(p.vB) + (long long)hu * vk, vk, bar);
+    bulk_g2s(s + L.off_v, static_cast<const char*>(p.vC) + (long long)hu * vv, vv, bar);
+}
+
+// One head from its stage.  After the row-maxima barrier no thread reads the
+// stage again, so thread 0 refills it there with head `refill` (if any).
 template <int DK, int BITS, int RND>
-__device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, int b, int h, int hu) {
+__device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* st, const KaStage& L, uint8_t* work,
+                                        uint32_t bar, int b, int h, int hu, int refill) {
     using K = KaCfg<DK>;
     constexpr int RPT = K::RPT;
     constexpr int BLOCK_BYTES = DK * kBlockCols * BITS / 8;
@@ -117,7 +156,7 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, in
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, nt = blockDim.x, nw = nt >> 5;
     const int g = lane >> 2, cw = lane & 3;
     const bool bf16 = p.in_bf16 != 0;
-    uint64_t* pq = reinterpret_cast<uint64_t*>(smem);
+    uint64_t* pq = reinterpret_cast<uint64_t*>(work);
     uint64_t* pkk = pq + K::PAIRS;   // k
     uint64_t* pks = pkk + K::PAIRS;  // s_i k_i
     uint64_t* pas = pks + K::PAIRS;  // alpha s_i
@@ -127,9 +166,9 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, in
 
     // ---- key-axis vectors and row scales as duplicated pairs (shared by all warps)
     for (int i = tid; i < DK; i += nt) {
-        const float q = ka_vec(p.vA, (long long)hu * DK + i, bf16);
-        const float k = ka_vec(p.vB, (long long)hu * DK + i, bf16);
-        const float s = __ldg(p.scales_in + (long long)hu * DK + i);
+        const float q = ka_vec(st + L.off_q, i, bf16);
+        const float k = ka_vec(st + L.off_k, i, bf16);
+        const float s = reinterpret_cast<const float*>(st + L.off_s)[i];
         const int pos = (i & (kR - 1)) * K::PST + i / kR;
         const float ks = __fmul_rn(s, k), as = __fmul_rn(alpha, s);
         pq[pos] = pk(q, q);
@@ -141,9 +180,8 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, in
 
     // ---- this warp's block: decode, update, read out -------------------------
     const int j0 = w * kBlockCols;
-    const long long rowoff = (long long)b * p.row_bytes + p.head_off[h] + (long long)w * BLOCK_BYTES;
     uint64_t S2[RPT][2];
-    load_codes<BITS, RPT>(p.codes_in + rowoff, g, cw, S2);
+    load_codes<BITS, RPT>(st + w * BLOCK_BYTES, g, cw, S2);
     const uint64_t* kq = pq + g * K::PST;
     const uint64_t* kk = pkk + g * K::PST;
     const uint64_t* kks = pks + g * K::PST;
@@ -162,7 +200,7 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, in
     float wj[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-        const float v = ka_vec(p.vC, (long long)hu * p.dv + j0 + 4 * cw + j, bf16);
+        const float v = ka_vec(st + L.off_v, j0 + 4 * cw + j, bf16);
         wj[j] = __fmul_rn(beta, __fmaf_rn(-alpha, uv[j], v));
     }
     const uint64_t W01 = pk(wj[0], wj[1]), W23 = pk(wj[2], wj[3]);
@@ -197,6 +235,12 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, in
         if (cw == 0) rowmax[w * DK + g + kR * k] = m;
     }
     __syncthreads();
+    // every read of the stage is behind the barrier above: refill it (the
+    // proxy fence orders those generic-proxy reads before the async writes)
+    if (tid == 0 && refill >= 0) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        ka_issue<DK>(p, refill, st, bar, L);
+    }
     for (int i = tid; i < DK; i += nt) {
         float m = 0.f;
         for (int ww = 0; ww < nw; ++ww) m = max_nan(m, rowmax[ww * DK + i]);
@@ -218,6 +262,7 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, in
     uint64_t invp[RPT];
 #pragma unroll
     for (int k = 0; k < RPT; ++k) invp[k] = ki[k];
+    const long long rowoff = (long long)b * p.row_bytes + p.head_off[h] + (long long)w * BLOCK_BYTES;
     uint8_t* dst = p.codes_out + rowoff;
     const uint32_t gcol = static_cast<uint32_t>(j0 / 4 + cw);
     ka_requantize_store<BITS, RND, RPT>(S2, invp, dst, g, cw, gcol, h, b, p.step, p.rk);
@@ -237,15 +282,67 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* smem, in
     }
 }
 
+// Shared memory: the stages, then the pair arrays and row maxima of the head in
+// work, then one mbarrier per stage.
+template <int DK>
+__host__ __device__ inline size_t ka_work_bytes(int nw) {
+    return 5 * KaCfg<DK>::PAIRS * sizeof(uint64_t) + static_cast<size_t>(nw) * DK * sizeof(float);
+}
+template <int DK>
+__host__ __device__ inline size_t ka_smem(int dv) {
+    return static_cast<size_t>(kKaStages) * KaStage(DK, dv).bytes + ka_work_bytes<DK>(dv / kBlockCols) +
+           kKaStages * 8;
+}
+
 template <int DK, int RND>
 __global__ void __launch_bounds__(512) rsq_decode_ka_kernel(const __grid_constant__ DecodeParams p) {
-    extern __shared__ __align__(16) uint8_t smem[];
-    const int hu = blockIdx.x;
-    const int b = hu / p.H, h = hu - b * p.H;
-    if (p.head_bits[h] == 8)
-        ka_head<DK, 8, RND>(p, smem, b, h, hu);
-    else
-        ka_head<DK, 4, RND>(p, smem, b, h, hu);
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x;
+    const int heads = p.B * p.H, grid = static_cast<int>(gridDim.x);
+    const KaStage L(DK, p.dv);
+    uint8_t* work = smem + kKaStages * L.bytes;
+    const uint32_t bar0 = smem_u32(work + ka_work_bytes<DK>(p.dv / kBlockCols));
+    if (tid == 0) {
+        for (int s = 0; s < kKaStages; ++s) mbar_init(bar0 + 8 * s, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid == 0)
+        for (int s = 0; s < kKaStages; ++s) {
+            const int hu = static_cast<int>(blockIdx.x) + s * grid;
+            if (hu < heads) ka_issue<DK>(p, hu, smem + s * L.bytes, bar0 + 8 * s, L);
+        }
+    int stage = 0;
+    uint32_t parity = 0;
+    for (int hu = static_cast<int>(blockIdx.x); hu < heads; hu += grid) {
+        const uint32_t bar = bar0 + 8 * stage;
+        const bool ok = mbar_wait(bar, parity, p.wait_iters);
+        if (!__syncthreads_and(ok)) {
+            // the whole CTA leaves; first wait (bounded) for every stage copy it
+            // issued that has not landed, so none writes into a CTA that is gone
+            if (tid == 0) {
+                atomicOr(p.flag, kFlagTimeout);
+                for (int s = 0; s < kKaStages; ++s) {
+                    const int ahead = (s - stage + kKaStages) % kKaStages;
+                    if (static_cast<long long>(hu) + static_cast<long long>(ahead) * grid >= heads) continue;
+                    mbar_wait(bar0 + 8 * s, s >= stage ? parity : (parity ^ 1u), kDrainIters);
+                }
+            }
+            return;
+        }
+        const int b = hu / p.H, h = hu - b * p.H;
+        const long long next = static_cast<long long>(hu) + static_cast<long long>(kKaStages) * grid;
+        const int refill = next < heads ? static_cast<int>(next) : -1;
+        uint8_t* st = smem + stage * L.bytes;
+        if (p.head_bits[h] == 8)
+            ka_head<DK, 8, RND>(p, st, L, work, bar, b, h, hu, refill);
+        else
+            ka_head<DK, 4, RND>(p, st, L, work, bar, b, h, hu, refill);
+        if (++stage == kKaStages) {
+            stage = 0;
+            parity ^= 1u;
+        }
+    }
 }
 
 // Quantize a full-precision head (natural [dk][dv] layout) with key-axis
@@ -308,7 +405,7 @@ __device__ __forceinline__ void ka_quantize_head(const QuantParams& p, uint8_t* 
 
 template <int DK>
 __global__ void __launch_bounds__(512) rsq_quantize_ka_kernel(const __grid_constant__ QuantParams p) {
-    extern __shared__ __align__(16) uint8_t smem[];
+    extern __shared__ __align__(128) uint8_t smem[];
     const int hu = blockIdx.x;
     const int b = hu / p.H, h = hu - b * p.H;
     const bool bits8 = p.head_bits[h] == 8;
@@ -334,25 +431,30 @@ int launch_quantize_ka_dk(const QuantParams& p, void* stream) {
 }
 
 template <int DK>
-size_t ka_smem(int nw) {
-    return 5 * KaCfg<DK>::PAIRS * sizeof(uint64_t) + static_cast<size_t>(nw) * DK * sizeof(float);
+const void* ka_func(int rnd) {
+    constexpr int kSr8 = kRndSr | kRndU8;
+    return rnd == kSr8    ? reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, kSr8>)
+           : rnd == kRndSr ? reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, kRndSr>)
+                           : reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, 0>);
 }
 
 template <int DK>
 int launch_ka_dk(const DecodeParams& p, void* stream) {
-    const int nw = p.dv / kBlockCols;
-    const size_t smem = ka_smem<DK>(nw);
-    constexpr int kSr8 = kRndSr | kRndU8;
-    const void* f = p.rnd == kSr8    ? reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, kSr8>)
-                    : p.rnd == kRndSr ? reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, kRndSr>)
-                                      : reinterpret_cast<const void*>(&rsq_decode_ka_kernel<DK, 0>);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(p.B * p.H);
-    cfg.blockDim = dim3(32 * nw);
-    cfg.dynamicSmemBytes = smem;
+    cfg.gridDim = dim3(p.grid);
+    cfg.blockDim = dim3(32 * (p.dv / kBlockCols));
+    cfg.dynamicSmemBytes = ka_smem<DK>(p.dv);
     cfg.stream = static_cast<cudaStream_t>(stream);
     void* args[] = {const_cast<DecodeParams*>(&p)};
-    return static_cast<int>(cudaLaunchKernelExC(&cfg, f, args));
+    return static_cast<int>(cudaLaunchKernelExC(&cfg, ka_func<DK>(p.rnd), args));
+}
+
+template <int DK>
+int ka_info_dk(int dv, int rnd, int* threads, size_t* smem, const void** func) {
+    *threads = 32 * (dv / kBlockCols);
+    *smem = ka_smem<DK>(dv);
+    *func = ka_func<DK>(rnd);
+    return 0;
 }
 
 }  // namespace
@@ -364,6 +466,16 @@ int launch_quantize_ka(int dk, const QuantParams& p, void* stream) {
         case 64: return launch_quantize_ka_dk<64>(p, stream);
         case 128: return launch_quantize_ka_dk<128>(p, stream);
         default: return static_cast<int>(cudaErrorInvalidValue);
+    }
+}
+
+int decode_ka_info(int dk, int dv, int rnd, int* threads, size_t* smem, const void** func) {
+    switch (dk) {
+        case 16: return ka_info_dk<16>(dv, rnd, threads, smem, func);
+        case 32: return ka_info_dk<32>(dv, rnd, threads, smem, func);
+        case 64: return ka_info_dk<64>(dv, rnd, threads, smem, func);
+        case 128: return ka_info_dk<128>(dv, rnd, threads, smem, func);
+        default: return -1;
     }
 }
 

@@ -884,13 +884,16 @@ int decode_info_rules(bool f32state, int rnd, int* threads, size_t* smem, const 
     return found;
 }
 
-// Two blocks per warp are built for d_k = 128 units of four blocks (not for the
-// pure-write window).
+// Two blocks per warp are built for d_k = 128 units of four blocks, but not for
+// the pure-write window nor for Bounded Directional Rounding: its second decode
+// of the previous codes does not fit two blocks' work into the registers of
+// six 64-thread CTAs per SM (the instances spilled 400-550 bytes per thread).
 template <int FAM, int... RNDS>
 int decode_info_family(int dk, int ub, int bpw, bool f32state, int rnd, int* threads, size_t* smem,
                        const void** func) {
+    constexpr bool kAnyBdr = (((RNDS & kRndBdr) != 0) || ...);
     if (bpw == 2) {
-        if constexpr (!is_pw_family(FAM)) {
+        if constexpr (!is_pw_family(FAM) && !kAnyBdr) {
             if (dk == 128 && ub == 4 && !f32state)
                 return decode_info_rules<FAM, 128, 4, 2, RNDS...>(f32state, rnd, threads, smem, func);
         }

@@ -22,6 +22,7 @@ struct rsq_ctx {
     int ub, ncb, units;   // 16-column blocks per unit, units per head, units per step
     int bpw;              // blocks each warp of the decode kernel takes per unit (1 or 2)
     int grid;        // persistent decode grid
+    int ka_grid;     // persistent grid of the key-axis kernel (key-axis scales)
     int device;
     unsigned* flag;  // device word: rsq::kFlag* bits
     uint32_t wait_iters;  // limit of the kernels' bounded barrier waits (0: the default)
@@ -71,7 +72,15 @@ int base_rule(int r) { return r & (rsq::kRndSr | rsq::kRndU8); }
 // 16-column blocks per work unit (at most): four, except stochastic rounding
 // at dk = 256, whose two-warp blocks run faster as 128-thread CTAs at three
 // per SM (168 registers, no spills) than as 256-thread CTAs at two.
-int unit_blocks(const rsq_config& c) { return (c.dk > 128 && (c.rounding & RSQ_SR)) ? 2 : 4; }
+// Blocks per work unit.  At d_k = 256 stochastic rounding takes two (three
+// 128-thread CTAs per SM at 168 registers, no spills) and BDR one: with two
+// blocks per unit its instances spilled 400-700 bytes per thread, with four
+// they take 255 registers and run one CTA per SM.
+int unit_blocks(const rsq_config& c) {
+    if (c.dk <= 128) return 4;
+    if (c.rounding & RSQ_BDR) return 1;
+    return (c.rounding & RSQ_SR) ? 2 : 4;
+}
 
 bool dk_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
 bool dv_ok(int d) { return d == 16 || d == 32 || d == 64 || d == 128 || d == 256; }
@@ -292,6 +301,24 @@ rsq_status rsq_create(const rsq_config* cfg, rsq_ctx** out) {
         return cuda_fail(err, "create");
     }
     ctx->grid = static_cast<int>(std::min<long long>(units, static_cast<long long>(sms) * per_sm));
+    if (c.key_axis) {
+        // the key-axis kernel: one head at a time per CTA, every resident CTA
+        int threads = 0, per_sm_ka = 0;
+        size_t smem = 0;
+        const void* func = nullptr;
+        int e = rsq::decode_ka_info(c.dk, c.dv, base_rule(c.rounding), &threads, &smem, &func);
+        if (e == 0) e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e == 0) e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm_ka, func, threads, smem);
+        if (e == 0 && per_sm_ka < 1) e = cudaErrorInvalidConfiguration;
+        if (e) {
+            release_flag(ctx);
+            delete ctx;
+            return e == -1 ? fail(RSQ_E_UNSUPPORTED, "create: no key-axis kernel for dk=%d", c.dk)
+                           : cuda_fail(e, "create: key-axis launch geometry");
+        }
+        ctx->ka_grid = static_cast<int>(std::min<long long>(static_cast<long long>(c.batch) * c.heads,
+                                                            static_cast<long long>(sms) * per_sm_ka));
+    }
     *out = ctx;
     return RSQ_OK;
 }
@@ -466,6 +493,7 @@ rsq_status decode_step_impl(const rsq_ctx* ctx, const rsq_state* state_in, const
     p.gb = ghu / c.heads;
     if (c.key_axis) {
         if (copy_absmax) return fail(RSQ_E_UNSUPPORTED, "decode_step_copy_scale: not with key-axis scales");
+        p.grid = ctx->ka_grid;
         const int e = rsq::launch_decode_ka(c.dk, p, stream);
         if (e) return cuda_fail(e, "decode_step launch");
         return RSQ_OK;

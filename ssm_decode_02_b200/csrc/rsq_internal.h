@@ -130,8 +130,10 @@ int decode_kernel_info(int family, int dk, int ub, int bpw, bool f32state, int r
                        const void** func);
 int launch_quantize(int dk, const QuantParams& p, void* stream);
 int launch_dequantize(int dk, const DequantParams& p, void* stream);
-// key-axis scale groups (one CTA per head)
+// key-axis scale groups (one head at a time per CTA; the decode kernel is
+// persistent over p.grid CTAs)
 int launch_decode_ka(int dk, const DecodeParams& p, void* stream);
+int decode_ka_info(int dk, int dv, int rnd, int* threads, size_t* smem, const void** func);
 int launch_quantize_ka(int dk, const QuantParams& p, void* stream);
 int launch_drift(const DriftParams& p, void* stream);
 
