@@ -165,7 +165,7 @@ SWEEP = (
     ("gdn_b64_h8_d256_int8_sr", "sr_bdr", 0, False), ("mamba2_b128_h80_p64_n256_int8_sr", None, 0, False),
     ("gdn_b64_h16_d128_int8_sr", "sr16", 0, False), ("gdn_b1024_h16_d128_int4_sr_long", "sr16", 0, False),
     ("gdn_b1024_h16_d128_int4_sr_long", "rtn", 0, False), ("gdn_b256_h32_d128_mixed_sr", "rtn", 0, False),
-    ("mamba2_b128_h80_p64_n128_int8_sr", "rtn", 0, False),
+    ("mamba2_b128_h80_p64_n128_int8_sr", "rtn", 0, False), ("gdn_b64_h8_d256_int8_sr", "bdr", 0, False),
 )
 
 

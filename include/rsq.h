@@ -151,7 +151,8 @@ typedef struct {
     int key_axis;    /* 0: one scale per value column (the method's grouping); 1: one scale
                         per key row, s_i = max_j |S_ij| / r ([LoReS] (1/4), the grouping
                         ablation).  Key-axis: Gated DeltaNet, 4/8-bit heads, RSQ_RTN,
-                        RSQ_SR or RSQ_SR8; scales are [B][H][dk]; one CTA per head. */
+                        RSQ_SR or RSQ_SR8; scales are [B][H][dk]; a CTA works on one head
+                        at a time (a row maximum spans every column). */
     rsq_alloc_fn alloc;      /* allocator hook (above); NULL with release NULL: cudaMalloc */
     rsq_release_fn release;  /* its release; set both or neither (else RSQ_E_INVAL) */
     void* alloc_user;        /* passed to both */
@@ -350,10 +351,12 @@ rsq_status rsq_check_flags(const rsq_ctx* ctx, int* seen, void* stream);
 
 /* Failure-detection hook for tests (no counterpart in the method's pages).
  * Sets the limit of this context's decode kernels' bounded barrier waits to
- * `wait_iters` polls (0: the default, 2^22) and, with withhold = 1, makes
- * the second warp of every two-warp
- * block (dk = 256) skip its arrivals on the block's exchange barrier, so that
- * both warps' waits on it run out.  A kernel whose wait runs out sets the
+ * `wait_iters` polls (0: the default, 2^22).  With withhold = 1 the second
+ * warp of every two-warp block (dk = 256) skips its arrivals on the block's
+ * exchange barrier, so that both warps' waits on it run out; and the
+ * key-axis kernel (key_axis = 1) never fills the first stage of its ring, so
+ * that its first stage wait runs out while the second stage's copies are in
+ * flight.  A kernel whose wait runs out sets the
  * context's timeout flag, waits (bounded) for the copies it still has in
  * flight towards its shared memory, and ends; that step's outputs are
  * incomplete and rsq_check_flags returns RSQ_E_CUDA.  withhold = 0 and

@@ -307,10 +307,12 @@ __global__ void __launch_bounds__(512) rsq_decode_ka_kernel(const __grid_constan
         fence_mbar_init();
     }
     __syncthreads();
+    // (failure-detection tests: with p.withhold the first stage is never
+    // filled, so its wait runs out while the second stage's copies are in flight)
     if (tid == 0)
         for (int s = 0; s < kKaStages; ++s) {
             const int hu = static_cast<int>(blockIdx.x) + s * grid;
-            if (hu < heads) ka_issue<DK>(p, hu, smem + s * L.bytes, bar0 + 8 * s, L);
+            if (hu < heads && !(p.withhold && s == 0)) ka_issue<DK>(p, hu, smem + s * L.bytes, bar0 + 8 * s, L);
         }
     int stage = 0;
     uint32_t parity = 0;

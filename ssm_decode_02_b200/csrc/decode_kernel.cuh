@@ -907,7 +907,11 @@ int decode_info_family(int dk, int ub, int bpw, bool f32state, int rnd, int* thr
     RSQ_CASE(64, 1) RSQ_CASE(64, 2) RSQ_CASE(64, 4)
     RSQ_CASE(128, 1) RSQ_CASE(128, 2) RSQ_CASE(128, 4)
     if constexpr (!is_pw_family(FAM)) {
-        RSQ_CASE(256, 1) RSQ_CASE(256, 2) RSQ_CASE(256, 4)
+        RSQ_CASE(256, 1)
+        // BDR at d_k = 256 runs one block per unit (the host never picks more)
+        if constexpr (!kAnyBdr) {
+            RSQ_CASE(256, 2) RSQ_CASE(256, 4)
+        }
     }
 #undef RSQ_CASE
     return -1;

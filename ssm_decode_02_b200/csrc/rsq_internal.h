@@ -77,7 +77,8 @@ struct DecodeParams {
     PhiloxKeys rk;                 // Philox round keys of (key0, key1)
     // bounded waits: polls before a barrier wait gives up (sets kFlagTimeout);
     // withhold = 1 (failure-detection tests only): the second warp of a
-    // two-warp block never arrives on the block's exchange barrier
+    // two-warp block never arrives on the block's exchange barrier, and the
+    // key-axis kernel never fills its first stage
     uint32_t wait_iters;
     int withhold;
     uint32_t head_off[RSQ_MAX_HEADS];  // byte offset of each head in a batch row

@@ -1,8 +1,9 @@
 """GPU parity of key-axis scale groups (LoReS "(1/4) Scale grouping": one scale
 per key row, the grouping ablation) against the CPU oracle.
 
-The key-axis decode kernel (one CTA per head) and its quantize / dequantize
-paths must match the oracle bit for bit on free-running trajectories.
+The key-axis decode kernel (persistent CTAs, one head at a time through a
+two-stage ring of bulk copies) and its quantize / dequantize paths must match
+the oracle bit for bit on free-running trajectories.
 """
 import dataclasses
 
@@ -99,3 +100,49 @@ def test_key_axis_quantize_dequantize_and_maxima(rounding):
     m = torch.empty((2, 3, 128), dtype=torch.float32, device="cuda")
     run.ctx.column_absmax(g, m)
     assert np.array_equal(host(m), np.abs(oracle.dequantize_ka(want)).max(axis=2))
+
+
+def test_key_axis_several_heads_per_cta_all_heads():
+    """More heads than resident CTAs (d_v = 256: 512-thread CTAs), so every
+    persistent CTA takes several heads through its two-stage ring; every head
+    compared, mixed widths."""
+    w = dataclasses.replace(W.WORKLOADS[1], B=40, H=8, dk=64, dv=256)
+    _trajectory(KaRun(w, [8, 4, 4, 8, 8, 4, 8, 4], rsq.RSQ_SR8), 3, seed=11)
+
+
+def test_key_axis_stage_wait_runs_out_and_is_reported():
+    """Failure detection without a fault: with the test hook the first stage of
+    every CTA's ring is never filled, so its bounded wait runs out while the
+    second stage's copies are in flight.  The kernel must wait for those
+    copies, end by itself, report the timeout, and leave the context usable."""
+    import time
+    w = dataclasses.replace(W.WORKLOADS[1], B=40, H=8, dk=64, dv=256)
+    bits = [8, 4, 4, 8, 8, 4, 8, 4]
+    run = KaRun(w, bits, rsq.RSQ_SR8)
+    rng = np.random.default_rng(2)
+    S = (rng.standard_normal((run.B, run.H, run.dk, run.dv)) * 0.2).astype(np.float32)
+    st = oracle.quantize_ka(S, run.bits, rounding=run.rounding, seed=w.sr_seed, step=0)
+    inp = run.inputs(0)
+    keep = {k: dev(v) for k, v in inp.items()}
+    ins = rsq.gdn_inputs(keep["q"], keep["k"], keep["v"], keep["alpha"], keep["beta"])
+    out = torch.empty((run.B, run.H, run.dv), dtype=torch.float32, device="cuda")
+    g = run.upload(st)
+    rsq.rsq_debug_waits(run.ctx.ctx, 1024, 1)
+    t0 = time.perf_counter()
+    run.ctx.decode_step(g, g, ins, out, 0)
+    torch.cuda.synchronize()                     # the kernel ended by itself
+    assert time.perf_counter() - t0 < 60.0
+    with pytest.raises(rsq.RsqError) as e:
+        run.ctx.check_flags()
+    assert e.value.status == rsq.RSQ_E_CUDA and "timed out" in str(e.value)
+    # hook cleared: the same context computes the step bit-exactly again
+    rsq.rsq_debug_waits(run.ctx.ctx, 0, 0)
+    assert run.ctx.check_flags() == 0            # the flag was cleared by the read above
+    g = run.upload(st)
+    run.ctx.decode_step(g, g, ins, out, 0)
+    torch.cuda.synchronize()
+    want, o = oracle.gdn_ka_step(st, inp, run.bits, rounding=run.rounding, seed=w.sr_seed, step=0)
+    allh = [(b, h) for b in range(run.B) for h in range(run.H)]
+    _assert_ka_equal(run.download(g), want, allh, "after the timeout")
+    assert_out_equal(host(out), o, what="after the timeout")
+    assert run.ctx.check_flags() == 0
