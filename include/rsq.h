@@ -390,10 +390,11 @@ int rsq_reduction_partials(int dk);
  * Its scratch (the decode kernel's flag word) lives in a statically allocated
  * device array of 64 words (256 bytes) that every GPU loading the library
  * holds until the process exits; a call needing more scratch than that is
- * rejected with RSQ_E_UNSUPPORTED.  All calls share the array: the flag word is
- * cleared on the stream at the start of every call, the flags it collects are
- * not reported (use a context and rsq_check_flags for that), and calls that
- * overlap on the GPU race on it.  The first call on a device looks up the
+ * rejected with RSQ_E_UNSUPPORTED.  All calls share the array.  The kernels
+ * only set bits in its flag word and nothing reads or clears it, so a
+ * non-finite column or a timed-out wait is not reported on this path (use a
+ * context and rsq_check_flags for that), and overlapping calls may set bits
+ * concurrently without harm.  The first call on a device looks up the
  * array's device address for that device, and the first call with a given
  * kernel sets its shared-memory attribute and queries its occupancy; make
  * those first calls before any stream capture.  The remembered address

@@ -1,12 +1,13 @@
 // decode_kernel.cuh -- fused quantized recurrent-state decode step (sm_100a).
 //
-// A work unit is one to four 16-column blocks of one head (all dk rows); the
-// CTA has one warp per block up to dk = 128, and each warp owns its block's
-// columns outright, so every reduction over the key axis stays inside the warp
-// and the loop has no CTA-wide barrier.  At dk = 256 two warps share a block
-// (half of the rows each) and combine their column totals through shared
-// memory behind a per-block mbarrier.  Persistent CTAs walk the units with a
-// grid stride.
+// A work unit is one to four 16-column blocks of one head (all dk rows); up to
+// dk = 128 the CTA has one warp per block (or, on large steps with units of
+// four blocks, one warp per two blocks, taken one after the other), and each
+// warp owns its block's columns outright, so every reduction over the key axis
+// stays inside the warp and the loop has no CTA-wide barrier.  At dk = 256 two
+// warps share a block (half of the rows each) and combine their column totals
+// through shared memory behind a per-block mbarrier.  Persistent CTAs walk the
+// units with a grid stride.
 // Units arrive in an NS-stage shared-memory ring filled by bulk asynchronous
 // (TMA) copies; the last warp to finish with a stage refills it with the unit
 // NS ahead.  Per block a warp:

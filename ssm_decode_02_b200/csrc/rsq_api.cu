@@ -752,9 +752,8 @@ extern "C" rsq_status rsq_decode_step_noalloc(const rsq_config* cfg, const rsq_s
     if (s) return s;
     ctx.grid = static_cast<int>(std::min<long long>(units, static_cast<long long>(sms) * per_sm));
 
-    // the flag word starts each call at zero (every call shares the array)
-    err = cudaMemsetAsync(scratch, 0, kNoallocWordsNeeded * sizeof(unsigned), static_cast<cudaStream_t>(stream));
-    if (err) return cuda_fail(err, "decode_step_noalloc: clear scratch");
+    // the kernels only set bits in the flag word and nothing reads it on this
+    // path, so it is never cleared (every call shares the array)
     ctx.flag = scratch;
     return rsq_decode_step(&ctx, state_in, state_out, inputs, out, step, stream);
 }
