@@ -146,3 +146,63 @@ def test_key_axis_stage_wait_runs_out_and_is_reported():
     _assert_ka_equal(run.download(g), want, allh, "after the timeout")
     assert_out_equal(host(out), o, what="after the timeout")
     assert run.ctx.check_flags() == 0
+
+
+@pytest.mark.parametrize("bits", [8, 4])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_SR8, rsq.RSQ_RTN])
+def test_key_axis_against_the_literal_order(bits, rounding):
+    """Key-axis groups against the oracle's literal order at the method's
+    tolerance ("(1/4) Scale grouping": s_i = max_j |S_ij| / r, codes
+    round(S / s); "(3/4) Rounding").  Teacher-forced on the benchmark head
+    shape: each step starts the GPU and the literal order from the canonical
+    oracle's state, which the GPU matches bit for bit.  At most 1e-5 of the
+    codes differ, each by one step, apart from nearest-rounding boundary cases
+    (held to 1e-3); scales agree to 1e-5 relative; outputs and the
+    dequantized state of the agreeing codes to 1e-3 normwise relative.  Row
+    groups are compared through the transpose, so a group's maximum is the
+    column maximum the boundary accounting expects."""
+    import plain_order
+    w = dataclasses.replace(W.WORKLOADS[1], B=8)
+    hb = np.full(w.H, bits, np.int8)
+    run = KaRun(w, hb, rounding)
+    rng = np.random.default_rng(21 + bits)
+    S = (rng.standard_normal((run.B, run.H, run.dk, run.dv)) * 0.2).astype(np.float32)
+    orc_rnd = oracle.SR8 if rounding == rsq.RSQ_SR8 else oracle.RTN
+    st = oracle.quantize_ka(S, hb, rounding=orc_rnd, seed=w.sr_seed, step=0)
+    b32 = np.full(w.H, 32, np.int8)
+    n_other = n_tie = n_tot = 0
+    for t in range(4):
+        inp = run.inputs(t)
+        keep = {k: dev(v) for k, v in inp.items()}
+        ins = rsq.gdn_inputs(keep["q"], keep["k"], keep["v"], keep["alpha"], keep["beta"])
+        out = torch.empty((run.B, run.H, run.dv), dtype=torch.float32, device="cuda")
+        g = run.upload(st)
+        run.ctx.decode_step(g, g, ins, out, t)
+        torch.cuda.synchronize()
+        gpu = run.download(g)
+        canon, canon_out = oracle.gdn_ka_step(st, inp, hb, rounding=orc_rnd, seed=w.sr_seed, step=t)
+        allh = [(b, h) for b in range(run.B) for h in range(run.H)]
+        _assert_ka_equal(gpu, canon, allh, "step %d" % t)
+        assert_out_equal(host(out), canon_out, what="step %d" % t)
+        plain, plain_out = oracle.gdn_ka_step(st, inp, hb, rounding=orc_rnd, seed=w.sr_seed, step=t,
+                                              mode=oracle.PLAIN)
+        # the literal order's full-precision S_t: the 32-bit plain step of the dequantized state
+        f = oracle.zero_state(run.B, run.H, run.dk, run.dv, fp32=True)
+        f["f"] = oracle.dequantize_ka(st)
+        lit, _ = oracle.gdn_step(f, inp, b32, rounding=oracle.RTN, seed=0, step=0, mode=oracle.PLAIN)
+        T = lambda x: np.ascontiguousarray(np.swapaxes(x, 2, 3))
+        o, ti, tot = plain_order.compare_codes(T(gpu["codes"]), T(plain["codes"]), T(lit["f"]), hb,
+                                               nearest=rounding == rsq.RSQ_RTN)
+        n_other, n_tie, n_tot = n_other + o, n_tie + ti, n_tot + tot
+        assert np.allclose(gpu["scales"], plain["scales"], rtol=1e-5, atol=0)
+        assert plain_order.max_rel(host(out), plain_out) <= 1e-3
+        same = gpu["codes"] == plain["codes"]
+        dg = np.where(same, oracle.dequantize_ka(gpu), 0.0)
+        dp = np.where(same, oracle.dequantize_ka(plain), 0.0)
+        rows = np.abs(oracle.dequantize_ka(plain)).max(axis=3, keepdims=True)
+        rows[rows == 0] = 1.0
+        assert np.max(np.abs(dg - dp) / rows) <= 1e-3
+        st = canon
+    assert n_tot > 0
+    assert n_other <= 1e-5 * n_tot, (n_other, n_tie, n_tot)
+    assert n_tie <= 1e-3 * n_tot, (n_other, n_tie, n_tot)
