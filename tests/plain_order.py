@@ -43,6 +43,9 @@ def literal_state(family: str, st: dict, inp: dict, head_bits, *, ngroups: int =
     elif family == "mamba2":
         out, _ = oracle.mamba2_step(f, inp, b32, rounding=oracle.RTN, seed=0, step=0, mode=oracle.PLAIN,
                                     ngroups=ngroups, decay=decay)
+    elif family in ("gla", "kda"):
+        step = oracle.gla_step if family == "gla" else oracle.kda_step
+        out, _ = step(f, inp, b32, rounding=oracle.RTN, seed=0, step=0, mode=oracle.PLAIN)
     else:
         raise ValueError(family)
     return out["f"]

@@ -36,7 +36,7 @@ def _decay(inp):
 def _against_plain(run: Run, steps: int, decay_override: bool = True, bit_exact: bool = True):
     """Teacher-forced: every step starts both sides from the canonical oracle's
     state.  Returns (codes differing away from ties, at ties, codes compared)."""
-    family = "gdn" if run.family == rsq.RSQ_GDN else "mamba2"
+    family = {rsq.RSQ_GDN: "gdn", rsq.RSQ_MAMBA2: "mamba2", rsq.RSQ_GLA: "gla", rsq.RSQ_KDA: "kda"}[run.family]
     nearest = run.rounding == rsq.RSQ_RTN
     st = run.zero()
     n_other = n_tie = n_tot = 0
@@ -141,3 +141,13 @@ def test_mixed_bit_map_from_the_runs_gates():
         assert_state_equal(run.download(g_out), st, run.head_bits, what="step %d" % t)
         assert_out_equal(out, ref_out, what="step %d" % t)
         g_in, g_out = g_out, g_in
+
+
+@pytest.mark.parametrize("name", ["gla_b64_h16_d128_int8_sr", "kda_b64_h16_d128_int8_sr"], ids=["gla", "kda"])
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("rounding", ["sr", "rtn"])
+def test_diag_families_plain(name, bits, rounding):
+    """GLA and KDA (a decay per key channel), 4- and 8-bit codes, stochastic
+    (8-bit uniforms) and nearest rounding, bf16 inputs."""
+    w = dataclasses.replace(W.BY_NAME[name], rounding=rounding)
+    _check(_against_plain(Run(w, np.full(w.H, bits, np.int8), B=8), 4))
