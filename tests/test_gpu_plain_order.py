@@ -151,3 +151,12 @@ def test_diag_families_plain(name, bits, rounding):
     (8-bit uniforms) and nearest rounding, bf16 inputs."""
     w = dataclasses.replace(W.BY_NAME[name], rounding=rounding)
     _check(_against_plain(Run(w, np.full(w.H, bits, np.int8), B=8), 4))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("rounding", ["sr", "rtn"])
+def test_dk256_plain(bits, rounding):
+    """d_k = 256 (two warps per block, the 16-partial canonical order), 4- and
+    8-bit codes, stochastic (8-bit uniforms) and nearest rounding."""
+    w = dataclasses.replace(W.BY_NAME["gdn_b64_h8_d256_int8_sr"], rounding=rounding)
+    _check(_against_plain(Run(w, np.full(w.H, bits, np.int8), B=8), 3))
