@@ -37,7 +37,7 @@ def _against_plain(run: Run, steps: int, decay_override: bool = True, bit_exact:
     """Teacher-forced: every step starts both sides from the canonical oracle's
     state.  Returns (codes differing away from ties, at ties, codes compared)."""
     family = {rsq.RSQ_GDN: "gdn", rsq.RSQ_MAMBA2: "mamba2", rsq.RSQ_GLA: "gla", rsq.RSQ_KDA: "kda"}[run.family]
-    nearest = run.rounding == rsq.RSQ_RTN
+    nearest = (run.rounding & rsq.RSQ_SR) == 0   # nearest rounding, with or without BDR
     st = run.zero()
     n_other = n_tie = n_tot = 0
     for t in range(steps):
@@ -160,3 +160,14 @@ def test_dk256_plain(bits, rounding):
     8-bit codes, stochastic (8-bit uniforms) and nearest rounding."""
     w = dataclasses.replace(W.BY_NAME["gdn_b64_h8_d256_int8_sr"], rounding=rounding)
     _check(_against_plain(Run(w, np.full(w.H, bits, np.int8), B=8), 3))
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_BDR, rsq.RSQ_SR8_BDR], ids=["bdr", "sr8_bdr"])
+def test_bdr_plain(bits, rounding):
+    """Bounded Directional Rounding on nearest and on stochastic rounding (8-bit
+    uniforms), 4- and 8-bit codes.  In the literal order the reversal test
+    compares c s_new with c_prev s_prev from the float scales and takes ceil or
+    floor of S / s; the canonical order uses the multiplier."""
+    w = W.WORKLOADS[1]
+    _check(_against_plain(Run(w, np.full(w.H, bits, np.int8), B=8, rounding=rounding), 4))
