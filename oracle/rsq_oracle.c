@@ -6,7 +6,10 @@
  * path (the CUDA library) never calls it and shares no code with it.
  *
  * Plain, single-threaded, obviously-correct C.  Every function cites the passage
- * of the method description it follows.  Sources:
+ * of the method description it follows, and every function is pinned by a
+ * test against something other than itself.  Parity unpinned: the drift
+ * *values* of the long-horizon study, which the pages describe only in words
+ * (the steps that produce them are pinned).  Sources:
  *   [LoReS]  "Quantizing Recurrent Language Models Is Easier Than You Think"
  *            (blog post of the LoReS paper): sections "(1/4) Scale grouping",
  *            "(2/4) Mixed precision", "(3/4) Rounding", "(4/4) Rotations".
