@@ -112,3 +112,58 @@ def test_window_entry_points_checked():
     a, b, sc = rsq.rsq_window_bytes(ctx.ctx)
     assert (a, b, sc) == (1 * 2 * 4 * 128, 1 * 2 * 4 * 128, 1 * 2 * 4 * 4)
     ctx.close()
+
+
+@pytest.mark.parametrize("bits", [4, 8])
+@pytest.mark.parametrize("rounding", [rsq.RSQ_SR8, rsq.RSQ_RTN])
+def test_window_against_the_literal_order(bits, rounding):
+    """The low-bit history of a window state against the oracle's literal order
+    at the method's tolerance, teacher-forced through the first merges (8 slots):
+    each step starts the GPU and both oracle orders from the canonical state,
+    which the GPU matches bit for bit.  The window's own arithmetic (the slot
+    propagation and its FP8 codes) is the same in both orders and must agree
+    exactly; of the history's codes at most 1e-5 differ, each by one step, apart
+    from nearest-rounding boundary cases (1e-3), judged against the literal
+    order's full-precision history after the merge."""
+    import plain_order
+    Wn = 8
+    w = dataclasses.replace(W.WORKLOADS[1], B=8)
+    hb = np.full(w.H, bits, np.int8)
+    b32 = np.full(w.H, 32, np.int8)
+    run = Run(w, hb, rounding=rounding)
+    ctx = rsq.Context(rsq.RSQ_GDN, run.B, run.H, run.dk, run.dv, head_bits=hb, rounding=rounding,
+                      in_dtype=run.in_dtype, seed=run.seed, window=Wn)
+    st = run.zero()
+    win = oracle.zero_window(run.B, run.H, Wn, run.dk, run.dv)
+    allh = [(b, h) for b in range(run.B) for h in range(run.H)]
+    n_other = n_tie = n_tot = 0
+    for t in range(Wn + 3):
+        inp = run.inputs(t)
+        ins, keep = run.dev_inputs(inp)
+        out = torch.empty((run.B, run.H, run.dv), dtype=torch.float32, device="cuda")
+        g_in, g_out = run.upload(st), run.upload(st)
+        w_in, w_out = _upload_window(win, run.dv), _upload_window(win, run.dv)
+        ctx.decode_step_window(g_in, g_out, w_in, w_out, ins, out, t)
+        torch.cuda.synchronize()
+        gpu, gwin = run.download(g_out), _download_window(w_out, run.dv)
+        canon, cwin, co = oracle.gdn_pw_step(st, win, inp, hb, rounding=rounding, seed=run.seed, step=t)
+        assert_state_equal(gpu, canon, hb, what="step %d" % t)
+        assert_out_equal(host(out), co, what="step %d" % t)
+        _assert_window_equal(gwin, cwin, allh, "step %d" % t)
+        plain, pwin, po = oracle.gdn_pw_step(st, win, inp, hb, rounding=rounding, seed=run.seed, step=t,
+                                             mode=oracle.PLAIN)
+        _assert_window_equal(pwin, cwin, allh, "step %d (literal order)" % t)
+        f = oracle.zero_state(run.B, run.H, run.dk, run.dv, fp32=True)
+        f["f"] = oracle.dequantize(st, hb)
+        lit, _, _ = oracle.gdn_pw_step(f, win, inp, b32, rounding=oracle.RTN, seed=0, step=t, mode=oracle.PLAIN)
+        o, ti, tot = plain_order.compare_codes(gpu["codes"], plain["codes"], lit["f"], hb,
+                                               nearest=rounding == rsq.RSQ_RTN)
+        n_other, n_tie, n_tot = n_other + o, n_tie + ti, n_tot + tot
+        assert np.allclose(gpu["scales"], plain["scales"], rtol=1e-5, atol=0)
+        assert plain_order.max_rel(host(out), po) <= 1e-3
+        st, win = canon, cwin
+        del keep
+    ctx.close()
+    assert n_tot > 0
+    assert n_other <= 1e-5 * n_tot, (n_other, n_tie, n_tot)
+    assert n_tie <= 1e-3 * n_tot, (n_other, n_tie, n_tot)
