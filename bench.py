@@ -559,7 +559,8 @@ def run_ours(args, w: W.Workload):
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "peak_kind": peak_kind,
                      "traffic": (profiled_traffic(w.name, kernel_tag)
-                                 if not args.window and not args.key_axis else None),
+                                 if not (args.window or args.key_axis or getattr(args, "state", None))
+                                 else None),
                      "algorithmic_bytes_per_launch": alg, "kernel": kernel_tag},
         "frac_of_8tbs_datasheet": achieved / 8000.0,
         "e2e": {"value": e2e_value, "unit": "head-updates/s", "h2d_bytes_per_step": h2d,
@@ -782,6 +783,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--rounding", choices=sorted(ROUNDING), default=None,
                     help="override the workload's requantization rule")
+    ap.add_argument("--state", choices=["int8", "int4", "fp32"], default=None,
+                    help="override the workload's state format with one width for every head")
     ap.add_argument("--window", type=int, default=0,
                     help="pure-write window slots (Gated DeltaNet): 0, 4, 8 or 16")
     ap.add_argument("--key-axis", action="store_true",
@@ -809,12 +812,14 @@ def main():
         with mp.get_context("spawn").Pool(max(1, min(32, (os.cpu_count() or 2) - 1))) as pool:
             return run_drift(args, w, pool)
     w = W.BY_NAME[args.workload]
-    if args.rounding or args.seed is not None:
+    if args.rounding or args.seed is not None or args.state:
         import dataclasses
         if args.rounding:
             w = dataclasses.replace(w, rounding=args.rounding)
         if args.seed is not None:
             w = dataclasses.replace(w, sr_seed=args.seed)
+        if args.state:
+            w = dataclasses.replace(w, state=args.state)
     if args.impl == "reference":
         return run_reference(args, w)
     return run_ours(args, w)
