@@ -11,7 +11,7 @@
 // a two-stage shared-memory ring by bulk asynchronous copies, so the next
 // head's copy overlaps this head's arithmetic.  Every thread takes the same
 // path through the barriers: the one early exit (a stage wait that ran out) is
-// decided for the whole CTA at once.
+// decided for the whole CTA at once, at the head's first barrier.
 //
 // Per head, in the canonical order the oracle follows:
 //   u_j = sum_i c_ij (s_i k_i)  (8 partials + XOR butterfly),
@@ -144,11 +144,15 @@ __device__ __forceinline__ void ka_issue(const DecodeParams& p, int hu, uint8_t*
     bulk_g2s(s + L.off_v, static_cast<const char*>(p.vC) + (long long)hu * vv, vv, bar);
 }
 
-// One head from its stage.  After the row-maxima barrier no thread reads the
-// stage again, so thread 0 refills it there with head `refill` (if any).
+// One head from its stage.  `ok`: this thread's wait for the stage succeeded;
+// the first barrier also decides, for the whole CTA, whether every thread's did
+// (false: nothing was computed, the caller stops).  After the row-maxima barrier
+// no thread reads the stage again, so thread 0 refills it there with head
+// `refill` (if any).  alpha, beta: the head's gates, loaded one head ahead.
 template <int DK, int BITS, int RND>
-__device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* st, const KaStage& L, uint8_t* work,
-                                        uint32_t bar, int b, int h, int hu, int refill) {
+__device__ __forceinline__ bool ka_head(const DecodeParams& p, uint8_t* st, const KaStage& L, uint8_t* work,
+                                        uint32_t bar, int b, int h, int hu, int refill, bool ok, float alpha,
+                                        float beta) {
     using K = KaCfg<DK>;
     constexpr int RPT = K::RPT;
     constexpr int BLOCK_BYTES = DK * kBlockCols * BITS / 8;
@@ -162,10 +166,9 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* st, cons
     uint64_t* pas = pks + K::PAIRS;  // alpha s_i
     uint64_t* pin = pas + K::PAIRS;  // inv_i (after the row maxima)
     float* rowmax = reinterpret_cast<float*>(pin + K::PAIRS);  // [nw][DK]
-    const float alpha = __ldg(p.g0 + hu), beta = __ldg(p.g1 + hu);
 
     // ---- key-axis vectors and row scales as duplicated pairs (shared by all warps)
-    for (int i = tid; i < DK; i += nt) {
+    for (int i = tid; i < DK && ok; i += nt) {
         const float q = ka_vec(st + L.off_q, i, bf16);
         const float k = ka_vec(st + L.off_k, i, bf16);
         const float s = reinterpret_cast<const float*>(st + L.off_s)[i];
@@ -176,7 +179,7 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* st, cons
         pks[pos] = pk(ks, ks);
         pas[pos] = pk(as, as);
     }
-    __syncthreads();
+    if (!__syncthreads_and(ok)) return false;
 
     // ---- this warp's block: decode, update, read out -------------------------
     const int j0 = w * kBlockCols;
@@ -280,6 +283,7 @@ __device__ __forceinline__ void ka_head(const DecodeParams& p, uint8_t* st, cons
             }
         ka_requantize_store<BITS, RND, RPT>(S2, invp, dst, g, cw, gcol, h, b, p.step, p.rk);
     }
+    return true;
 }
 
 // Shared memory: the stages, then the pair arrays and row maxima of the head in
@@ -316,12 +320,31 @@ __global__ void __launch_bounds__(512) rsq_decode_ka_kernel(const __grid_constan
         }
     int stage = 0;
     uint32_t parity = 0;
+    // the gates of the CTA's first head; each iteration loads the next head's
+    float alpha = 0.f, beta = 0.f;
+    if (static_cast<int>(blockIdx.x) < heads) {
+        alpha = __ldg(p.g0 + blockIdx.x);
+        beta = __ldg(p.g1 + blockIdx.x);
+    }
     for (int hu = static_cast<int>(blockIdx.x); hu < heads; hu += grid) {
         const uint32_t bar = bar0 + 8 * stage;
         const bool ok = mbar_wait(bar, parity, p.wait_iters);
-        if (!__syncthreads_and(ok)) {
-            // the whole CTA leaves; first wait (bounded) for every stage copy it
-            // issued that has not landed, so none writes into a CTA that is gone
+        float na = 0.f, nb = 0.f;
+        if (hu + grid < heads) {
+            na = __ldg(p.g0 + hu + grid);
+            nb = __ldg(p.g1 + hu + grid);
+        }
+        const int b = hu / p.H, h = hu - b * p.H;
+        const long long next = static_cast<long long>(hu) + static_cast<long long>(kKaStages) * grid;
+        const int refill = next < heads ? static_cast<int>(next) : -1;
+        uint8_t* st = smem + stage * L.bytes;
+        const bool done = (p.head_bits[h] == 8)
+                              ? ka_head<DK, 8, RND>(p, st, L, work, bar, b, h, hu, refill, ok, alpha, beta)
+                              : ka_head<DK, 4, RND>(p, st, L, work, bar, b, h, hu, refill, ok, alpha, beta);
+        if (!done) {
+            // a stage wait ran out (decided for the whole CTA): the CTA leaves,
+            // first waiting (bounded) for every stage copy it issued that has
+            // not landed, so none writes into a CTA that is gone
             if (tid == 0) {
                 atomicOr(p.flag, kFlagTimeout);
                 for (int s = 0; s < kKaStages; ++s) {
@@ -332,14 +355,8 @@ __global__ void __launch_bounds__(512) rsq_decode_ka_kernel(const __grid_constan
             }
             return;
         }
-        const int b = hu / p.H, h = hu - b * p.H;
-        const long long next = static_cast<long long>(hu) + static_cast<long long>(kKaStages) * grid;
-        const int refill = next < heads ? static_cast<int>(next) : -1;
-        uint8_t* st = smem + stage * L.bytes;
-        if (p.head_bits[h] == 8)
-            ka_head<DK, 8, RND>(p, st, L, work, bar, b, h, hu, refill);
-        else
-            ka_head<DK, 4, RND>(p, st, L, work, bar, b, h, hu, refill);
+        alpha = na;
+        beta = nb;
         if (++stage == kKaStages) {
             stage = 0;
             parity ^= 1u;
